@@ -183,6 +183,9 @@ def _lloyd_max(bits: int, tol: float, max_iter: int):
             break
     else:
         raise RuntimeError("Lloyd-Max did not converge")
+    # N(0,1) is symmetric, so the fixed point is: c_j = -c_{L-1-j}. Make that exact, which
+    # puts the middle boundary exactly at 0 (a zero coordinate then ties to the lower level).
+    c = [(c[j] - c[levels - 1 - j]) / 2.0 for j in range(levels)]
     beta = [(c[j] + c[j + 1]) / 2.0 for j in range(levels - 1)]
     edges = [-math.inf] + beta + [math.inf]
     dist = 1.0 - sum(c[j] ** 2 * (_cdf(edges[j + 1]) - _cdf(edges[j])) for j in range(levels))
