@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of the compressed-KV decode hot path on B200.
+
+A step is one decode step of one attention layer of the workload: the new token's K and V
+are quantised into the packed cache (tq_quantize_kv at position T-1), then decode attention
+runs over all T cached tokens (tq_decode_attention: split-K kernel + combine). The headline
+value is packed-KV bytes read per step / step time (GB/s), summed over ranks (one replica
+per GPU, weak scaling). Inputs are seeded synthetic tensors resident in HBM; the packed
+cache (419 MB for the default workload) is larger than the 126 MB L2, so no flush is needed.
+
+Side measurements on rank 0 (outside the timed loop): the decode call alone (roofline), the
+bulk quantise of the whole layer (Mtok/s), the bf16 kernel of the same design (speedup),
+an end-to-end run from pinned host buffers, the oracle on a bounded sample (cpu_baseline),
+and nvidia-smi clocks sampled during the timed loop.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn GB/s & % of B200 HBM peak on packed KV; quantize Mtok/s"
+DEFAULT_WORKLOAD = "llama3_8b_decode_32k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-side", action="store_true", help="skip side measurements")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+def kernel_traffic():
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary, if the
+    decode source is unchanged since the capture (else null)."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, "quantized_decode_attention_kv_b200", "csrc", "decode.cu")
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if rec.get("decode_cu_sha256") != digest:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class Clocks:
+    """nvidia-smi samples every 200 ms while the timed loop runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        load = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) arm
+def oracle_sample(w, heads: int):
+    """Records and queries for `heads` (b, KV-head) slices of the workload, full context."""
+    import numpy as np
+
+    import oracle as O
+    from quantized_decode_attention_kv_b200.workloads import make_inputs
+    K, V, q = make_inputs(w, B=1, Hkv=heads, Hq=heads * w.G)
+    samples = []
+    for h in range(heads):
+        Kn = K[0, h].float().numpy().astype(np.float64)
+        Vn = V[0, h].float().numpy().astype(np.float64)
+        kr = O.quantize(Kn, w.k_bits, w.k_mode, seed=w.seed, qjl_seed=w.qjl_seed, m=w.qjl_m or None)
+        vr = O.quantize(Vn, w.v_bits, w.v_mode, seed=w.seed, qjl_seed=w.qjl_seed, m=w.qjl_m or None)
+        qs = q[:, h * w.G:(h + 1) * w.G].float().numpy().astype(np.float64)
+        samples.append((qs, kr, vr))
+    rec_bytes = (O.record_bytes(w.d, w.k_bits, w.k_mode, w.qjl_m or None)
+                 + O.record_bytes(w.d, w.v_bits, w.v_mode, w.qjl_m or None))
+    return samples, rec_bytes * w.T
+
+
+def oracle_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:  # noqa: BLE001
+        blas = 1
+    return blas, len(os.sched_getaffinity(0))
+
+
+def time_oracle_decode(w, budget_s: float = 12.0):
+    import oracle as O
+    samples, per_head_bytes = oracle_sample(w, heads=2)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        qs, kr, vr = samples[reps % len(samples)]
+        O.decode_compressed(qs, [kr], [vr], 1, 1, w.scale)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 200:
+            break
+    blas, aff = oracle_cores()
+    return {"value": per_head_bytes * reps / el / 1e9, "unit": "GB/s", "cores": blas,
+            "kind": "oracle",
+            "sample": (f"{reps} oracle decode steps of one (batch, KV head) slice each: dequantise "
+                       f"{w.T} K and V records (float64, explicit Hadamard) + two-pass softmax for "
+                       f"{w.G} query heads; {per_head_bytes} packed bytes per slice; "
+                       f"{blas} BLAS threads of {aff} cores in affinity")}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from quantized_decode_attention_kv_b200.workloads import WORKLOADS
+    import oracle as O
+    w = WORKLOADS[args.workload]
+    samples, per_head_bytes = oracle_sample(w, heads=2)
+    times = []
+    for i in range(args.warmup + args.steps):
+        qs, kr, vr = samples[i % len(samples)]
+        t0 = time.perf_counter()
+        O.decode_compressed(qs, [kr], [vr], 1, 1, w.scale)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    step = statistics.mean(times)
+    value = per_head_bytes / step / 1e9
+    blas, aff = oracle_cores()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "sample": "one (batch, KV head) slice per step, full context",
+                       "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "k_bits": w.k_bits,
+                       "v_bits": w.v_bits},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": blas, "kind": "oracle",
+                             "sample": f"oracle decode of one (b, KV head) slice of {w.T} tokens per step; "
+                                       f"{blas} BLAS threads of {aff} cores"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ CUDA arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_decode_attention_kv_b200 import tq
+    from quantized_decode_attention_kv_b200.workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = WORKLOADS[args.workload]
+    K, V, q = make_inputs(w, device="cuda", layer=rank)
+    cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, w.k_mode, w.v_mode, w.qjl_m,
+                       w.qjl_m, seed=w.seed, qjl_seed=w.qjl_seed)
+    tq.tq_quantize_kv(K, V, cache)  # prefill the whole context
+    k_new = K[:, :, w.T - 1:].contiguous()
+    v_new = V[:, :, w.T - 1:].contiguous()
+    out = torch.empty(w.B, w.Hq, w.d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, w.Hq, w.T))
+    stream = torch.cuda.current_stream()
+    packed = cache.packed_bytes(w.T)
+
+    def step():
+        tq.tq_quantize_kv(k_new, v_new, cache, t_offset=w.T - 1, stream=stream)
+        tq.tq_decode_attention(q, cache, w.T, w.scale, out, ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = Clocks(local)
+    with clocks:
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * packed / (ms * 1e-3) / 1e9
+    launches_per_step = 4  # quantise K, quantise V, split-K decode, combine
+
+    side = {}
+    if rank == 0 and not args.no_side:
+        side = side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new, packed, stream)
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    hbm, hbm_src = peaks()
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
+                   "k": f"{w.k_bits}-bit {'MSE' if w.k_mode == 0 else 'PROD'}",
+                   "v": f"{w.v_bits}-bit {'MSE' if w.v_mode == 0 else 'PROD'}",
+                   "packed_bytes_per_step": packed,
+                   "step": "quantise 1 new token (K,V) + decode attention over T tokens",
+                   "arithmetic": "u8 packed codes, f32 scores/softmax/accumulation, bf16 query",
+                   "l2": "no flush: packed cache per step larger than the 126 MB L2",
+                   "parallelism": f"{world} independent replica(s), one per GPU"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if side:
+        dec_gbs = packed / side["decode_s"] / 1e9
+        line["roofline"] = {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
+                            "frac": dec_gbs / hbm, "traffic": kernel_traffic(),
+                            "kernel": "tq_decode_attention (split-K kernel + combine), CUDA events",
+                            "peak_source": hbm_src}
+        line["e2e"] = side["e2e"]
+        line["cpu_baseline"] = side["cpu_baseline"]
+        line["decode_us"] = side["decode_s"] * 1e6
+        line["quantize"] = side["quantize"]
+        line["bf16_decode"] = side["bf16"]
+        line["speedup_vs_bf16"] = side["bf16"]["us"] / (side["decode_s"] * 1e6)
+    print(json.dumps(line), flush=True)
+
+
+def _time(fn, stream, reps, torch):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fn()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps * 1e-3
+
+
+def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new, packed, stream):
+    hbm, _ = peaks()
+    res = {}
+    # decode call alone (split-K kernel + combine)
+    res["decode_s"] = _time(lambda: tq.tq_decode_attention(q, cache, w.T, w.scale, out, ws, stream=stream),
+                            stream, max(args.steps, 20), torch)
+    # bulk quantise of the whole layer: B*T token positions, all KV heads, K and V
+    qs = _time(lambda: tq.tq_quantize_kv(K, V, cache, stream=stream), stream, 5, torch)
+    in_bytes = (K.numel() + V.numel()) * K.element_size()
+    q_bytes = in_bytes + packed
+    res["quantize"] = {"us": qs * 1e6, "mtok_s": w.B * w.T / qs / 1e6, "gbs": q_bytes / qs / 1e9,
+                       "frac": q_bytes / qs / 1e9 / hbm, "bytes": q_bytes,
+                       "token": "one (sequence, position) of one layer: all KV heads, K and V"}
+    # the same split-K design over the unquantised bf16 cache
+    if K.dtype == torch.bfloat16:
+        wsb = tq.workspace(tq.tq_decode_bf16_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.d))
+        qb = q.to(torch.bfloat16)
+        bs = _time(lambda: tq.tq_decode_attention_bf16(qb, K, V, w.T, w.scale, out, wsb, stream=stream),
+                   stream, 10, torch)
+        bbytes = (K.numel() + V.numel()) * 2
+        res["bf16"] = {"us": bs * 1e6, "gbs": bbytes / bs / 1e9, "frac": bbytes / bs / 1e9 / hbm,
+                       "bytes": bbytes}
+    else:
+        res["bf16"] = {"us": float("nan")}
+    # end to end through the C ABI from pinned host buffers: H2D of the step's inputs (query,
+    # new token's K and V), the two calls, D2H of the attention output
+    hq = q.cpu().pin_memory()
+    hk = k_new.cpu().pin_memory()
+    hv = v_new.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        tq.tq_quantize_kv(dk, dv, cache, t_offset=w.T - 1, stream=stream)
+        tq.tq_decode_attention(dq, cache, w.T, w.scale, out, ws, stream=stream)
+        hout.copy_(out, non_blocking=True)
+
+    es = _time(e2e_step, stream, max(args.steps, 10), torch)
+    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+    res["e2e"] = {"value": packed / es / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                  "d2h_bytes_per_step": hout.numel() * hout.element_size(), "ms_per_step": es * 1e3}
+    # the oracle on the host cores, bounded sample
+    if args.gpus == 1:
+        res["cpu_baseline"] = time_oracle_decode(w)
+    return res
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+/*
+ * tq.h -- C ABI of libtq: TurboQuant-style KV-cache compression and decode attention over
+ * the compressed cache, for one NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages on TurboQuant):
+ *   "Closing - The Three-Step Summary", Step 1 Rotate: a Walsh-Hadamard transform with
+ *     random signs is applied to each K/V vector; it preserves inner products.
+ *   Step 2 Quantize: each rotated coordinate gets a Lloyd-Max scalar code for the Gaussian,
+ *     centroids scaled by 1/sqrt(d).
+ *   Step 3 Correct: below 3 bits, (b-1)-bit codes plus a 1-bit QJL sketch of the residual
+ *     (TurboQuant_prod); at 3+ bits, codes only (TurboQuant_mse).
+ *   "What the Paper Doesn't Tell You", Finding 1: keys and values take separate bit-widths.
+ *   "Where This Fits in the Inference Stack", TensorRT-LLM section: dequantisation happens
+ *     inside the attention kernel, in registers, while K/V tiles stream from HBM.
+ *   "Why the KV Cache Exists", What's in the KV Cache: per layer and KV head, K and V are
+ *     [T x d] matrices; a decode query attends to all T cached tokens.
+ *
+ * Conventions shared by every entry point
+ *   - Return: int status, TQ_OK (0) on success. On failure nothing is launched and
+ *     tq_last_error() returns a message (thread-local; valid until the next failing call on
+ *     the same thread). Size queries return 0 on invalid arguments.
+ *   - Memory: every pointer is caller-owned. The library never allocates, frees or
+ *     synchronises; device work is enqueued on the given stream (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream) and is asynchronous. Device pointers must be
+ *     16-byte aligned. Host pointers have no alignment rule.
+ *   - Shapes: d (head_dim) is a power of two in 16..256. Bit-widths are 1..4.
+ *     qjl_m (QJL sketch length) is 0 (meaning d) or a multiple of 8 in 8..256.
+ *   - Arrays are row-major and C-contiguous. The cache is token-major per (batch, KV head):
+ *     element (b, h, t) of a cache array lives at index (b*Hkv + h)*T_cap + t.
+ *   - GQA: query head hq reads KV head hq / (Hq/Hkv) (consecutive query heads share a KV
+ *     head); Hq must be a multiple of Hkv.
+ *   - Rotation: R x = H D x / sqrt(d), H the natural-order (Sylvester) Hadamard matrix,
+ *     D = diag(+-1) with D_ii = -1 iff bit i of the SplitMix64(seed) stream is set (bit i%64
+ *     of output i/64). One sign vector per cache, shared by K, V and the query.
+ *   - Codes: code i of a record occupies bits [i*w, i*w+w) of a little-endian bit stream
+ *     (stream bit k = bit k%8 of byte k/8); codes index the Lloyd-Max levels in ascending
+ *     order; a coordinate exactly on a boundary takes the lower level. QJL bit j = 1 iff
+ *     (S r)_j < 0.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ_OK 0
+#define TQ_ERR_INVALID_ARG 1 /* null pointer, bad size or shape, misaligned pointer      */
+#define TQ_ERR_UNSUPPORTED 2 /* d, bits, mode or qjl_m outside the supported set          */
+#define TQ_ERR_WORKSPACE 3   /* workspace missing or smaller than the size query says      */
+#define TQ_ERR_CUDA 4        /* a CUDA runtime call or kernel launch failed                */
+
+#define TQ_MSE 0  /* TurboQuant_mse: b-bit Lloyd-Max codes                                  */
+#define TQ_PROD 1 /* TurboQuant_prod: (b-1)-bit codes + 1-bit QJL residual sketch + ||r||   */
+
+#define TQ_F32 0
+#define TQ_BF16 1
+#define TQ_F16 2
+
+/* Quantiser of one tensor (keys or values). */
+typedef struct {
+  int bits;  /* total bits per coordinate, 1..4                                          */
+  int mode;  /* TQ_MSE or TQ_PROD ("Closing", Step 3: PROD is meant for bits <= 2)        */
+  int qjl_m; /* PROD only: QJL rows m (0 = d); ignored for TQ_MSE                          */
+} tq_qcfg;
+
+/* One layer's compressed KV cache. All pointers are device pointers owned by the caller.
+ * Per (b, h, t) record, for each of K and V:
+ *   codes  [B][Hkv][T_cap][tq_code_bytes]  uint8   Lloyd-Max codes (absent when 0 bits)
+ *   norm   [B][Hkv][T_cap]                 uint16  IEEE fp16 bits of ||x||
+ *   signs  [B][Hkv][T_cap][tq_sign_bytes]  uint8   PROD only: QJL sign bits, else NULL
+ *   rnorm  [B][Hkv][T_cap]                 uint16  PROD only: fp16 ||r||, else NULL
+ *   qjl    [m][d]                          float   PROD only: the projection S (fill it
+ *                                                  with tq_make_qjl_matrix), else NULL  */
+typedef struct {
+  int B, Hkv, T_cap, d;
+  uint64_t seed; /* rotation seed: fixed per model load, so records are reproducible    */
+  tq_qcfg kc, vc;
+  uint8_t *k_codes, *v_codes;
+  uint16_t *k_norm, *v_norm;
+  uint8_t *k_signs, *v_signs;
+  uint16_t *k_rnorm, *v_rnorm;
+  const float *k_qjl, *v_qjl;
+} tq_cache;
+
+/* Message for the last failure on the calling thread ("" if none). */
+const char *tq_last_error(void);
+
+/* ---------------------------------------------------------------- host-side helpers */
+
+/* Gaussian Lloyd-Max codebook for `bits` (1..4) at head dimension d ("Closing", Step 2):
+ * writes 2^bits centroids (ascending) and 2^bits - 1 decision boundaries, both already
+ * scaled by 1/sqrt(d) (the unit-norm vector's scale), into caller host arrays. Computed in
+ * double by alternating the midpoint and conditional-mean conditions to a 1e-13 fixed
+ * point. Errors: TQ_ERR_UNSUPPORTED, TQ_ERR_INVALID_ARG (null outputs). */
+int tq_make_codebook(int bits, int d, float *centroids, float *bounds);
+
+/* The rotation's sign vector as d bits (d/8 bytes, host): bit i set means D_ii = -1.
+ * 16 bytes at d = 128 ("What the Paper Doesn't Tell You", Finding 4). */
+int tq_make_signs(uint64_t seed, int d, uint8_t *signs);
+
+/* QJL projection S [m][d] (host, row-major float32), i.i.d. N(0,1): entries 2k, 2k+1 are
+ * the Box-Muller pair of the SplitMix64(seed) uniforms u = (word >> 11) * 2^-53 numbered
+ * 2k, 2k+1 (rho = sqrt(-2 ln(1-u_2k)), theta = 2 pi u_2k+1), computed in double and rounded
+ * to float32. m*d must be even; m, d in the supported ranges ("Closing", Step 3). */
+int tq_make_qjl_matrix(uint64_t seed, int m, int d, float *S);
+
+/* Bytes per vector: packed codes (d * Lloyd-Max bits / 8), QJL sign bytes (m/8 in PROD,
+ * else 0), and the whole stored record (codes + signs + 2-byte norm [+ 2-byte rnorm]).
+ * At d = 128 a 3-bit MSE record is 50 bytes ("Finding 3": 5.12x vs fp16). 0 if invalid. */
+size_t tq_code_bytes(int d, tq_qcfg c);
+size_t tq_sign_bytes(int d, tq_qcfg c);
+size_t tq_record_bytes(int d, tq_qcfg c);
+
+/* ---------------------------------------------------------------- device entry points */
+
+/* Quantise-on-write ("Closing", Steps 1-3). K and V are device arrays [B][Hkv][T][d] of
+ * `dtype` (TQ_F32 / TQ_BF16 / TQ_F16); either may be NULL to write only the other. Token t
+ * is stored at cache position t_offset + t (0 <= t_offset, t_offset + T <= T_cap). T = 0
+ * is a no-op. Per vector: n = ||x|| (fp32, stored fp16); z = H D x / n; codes by the
+ * boundary count (fp32 decisions); PROD: r = (z - c[code]) / sqrt(d), rnorm = ||r||,
+ * QJL bits of S r. A zero vector stores norm 0 (its reconstruction is 0). */
+int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
+                   const tq_cache *cache, void *stream);
+
+/* Workspace bytes tq_decode_attention needs for this shape (split-K partials: running
+ * max, running sum and the rotated-domain accumulator per split and query head). 0 if
+ * invalid. Depends on the current device's SM count. */
+size_t tq_decode_workspace_bytes(int B, int Hq, int T_len, const tq_cache *cache);
+
+/* Decode attention over cache positions [0, T_len) of every (b, KV head) ("Where This
+ * Fits", TensorRT-LLM section: dequantise in registers inside the attention kernel).
+ * q [B][Hq][d] of `dtype`; out [B][Hq][d] float32; scale is the softmax scale (e.g.
+ * 1/sqrt(d)). The query is rotated once (q~ = scale H D q / d), so that
+ * scale q.k_hat = ||k|| sum_i q~_i c[code_i] (+ the QJL term); split-K online softmax;
+ * values accumulate in the rotated domain; one inverse rotation per output. Needs
+ * T_len >= 1 and ws_bytes >= tq_decode_workspace_bytes(...). Errors as above plus
+ * TQ_ERR_WORKSPACE. */
+int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale,
+                        const tq_cache *cache, float *out, void *ws, size_t ws_bytes,
+                        void *stream);
+
+/* Dequantise cache positions [0, T_len) of K (which = 0) or V (which = 1) into out
+ * [B][Hkv][T_len][d] of `dtype` in the original domain: x_hat = n D H c / d (MSE), plus
+ * the QJL residual estimate sqrt(d) gamma sqrt(pi/2)/m S^T s inside the bracket (PROD). */
+int tq_dequantize(const tq_cache *cache, int which, int T_len, void *out, int dtype,
+                  void *stream);
+
+/* Same split-K design over an unquantised bf16 cache: K, V [B][Hkv][T_cap][d] bf16
+ * (positions [0, T_len) are read), q [B][Hq][d] bf16, out [B][Hq][d] float32. The
+ * comparator for the compressed kernel and the path for layers kept at full precision
+ * ("What the Paper Doesn't Tell You", Finding 1: boundary layers). */
+size_t tq_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int T_len, int d);
+int tq_decode_attention_bf16(const void *q, int Hq, const void *K, const void *V, int B,
+                             int Hkv, int T_cap, int T_len, int d, float scale, float *out,
+                             void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

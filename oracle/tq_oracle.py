@@ -42,6 +42,7 @@ MSE = 0   # TurboQuant_mse: b-bit Lloyd-Max codes only
 PROD = 1  # TurboQuant_prod: (b-1)-bit Lloyd-Max codes + 1-bit QJL residual sketch
 
 _MASK64 = (1 << 64) - 1
+_ROWS = 1024  # vectors per chunk in quantize/boundary_distance (memory only)
 _GAMMA = 0x9E3779B97F4A7C15
 
 
@@ -277,6 +278,7 @@ class Records:
     z: np.ndarray            # [N, d] rotated coordinates on the N(0,1) scale (H D x / ||x||)
     proj: np.ndarray         # [N, m] S r (PROD) or [N, 0]
     rnorm: np.ndarray        # [N] exact residual norm (PROD) or zeros
+    norm: np.ndarray         # [N] exact float64 norm ||x||
 
 
 def quantize(x: np.ndarray, bits: int, mode: int = MSE, seed: int = 0, qjl_seed: int = 1,
@@ -312,10 +314,14 @@ def quantize(x: np.ndarray, bits: int, mode: int = MSE, seed: int = 0, qjl_seed:
 
     if wbits > 0:
         cent, beta, _ = lloyd_max_gaussian(wbits)
-        codes = np.argmin(np.abs(z[:, :, None] - cent[None, None, :]), axis=2)
-        counted = np.searchsorted(beta, z, side="left")
-        exact_tie = np.min(np.abs(z[:, :, None] - beta[None, None, :]), axis=2) < 1e-12
-        assert np.all((codes == counted) | exact_tie), "nearest centroid != boundary count"
+        codes = np.empty(z.shape, dtype=np.int64)
+        for lo in range(0, n_vec, _ROWS):  # rows are independent; chunks bound the temporaries
+            zc = z[lo:lo + _ROWS]
+            codes[lo:lo + _ROWS] = np.argmin(np.abs(zc[:, :, None] - cent[None, None, :]), axis=2)
+            counted = np.searchsorted(beta, zc, side="left")
+            exact_tie = np.min(np.abs(zc[:, :, None] - beta[None, None, :]), axis=2) < 1e-12
+            assert np.all((codes[lo:lo + _ROWS] == counted) | exact_tie), \
+                "nearest centroid != boundary count"
         chat = cent[codes]
     else:
         codes = np.zeros((n_vec, d), dtype=np.int64)
@@ -337,7 +343,7 @@ def quantize(x: np.ndarray, bits: int, mode: int = MSE, seed: int = 0, qjl_seed:
         qpacked = np.zeros((n_vec, 0), dtype=np.uint8)
         rnorm16 = np.zeros(n_vec, dtype=np.float16)
     return Records(bits, mode, d, m, seed, qjl_seed, codes, packed, norm16, qbits, qpacked,
-                   rnorm16, z, proj, rnorm)
+                   rnorm16, z, proj, rnorm, norm)
 
 
 def records_from_packed(bits: int, mode: int, d: int, packed: np.ndarray, norm16: np.ndarray,
@@ -357,7 +363,8 @@ def records_from_packed(bits: int, mode: int, d: int, packed: np.ndarray, norm16
     return Records(bits, mode, d, m, seed, qjl_seed, codes, np.asarray(packed),
                    np.asarray(norm16, dtype=np.float16), qbits, np.asarray(qjl_packed),
                    np.asarray(rnorm16, dtype=np.float16), np.zeros((n_vec, d)),
-                   np.zeros((n_vec, 0)), np.zeros(n_vec))
+                   np.zeros((n_vec, 0)), np.zeros(n_vec),
+                   np.asarray(norm16, dtype=np.float16).astype(np.float64))
 
 
 def dequantize(rec: Records) -> np.ndarray:
@@ -390,7 +397,11 @@ def boundary_distance(rec: Records) -> np.ndarray:
     if wbits == 0:
         return np.full(rec.z.shape, np.inf)
     beta = lloyd_max_gaussian(wbits)[1]
-    return np.min(np.abs(rec.z[:, :, None] - beta[None, None, :]), axis=2)
+    out = np.empty(rec.z.shape)
+    for lo in range(0, rec.z.shape[0], _ROWS):
+        zc = rec.z[lo:lo + _ROWS]
+        out[lo:lo + _ROWS] = np.min(np.abs(zc[:, :, None] - beta[None, None, :]), axis=2)
+    return out
 
 
 # ----------------------------------------------------------------------------------------

@@ -1,0 +1,441 @@
+// C-ABI host layer of libtq: argument validation, the Gaussian Lloyd-Max codebook (double),
+// the seeded sign vector and QJL matrix (SplitMix64 + Box-Muller), split planning, and the
+// calls into the CUDA launchers. Nothing here allocates device memory or synchronises.
+#include "../../include/tq.h"
+#include "tq_internal.h"
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+// ---------------------------------------------------------------- SplitMix64
+// Steele, Lea & Flood, "Fast splittable pseudorandom number generators" (OOPSLA 2014):
+// output k (k >= 0) from seed s is mix(s + (k+1) * 0x9E3779B97F4A7C15).
+uint64_t splitmix64_at(uint64_t seed, uint64_t k) {
+  uint64_t z = seed + (k + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+// ---------------------------------------------------------------- Lloyd-Max (double)
+// Gaussian Lloyd-Max quantiser ("Closing - The Three-Step Summary", Step 2): alternate
+// boundaries = midpoints of neighbouring centroids and centroids = conditional means of
+// N(0,1) on their cells, until no centroid moves by more than 1e-13.
+double npdf(double x) { return std::isinf(x) ? 0.0 : std::exp(-0.5 * x * x) * 0.3989422804014327; }
+double ncdf(double x) { return 0.5 * std::erfc(-x * 0.7071067811865476); }
+
+double ninv(double p) { // bisection on the CDF; only the starting point depends on it
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 200; ++i) {
+    double mid = 0.5 * (lo + hi);
+    (ncdf(mid) < p ? lo : hi) = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+struct DoubleCodebook {
+  double c[16], beta[15];
+  int levels;
+  bool ok;
+};
+
+DoubleCodebook compute_lloyd_max(int wbits) {
+  DoubleCodebook cb{};
+  const int L = 1 << wbits;
+  cb.levels = L;
+  double c[16], nc[16], edges[17];
+  for (int j = 0; j < L; ++j) c[j] = ninv((j + 0.5) / L);
+  cb.ok = false;
+  for (int it = 0; it < 200000; ++it) {
+    edges[0] = -INFINITY;
+    edges[L] = INFINITY;
+    for (int j = 0; j + 1 < L; ++j) edges[j + 1] = 0.5 * (c[j] + c[j + 1]);
+    double moved = 0.0;
+    for (int j = 0; j < L; ++j) {
+      nc[j] = (npdf(edges[j]) - npdf(edges[j + 1])) / (ncdf(edges[j + 1]) - ncdf(edges[j]));
+      moved = std::fmax(moved, std::fabs(nc[j] - c[j]));
+    }
+    std::memcpy(c, nc, sizeof(double) * L);
+    if (moved < 1e-13) {
+      cb.ok = true;
+      break;
+    }
+  }
+  // The Gaussian is symmetric, so the fixed point satisfies c_j = -c_{L-1-j}; enforce it
+  // exactly so the middle boundary is exactly 0 (a zero coordinate takes the lower level).
+  for (int j = 0; j < L / 2; ++j) {
+    const double s = 0.5 * (c[L - 1 - j] - c[j]);
+    c[L - 1 - j] = s;
+    c[j] = -s;
+  }
+  for (int j = 0; j < L; ++j) cb.c[j] = c[j];
+  for (int j = 0; j + 1 < L; ++j) cb.beta[j] = 0.5 * (c[j] + c[j + 1]);
+  return cb;
+}
+
+const DoubleCodebook &lloyd_max(int wbits) { // wbits in 1..4, computed once
+  static DoubleCodebook table[5];
+  static std::once_flag once[5];
+  std::call_once(once[wbits], [wbits] { table[wbits] = compute_lloyd_max(wbits); });
+  return table[wbits];
+}
+
+// ---------------------------------------------------------------- validation helpers
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_qcfg(int d, const tq_qcfg &c, const char *name) {
+  if (!pow2_in(d, 16, 256))
+    return fail(TQ_ERR_UNSUPPORTED, "d=%d: head_dim must be a power of two in 16..256", d);
+  if (c.bits < 1 || c.bits > 4)
+    return fail(TQ_ERR_UNSUPPORTED, "%s.bits=%d: bits must be 1..4", name, c.bits);
+  if (c.mode != TQ_MSE && c.mode != TQ_PROD)
+    return fail(TQ_ERR_UNSUPPORTED, "%s.mode=%d: mode must be TQ_MSE or TQ_PROD", name, c.mode);
+  if (c.mode == TQ_PROD) {
+    int m = c.qjl_m == 0 ? d : c.qjl_m;
+    if (m < 8 || m > tq::kMaxM || m % 8)
+      return fail(TQ_ERR_UNSUPPORTED, "%s.qjl_m=%d: must be 0 or a multiple of 8 in 8..%d",
+                  name, c.qjl_m, tq::kMaxM);
+  }
+  return TQ_OK;
+}
+
+int resolve_tensor(const tq_cache &c, int which, tq::TensorArgs *t) {
+  const tq_qcfg &q = which == 0 ? c.kc : c.vc;
+  const char *name = which == 0 ? "kc" : "vc";
+  int st = check_qcfg(c.d, q, name);
+  if (st) return st;
+  std::memset(t, 0, sizeof *t);
+  t->bits = q.bits;
+  t->mode = q.mode;
+  t->wbits = q.mode == TQ_MSE ? q.bits : q.bits - 1;
+  t->m = q.mode == TQ_PROD ? (q.qjl_m == 0 ? c.d : q.qjl_m) : 0;
+  t->code_bytes = c.d * t->wbits / 8;
+  t->sign_bytes = t->m / 8;
+  t->codes = which == 0 ? c.k_codes : c.v_codes;
+  t->norm = which == 0 ? c.k_norm : c.v_norm;
+  t->signs = which == 0 ? c.k_signs : c.v_signs;
+  t->rnorm = which == 0 ? c.k_rnorm : c.v_rnorm;
+  t->S = which == 0 ? c.k_qjl : c.v_qjl;
+  const char *tn = which == 0 ? "K" : "V";
+  if (t->wbits > 0 && (!t->codes || !aligned16(t->codes)))
+    return fail(TQ_ERR_INVALID_ARG, "%s codes pointer is NULL or not 16-byte aligned", tn);
+  if (!t->norm || !aligned16(t->norm))
+    return fail(TQ_ERR_INVALID_ARG, "%s norm pointer is NULL or not 16-byte aligned", tn);
+  if (q.mode == TQ_PROD) {
+    if (!t->signs || !aligned16(t->signs) || !t->rnorm || !aligned16(t->rnorm) || !t->S ||
+        !aligned16(t->S))
+      return fail(TQ_ERR_INVALID_ARG,
+                  "%s is TQ_PROD: signs, rnorm and qjl pointers must be non-NULL and 16-byte "
+                  "aligned", tn);
+  }
+  tq::Codebook &cb = t->cb;
+  std::memset(&cb, 0, sizeof cb);
+  if (t->wbits == 0) {
+    cb.levels = 1;
+  } else {
+    const DoubleCodebook &d = lloyd_max(t->wbits);
+    if (!d.ok) return fail(TQ_ERR_UNSUPPORTED, "Lloyd-Max iteration did not converge");
+    cb.levels = d.levels;
+    for (int j = 0; j < d.levels; ++j) cb.c[j] = static_cast<float>(d.c[j]);
+    for (int j = 0; j + 1 < d.levels; ++j) cb.beta[j] = static_cast<float>(d.beta[j]);
+  }
+  return TQ_OK;
+}
+
+int check_cache(const tq_cache *c) {
+  if (!c) return fail(TQ_ERR_INVALID_ARG, "cache is NULL");
+  if (c->B < 1 || c->Hkv < 1 || c->T_cap < 1)
+    return fail(TQ_ERR_INVALID_ARG, "cache shape B=%d Hkv=%d T_cap=%d must be positive", c->B,
+                c->Hkv, c->T_cap);
+  if (!pow2_in(c->d, 16, 256))
+    return fail(TQ_ERR_UNSUPPORTED, "d=%d: head_dim must be a power of two in 16..256", c->d);
+  if ((long long)c->B * c->Hkv * c->T_cap > (1ll << 40))
+    return fail(TQ_ERR_INVALID_ARG, "cache too large");
+  if (c->B > 65535 || c->Hkv > 4096)
+    return fail(TQ_ERR_INVALID_ARG, "B=%d must be <= 65535 and Hkv=%d <= 4096", c->B, c->Hkv);
+  return TQ_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+int cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return TQ_OK;
+  return fail(TQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool dtype_ok(int dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
+
+} // namespace
+
+extern "C" {
+
+const char *tq_last_error(void) { return g_err.c_str(); }
+
+int tq_make_codebook(int bits, int d, float *centroids, float *bounds) {
+  if (bits < 1 || bits > 4) return fail(TQ_ERR_UNSUPPORTED, "bits=%d: must be 1..4", bits);
+  if (!pow2_in(d, 16, 256))
+    return fail(TQ_ERR_UNSUPPORTED, "d=%d: head_dim must be a power of two in 16..256", d);
+  if (!centroids || !bounds) return fail(TQ_ERR_INVALID_ARG, "output pointer is NULL");
+  const DoubleCodebook &cb = lloyd_max(bits);
+  if (!cb.ok) return fail(TQ_ERR_UNSUPPORTED, "Lloyd-Max iteration did not converge");
+  const double s = 1.0 / std::sqrt(static_cast<double>(d));
+  for (int j = 0; j < cb.levels; ++j) centroids[j] = static_cast<float>(cb.c[j] * s);
+  for (int j = 0; j + 1 < cb.levels; ++j) bounds[j] = static_cast<float>(cb.beta[j] * s);
+  return TQ_OK;
+}
+
+int tq_make_signs(uint64_t seed, int d, uint8_t *signs) {
+  if (!pow2_in(d, 16, 256))
+    return fail(TQ_ERR_UNSUPPORTED, "d=%d: head_dim must be a power of two in 16..256", d);
+  if (!signs) return fail(TQ_ERR_INVALID_ARG, "signs is NULL");
+  for (int byte = 0; byte < d / 8; ++byte) {
+    uint64_t w = splitmix64_at(seed, static_cast<uint64_t>(byte / 8));
+    signs[byte] = static_cast<uint8_t>(w >> (8 * (byte % 8)));
+  }
+  return TQ_OK;
+}
+
+int tq_make_qjl_matrix(uint64_t seed, int m, int d, float *S) {
+  if (!pow2_in(d, 16, 256))
+    return fail(TQ_ERR_UNSUPPORTED, "d=%d: head_dim must be a power of two in 16..256", d);
+  if (m < 8 || m > tq::kMaxM || m % 8)
+    return fail(TQ_ERR_UNSUPPORTED, "m=%d: must be a multiple of 8 in 8..%d", m, tq::kMaxM);
+  if (!S) return fail(TQ_ERR_INVALID_ARG, "S is NULL");
+  const long n = static_cast<long>(m) * d;
+  const double two_pi = 6.283185307179586;
+  for (long k = 0; k < n / 2; ++k) {
+    double u0 = static_cast<double>(splitmix64_at(seed, 2 * k) >> 11) * 0x1.0p-53;
+    double u1 = static_cast<double>(splitmix64_at(seed, 2 * k + 1) >> 11) * 0x1.0p-53;
+    double rho = std::sqrt(-2.0 * std::log(1.0 - u0));
+    double th = two_pi * u1;
+    S[2 * k] = static_cast<float>(rho * std::cos(th));
+    S[2 * k + 1] = static_cast<float>(rho * std::sin(th));
+  }
+  return TQ_OK;
+}
+
+size_t tq_code_bytes(int d, tq_qcfg c) {
+  if (check_qcfg(d, c, "cfg")) return 0;
+  int w = c.mode == TQ_MSE ? c.bits : c.bits - 1;
+  return static_cast<size_t>(d) * w / 8;
+}
+
+size_t tq_sign_bytes(int d, tq_qcfg c) {
+  if (check_qcfg(d, c, "cfg")) return 0;
+  return c.mode == TQ_PROD ? static_cast<size_t>(c.qjl_m == 0 ? d : c.qjl_m) / 8 : 0;
+}
+
+size_t tq_record_bytes(int d, tq_qcfg c) {
+  if (check_qcfg(d, c, "cfg")) return 0;
+  return tq_code_bytes(d, c) + tq_sign_bytes(d, c) + (c.mode == TQ_PROD ? 4 : 2);
+}
+
+int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
+                   const tq_cache *cache, void *stream) {
+  int st = check_cache(cache);
+  if (st) return st;
+  if (!dtype_ok(dtype)) return fail(TQ_ERR_INVALID_ARG, "dtype=%d is not F32/BF16/F16", dtype);
+  if (T < 0 || t_offset < 0 || (long long)t_offset + T > cache->T_cap)
+    return fail(TQ_ERR_INVALID_ARG, "positions [%d, %d) fall outside T_cap=%d", t_offset,
+                t_offset + T, cache->T_cap);
+  if (!K && !V) return fail(TQ_ERR_INVALID_ARG, "K and V are both NULL");
+  if ((K && !aligned16(K)) || (V && !aligned16(V)))
+    return fail(TQ_ERR_INVALID_ARG, "K/V input pointers must be 16-byte aligned");
+  tq::QuantArgs a[2];
+  for (int which = 0; which < 2; ++which) {
+    const void *x = which == 0 ? K : V;
+    if (!x) continue;
+    st = resolve_tensor(*cache, which, &a[which].t);
+    if (st) return st;
+  }
+  if (T == 0) return TQ_OK;
+  for (int which = 0; which < 2; ++which) {
+    const void *x = which == 0 ? K : V;
+    if (!x) continue;
+    tq::QuantArgs &q = a[which];
+    q.x = x;
+    q.dtype = dtype;
+    q.B = cache->B;
+    q.Hkv = cache->Hkv;
+    q.T = T;
+    q.T_cap = cache->T_cap;
+    q.t_offset = t_offset;
+    q.d = cache->d;
+    q.seed = cache->seed;
+    st = cuda_status(tq::launch_quantize(q, static_cast<cudaStream_t>(stream)), "quantize launch");
+    if (st) return st;
+  }
+  return TQ_OK;
+}
+
+size_t tq_decode_workspace_bytes(int B, int Hq, int T_len, const tq_cache *cache) {
+  if (check_cache(cache)) return 0;
+  if (Hq < 1 || Hq % cache->Hkv || T_len < 1 || T_len > cache->T_cap) {
+    fail(TQ_ERR_INVALID_ARG, "bad Hq=%d or T_len=%d", Hq, T_len);
+    return 0;
+  }
+  if (B != cache->B) {
+    fail(TQ_ERR_INVALID_ARG, "B=%d differs from cache B=%d", B, cache->B);
+    return 0;
+  }
+  if (check_qcfg(cache->d, cache->kc, "kc") || check_qcfg(cache->d, cache->vc, "vc")) return 0;
+  int sms = sm_count();
+  if (sms <= 0) {
+    fail(TQ_ERR_CUDA, "cannot query the device's SM count");
+    return 0;
+  }
+  int vm = cache->vc.mode == TQ_PROD ? (cache->vc.qjl_m ? cache->vc.qjl_m : cache->d) : 0;
+  return tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, vm, sms, false).ws_bytes;
+}
+
+int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale,
+                        const tq_cache *cache, float *out, void *ws, size_t ws_bytes,
+                        void *stream) {
+  int st = check_cache(cache);
+  if (st) return st;
+  if (!dtype_ok(dtype)) return fail(TQ_ERR_INVALID_ARG, "dtype=%d is not F32/BF16/F16", dtype);
+  if (!q || !out || !aligned16(q) || !aligned16(out))
+    return fail(TQ_ERR_INVALID_ARG, "q/out must be non-NULL and 16-byte aligned");
+  if (Hq < 1 || Hq % cache->Hkv || Hq > 65535)
+    return fail(TQ_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d (<= 65535)", Hq,
+                cache->Hkv);
+  if (T_len < 1 || T_len > cache->T_cap)
+    return fail(TQ_ERR_INVALID_ARG, "T_len=%d must be in 1..T_cap=%d", T_len, cache->T_cap);
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale is not finite");
+  tq::DecodeArgs a;
+  std::memset(&a, 0, sizeof a);
+  st = resolve_tensor(*cache, 0, &a.k);
+  if (st) return st;
+  st = resolve_tensor(*cache, 1, &a.v);
+  if (st) return st;
+  int sms = sm_count();
+  if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
+  a.plan = tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, a.v.m, sms, false);
+  if (!ws || !aligned16(ws) || ws_bytes < a.plan.ws_bytes)
+    return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
+                a.plan.ws_bytes, ws ? ws_bytes : 0);
+  a.q = q;
+  a.q_dtype = dtype;
+  a.B = cache->B;
+  a.Hq = Hq;
+  a.Hkv = cache->Hkv;
+  a.d = cache->d;
+  a.T_len = T_len;
+  a.T_cap = cache->T_cap;
+  a.scale = scale;
+  a.seed = cache->seed;
+  a.out = out;
+  a.ws = static_cast<float *>(ws);
+  return cuda_status(tq::launch_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
+}
+
+int tq_dequantize(const tq_cache *cache, int which, int T_len, void *out, int dtype,
+                  void *stream) {
+  int st = check_cache(cache);
+  if (st) return st;
+  if (which != 0 && which != 1) return fail(TQ_ERR_INVALID_ARG, "which=%d must be 0 or 1", which);
+  if (!dtype_ok(dtype)) return fail(TQ_ERR_INVALID_ARG, "dtype=%d is not F32/BF16/F16", dtype);
+  if (T_len < 0 || T_len > cache->T_cap)
+    return fail(TQ_ERR_INVALID_ARG, "T_len=%d must be in 0..T_cap=%d", T_len, cache->T_cap);
+  if (!out || !aligned16(out))
+    return fail(TQ_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
+  tq::DequantArgs a;
+  std::memset(&a, 0, sizeof a);
+  st = resolve_tensor(*cache, which, &a.t);
+  if (st) return st;
+  if (T_len == 0) return TQ_OK;
+  a.out = out;
+  a.dtype = dtype;
+  a.B = cache->B;
+  a.Hkv = cache->Hkv;
+  a.T_len = T_len;
+  a.T_cap = cache->T_cap;
+  a.d = cache->d;
+  a.seed = cache->seed;
+  return cuda_status(tq::launch_dequantize(a, static_cast<cudaStream_t>(stream)),
+                     "dequantize launch");
+}
+
+size_t tq_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int T_len, int d) {
+  if (B < 1 || Hkv < 1 || Hq < 1 || Hq % Hkv || T_len < 1 || !pow2_in(d, 16, 256)) {
+    fail(TQ_ERR_INVALID_ARG, "bad shape B=%d Hq=%d Hkv=%d T_len=%d d=%d", B, Hq, Hkv, T_len, d);
+    return 0;
+  }
+  int sms = sm_count();
+  if (sms <= 0) {
+    fail(TQ_ERR_CUDA, "cannot query the device's SM count");
+    return 0;
+  }
+  return tq::plan_decode(B, Hq, Hkv, d, T_len, 0, sms, true).ws_bytes;
+}
+
+int tq_decode_attention_bf16(const void *q, int Hq, const void *K, const void *V, int B,
+                             int Hkv, int T_cap, int T_len, int d, float scale, float *out,
+                             void *ws, size_t ws_bytes, void *stream) {
+  if (B < 1 || Hkv < 1 || T_cap < 1 || B > 65535 || Hkv > 4096)
+    return fail(TQ_ERR_INVALID_ARG, "shape B=%d Hkv=%d T_cap=%d must be positive (B <= 65535, "
+                "Hkv <= 4096)", B, Hkv, T_cap);
+  if (!pow2_in(d, 16, 256))
+    return fail(TQ_ERR_UNSUPPORTED, "d=%d: head_dim must be a power of two in 16..256", d);
+  if (Hq < 1 || Hq % Hkv || Hq > 65535)
+    return fail(TQ_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d (<= 65535)", Hq,
+                Hkv);
+  if (T_len < 1 || T_len > T_cap)
+    return fail(TQ_ERR_INVALID_ARG, "T_len=%d must be in 1..T_cap=%d", T_len, T_cap);
+  if (!q || !K || !V || !out || !aligned16(q) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(out))
+    return fail(TQ_ERR_INVALID_ARG, "q/K/V/out must be non-NULL and 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale is not finite");
+  int sms = sm_count();
+  if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
+  tq::DecodeBf16Args a;
+  std::memset(&a, 0, sizeof a);
+  a.plan = tq::plan_decode(B, Hq, Hkv, d, T_len, 0, sms, true);
+  if (!ws || !aligned16(ws) || ws_bytes < a.plan.ws_bytes)
+    return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
+                a.plan.ws_bytes, ws ? ws_bytes : 0);
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.T_len = T_len;
+  a.T_cap = T_cap;
+  a.scale = scale;
+  a.out = out;
+  a.ws = static_cast<float *>(ws);
+  return cuda_status(tq::launch_decode_bf16(a, static_cast<cudaStream_t>(stream)),
+                     "bf16 decode launch");
+}
+
+} // extern "C"

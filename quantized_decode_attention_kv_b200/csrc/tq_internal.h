@@ -1,0 +1,92 @@
+// Private interface between the C-ABI host layer (host.cpp) and the CUDA launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace tq {
+
+constexpr int kMaxM = 256;       // longest QJL sketch supported
+constexpr int kMaxSplits = 1024; // split-K upper bound per (b, q-head)
+
+// Lloyd-Max codebook on the N(0,1) scale (the kernels work on z = H D x / ||x||).
+struct Codebook {
+  float c[16];    // centroids, ascending (levels entries used)
+  float beta[15]; // decision boundaries, ascending (levels - 1 used)
+  int levels;     // 2^wbits; 1 when a PROD record carries no Lloyd-Max codes
+};
+
+// One tensor (K or V) of a cache, resolved from tq_cache + tq_qcfg.
+struct TensorArgs {
+  int bits, mode;  // as given
+  int wbits;       // Lloyd-Max bits per coordinate (bits, or bits - 1 in PROD)
+  int m;           // QJL rows (PROD), else 0
+  int code_bytes;  // d * wbits / 8
+  int sign_bytes;  // m / 8 (PROD), else 0
+  uint8_t *codes;
+  uint16_t *norm;
+  uint8_t *signs;
+  uint16_t *rnorm;
+  const float *S;  // [m][d] (PROD)
+  Codebook cb;
+};
+
+struct QuantArgs {
+  const void *x;
+  int dtype;
+  int B, Hkv, T, T_cap, t_offset, d;
+  uint64_t seed;
+  TensorArgs t;
+};
+
+struct DequantArgs {
+  void *out;
+  int dtype;
+  int B, Hkv, T_len, T_cap, d;
+  uint64_t seed;
+  TensorArgs t;
+};
+
+struct DecodePlan {
+  int tile;      // tokens per pipeline tile
+  int splits;    // context splits per (b, KV head)
+  int chunk;     // tokens per split (a multiple of tile)
+  int gc;        // query heads handled by one CTA (power of two)
+  int ws_stride; // floats per (b, q-head, split) partial record
+  size_t ws_bytes;
+};
+
+struct DecodeArgs {
+  const void *q;
+  int q_dtype;
+  int B, Hq, Hkv, d, T_len, T_cap;
+  float scale;
+  uint64_t seed;
+  TensorArgs k, v;
+  float *out;
+  float *ws;
+  DecodePlan plan;
+};
+
+struct DecodeBf16Args {
+  const void *q, *K, *V;
+  int B, Hq, Hkv, d, T_len, T_cap;
+  float scale;
+  float *out;
+  float *ws;
+  DecodePlan plan;
+};
+
+// Launchers (quantize.cu, decode.cu). Return the launch status.
+cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t s);
+cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s);
+
+// Split-K plan for the compressed and bf16 decode kernels (decode.cu).
+DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count,
+                       bool bf16);
+
+} // namespace tq

@@ -1,0 +1,246 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs, at sizes the oracle finishes in seconds that still span several tiles and a ragged
+tail, plus edge cases. Full-size workloads are in test_gpu_workloads.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - the GPU tier always has a device
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from quantized_decode_attention_kv_b200 import tq  # noqa: E402
+from quantized_decode_attention_kv_b200.workloads import random_kv  # noqa: E402
+
+DT = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
+
+
+def _inputs(B, Hkv, T, d, dtype, seed, outliers=False, zero_at=None, scale=1.0):
+    K, V = random_kv(B, Hkv, T, d, dtype=torch.float32, seed=seed, scale=scale)
+    if outliers:
+        K[..., :3] *= 20.0
+    if zero_at is not None:
+        K[0, 0, zero_at] = 0.0
+        V[0, 0, zero_at] = 0.0
+    return K.to(dtype), V.to(dtype)
+
+
+# ------------------------------------------------------------------ quantize
+QUANT_CASES = [
+    # d, k(bits, mode), v(bits, mode), m
+    (128, (4, O.MSE), (2, O.MSE), 0),
+    (128, (3, O.MSE), (3, O.MSE), 0),
+    (128, (1, O.MSE), (4, O.MSE), 0),
+    (64, (2, O.PROD), (2, O.PROD), 64),
+    (64, (1, O.PROD), (3, O.PROD), 32),
+    (16, (3, O.MSE), (1, O.MSE), 0),
+    (16, (2, O.PROD), (4, O.PROD), 8),
+    (32, (4, O.MSE), (2, O.PROD), 0),
+    (256, (4, O.MSE), (3, O.MSE), 0),
+    (256, (2, O.PROD), (2, O.MSE), 256),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("case", QUANT_CASES, ids=lambda c: f"d{c[0]}-k{c[1]}-v{c[2]}-m{c[3]}")
+def test_quantize_matches_oracle(case, dtype):
+    d, (kb, km), (vb, vm), m = case
+    B, Hkv, T, T_cap, t_off = 2, 3, 37, 50, 6
+    K, V = _inputs(B, Hkv, T, d, DT[dtype], seed=d + kb, outliers=True, zero_at=5)
+    cache = tq.TQCache(B, Hkv, T_cap, d, kb, vb, km, vm, m, m, seed=11, qjl_seed=5)
+    tq.tq_quantize_kv(K.cuda(), V.cuda(), cache, t_offset=t_off)
+    torch.cuda.synchronize()
+    for side, X, bits, mode in (("k", K, kb, km), ("v", V, vb, vm)):
+        recs = P.oracle_records(P.to_np(X), bits, mode, 11, 5, m or None)
+        st = P.compare_records(cache, side, recs, t_offset=t_off)
+        assert st["flipped_near_boundary"] <= st["near_boundary"]
+    # positions outside [t_off, t_off + T) stay untouched (zero)
+    assert int(cache["k_norm"][:, :, :t_off].abs().sum()) == 0
+    assert int(cache["v_norm"][:, :, t_off + T:].abs().sum()) == 0
+
+
+def test_quantize_only_keys_or_values():
+    d = 64
+    K, V = _inputs(1, 2, 20, d, torch.bfloat16, seed=3)
+    cache = tq.TQCache(1, 2, 20, d, 4, 2)
+    tq.tq_quantize_kv(None, V.cuda(), cache)
+    torch.cuda.synchronize()
+    assert int(cache["k_norm"].abs().sum()) == 0
+    P.compare_records(cache, "v", P.oracle_records(P.to_np(V), 2, O.MSE, 0, 1, None))
+    tq.tq_quantize_kv(K.cuda(), None, cache)
+    torch.cuda.synchronize()
+    P.compare_records(cache, "k", P.oracle_records(P.to_np(K), 4, O.MSE, 0, 1, None))
+
+
+def test_quantize_is_deterministic_and_per_head_independent():
+    d, B, H, T = 128, 2, 4, 300
+    K, V = _inputs(B, H, T, d, torch.bfloat16, seed=9, outliers=True)
+    c1 = tq.TQCache(B, H, T, d, 4, 2)
+    c2 = tq.TQCache(B, H, T, d, 4, 2)
+    tq.tq_quantize_kv(K.cuda(), V.cuda(), c1)
+    tq.tq_quantize_kv(K.cuda(), V.cuda(), c2)
+    one = tq.TQCache(1, 1, T, d, 4, 2)
+    tq.tq_quantize_kv(K[1:2, 2:3].contiguous().cuda(), V[1:2, 2:3].contiguous().cuda(), one)
+    torch.cuda.synchronize()
+    for key in ("k_codes", "v_codes", "k_norm", "v_norm"):
+        assert torch.equal(c1[key], c2[key])
+        assert torch.equal(c1[key][1, 2], one[key][0, 0])
+
+
+# ------------------------------------------------------------------ dequantize
+@pytest.mark.parametrize("case", QUANT_CASES, ids=lambda c: f"d{c[0]}-k{c[1]}-v{c[2]}-m{c[3]}")
+def test_dequantize_matches_oracle(case):
+    d, (kb, km), (vb, vm), m = case
+    B, Hkv, T = 2, 2, 45
+    K, V = _inputs(B, Hkv, T, d, torch.float32, seed=d * 3 + vb, scale=7.0)
+    cache = tq.TQCache(B, Hkv, T + 3, d, kb, vb, km, vm, m, m, seed=4, qjl_seed=9)
+    for side, X, bits, mode in (("k", K, kb, km), ("v", V, vb, vm)):
+        recs = P.oracle_records(P.to_np(X), bits, mode, 4, 9, m or None)
+        P.upload(cache, side, recs)
+        out = torch.empty(B, Hkv, T, d, device="cuda", dtype=torch.float32)
+        tq.tq_dequantize(cache, 0 if side == "k" else 1, T, out)
+        torch.cuda.synchronize()
+        want = np.stack([O.dequantize(r) for r in recs]).reshape(B, Hkv, T, d)
+        n16 = np.stack([r.norm16.astype(np.float64) for r in recs]).reshape(B, Hkv, T, 1)
+        err = np.abs(P.to_np(out) - want) / np.maximum(n16, 1e-30)
+        assert err.max() <= P.DEQUANT_ATOL, err.max()
+        for dt in (torch.bfloat16, torch.float16):
+            o2 = torch.empty(B, Hkv, T, d, device="cuda", dtype=dt)
+            tq.tq_dequantize(cache, 0 if side == "k" else 1, T, o2)
+            assert torch.allclose(o2.float(), out.to(dt).float(), rtol=0, atol=0)
+
+
+# ------------------------------------------------------------------ decode
+DECODE_CASES = [
+    # d, G, Hkv, k(bits, mode), v(bits, mode), m, T_len, T_cap
+    (128, 4, 2, (4, O.MSE), (2, O.MSE), 0, 1000, 1030),
+    (128, 1, 1, (4, O.MSE), (4, O.MSE), 0, 1024, 1024),
+    (128, 8, 1, (3, O.MSE), (3, O.MSE), 0, 777, 800),
+    (128, 5, 2, (4, O.MSE), (2, O.MSE), 0, 300, 300),
+    (64, 1, 3, (2, O.PROD), (2, O.PROD), 64, 520, 520),
+    (64, 2, 2, (1, O.PROD), (3, O.PROD), 32, 129, 140),
+    (16, 4, 2, (3, O.MSE), (1, O.MSE), 0, 257, 260),
+    (32, 16, 1, (4, O.MSE), (2, O.PROD), 0, 200, 200),
+    (256, 2, 2, (4, O.MSE), (2, O.MSE), 0, 390, 400),
+    (256, 3, 1, (2, O.PROD), (4, O.MSE), 128, 128, 128),
+    (128, 32, 1, (4, O.MSE), (2, O.MSE), 0, 64, 64),
+    (128, 4, 2, (4, O.MSE), (2, O.MSE), 0, 1, 10),
+]
+
+
+def _decode_case(case, q_dtype, k_scale=1.0, seed=0):
+    d, G, Hkv, (kb, km), (vb, vm), m, T_len, T_cap = case
+    B = 2
+    Hq = G * Hkv
+    K, V = _inputs(B, Hkv, T_cap, d, torch.float32, seed=seed + d + G, outliers=True, scale=k_scale)
+    g = torch.Generator().manual_seed(seed + 17)
+    q = torch.randn(B, Hq, d, generator=g).to(q_dtype)
+    return B, Hq, K, V, q
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=lambda c: f"d{c[0]}-G{c[1]}-H{c[2]}-k{c[3]}-v{c[4]}-T{c[6]}")
+def test_decode_over_oracle_records_matches_oracle(case):
+    d, G, Hkv, (kb, km), (vb, vm), m, T_len, T_cap = case
+    B, Hq, K, V, q = _decode_case(case, torch.bfloat16)
+    scale = 1.0 / math.sqrt(d)
+    cache = tq.TQCache(B, Hkv, T_cap, d, kb, vb, km, vm, m, m, seed=21, qjl_seed=2)
+    k_recs = P.oracle_records(P.to_np(K), kb, km, 21, 2, m or None)
+    v_recs = P.oracle_records(P.to_np(V), vb, vm, 21, 2, m or None)
+    P.upload(cache, "k", k_recs)
+    P.upload(cache, "v", v_recs)
+    out = torch.empty(B, Hq, d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, T_len))
+    tq.tq_decode_attention(q.cuda(), cache, T_len, scale, out, ws)
+    torch.cuda.synchronize()
+    want = P.oracle_decode(P.to_np(q), k_recs, v_recs, B, Hkv, scale, T_len)
+    P.assert_attention_close(P.to_np(out), want)
+
+
+@pytest.mark.parametrize("q_dtype", [torch.float32, torch.float16])
+def test_decode_query_dtypes(q_dtype):
+    case = DECODE_CASES[0]
+    d, G, Hkv, (kb, km), (vb, vm), m, T_len, T_cap = case
+    B, Hq, K, V, q = _decode_case(case, q_dtype, seed=5)
+    cache = tq.TQCache(B, Hkv, T_cap, d, kb, vb, km, vm)
+    k_recs = P.oracle_records(P.to_np(K), kb, km, 0, 1, None)
+    v_recs = P.oracle_records(P.to_np(V), vb, vm, 0, 1, None)
+    P.upload(cache, "k", k_recs)
+    P.upload(cache, "v", v_recs)
+    out = torch.empty(B, Hq, d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, T_len))
+    tq.tq_decode_attention(q.cuda(), cache, T_len, 0.3, out, ws)
+    torch.cuda.synchronize()
+    P.assert_attention_close(P.to_np(out), P.oracle_decode(P.to_np(q), k_recs, v_recs, B, Hkv, 0.3, T_len))
+
+
+def test_decode_with_large_key_norms():
+    # keys 50x the values' norm ("What the Paper Doesn't Tell You", Finding 1): near-one-hot
+    # softmax, where score precision decides the output
+    case = (128, 8, 1, (4, O.MSE), (2, O.MSE), 0, 700, 700)
+    B, Hq, K, V, q = _decode_case(case, torch.bfloat16, k_scale=50.0, seed=3)
+    cache = tq.TQCache(B, 1, 700, 128, 4, 2)
+    k_recs = P.oracle_records(P.to_np(K), 4, O.MSE, 0, 1, None)
+    v_recs = P.oracle_records(P.to_np(V), 2, O.MSE, 0, 1, None)
+    P.upload(cache, "k", k_recs)
+    P.upload(cache, "v", v_recs)
+    out = torch.empty(B, Hq, 128, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, 700))
+    tq.tq_decode_attention(q.cuda(), cache, 700, 128 ** -0.5, out, ws)
+    torch.cuda.synchronize()
+    P.assert_attention_close(P.to_np(out), P.oracle_decode(P.to_np(q), k_recs, v_recs, B, 1, 128 ** -0.5))
+
+
+@pytest.mark.parametrize("case", DECODE_CASES[:6], ids=lambda c: f"d{c[0]}-G{c[1]}-k{c[3]}-v{c[4]}")
+def test_quantize_then_decode_end_to_end(case):
+    d, G, Hkv, (kb, km), (vb, vm), m, T_len, T_cap = case
+    B, Hq, K, V, q = _decode_case(case, torch.bfloat16, seed=8)
+    Kb, Vb = K.to(torch.bfloat16), V.to(torch.bfloat16)
+    cache = tq.TQCache(B, Hkv, T_cap, d, kb, vb, km, vm, m, m, seed=6, qjl_seed=3)
+    # prefill T_len - 1 tokens, then append the last one (decode-time write)
+    tq.tq_quantize_kv(Kb[:, :, : T_len - 1].contiguous().cuda(), Vb[:, :, : T_len - 1].contiguous().cuda(),
+                      cache, 0) if T_len > 1 else None
+    tq.tq_quantize_kv(Kb[:, :, T_len - 1:T_len].contiguous().cuda(), Vb[:, :, T_len - 1:T_len].contiguous().cuda(),
+                      cache, T_len - 1)
+    out = torch.empty(B, Hq, d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, T_len))
+    tq.tq_decode_attention(q.cuda(), cache, T_len, d ** -0.5, out, ws)
+    torch.cuda.synchronize()
+    k_recs = P.oracle_records(P.to_np(Kb[:, :, :T_len]), kb, km, 6, 3, m or None)
+    v_recs = P.oracle_records(P.to_np(Vb[:, :, :T_len]), vb, vm, 6, 3, m or None)
+    want = P.oracle_decode(P.to_np(q), k_recs, v_recs, B, Hkv, d ** -0.5)
+    P.assert_attention_close(P.to_np(out), want)
+
+
+def test_decode_rejects_small_workspace_and_empty_context():
+    cache = tq.TQCache(1, 1, 64, 128, 4, 2)
+    q = torch.zeros(1, 4, 128, device="cuda", dtype=torch.bfloat16)
+    out = torch.empty(1, 4, 128, device="cuda")
+    need = tq.tq_decode_workspace_bytes(cache, 4, 64)
+    small = tq.workspace(need - 64)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_decode_attention(q, cache, 64, 0.1, out, small[: (need - 64) // 4 - 8])
+    assert e.value.status == tq.TQ_ERR_WORKSPACE
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_decode_attention(q, cache, 0, 0.1, out, tq.workspace(need))
+    assert e.value.status == tq.TQ_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ bf16 comparator
+@pytest.mark.parametrize("d,G,Hkv,T_len,T_cap", [(128, 4, 2, 1000, 1024), (64, 1, 3, 129, 140),
+                                                  (256, 8, 1, 300, 300), (16, 2, 2, 1, 4)])
+def test_bf16_decode_matches_oracle(d, G, Hkv, T_len, T_cap):
+    B, Hq = 2, G * Hkv
+    K, V = _inputs(B, Hkv, T_cap, d, torch.bfloat16, seed=d + G, outliers=True)
+    q = torch.randn(B, Hq, d, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    out = torch.empty(B, Hq, d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_bf16_workspace_bytes(B, Hq, Hkv, T_len, d))
+    tq.tq_decode_attention_bf16(q.cuda(), K.cuda(), V.cuda(), T_len, d ** -0.5, out, ws)
+    torch.cuda.synchronize()
+    want = O.gqa_decode(P.to_np(q), P.to_np(K)[:, :, :T_len], P.to_np(V)[:, :, :T_len], d ** -0.5)
+    P.assert_attention_close(P.to_np(out), want)

@@ -1,0 +1,78 @@
+"""Full-size workloads on the GPU, in the launch configuration bench.py times: every
+workload is quantised and decoded at its real size through the C ABI, and sampled
+(batch, KV head) slices are checked against the oracle (codes, norms, and the attention of
+that KV head's query heads over the full context)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from quantized_decode_attention_kv_b200 import tq  # noqa: E402
+from quantized_decode_attention_kv_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+
+def _cache_for(w):
+    return tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, w.k_mode, w.v_mode, w.qjl_m,
+                      w.qjl_m, seed=w.seed, qjl_seed=w.qjl_seed)
+
+
+def _check_full(w, layer=0, samples=((0, 0), (-1, -1))):
+    K, V, q = make_inputs(w, device="cuda", layer=layer)
+    cache = _cache_for(w)
+    tq.tq_quantize_kv(K, V, cache)
+    out = torch.empty(w.B, w.Hq, w.d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, w.Hq, w.T))
+    tq.tq_decode_attention(q, cache, w.T, w.scale, out, ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    G = w.G
+    stats = []
+    for b, h in samples:
+        b %= w.B
+        h %= w.Hkv
+        recs = {}
+        for side, X, bits, mode in (("k", K, w.k_bits, w.k_mode), ("v", V, w.v_bits, w.v_mode)):
+            r = O.quantize(P.to_np(X[b, h]), bits, mode, seed=w.seed, qjl_seed=w.qjl_seed,
+                           m=w.qjl_m or None)
+            stats.append(P.compare_records(cache, side, [r], heads=[(b, h)]))
+            recs[side] = r
+        qs = P.to_np(q[b:b + 1, h * G:(h + 1) * G])
+        want = O.decode_compressed(qs, [recs["k"]], [recs["v"]], 1, 1, w.scale)
+        P.assert_attention_close(P.to_np(out[b:b + 1, h * G:(h + 1) * G]), want)
+    del K, V, cache
+    torch.cuda.empty_cache()
+    return stats
+
+
+@pytest.mark.parametrize("name", ["tiny_single_head_fp32", "llama3_8b_decode_32k", "gpt2_prod_2bit",
+                                  "llama3_8b_128k_3bit", "llama70b_asym_16k"])
+def test_full_size_workload_sampled_parity(name):
+    w = WORKLOADS[name]
+    stats = _check_full(w)
+    near = sum(s["near_boundary"] for s in stats)
+    coords = sum(s["coords"] for s in stats)
+    # the exemption band is 2e-5 wide around each boundary: for near-Gaussian z that is about
+    # 2e-5 * sum_j pdf(beta_j) < 1e-4 of the coordinates
+    assert near <= 3e-4 * coords
+
+
+def test_full_size_bf16_boundary_layer():
+    # layers kept unquantised in the 70B-shaped workload run the bf16 kernel at full size
+    w = WORKLOADS["llama70b_asym_16k"]
+    K, V, q = make_inputs(w, device="cuda", layer=0)
+    out = torch.empty(w.B, w.Hq, w.d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_bf16_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.d))
+    tq.tq_decode_attention_bf16(q, K, V, w.T, w.scale, out, ws)
+    torch.cuda.synchronize()
+    G = w.G
+    for b, h in ((0, 0), (w.B - 1, w.Hkv - 1)):
+        want = O.gqa_decode(P.to_np(q[b:b + 1, h * G:(h + 1) * G]), P.to_np(K[b:b + 1, h:h + 1]),
+                            P.to_np(V[b:b + 1, h:h + 1]), w.scale)
+        P.assert_attention_close(P.to_np(out[b:b + 1, h * G:(h + 1) * G]), want)
