@@ -143,6 +143,23 @@ int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale
                         const tq_cache *cache, float *out, void *ws, size_t ws_bytes,
                         void *stream);
 
+/* Decode attention without a workspace and without any allocation. The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device memory at this
+ * point: runtimes that hand out all device memory from their own pool and forbid a library
+ * to call cudaMalloc, decode loops that cannot afford cudaMalloc/cudaFree (they can stall
+ * the whole device), and plugin interfaces that pass a kernel only its inputs and outputs.
+ * Arguments, results and errors are those of tq_decode_attention; q, out and the cache stay
+ * caller-owned. The split-K partials live in one fixed 8 MiB device array inside libtq
+ * (present on every GPU that loads the library, until the process exits); a shape whose
+ * tq_decode_workspace_bytes exceeds 8 MiB is rejected with TQ_ERR_WORKSPACE and nothing is
+ * launched. The first call on a device looks up the array's device address with that device
+ * current; make that first call before any stream capture. Every call on a device shares the
+ * same array and leaves its partials behind; a call writes every element it later reads, so
+ * nothing needs clearing, but calls that overlap on the GPU (other streams, other host
+ * threads) race on the array and must be serialised by the caller. */
+int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, float scale,
+                                const tq_cache *cache, float *out, void *stream);
+
 /* Dequantise cache positions [0, T_len) of K (which = 0) or V (which = 1) into out
  * [B][Hkv][T_len][d] of `dtype` in the original domain: x_hat = n D H c / d (MSE), plus
  * the QJL residual estimate sqrt(d) gamma sqrt(pi/2)/m S^T s inside the bracket (PROD). */

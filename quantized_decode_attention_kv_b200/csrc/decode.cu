@@ -16,6 +16,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 namespace tq {
 namespace {
@@ -595,6 +596,41 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) { TQ_DISPATCH_DEC
 
 cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s) {
   TQ_DISPATCH_DEC(run_decode_bf16)
+}
+
+} // namespace tq
+
+// ------------------------------------------------------------------ fixed scratch
+// Backing store for tq_decode_attention_noalloc: the split-K partials of one call live in
+// this file-scope device array instead of a caller workspace. Every GPU that loads the
+// library holds it for the life of the process. Host code must not pass the symbol itself
+// to a kernel (in host code it names a host-side stand-in); fixed_scratch() fetches the real
+// device address once per device and caches it.
+namespace tq {
+namespace {
+constexpr size_t kFixedScratchBytes = size_t(8) << 20; // 8 MiB
+constexpr int kMaxDevices = 64;
+} // namespace
+
+static __device__ __align__(256) float g_fixed_scratch[kFixedScratchBytes / sizeof(float)];
+
+cudaError_t fixed_scratch(float **ptr, size_t *bytes) {
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fixed_scratch); // with `dev` current
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = static_cast<float *>(addr[dev]);
+  *bytes = kFixedScratchBytes;
+  return cudaSuccess;
 }
 
 } // namespace tq

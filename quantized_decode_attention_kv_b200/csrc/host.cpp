@@ -357,6 +357,55 @@ int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale
   return cuda_status(tq::launch_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
 }
 
+int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, float scale,
+                                const tq_cache *cache, float *out, void *stream) {
+  // Same arguments and checks as tq_decode_attention, minus the workspace: the split-K
+  // partials go to the library's fixed device scratch, so this call allocates nothing.
+  int st = check_cache(cache);
+  if (st) return st;
+  if (!dtype_ok(dtype)) return fail(TQ_ERR_INVALID_ARG, "dtype=%d is not F32/BF16/F16", dtype);
+  if (!q || !out || !aligned16(q) || !aligned16(out))
+    return fail(TQ_ERR_INVALID_ARG, "q/out must be non-NULL and 16-byte aligned");
+  if (Hq < 1 || Hq % cache->Hkv || Hq > 65535)
+    return fail(TQ_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d (<= 65535)", Hq,
+                cache->Hkv);
+  if (T_len < 1 || T_len > cache->T_cap)
+    return fail(TQ_ERR_INVALID_ARG, "T_len=%d must be in 1..T_cap=%d", T_len, cache->T_cap);
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale is not finite");
+  tq::DecodeArgs a;
+  std::memset(&a, 0, sizeof a);
+  st = resolve_tensor(*cache, 0, &a.k);
+  if (st) return st;
+  st = resolve_tensor(*cache, 1, &a.v);
+  if (st) return st;
+  int sms = sm_count();
+  if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
+  a.plan = tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, a.v.m, sms, false);
+  float *scratch = nullptr;
+  size_t cap = 0;
+  st = cuda_status(tq::fixed_scratch(&scratch, &cap), "fixed scratch lookup");
+  if (st) return st;
+  if (a.plan.ws_bytes > cap)
+    return fail(TQ_ERR_WORKSPACE,
+                "this shape needs %zu bytes of split-K scratch but the fixed scratch holds %zu; "
+                "call tq_decode_attention with a caller-owned workspace instead",
+                a.plan.ws_bytes, cap);
+  a.q = q;
+  a.q_dtype = dtype;
+  a.B = cache->B;
+  a.Hq = Hq;
+  a.Hkv = cache->Hkv;
+  a.d = cache->d;
+  a.T_len = T_len;
+  a.T_cap = cache->T_cap;
+  a.scale = scale;
+  a.seed = cache->seed;
+  a.out = out;
+  a.ws = scratch;
+  return cuda_status(tq::launch_decode(a, static_cast<cudaStream_t>(stream)),
+                     "decode (fixed scratch) launch");
+}
+
 int tq_dequantize(const tq_cache *cache, int which, int T_len, void *out, int dtype,
                   void *stream) {
   int st = check_cache(cache);

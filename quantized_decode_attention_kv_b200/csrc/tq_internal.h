@@ -85,6 +85,11 @@ cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s);
 
+// Device address and size (bytes) of the fixed scratch array behind
+// tq_decode_attention_noalloc (decode.cu). The first call on a device looks the address up
+// with that device current; later calls return the cached address.
+cudaError_t fixed_scratch(float **ptr, size_t *bytes);
+
 // Split-K plan for the compressed and bf16 decode kernels (decode.cu).
 DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count,
                        bool bf16);

@@ -61,6 +61,9 @@ EXPORTS = {
     "tq_decode_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_float, ctypes.POINTER(tq_cache), ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tq_decode_attention_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_float, ctypes.POINTER(tq_cache),
+                                                   ctypes.c_void_p, ctypes.c_void_p]),
     "tq_dequantize": (ctypes.c_int, [ctypes.POINTER(tq_cache), ctypes.c_int, ctypes.c_int,
                                      ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "tq_decode_bf16_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -231,6 +234,18 @@ def tq_decode_attention(q: torch.Tensor, cache: TQCache, T_len: int, scale: floa
     _check(lib.tq_decode_attention(_dev(q, "q"), dt, q.shape[1], T_len, scale, ctypes.byref(cache.struct),
                                    _dev(out, "out"), _dev(ws, "ws"), ws.numel() * ws.element_size(),
                                    _stream(stream)))
+
+
+def tq_decode_attention_noalloc(q: torch.Tensor, cache: TQCache, T_len: int, scale: float,
+                                out: torch.Tensor, stream=None) -> None:
+    """tq_decode_attention without a workspace: libtq keeps the split-K partials in its own
+    fixed device scratch (8 MiB), so nothing is allocated. For callers that may not allocate
+    device memory; calls that overlap on the GPU must be serialised by the caller."""
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise TQError(TQ_ERR_INVALID_ARG, f"unsupported dtype {q.dtype}")
+    _check(lib.tq_decode_attention_noalloc(_dev(q, "q"), dt, q.shape[1], T_len, scale,
+                                           ctypes.byref(cache.struct), _dev(out, "out"), _stream(stream)))
 
 
 def tq_dequantize(cache: TQCache, which: int, T_len: int, out: torch.Tensor, stream=None) -> None:
