@@ -569,9 +569,14 @@ cudaError_t run_decode_bf16(const DecodeBf16Args &a, cudaStream_t s) {
 
 } // namespace
 
-DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count, bool bf16) {
-  (void)bf16;
+DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count, bool bf16,
+                       bool fast) {
   DecodePlan p{};
+  if (fast && !bf16) {
+    plan_fast(B, Hq, Hkv, T_len, sm_count, &p);
+    return p;
+  }
+  p.path = 0;
   p.tile = kTile;
   const int G = Hq / Hkv;
   int gc = 1;
@@ -592,7 +597,10 @@ DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm
   return p;
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) { TQ_DISPATCH_DEC(run_decode) }
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
+  if (a.plan.path == 1) return launch_fast_decode(a, s);
+  TQ_DISPATCH_DEC(run_decode)
+}
 
 cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s) {
   TQ_DISPATCH_DEC(run_decode_bf16)

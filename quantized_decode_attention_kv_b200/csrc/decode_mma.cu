@@ -1,0 +1,567 @@
+// Tensor-core decode attention over the compressed cache (head_dim 128, 4-bit keys, 2-bit
+// values, TurboQuant_mse, up to 8 query heads per KV head).
+//
+// "Where This Fits in the Inference Stack", TensorRT-LLM section: dequantise in registers
+// inside the attention kernel. Here the dequantised codes are written straight into the
+// operand registers of warp-level tensor-core MMAs (mma.sync m16n8k16, fp16 x fp16 -> fp32):
+//
+//   scores  S[16 tokens x (hi, lo) per head] = K^[16 x 128] . [q^_hi | q^_lo]
+//     K^ comes from a shared-memory LUT indexed by one code byte (two 4-bit codes): each entry
+//     holds the two centroids as fp16 (hi) and their fp16 rounding residuals scaled by 2^12
+//     (lo); two MMAs (hi, lo) give scores good to ~2^-21 relative, as fp32 scoring would.
+//     The query side is split the same way by the query-prep kernel.
+//   values  O^T[128 x heads] += V^T[128 x 16 tokens] . P'^T[16 tokens x heads]
+//     V^ comes from a 4-entry fp16 table held in two registers and indexed with PRMT, one
+//     PRMT per pair of tokens; P' = p * ||v_t|| in fp16.
+//
+// The contraction order is free along k, so each thread owns a contiguous 16-byte slice of
+// every key record and one 32-bit word of every value record: all loads are 16- or 4-byte,
+// and the permutation is undone when the partial accumulators are written.
+//
+// Work split: the (batch, KV head, 16-token tile) space is flattened and cut into equal
+// contiguous ranges, one per persistent CTA of 4 warps; within a range each maximal run of
+// one (batch, KV head) is a segment, its tiles dealt round-robin to the warps, each warp
+// keeping its own online-softmax state (log2 domain); the warps merge through shared memory
+// at the end of the segment and write one partial record per query head.
+#include "tq_device.cuh"
+
+#include <algorithm>
+#include <mutex>
+
+namespace tq {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kD = 128;
+constexpr float kLoScale = 4096.0f; // residual scaling 2^12 (keeps residuals normal in fp16)
+constexpr float kLoInv = 1.0f / 4096.0f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kLutBytes = 256 * 32 * 8; // [code byte][lane] uint2
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg_nc16(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_nc4(const void *p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_nc2(const void *p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t smem_addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr));
+  return v;
+}
+
+// Per-tile registers of one warp lane.
+struct Tile {
+  uint4 k0, k1;   // key bytes [16c, 16c+16) of tokens r and r+8
+  uint32_t v[4];  // value word r of tokens 2c, 2c+1, 2c+8, 2c+9
+  uint32_t kn[2]; // key norms (fp16 bits) of tokens r, r+8
+  uint32_t vn[2]; // value norms (fp16 bits) of tokens r, r+8
+};
+
+} // namespace
+
+// Query prep: rotate once (q'' = H D q), scale (q~ = scale q'' / d), normalise by a power of
+// two so max|q^| is in [1, 2), split into fp16 hi and 2^12-scaled fp16 residual.
+struct QPrep {
+  uint16_t hi[kD];
+  uint16_t lo[kD];
+  float inv; // 1 / (power-of-two factor): score = ||k|| * inv * (K^ . q^)
+  float pad[3];
+};
+
+namespace {
+
+__global__ void __launch_bounds__(kD) qprep_kernel(const void *q, int dtype, float scale,
+                                                   uint64_t seed, QPrep *out) {
+  __shared__ float v[kD];
+  __shared__ float red[4];
+  const int i = threadIdx.x;
+  const size_t bq = blockIdx.x;
+  float x = load_scalar(q, dtype, bq * kD + i);
+  if (sign_is_neg(seed, i)) x = -x;
+  v[i] = x;
+  __syncthreads();
+  for (int hs = 1; hs < kD; hs <<= 1) {
+    float a = 0.f, b = 0.f;
+    const bool lower = (i & hs) == 0;
+    if (lower) {
+      a = v[i];
+      b = v[i + hs];
+    }
+    __syncthreads();
+    if (lower) {
+      v[i] = a + b;
+      v[i + hs] = a - b;
+    }
+    __syncthreads();
+  }
+  const float qt = v[i] * (scale / static_cast<float>(kD));
+  float mx = warp_max(fabsf(qt));
+  if ((i & 31) == 0) red[i >> 5] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float factor = 1.0f;
+  if (mx > 0.f && isfinite(mx)) {
+    int ex;
+    frexpf(mx, &ex);             // mx = f * 2^ex, f in [0.5, 1)
+    factor = ldexpf(1.0f, 1 - ex); // mx * factor in [1, 2)
+  }
+  const float qh = qt * factor;
+  const __half hi = __float2half_rn(qh);
+  const __half lo = __float2half_rn((qh - __half2float(hi)) * kLoScale);
+  out[bq].hi[i] = __half_as_ushort(hi);
+  out[bq].lo[i] = __half_as_ushort(lo);
+  if (i == 0) out[bq].inv = 1.0f / factor;
+}
+
+struct FastArgs {
+  const uint8_t *kc, *vc;
+  const uint16_t *kn, *vn;
+  const QPrep *qp;
+  float *part; // partial records [cta][slot][G][stride]
+  int Hq, Hkv, G, T_len, T_cap;
+  int tiles_per_bh, tiles_per_cta, slots, stride;
+  long long total_tiles;
+  float kcent[16];
+  float vcent[4];
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint2 *lut = reinterpret_cast<uint2 *>(smem);
+  float *mst = reinterpret_cast<float *>(smem + kLutBytes); // [kWarps][8] running max
+  float *gmx = mst + kWarps * 8;                            // [8] merged max
+  float *lsum = gmx + 8;                                    // [8] merged sum
+  float *obuf = lsum + 8;                                   // [G][128] merged accumulator
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = lane >> 2, c = lane & 3;
+
+  for (int idx = tid; idx < 256 * 32; idx += kThreads) {
+    const int e = idx >> 5;
+    const float c0 = a.kcent[e & 15], c1 = a.kcent[e >> 4];
+    const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
+    lut[idx] = make_uint2(pack_h2(c0, c1), pack_h2((c0 - h0) * kLoScale, (c1 - h1) * kLoScale));
+  }
+  const uint32_t vt0 = pack_h2(a.vcent[0], a.vcent[1]);
+  const uint32_t vt1 = pack_h2(a.vcent[2], a.vcent[3]);
+  const uint32_t lut_base = static_cast<uint32_t>(__cvta_generic_to_shared(lut));
+  const uint32_t lanebase = static_cast<uint32_t>(lane) << 3;
+  __syncthreads();
+
+  const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
+  const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
+  int slot = 0;
+  for (long long seg = range0; seg < range1; ++slot) {
+    const long long bh = seg / a.tiles_per_bh;
+    const long long seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
+    const int tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+    const int ntiles = static_cast<int>(seg_end - seg);
+    seg = seg_end;
+    const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
+
+    // ---- B operands of the score MMA: column n = r of n-tile nt is head g = 4 nt + r/2,
+    //      hi (r even) or residual (r odd); thread c holds coordinates [32c, 32c+32).
+    uint32_t qb[NT][16];
+    float qscale[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int g = nt * 4 + (r >> 1);
+      if (g < a.G) {
+        const QPrep *p = a.qp + static_cast<size_t>(b) * a.Hq + h * a.G + g;
+        const uint4 *src = reinterpret_cast<const uint4 *>(((r & 1) ? p->lo : p->hi) + 32 * c);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 w = __ldg(src + k);
+          qb[nt][4 * k] = w.x;
+          qb[nt][4 * k + 1] = w.y;
+          qb[nt][4 * k + 2] = w.z;
+          qb[nt][4 * k + 3] = w.w;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) qb[nt][k] = 0u;
+      }
+      const int gs = nt * 4 + c; // head of this lane's score columns
+      qscale[nt] = gs < a.G ? __ldg(&a.qp[static_cast<size_t>(b) * a.Hq + h * a.G + gs].inv) * kLog2e
+                            : 0.f;
+    }
+
+    float m_run[NT], l_run[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m_run[nt] = -INFINITY;
+      l_run[nt] = 0.f;
+    }
+    float o[8][4];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+
+    const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
+    const uint8_t *kbase = a.kc + rec0 * 64 + 16 * c;
+    const uint8_t *vbase = a.vc + rec0 * 32 + 4 * r;
+    const uint16_t *knb = a.kn + rec0;
+    const uint16_t *vnb = a.vn + rec0;
+    const int tlast = a.T_len - 1;
+
+    auto load = [&](int jt, Tile &T) {
+      const int t0 = (tile0 + jt) * 16;
+      const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
+      T.k0 = ldg_nc16(kbase + static_cast<size_t>(tr) * 64);
+      T.k1 = ldg_nc16(kbase + static_cast<size_t>(tr8) * 64);
+      const int tv = t0 + 2 * c;
+      T.v[0] = ldg_nc4(vbase + static_cast<size_t>(min(tv, tlast)) * 32);
+      T.v[1] = ldg_nc4(vbase + static_cast<size_t>(min(tv + 1, tlast)) * 32);
+      T.v[2] = ldg_nc4(vbase + static_cast<size_t>(min(tv + 8, tlast)) * 32);
+      T.v[3] = ldg_nc4(vbase + static_cast<size_t>(min(tv + 9, tlast)) * 32);
+      T.kn[0] = ldg_nc2(knb + tr);
+      T.kn[1] = ldg_nc2(knb + tr8);
+      T.vn[0] = ldg_nc2(vnb + tr);
+      T.vn[1] = ldg_nc2(vnb + tr8);
+    };
+
+    Tile cur, nxt;
+    int jt = warp;
+    if (jt < ntiles) load(jt, cur);
+    for (; jt < ntiles; jt += kWarps) {
+      if (jt + kWarps < ntiles) load(jt + kWarps, nxt);
+      const int t0 = (tile0 + jt) * 16;
+
+      // ---- scores: two MMAs per k-step (centroid hi and residual) per n-tile
+      float c1[NT][4], c2[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c1[nt][e] = c2[nt][e] = 0.f;
+      const uint32_t w0[4] = {cur.k0.x, cur.k0.y, cur.k0.z, cur.k0.w};
+      const uint32_t w1[4] = {cur.k1.x, cur.k1.y, cur.k1.z, cur.k1.w};
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const uint32_t sel0 = 0x7604u | (static_cast<uint32_t>((2 * s) & 3) << 4);
+        const uint32_t sel1 = 0x7604u | (static_cast<uint32_t>((2 * s + 1) & 3) << 4);
+        const uint2 e0 = lds64(lut_base + prmt(w0[s >> 1], lanebase, sel0)); // token r, k 2c..
+        const uint2 e1 = lds64(lut_base + prmt(w1[s >> 1], lanebase, sel0)); // token r+8
+        const uint2 e2 = lds64(lut_base + prmt(w0[s >> 1], lanebase, sel1)); // token r, k 2c+8..
+        const uint2 e3 = lds64(lut_base + prmt(w1[s >> 1], lanebase, sel1)); // token r+8
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma16816(c1[nt], e0.x, e1.x, e2.x, e3.x, qb[nt][2 * s], qb[nt][2 * s + 1]);
+          mma16816(c2[nt], e0.y, e1.y, e2.y, e3.y, qb[nt][2 * s], qb[nt][2 * s + 1]);
+        }
+      }
+
+      // ---- online softmax (log2 domain); lane (r, c) owns head 4 nt + c, tokens r, r+8
+      const float kn0 = f16_bits_to_f32(static_cast<uint16_t>(cur.kn[0]));
+      const float kn1 = f16_bits_to_f32(static_cast<uint16_t>(cur.kn[1]));
+      const float vn0 = f16_bits_to_f32(static_cast<uint16_t>(cur.vn[0]));
+      const float vn1 = f16_bits_to_f32(static_cast<uint16_t>(cur.vn[1]));
+      const bool ok0 = t0 + r < a.T_len, ok1 = t0 + r + 8 < a.T_len;
+      uint32_t pk[NT];
+      float alpha[NT];
+      bool rescale = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float s0 = ok0 ? kn0 * qscale[nt] * fmaf(c1[nt][1] + c2[nt][0], kLoInv, c1[nt][0])
+                             : -INFINITY;
+        const float s1 = ok1 ? kn1 * qscale[nt] * fmaf(c1[nt][3] + c2[nt][2], kLoInv, c1[nt][2])
+                             : -INFINITY;
+        float mx = fmaxf(s0, s1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float mn = fmaxf(m_run[nt], mx);
+        alpha[nt] = exp2f(m_run[nt] - mn);
+        rescale |= mn != m_run[nt];
+        m_run[nt] = mn;
+        const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
+        l_run[nt] = fmaf(l_run[nt], alpha[nt], p0 + p1);
+        pk[nt] = pack_h2(p0 * vn0, p1 * vn1);
+      }
+      // rescale the value accumulators (lane owns heads 2c, 2c+1) when any max moved
+      if (__any_sync(0xffffffffu, rescale)) {
+        float a0[NT], a1[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          a0[nt] = __shfl_sync(0xffffffffu, alpha[nt], (2 * c) & 3);
+          a1[nt] = __shfl_sync(0xffffffffu, alpha[nt], (2 * c + 1) & 3);
+        }
+        const float al0 = NT == 2 && c >= 2 ? a0[NT - 1] : a0[0];
+        const float al1 = NT == 2 && c >= 2 ? a1[NT - 1] : a1[0];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          o[m][0] *= al0;
+          o[m][1] *= al1;
+          o[m][2] *= al0;
+          o[m][3] *= al1;
+        }
+      }
+
+      // ---- P'^T as the B operand: lane (r, c) needs head g = r at tokens 2c, 2c+1, 2c+8, 2c+9
+      const int src0 = 8 * c + (r & 3);
+      uint32_t x0 = __shfl_sync(0xffffffffu, pk[0], src0);
+      uint32_t x1 = __shfl_sync(0xffffffffu, pk[0], src0 + 4);
+      if (NT == 2) {
+        const uint32_t y0 = __shfl_sync(0xffffffffu, pk[NT - 1], src0);
+        const uint32_t y1 = __shfl_sync(0xffffffffu, pk[NT - 1], src0 + 4);
+        if (r >= 4) {
+          x0 = y0;
+          x1 = y1;
+        }
+      }
+      if (r >= a.G) x0 = x1 = 0u;
+      const uint32_t pb0 = prmt(x0, x1, 0x5410u); // tokens 2c, 2c+1
+      const uint32_t pb1 = prmt(x0, x1, 0x7632u); // tokens 2c+8, 2c+9
+
+      // ---- values: pair-of-token PRMT lookups straight into the A operand, then P'.V
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t xsel = half ? 0x7362u : 0x5140u;
+        const uint32_t xa = prmt(cur.v[0], cur.v[1], xsel); // tokens 2c, 2c+1: codes 8half..+7
+        const uint32_t xb = prmt(cur.v[2], cur.v[3], xsel); // tokens 2c+8, 2c+9
+        uint32_t A01[8], A89[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t ya = (xa >> (2 * k)) & 0x03030303u;
+          const uint32_t yb = (xb >> (2 * k)) & 0x03030303u;
+          const uint32_t za = ya * 0x22u + 0x10101010u;
+          const uint32_t zb = yb * 0x22u + 0x10101010u;
+          A01[k] = prmt(vt0, vt1, za);           // code 8half + k
+          A01[k + 4] = prmt(vt0, vt1, za >> 16); // code 8half + k + 4
+          A89[k] = prmt(vt0, vt1, zb);
+          A89[k + 4] = prmt(vt0, vt1, zb >> 16);
+        }
+        // m-tile m covers codes 2m (rows r) and 2m+1 (rows r+8) of the lane's word
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          const int m = 4 * half + mm;
+          mma16816(o[m], A01[2 * mm], A01[2 * mm + 1], A89[2 * mm], A89[2 * mm + 1], pb0, pb1);
+        }
+      }
+      cur = nxt;
+    }
+
+    // ---- merge the warps: common max per head, rescale, accumulate in shared memory
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float l = l_run[nt];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      l_run[nt] = l;
+      if (r == 0) mst[warp * 8 + nt * 4 + c] = m_run[nt];
+    }
+    for (int idx = tid; idx < a.G * kD; idx += kThreads) obuf[idx] = 0.f;
+    if (tid < 8) lsum[tid] = 0.f;
+    __syncthreads();
+    if (tid < 8) {
+      float M = -INFINITY;
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mst[w * 8 + tid]);
+      gmx[tid] = M;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int g = nt * 4 + c;
+      if (r == 0 && g < a.G) atomicAdd(&lsum[g], l_run[nt] * exp2f(m_run[nt] - gmx[g]));
+    }
+    {
+      const int g0 = 2 * c, g1 = 2 * c + 1;
+      const float f0 = g0 < a.G ? exp2f(mst[warp * 8 + g0] - gmx[g0]) : 0.f;
+      const float f1 = g1 < a.G ? exp2f(mst[warp * 8 + g1] - gmx[g1]) : 0.f;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int i0 = 16 * r + 2 * m;
+        if (g0 < a.G) {
+          atomicAdd(&obuf[g0 * kD + i0], o[m][0] * f0);
+          atomicAdd(&obuf[g0 * kD + i0 + 1], o[m][2] * f0);
+        }
+        if (g1 < a.G) {
+          atomicAdd(&obuf[g1 * kD + i0], o[m][1] * f1);
+          atomicAdd(&obuf[g1 * kD + i0 + 1], o[m][3] * f1);
+        }
+      }
+    }
+    __syncthreads();
+    float *dst = a.part + (static_cast<size_t>(blockIdx.x) * a.slots + slot) * a.G * a.stride;
+    for (int idx = tid; idx < a.G * kD; idx += kThreads) {
+      const int g = idx / kD, i = idx - g * kD;
+      dst[static_cast<size_t>(g) * a.stride + 2 + i] = obuf[idx];
+    }
+    if (tid < a.G) {
+      dst[static_cast<size_t>(tid) * a.stride] = gmx[tid];
+      dst[static_cast<size_t>(tid) * a.stride + 1] = lsum[tid];
+    }
+    __syncthreads();
+  }
+}
+
+// Merge the partial records of one (b, q-head) (log2-domain maxima), apply the inverse
+// rotation D H / d once and divide by the softmax sum.
+__global__ void __launch_bounds__(kD) combine_fast_kernel(const float *part, int Hkv, int G,
+                                                          int tiles_per_bh, int tiles_per_cta,
+                                                          int slots, int stride, uint64_t seed,
+                                                          float *out) {
+  __shared__ float o[kD];
+  const int i = threadIdx.x;
+  const int hq = blockIdx.x, b = blockIdx.y;
+  const int Hq = Hkv * G;
+  const int h = hq / G, g = hq - h * G;
+  const long long bh = static_cast<long long>(b) * Hkv + h;
+  const long long first = bh * tiles_per_bh, last = first + tiles_per_bh - 1;
+  const int cta0 = static_cast<int>(first / tiles_per_cta), cta1 = static_cast<int>(last / tiles_per_cta);
+  float M = -INFINITY;
+  for (int cta = cta0; cta <= cta1; ++cta) {
+    const long long bh0 = static_cast<long long>(cta) * tiles_per_cta / tiles_per_bh;
+    const float *p = part + ((static_cast<size_t>(cta) * slots + (bh - bh0)) * G + g) * stride;
+    M = fmaxf(M, p[0]);
+  }
+  float L = 0.f, acc = 0.f;
+  for (int cta = cta0; cta <= cta1; ++cta) {
+    const long long bh0 = static_cast<long long>(cta) * tiles_per_cta / tiles_per_bh;
+    const float *p = part + ((static_cast<size_t>(cta) * slots + (bh - bh0)) * G + g) * stride;
+    const float e = exp2f(p[0] - M);
+    L = fmaf(e, p[1], L);
+    acc = fmaf(e, p[2 + i], acc);
+  }
+  o[i] = acc;
+  __syncthreads();
+  for (int hs = 1; hs < kD; hs <<= 1) {
+    float x0 = 0.f, x1 = 0.f;
+    const bool lower = (i & hs) == 0;
+    if (lower) {
+      x0 = o[i];
+      x1 = o[i + hs];
+    }
+    __syncthreads();
+    if (lower) {
+      o[i] = x0 + x1;
+      o[i + hs] = x0 - x1;
+    }
+    __syncthreads();
+  }
+  const float v = o[i] / (static_cast<float>(kD) * L);
+  out[(static_cast<size_t>(b) * Hq + hq) * kD + i] = sign_is_neg(seed, i) ? -v : v;
+}
+
+int fast_ctas_per_sm() {
+  static std::once_flag once;
+  static int n = 0;
+  std::call_once(once, [] {
+    int v = 0;
+    const int smem = kLutBytes + (kWarps * 8 + 16 + 8 * kD) * 4;
+    if (cudaFuncSetAttribute(decode_k4v2_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) == cudaSuccess &&
+        cudaFuncSetAttribute(decode_k4v2_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, decode_k4v2_kernel<2>, kThreads, smem) ==
+            cudaSuccess)
+      n = std::max(1, v);
+    else
+      n = 1;
+  });
+  return n;
+}
+
+} // namespace
+
+bool fast_decode_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G) {
+  return d == kD && k_mode == TQ_MSE && k_wbits == 4 && v_mode == TQ_MSE && v_wbits == 2 &&
+         G >= 1 && G <= 8;
+}
+
+// Layout of the fast path's workspace: [partials][query prep].
+void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p) {
+  const int G = Hq / Hkv;
+  p->path = 1;
+  p->tile = 16;
+  p->gc = G;
+  p->ws_stride = 2 + kD + 2; // 132 floats
+  p->tiles_per_bh = (T_len + 15) / 16;
+  const long long total = static_cast<long long>(B) * Hkv * p->tiles_per_bh;
+  long long ctas = static_cast<long long>(sm_count) * 3;
+  ctas = std::min<long long>(ctas, (total + 7) / 8); // at least 8 tiles per CTA
+  ctas = std::max<long long>(ctas, 1);
+  p->tiles_per_cta = static_cast<int>((total + ctas - 1) / ctas);
+  p->ctas = static_cast<int>((total + p->tiles_per_cta - 1) / p->tiles_per_cta);
+  p->slots = (p->tiles_per_cta + p->tiles_per_bh - 1) / p->tiles_per_bh + 1;
+  p->splits = 0;
+  p->chunk = 0;
+  p->part_bytes = static_cast<size_t>(p->ctas) * p->slots * G * p->ws_stride * sizeof(float);
+  p->part_bytes = (p->part_bytes + 255) / 256 * 256;
+  p->ws_bytes = p->part_bytes + static_cast<size_t>(B) * Hq * sizeof(QPrep);
+}
+
+cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
+  const DecodePlan &p = a.plan;
+  QPrep *qp = reinterpret_cast<QPrep *>(reinterpret_cast<uint8_t *>(a.ws) + p.part_bytes);
+  qprep_kernel<<<a.B * a.Hq, kD, 0, s>>>(a.q, a.q_dtype, a.scale, a.seed, qp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  FastArgs f;
+  f.kc = a.k.codes;
+  f.vc = a.v.codes;
+  f.kn = a.k.norm;
+  f.vn = a.v.norm;
+  f.qp = qp;
+  f.part = a.ws;
+  f.Hq = a.Hq;
+  f.Hkv = a.Hkv;
+  f.G = a.Hq / a.Hkv;
+  f.T_len = a.T_len;
+  f.T_cap = a.T_cap;
+  f.tiles_per_bh = p.tiles_per_bh;
+  f.tiles_per_cta = p.tiles_per_cta;
+  f.slots = p.slots;
+  f.stride = p.ws_stride;
+  f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
+  for (int j = 0; j < 16; ++j) f.kcent[j] = a.k.cb.c[j];
+  for (int j = 0; j < 4; ++j) f.vcent[j] = a.v.cb.c[j];
+  const int smem = kLutBytes + (kWarps * 8 + 16 + 8 * kD) * 4;
+  (void)fast_ctas_per_sm();
+  if (f.G <= 4)
+    decode_k4v2_kernel<1><<<p.ctas, kThreads, smem, s>>>(f);
+  else
+    decode_k4v2_kernel<2><<<p.ctas, kThreads, smem, s>>>(f);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  combine_fast_kernel<<<dim3(a.Hq, a.B), kD, 0, s>>>(a.ws, a.Hkv, f.G, p.tiles_per_bh,
+                                                      p.tiles_per_cta, p.slots, p.ws_stride, a.seed,
+                                                      a.out);
+  return cudaGetLastError();
+}
+
+} // namespace tq

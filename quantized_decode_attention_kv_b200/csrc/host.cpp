@@ -193,6 +193,13 @@ int cuda_status(cudaError_t e, const char *what) {
 
 bool dtype_ok(int dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
 
+// Whether the cache's bit-widths and shape take the tensor-core decode kernel.
+bool fast_path(const tq_cache &c, int Hq) {
+  const int kw = c.kc.mode == TQ_MSE ? c.kc.bits : c.kc.bits - 1;
+  const int vw = c.vc.mode == TQ_MSE ? c.vc.bits : c.vc.bits - 1;
+  return tq::fast_decode_supported(c.d, c.kc.mode, kw, c.vc.mode, vw, Hq / c.Hkv);
+}
+
 } // namespace
 
 extern "C" {
@@ -313,7 +320,8 @@ size_t tq_decode_workspace_bytes(int B, int Hq, int T_len, const tq_cache *cache
     return 0;
   }
   int vm = cache->vc.mode == TQ_PROD ? (cache->vc.qjl_m ? cache->vc.qjl_m : cache->d) : 0;
-  return tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, vm, sms, false).ws_bytes;
+  return tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, vm, sms, false,
+                         fast_path(*cache, Hq)).ws_bytes;
 }
 
 int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale,
@@ -338,7 +346,8 @@ int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale
   if (st) return st;
   int sms = sm_count();
   if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
-  a.plan = tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, a.v.m, sms, false);
+  a.plan = tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, a.v.m, sms, false,
+                           fast_path(*cache, Hq));
   if (!ws || !aligned16(ws) || ws_bytes < a.plan.ws_bytes)
     return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
                 a.plan.ws_bytes, ws ? ws_bytes : 0);
@@ -380,7 +389,8 @@ int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, flo
   if (st) return st;
   int sms = sm_count();
   if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
-  a.plan = tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, a.v.m, sms, false);
+  a.plan = tq::plan_decode(cache->B, Hq, cache->Hkv, cache->d, T_len, a.v.m, sms, false,
+                           fast_path(*cache, Hq));
   float *scratch = nullptr;
   size_t cap = 0;
   st = cuda_status(tq::fixed_scratch(&scratch, &cap), "fixed scratch lookup");

@@ -50,11 +50,15 @@ struct DequantArgs {
 };
 
 struct DecodePlan {
+  int path;      // 0: generic split-K kernel; 1: tensor-core kernel (decode_mma.cu)
   int tile;      // tokens per pipeline tile
-  int splits;    // context splits per (b, KV head)
-  int chunk;     // tokens per split (a multiple of tile)
-  int gc;        // query heads handled by one CTA (power of two)
-  int ws_stride; // floats per (b, q-head, split) partial record
+  int splits;    // context splits per (b, KV head) (path 0)
+  int chunk;     // tokens per split (a multiple of tile) (path 0)
+  int gc;        // query heads handled by one CTA (path 0: power of two; path 1: G)
+  int ws_stride; // floats per partial record
+  // path 1: the (b, KV head, 16-token tile) space is cut into `ctas` equal ranges
+  int tiles_per_bh, tiles_per_cta, ctas, slots;
+  size_t part_bytes; // bytes of partial records (the query-prep area follows)
   size_t ws_bytes;
 };
 
@@ -90,8 +94,15 @@ cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s);
 // with that device current; later calls return the cached address.
 cudaError_t fixed_scratch(float **ptr, size_t *bytes);
 
-// Split-K plan for the compressed and bf16 decode kernels (decode.cu).
+// Split-K plan for the compressed and bf16 decode kernels (decode.cu). `fast` selects the
+// tensor-core kernel (see fast_decode_supported).
 DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count,
-                       bool bf16);
+                       bool bf16, bool fast = false);
+
+// Tensor-core decode (decode_mma.cu): head_dim 128, 4-bit MSE keys, 2-bit MSE values,
+// 1..8 query heads per KV head.
+bool fast_decode_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G);
+void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p);
+cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s);
 
 } // namespace tq
