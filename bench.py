@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import dataclasses
 import datetime
 import hashlib
 import io
@@ -45,6 +46,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-side", action="store_true", help="skip side measurements")
+    ap.add_argument("--T", type=int, default=0,
+                    help="override the context length (profiling runs on smaller cases)")
     return ap.parse_args()
 
 
@@ -225,6 +228,8 @@ def run_ours(args):
             dist.barrier()
 
     w = WORKLOADS[args.workload]
+    if args.T:
+        w = dataclasses.replace(w, T=args.T)
     K, V, q = make_inputs(w, device="cuda", layer=rank)
     cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, w.k_mode, w.v_mode, w.qjl_m,
                        w.qjl_m, seed=w.seed, qjl_seed=w.qjl_seed)
