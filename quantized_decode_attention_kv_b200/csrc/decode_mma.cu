@@ -44,6 +44,25 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// a * b + c on the IMAD pipe (keeps adds and small multiplies off the integer ALU pipe)
+__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t smem_addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t smem_addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -59,36 +78,12 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ldg_nc16(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint32_t ldg_nc4(const void *p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint32_t ldg_nc2(const void *p) {
-  unsigned short v;
-  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ uint2 lds64(uint32_t smem_addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr));
-  return v;
-}
-
 // Per-tile registers of one warp lane.
 struct Tile {
   uint4 k0, k1;   // key bytes [16c, 16c+16) of tokens r and r+8
   uint32_t v[4];  // value word r of tokens 2c, 2c+1, 2c+8, 2c+9
-  uint32_t kn[2]; // key norms (fp16 bits) of tokens r, r+8
-  uint32_t vn[2]; // value norms (fp16 bits) of tokens r, r+8
+  uint16_t kn[2]; // key norms (fp16 bits) of tokens r, r+8
+  uint16_t vn[2]; // value norms (fp16 bits) of tokens r, r+8
 };
 
 } // namespace
@@ -157,6 +152,7 @@ struct FastArgs {
   long long total_tiles;
   float kcent[16];
   float vcent[4];
+  uint32_t one;
 };
 
 template <int NT>
@@ -171,16 +167,21 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
 
+  // Row e (one code byte) = 32 lane copies of the hi pair, then 32 lane copies of the lo pair
+  // (256 bytes); a lane reads word `lane` of each half, so lookups never share a bank.
+  uint32_t *lutw = reinterpret_cast<uint32_t *>(smem);
   for (int idx = tid; idx < 256 * 32; idx += kThreads) {
-    const int e = idx >> 5;
+    const int e = idx >> 5, l = idx & 31;
     const float c0 = a.kcent[e & 15], c1 = a.kcent[e >> 4];
     const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
-    lut[idx] = make_uint2(pack_h2(c0, c1), pack_h2((c0 - h0) * kLoScale, (c1 - h1) * kLoScale));
+    lutw[e * 64 + l] = pack_h2(c0, c1);
+    lutw[e * 64 + 32 + l] = pack_h2((c0 - h0) * kLoScale, (c1 - h1) * kLoScale);
   }
   const uint32_t vt0 = pack_h2(a.vcent[0], a.vcent[1]);
   const uint32_t vt1 = pack_h2(a.vcent[2], a.vcent[3]);
+  const uint32_t lanebase = static_cast<uint32_t>(lane) << 2;
   const uint32_t lut_base = static_cast<uint32_t>(__cvta_generic_to_shared(lut));
-  const uint32_t lanebase = static_cast<uint32_t>(lane) << 3;
+  const uint32_t one = a.one; // 1, opaque to the compiler so the add stays an IMAD
   __syncthreads();
 
   const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
@@ -232,73 +233,115 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
     for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
 
     const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
-    const uint8_t *kbase = a.kc + rec0 * 64 + 16 * c;
-    const uint8_t *vbase = a.vc + rec0 * 32 + 4 * r;
-    const uint16_t *knb = a.kn + rec0;
-    const uint16_t *vnb = a.vn + rec0;
     const int tlast = a.T_len - 1;
+    // Lane pointers of the next tile this warp loads; a warp advances 4 tiles (64 tokens).
+    int jl = warp;
+    const int tw0 = (tile0 + warp) * 16;
+    const uint8_t *kp = a.kc + (rec0 + tw0 + r) * 64 + 16 * c;
+    const uint8_t *vp = a.vc + (rec0 + tw0 + 2 * c) * 32 + 4 * r;
+    const uint16_t *knp = a.kn + rec0 + tw0 + r;
+    const uint16_t *vnp = a.vn + rec0 + tw0 + r;
 
-    auto load = [&](int jt, Tile &T) {
-      const int t0 = (tile0 + jt) * 16;
-      const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
-      T.k0 = ldg_nc16(kbase + static_cast<size_t>(tr) * 64);
-      T.k1 = ldg_nc16(kbase + static_cast<size_t>(tr8) * 64);
-      const int tv = t0 + 2 * c;
-      T.v[0] = ldg_nc4(vbase + static_cast<size_t>(min(tv, tlast)) * 32);
-      T.v[1] = ldg_nc4(vbase + static_cast<size_t>(min(tv + 1, tlast)) * 32);
-      T.v[2] = ldg_nc4(vbase + static_cast<size_t>(min(tv + 8, tlast)) * 32);
-      T.v[3] = ldg_nc4(vbase + static_cast<size_t>(min(tv + 9, tlast)) * 32);
-      T.kn[0] = ldg_nc2(knb + tr);
-      T.kn[1] = ldg_nc2(knb + tr8);
-      T.vn[0] = ldg_nc2(vnb + tr);
-      T.vn[1] = ldg_nc2(vnb + tr8);
+    // Full tiles load at fixed offsets from the lane pointers; the ragged last tile of a
+    // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
+    auto load_next = [&](Tile &T) {
+      const int t0 = (tile0 + jl) * 16;
+      if (t0 + 16 <= a.T_len) {
+        T.k0 = __ldcs(reinterpret_cast<const uint4 *>(kp));
+        T.k1 = __ldcs(reinterpret_cast<const uint4 *>(kp + 8 * 64));
+        const uint32_t *vq = reinterpret_cast<const uint32_t *>(vp);
+        T.v[0] = __ldcs(vq);
+        T.v[1] = __ldcs(vq + 8);
+        T.v[2] = __ldcs(vq + 64);
+        T.v[3] = __ldcs(vq + 72);
+        T.kn[0] = __ldcs(knp);
+        T.kn[1] = __ldcs(knp + 8);
+        T.vn[0] = __ldcs(vnp);
+        T.vn[1] = __ldcs(vnp + 8);
+      } else {
+        const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
+        const uint8_t *kb = a.kc + rec0 * 64 + 16 * c;
+        T.k0 = __ldcs(reinterpret_cast<const uint4 *>(kb + static_cast<size_t>(tr) * 64));
+        T.k1 = __ldcs(reinterpret_cast<const uint4 *>(kb + static_cast<size_t>(tr8) * 64));
+        const uint8_t *vb = a.vc + rec0 * 32 + 4 * r;
+        const int tv = t0 + 2 * c;
+        T.v[0] = __ldcs(reinterpret_cast<const uint32_t *>(vb + static_cast<size_t>(min(tv, tlast)) * 32));
+        T.v[1] = __ldcs(reinterpret_cast<const uint32_t *>(vb + static_cast<size_t>(min(tv + 1, tlast)) * 32));
+        T.v[2] = __ldcs(reinterpret_cast<const uint32_t *>(vb + static_cast<size_t>(min(tv + 8, tlast)) * 32));
+        T.v[3] = __ldcs(reinterpret_cast<const uint32_t *>(vb + static_cast<size_t>(min(tv + 9, tlast)) * 32));
+        T.kn[0] = __ldcs(a.kn + rec0 + tr);
+        T.kn[1] = __ldcs(a.kn + rec0 + tr8);
+        T.vn[0] = __ldcs(a.vn + rec0 + tr);
+        T.vn[1] = __ldcs(a.vn + rec0 + tr8);
+      }
+      kp += 64 * 64;
+      vp += 64 * 32;
+      knp += 64;
+      vnp += 64;
+      jl += kWarps;
     };
 
-    Tile cur, nxt;
-    int jt = warp;
-    if (jt < ntiles) load(jt, cur);
-    for (; jt < ntiles; jt += kWarps) {
-      if (jt + kWarps < ntiles) load(jt + kWarps, nxt);
-      const int t0 = (tile0 + jt) * 16;
-
+    auto compute = [&](const Tile &T, int t0) {
       // ---- scores: two MMAs per k-step (centroid hi and residual) per n-tile
-      float c1[NT][4], c2[NT][4];
+      constexpr int SPL = NT == 1 ? 2 : 1; // independent accumulator chains
+      float c1[SPL][NT][4], c2[SPL][NT][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int u = 0; u < SPL; ++u)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) c1[nt][e] = c2[nt][e] = 0.f;
-      const uint32_t w0[4] = {cur.k0.x, cur.k0.y, cur.k0.z, cur.k0.w};
-      const uint32_t w1[4] = {cur.k1.x, cur.k1.y, cur.k1.z, cur.k1.w};
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c1[u][nt][e] = c2[u][nt][e] = 0.f;
+      const uint32_t w0[4] = {T.k0.x, T.k0.y, T.k0.z, T.k0.w};
+      const uint32_t w1[4] = {T.k1.x, T.k1.y, T.k1.z, T.k1.w};
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         const uint32_t sel0 = 0x7604u | (static_cast<uint32_t>((2 * s) & 3) << 4);
         const uint32_t sel1 = 0x7604u | (static_cast<uint32_t>((2 * s + 1) & 3) << 4);
-        const uint2 e0 = lds64(lut_base + prmt(w0[s >> 1], lanebase, sel0)); // token r, k 2c..
-        const uint2 e1 = lds64(lut_base + prmt(w1[s >> 1], lanebase, sel0)); // token r+8
-        const uint2 e2 = lds64(lut_base + prmt(w0[s >> 1], lanebase, sel1)); // token r, k 2c+8..
-        const uint2 e3 = lds64(lut_base + prmt(w1[s >> 1], lanebase, sel1)); // token r+8
+        // LUT row (code byte << 8) + lane word; the table base is added on the IMAD pipe. The
+        // four lookups land directly in the A-operand registers of the hi and lo MMAs.
+        const uint32_t ad0 = imad(prmt(w0[s >> 1], lanebase, sel0), one, lut_base); // token r
+        const uint32_t ad1 = imad(prmt(w1[s >> 1], lanebase, sel0), one, lut_base); // token r+8
+        const uint32_t ad2 = imad(prmt(w0[s >> 1], lanebase, sel1), one, lut_base);
+        const uint32_t ad3 = imad(prmt(w1[s >> 1], lanebase, sel1), one, lut_base);
+        uint32_t ah[4], al[4];
+        ah[0] = lds32(ad0);
+        ah[1] = lds32(ad1);
+        ah[2] = lds32(ad2);
+        ah[3] = lds32(ad3);
+        al[0] = lds32(ad0 + 128);
+        al[1] = lds32(ad1 + 128);
+        al[2] = lds32(ad2 + 128);
+        al[3] = lds32(ad3 + 128);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          mma16816(c1[nt], e0.x, e1.x, e2.x, e3.x, qb[nt][2 * s], qb[nt][2 * s + 1]);
-          mma16816(c2[nt], e0.y, e1.y, e2.y, e3.y, qb[nt][2 * s], qb[nt][2 * s + 1]);
+          mma16816(c1[s % SPL][nt], ah[0], ah[1], ah[2], ah[3], qb[nt][2 * s], qb[nt][2 * s + 1]);
+          mma16816(c2[s % SPL][nt], al[0], al[1], al[2], al[3], qb[nt][2 * s], qb[nt][2 * s + 1]);
         }
       }
 
       // ---- online softmax (log2 domain); lane (r, c) owns head 4 nt + c, tokens r, r+8
-      const float kn0 = f16_bits_to_f32(static_cast<uint16_t>(cur.kn[0]));
-      const float kn1 = f16_bits_to_f32(static_cast<uint16_t>(cur.kn[1]));
-      const float vn0 = f16_bits_to_f32(static_cast<uint16_t>(cur.vn[0]));
-      const float vn1 = f16_bits_to_f32(static_cast<uint16_t>(cur.vn[1]));
+      const float kn0 = f16_bits_to_f32(T.kn[0]);
+      const float kn1 = f16_bits_to_f32(T.kn[1]);
+      const float vn0 = f16_bits_to_f32(T.vn[0]);
+      const float vn1 = f16_bits_to_f32(T.vn[1]);
       const bool ok0 = t0 + r < a.T_len, ok1 = t0 + r + 8 < a.T_len;
       uint32_t pk[NT];
       float alpha[NT];
       bool rescale = false;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const float s0 = ok0 ? kn0 * qscale[nt] * fmaf(c1[nt][1] + c2[nt][0], kLoInv, c1[nt][0])
-                             : -INFINITY;
-        const float s1 = ok1 ? kn1 * qscale[nt] * fmaf(c1[nt][3] + c2[nt][2], kLoInv, c1[nt][2])
-                             : -INFINITY;
+        float hh0 = c1[0][nt][0], hl0 = c1[0][nt][1], lh0 = c2[0][nt][0];
+        float hh1 = c1[0][nt][2], hl1 = c1[0][nt][3], lh1 = c2[0][nt][2];
+        if (SPL == 2) {
+          hh0 += c1[SPL - 1][nt][0];
+          hl0 += c1[SPL - 1][nt][1];
+          lh0 += c2[SPL - 1][nt][0];
+          hh1 += c1[SPL - 1][nt][2];
+          hl1 += c1[SPL - 1][nt][3];
+          lh1 += c2[SPL - 1][nt][2];
+        }
+        const float s0 = ok0 ? kn0 * qscale[nt] * fmaf(hl0 + lh0, kLoInv, hh0) : -INFINITY;
+        const float s1 = ok1 ? kn1 * qscale[nt] * fmaf(hl1 + lh1, kLoInv, hh1) : -INFINITY;
         float mx = fmaxf(s0, s1);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -350,28 +393,40 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const uint32_t xsel = half ? 0x7362u : 0x5140u;
-        const uint32_t xa = prmt(cur.v[0], cur.v[1], xsel); // tokens 2c, 2c+1: codes 8half..+7
-        const uint32_t xb = prmt(cur.v[2], cur.v[3], xsel); // tokens 2c+8, 2c+9
-        uint32_t A01[8], A89[8];
+        const uint32_t xa = prmt(T.v[0], T.v[1], xsel); // tokens 2c, 2c+1: codes 8half..+7
+        const uint32_t xb = prmt(T.v[2], T.v[3], xsel); // tokens 2c+8, 2c+9
+        // operand quads of the four m-tiles of this half: codes 2m (rows r) and 2m+1 (rows
+        // r+8), tokens (2c, 2c+1) and (2c+8, 2c+9)
+        uint32_t aq[4][4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t ya = (xa >> (2 * k)) & 0x03030303u;
-          const uint32_t yb = (xb >> (2 * k)) & 0x03030303u;
-          const uint32_t za = ya * 0x22u + 0x10101010u;
-          const uint32_t zb = yb * 0x22u + 0x10101010u;
-          A01[k] = prmt(vt0, vt1, za);           // code 8half + k
-          A01[k + 4] = prmt(vt0, vt1, za >> 16); // code 8half + k + 4
-          A89[k] = prmt(vt0, vt1, zb);
-          A89[k + 4] = prmt(vt0, vt1, zb >> 16);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t ya = (xa >> (2 * kk)) & 0x03030303u;
+          const uint32_t yb = (xb >> (2 * kk)) & 0x03030303u;
+          const uint32_t za = imad(ya, 0x22u, 0x10101010u);
+          const uint32_t zb = imad(yb, 0x22u, 0x10101010u);
+          aq[kk >> 1][kk & 1] = prmt(vt0, vt1, za);
+          aq[kk >> 1][2 + (kk & 1)] = prmt(vt0, vt1, zb);
+          aq[2 + (kk >> 1)][kk & 1] = prmt(vt0, vt1, za >> 16);
+          aq[2 + (kk >> 1)][2 + (kk & 1)] = prmt(vt0, vt1, zb >> 16);
         }
-        // m-tile m covers codes 2m (rows r) and 2m+1 (rows r+8) of the lane's word
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-          const int m = 4 * half + mm;
-          mma16816(o[m], A01[2 * mm], A01[2 * mm + 1], A89[2 * mm], A89[2 * mm + 1], pb0, pb1);
-        }
+        for (int mm = 0; mm < 4; ++mm)
+          mma16816(o[4 * half + mm], aq[mm][0], aq[mm][1], aq[mm][2], aq[mm][3], pb0, pb1);
       }
-      cur = nxt;
+    };
+
+    // Two tile buffers in turn: the next tile loads while the current one computes.
+    Tile ta, tb;
+    int jt = warp;
+    if (jl < ntiles) load_next(ta);
+    while (jt < ntiles) {
+      if (jl < ntiles) load_next(tb);
+      compute(ta, (tile0 + jt) * 16);
+      jt += kWarps;
+      if (jt >= ntiles) break;
+      if (jl < ntiles) load_next(ta);
+      compute(tb, (tile0 + jt) * 16);
+      jt += kWarps;
     }
 
     // ---- merge the warps: common max per head, rescale, accumulate in shared memory
@@ -550,6 +605,7 @@ cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
   for (int j = 0; j < 16; ++j) f.kcent[j] = a.k.cb.c[j];
   for (int j = 0; j < 4; ++j) f.vcent[j] = a.v.cb.c[j];
+  f.one = 1u;
   const int smem = kLutBytes + (kWarps * 8 + 16 + 8 * kD) * 4;
   (void)fast_ctas_per_sm();
   if (f.G <= 4)

@@ -56,8 +56,8 @@ struct DecodePlan {
   int chunk;     // tokens per split (a multiple of tile) (path 0)
   int gc;        // query heads handled by one CTA (path 0: power of two; path 1: G)
   int ws_stride; // floats per partial record
-  // path 1: the (b, KV head, 16-token tile) space is cut into `ctas` equal ranges
-  int tiles_per_bh, tiles_per_cta, ctas, slots;
+  // path 1: the (b, KV head, 16-token tile) space is cut into equal per-warp ranges
+  int tiles_per_bh, tiles_per_cta, tiles_per_warp, ctas, slots;
   size_t part_bytes; // bytes of partial records (the query-prep area follows)
   size_t ws_bytes;
 };
