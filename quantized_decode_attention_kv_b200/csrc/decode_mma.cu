@@ -37,7 +37,13 @@ constexpr int kD = 128;
 constexpr float kLoScale = 4096.0f; // residual scaling 2^12 (keeps residuals normal in fp16)
 constexpr float kLoInv = 1.0f / 4096.0f;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kLutBytes = 256 * 32 * 8; // [code byte][lane] uint2
+constexpr int kLutBytes = 256 * 32 * 8; // [code byte][hi, lo][lane] fp16x2
+#ifndef TQ_DECODE_PREFETCH
+#define TQ_DECODE_PREFETCH 2
+#endif
+// A warp asks L2 for the tile it will load this many of its own steps later (0: no prefetch):
+// loads one step ahead in registers only cover part of the DRAM latency.
+constexpr int kPrefetchSteps = TQ_DECODE_PREFETCH;
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
@@ -244,7 +250,30 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
 
     // Full tiles load at fixed offsets from the lane pointers; the ragged last tile of a
     // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
+    // L2 prefetch lanes: 0-7 the eight 128-byte lines of the key codes of a tile, 8-11 the
+    // four lines of its value codes, 12 and 13 its key and value norms.
+    const int tp0 = tw0 + kPrefetchSteps * kWarps * 16;
+    const char *pfp;
+    size_t pfstep;
+    if (lane < 8) {
+      pfp = reinterpret_cast<const char *>(a.kc + (rec0 + tp0) * 64 + 128 * lane);
+      pfstep = 64 * 64;
+    } else if (lane < 12) {
+      pfp = reinterpret_cast<const char *>(a.vc + (rec0 + tp0) * 32 + 128 * (lane - 8));
+      pfstep = 64 * 32;
+    } else {
+      pfp = reinterpret_cast<const char *>((lane == 12 ? a.kn : a.vn) + rec0 + tp0);
+      pfstep = 64 * 2;
+    }
+    int tpf = tp0;
+
     auto load_next = [&](Tile &T) {
+      if (kPrefetchSteps > 0) {
+        if (lane < 14 && tpf + 16 <= a.T_len && tpf < (tile0 + ntiles) * 16)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
+        pfp += pfstep;
+        tpf += kWarps * 16;
+      }
       const int t0 = (tile0 + jl) * 16;
       if (t0 + 16 <= a.T_len) {
         T.k0 = __ldcs(reinterpret_cast<const uint4 *>(kp));
