@@ -297,7 +297,26 @@ int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
     q.t_offset = t_offset;
     q.d = cache->d;
     q.seed = cache->seed;
-    st = cuda_status(tq::launch_quantize(q, static_cast<cudaStream_t>(stream)), "quantize launch");
+    for (int k = 0; k < 4; ++k) q.sign_words[k] = splitmix64_at(cache->seed, static_cast<uint64_t>(k));
+  }
+  // 16-bit MSE tensors take the streaming kernel (both in one launch); the rest, the
+  // per-vector kernel.
+  const tq::QuantArgs *fast[2] = {nullptr, nullptr};
+  for (int which = 0; which < 2; ++which) {
+    const void *x = which == 0 ? K : V;
+    if (x && tq::quantize_fast_supported(a[which])) fast[which] = &a[which];
+  }
+  if (fast[0] || fast[1]) {
+    const int sms = sm_count();
+    if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
+    st = cuda_status(tq::launch_quantize_fast(fast[0], fast[1], sms, static_cast<cudaStream_t>(stream)),
+                     "quantize launch");
+    if (st) return st;
+  }
+  for (int which = 0; which < 2; ++which) {
+    const void *x = which == 0 ? K : V;
+    if (!x || fast[which]) continue;
+    st = cuda_status(tq::launch_quantize(a[which], static_cast<cudaStream_t>(stream)), "quantize launch");
     if (st) return st;
   }
   return TQ_OK;

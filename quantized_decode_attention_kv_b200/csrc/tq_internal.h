@@ -38,6 +38,7 @@ struct QuantArgs {
   int dtype;
   int B, Hkv, T, T_cap, t_offset, d;
   uint64_t seed;
+  uint64_t sign_words[4]; // SplitMix64 outputs 0..3 of `seed`: bit i set <=> D_ii = -1
   TensorArgs t;
 };
 
@@ -85,6 +86,13 @@ struct DecodeBf16Args {
 
 // Launchers (quantize.cu, decode.cu). Return the launch status.
 cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t s);
+
+// Streaming quantiser (quantize_fast.cu): MSE records of bf16/f16 input, head_dim 64 or 128.
+// K and V (either may be NULL, both must be supported and share dtype, d and seed) are
+// written by one launch.
+bool quantize_fast_supported(const QuantArgs &a);
+cudaError_t launch_quantize_fast(const QuantArgs *k, const QuantArgs *v, int sm_count,
+                                 cudaStream_t s);
 cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s);
