@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -68,15 +68,22 @@ def kernel_traffic():
         return None
     with open(path) as f:
         rec = json.load(f)
-    src = os.path.join(ROOT, "quantized_decode_attention_kv_b200", "csrc", "decode.cu")
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if rec.get("decode_cu_sha256") != digest:
+    if rec.get("sources_sha256") != decode_sources_digest():
         return None
     return rec.get("dram_bytes_per_launch")
 
 
+def decode_sources_digest() -> str:
+    """sha256 over the decode kernels' sources (the split-K and tensor-core decode files)."""
+    h = hashlib.sha256()
+    for name in ("decode.cu", "decode_mma.cu"):
+        with open(os.path.join(ROOT, "quantized_decode_attention_kv_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 class Clocks:
-    """nvidia-smi samples every 200 ms while the timed loop runs."""
+    """nvidia-smi samples every 100 ms while the timed loop runs."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -90,7 +97,7 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -266,7 +273,8 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     value = world * packed / (ms * 1e-3) / 1e9
-    launches_per_step = 4  # quantise K, quantise V, split-K decode, combine
+    nq, nd = tq.tq_launch_counts(cache, k_new.dtype, 1, w.Hq, w.T)
+    launches_per_step = nq + nd
 
     side = {}
     if rank == 0 and not args.no_side:
@@ -280,13 +288,14 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f16-mma/f32", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
                    "k": f"{w.k_bits}-bit {'MSE' if w.k_mode == 0 else 'PROD'}",
                    "v": f"{w.v_bits}-bit {'MSE' if w.v_mode == 0 else 'PROD'}",
                    "packed_bytes_per_step": packed,
                    "step": "quantise 1 new token (K,V) + decode attention over T tokens",
-                   "arithmetic": "u8 packed codes, f32 scores/softmax/accumulation, bf16 query",
+                   "arithmetic": ("u8 packed codes; scores and P.V on f16 tensor cores with f32 "
+                                  "accumulation (hi/lo split centroids and query); f32 softmax"),
                    "l2": "no flush: packed cache per step larger than the 126 MB L2",
                    "parallelism": f"{world} independent replica(s), one per GPU"},
         "gpu_launches": launches_per_step * args.steps,

@@ -160,6 +160,14 @@ int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale
 int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, float scale,
                                 const tq_cache *cache, float *out, void *stream);
 
+/* How many kernels tq_quantize_kv (K and V both given, `dtype` input, T new positions) and
+ * tq_decode_attention (Hq query heads over T_len positions) launch for this cache on the
+ * current device. The pages have no counterpart to this call; benchmarks use it to count the
+ * library's launches. Writes *quantize_launches and *decode_launches (either may be NULL);
+ * returns TQ_OK, or the error the two calls would return for these arguments. */
+int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,
+                     int *quantize_launches, int *decode_launches);
+
 /* Dequantise cache positions [0, T_len) of K (which = 0) or V (which = 1) into out
  * [B][Hkv][T_len][d] of `dtype` in the original domain: x_hat = n D H c / d (MSE), plus
  * the QJL residual estimate sqrt(d) gamma sqrt(pi/2)/m S^T s inside the bracket (PROD). */

@@ -435,6 +435,33 @@ int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, flo
                      "decode (fixed scratch) launch");
 }
 
+int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,
+                     int *quantize_launches, int *decode_launches) {
+  int st = check_cache(cache);
+  if (st) return st;
+  if (!dtype_ok(dtype)) return fail(TQ_ERR_INVALID_ARG, "dtype=%d is not F32/BF16/F16", dtype);
+  if (T < 0 || T > cache->T_cap) return fail(TQ_ERR_INVALID_ARG, "T=%d outside [0, T_cap]", T);
+  if (Hq < 1 || Hq % cache->Hkv || Hq > 65535 || T_len < 1 || T_len > cache->T_cap)
+    return fail(TQ_ERR_INVALID_ARG, "bad Hq=%d or T_len=%d", Hq, T_len);
+  int nq = 0;
+  bool any_fast = false;
+  for (int which = 0; which < 2 && T > 0; ++which) {
+    tq::QuantArgs q{};
+    st = resolve_tensor(*cache, which, &q.t);
+    if (st) return st;
+    q.dtype = dtype;
+    q.B = cache->B;
+    q.Hkv = cache->Hkv;
+    q.T = T;
+    q.d = cache->d;
+    if (tq::quantize_fast_supported(q)) any_fast = true;
+    else ++nq;
+  }
+  if (quantize_launches) *quantize_launches = nq + (any_fast ? 1 : 0);
+  if (decode_launches) *decode_launches = fast_path(*cache, Hq) ? 3 : 2; // (query prep,) split-K, combine
+  return TQ_OK;
+}
+
 int tq_dequantize(const tq_cache *cache, int which, int T_len, void *out, int dtype,
                   void *stream) {
   int st = check_cache(cache);

@@ -87,16 +87,27 @@ __device__ __forceinline__ uint4 lds128(const uint8_t *p) {
   return *reinterpret_cast<const uint4 *>(p);
 }
 
-// OR `code` (WB bits) into the record at coordinate i.
+// Add `code` (WB bits) into the record at coordinate i (the record starts zeroed and codes
+// occupy disjoint bits, so the add is an OR that can fold into one shift-add).
 template <int WB>
 __device__ __forceinline__ void put_code(uint32_t *words, int i, uint32_t code) {
   const int bit = i * WB, wi = bit >> 5, sh = bit & 31;
-  words[wi] |= code << sh;
-  if (sh + WB > 32) words[wi + 1] |= code >> (32 - sh);
+  words[wi] += code << sh;
+  if (sh + WB > 32) words[wi + 1] += code >> (32 - sh);
+}
+
+// Cell-table entry {boundary bits, base code} for the cell index held in the low mantissa
+// bits of u: (u & 0x7F8) | table is one LOP3 because the table is 2048-byte aligned.
+__device__ __forceinline__ uint2 cell_entry(float u, uint32_t table) {
+  uint32_t addr;
+  asm("lop3.b32 %0, %1, 0x7F8, %2, 0xEA;" : "=r"(addr) : "r"(__float_as_uint(u)), "r"(table));
+  uint2 e;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(e.x), "=r"(e.y) : "r"(addr));
+  return e;
 }
 
 template <int D, int WB, bool BF16>
-__device__ __forceinline__ void quantize_row(const uint8_t *row, const uint8_t *cells,
+__device__ __forceinline__ void quantize_row(const uint8_t *row, uint32_t cells,
                                              const FastQuantArgs &a, const FastTensor &t,
                                              unsigned v) {
   constexpr int H = D / 2; // pair stride: P[j] = (x_j, x_{j+H})
@@ -156,8 +167,8 @@ __device__ __forceinline__ void quantize_row(const uint8_t *row, const uint8_t *
     float z0, z1, u0, u1;
     f2_split(z2, z0, z1);
     f2_split(u2, u0, u1);
-    const uint2 e0 = *reinterpret_cast<const uint2 *>(cells + (__float_as_uint(u0) & 0x7F8u));
-    const uint2 e1 = *reinterpret_cast<const uint2 *>(cells + (__float_as_uint(u1) & 0x7F8u));
+    const uint2 e0 = cell_entry(u0, cells);
+    const uint2 e1 = cell_entry(u1, cells);
     put_code<WB>(words, j, e0.y + (z0 > __uint_as_float(e0.x) ? 1u : 0u));
     put_code<WB>(words, j + H, e1.y + (z1 > __uint_as_float(e1.x) ? 1u : 0u));
   }
@@ -185,8 +196,13 @@ __global__ void __launch_bounds__(kQThreads, 3) quantize_fast_kernel(const FastQ
   constexpr int BUF = kQThreads * ROW;   // one staging buffer
   constexpr int CPR = 2 * D / 16;        // 16-byte chunks per row
   extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t *cells = smem;                 // [2 tensors][256 cells] {boundary bits, base code}
-  uint8_t *stage = smem + 2 * kCells * 8;
+  // [2 tensors][256 cells] {boundary bits, base code} at the first 2048-byte aligned shared
+  // address, then the two staging buffers
+  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const uint32_t pad = ((sbase + 2047u) & ~2047u) - sbase;
+  uint8_t *cells = smem + pad;
+  const uint32_t cells_s = sbase + pad;
+  uint8_t *stage = cells + 2 * kCells * 8;
   const int tid = threadIdx.x;
 
   // Cell k covers z in [(8k - 1024.5) / 32, (8k - 1016.5) / 32): the FMA z * 32 + 1.5 * 2^23
@@ -213,8 +229,17 @@ __global__ void __launch_bounds__(kQThreads, 3) quantize_fast_kernel(const FastQ
     const int nv = static_cast<int>(min(static_cast<unsigned>(kQThreads), t.nvec - v0));
     const uint8_t *src = t.x + static_cast<size_t>(v0) * (2 * D);
     const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage + buf * BUF));
-    for (int j = tid; j < nv * CPR; j += kQThreads)
-      cp_async16(dst + (j / CPR) * ROW + (j % CPR) * 16, src + static_cast<size_t>(j) * 16);
+    if (nv == kQThreads) {
+      // chunk j = tid + 128 k: row tid / CPR + k * 128 / CPR, column tid % CPR
+      const uint32_t d0 = dst + (tid / CPR) * ROW + (tid % CPR) * 16;
+      const uint8_t *s0 = src + tid * 16;
+#pragma unroll
+      for (int k = 0; k < CPR; ++k)
+        cp_async16(d0 + k * (kQThreads / CPR) * ROW, s0 + k * kQThreads * 16);
+    } else {
+      for (int j = tid; j < nv * CPR; j += kQThreads)
+        cp_async16(dst + (j / CPR) * ROW + (j % CPR) * 16, src + static_cast<size_t>(j) * 16);
+    }
   };
 
   long long g = blockIdx.x;
@@ -233,7 +258,7 @@ __global__ void __launch_bounds__(kQThreads, 3) quantize_fast_kernel(const FastQ
     const unsigned v = static_cast<unsigned>(lb * kQThreads) + tid;
     if (v < t.nvec) {
       const uint8_t *row = stage + buf * BUF + tid * ROW;
-      const uint8_t *cl = cells + ti * kCells * 8;
+      const uint32_t cl = cells_s + ti * kCells * 8;
       switch (t.wbits) {
       case 1: quantize_row<D, 1, BF16>(row, cl, a, t, v); break;
       case 2: quantize_row<D, 2, BF16>(row, cl, a, t, v); break;
@@ -245,9 +270,107 @@ __global__ void __launch_bounds__(kQThreads, 3) quantize_fast_kernel(const FastQ
   }
 }
 
+// Few vectors (a decode step's new token): one warp per vector with compact, looped code, so
+// that a launch that finds its instructions evicted from L2 by the decode stream still starts
+// fast. Lane l holds coordinates [E l, E l + E); the butterflies of span >= E run across
+// lanes with shuffles; codes count the boundaries below z; the packed record is assembled in
+// shared memory and written by the first lanes.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kQThreads) quantize_small_kernel(const FastQuantArgs a) {
+  constexpr int E = D / 32;        // coordinates per lane
+  constexpr int WPB = kQThreads / 32;
+  __shared__ uint32_t rec_words[WPB][D * 4 / 32];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const unsigned gv = blockIdx.x * WPB + wib;
+  const unsigned nv0 = a.t[0].nvec;
+  const int ti = gv < nv0 ? 0 : 1;
+  const FastTensor &t = a.t[ti];
+  const unsigned v = gv - (ti ? nv0 : 0u);
+  if (ti == 1 && (a.nbatch_total == a.t[0].nbatch || v >= t.nvec)) return;
+
+  float x[E];
+  const uint8_t *src = t.x + (static_cast<size_t>(v) * D + E * lane) * 2;
+  uint32_t w[E / 2];
+  if constexpr (E == 4) {
+    const uint2 q = *reinterpret_cast<const uint2 *>(src);
+    w[0] = q.x;
+    w[1] = q.y;
+  } else {
+    w[0] = *reinterpret_cast<const uint32_t *>(src);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int p = 0; p < E / 2; ++p) {
+    const int pp = (E * lane) / 2 + p; // 16-bit pair index within the vector
+    float lo, hi;
+    if (BF16) {
+      lo = __uint_as_float(w[p] << 16);
+      hi = __uint_as_float(w[p] & 0xFFFF0000u);
+    } else {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[p]));
+      lo = f.x;
+      hi = f.y;
+    }
+    x[2 * p] = __uint_as_float(__float_as_uint(lo) ^ a.sgn_lo[pp]);
+    x[2 * p + 1] = __uint_as_float(__float_as_uint(hi) ^ a.sgn_hi[pp]);
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  // butterflies within the lane
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if ((e & h) == 0) {
+        const float u = x[e], y = x[e + h];
+        x[e] = u + y;
+        x[e + h] = u - y;
+      }
+  // butterflies across lanes: the lane with the span bit set keeps partner - own
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
+      x[e] = upper ? o - x[e] : x[e] + o;
+    }
+  }
+  const float n = sqrtf(ss);
+  const float inv = n > 0.f ? 1.0f / n : 0.0f;
+  const int WB = t.wbits;
+  uint32_t bits = 0; // this lane's E codes, E * WB bits
+  for (int e = 0; e < E; ++e) {
+    const float z = x[e] * inv;
+    uint32_t code = 0;
+    for (int j = 0; j < t.nbeta; ++j) code += z > t.beta[j] ? 1u : 0u;
+    bits |= code << (e * WB);
+  }
+  const int nw = D * WB / 32;
+  uint32_t *rw = rec_words[wib];
+  if (lane < nw) rw[lane] = 0u;
+  __syncwarp();
+  const int bit = lane * E * WB, wi = bit >> 5, sh = bit & 31;
+  atomicOr(&rw[wi], bits << sh);
+  if (sh + E * WB > 32) atomicOr(&rw[wi + 1], bits >> (32 - sh));
+  __syncwarp();
+  const unsigned bh = v / static_cast<unsigned>(t.T);
+  const unsigned tt = v - bh * static_cast<unsigned>(t.T);
+  const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
+  if (lane < nw) reinterpret_cast<uint32_t *>(t.codes + rec * (nw * 4))[lane] = rw[lane];
+  if (lane == 0) t.norm[rec] = f32_to_f16_bits(n);
+}
+
 template <int D, bool BF16>
 cudaError_t run_fast(const FastQuantArgs &f, int sms, cudaStream_t s) {
-  const int smem = 2 * kCells * 8 + 2 * kQThreads * (2 * D + 16);
+  const unsigned nvec = f.t[0].nvec + (f.nbatch_total > f.t[0].nbatch ? f.t[1].nvec : 0u);
+  if (f.nbatch_total < sms) { // fewer than one 128-vector batch per SM
+    const unsigned blocks = (nvec + kQThreads / 32 - 1) / (kQThreads / 32);
+    quantize_small_kernel<D, BF16><<<blocks, kQThreads, 0, s>>>(f);
+    return cudaGetLastError();
+  }
+  const int smem = 2048 + 2 * kCells * 8 + 2 * kQThreads * (2 * D + 16); // 2048: alignment slack
   cudaError_t e = cudaFuncSetAttribute(quantize_fast_kernel<D, BF16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

@@ -56,6 +56,8 @@ EXPORTS = {
     "tq_record_bytes": (ctypes.c_size_t, [ctypes.c_int, tq_qcfg]),
     "tq_quantize_kv": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ctypes.POINTER(tq_cache), ctypes.c_void_p]),
+    "tq_launch_counts": (ctypes.c_int, [ctypes.POINTER(tq_cache), ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "tq_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                     ctypes.POINTER(tq_cache)]),
     "tq_decode_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -217,6 +219,18 @@ def tq_quantize_kv(K: torch.Tensor | None, V: torch.Tensor | None, cache: TQCach
     kp = _dev(K, "K") if K is not None else None
     vp = _dev(V, "V") if V is not None else None
     _check(lib.tq_quantize_kv(kp, vp, dt, T, t_offset, ctypes.byref(cache.struct), _stream(stream)))
+
+
+def tq_launch_counts(cache: TQCache, dtype: torch.dtype, T: int, Hq: int, T_len: int) -> tuple[int, int]:
+    """(kernels one tq_quantize_kv of T positions launches, kernels one tq_decode_attention
+    over T_len positions launches) for this cache on the current device."""
+    dt = _DTYPES.get(dtype)
+    if dt is None:
+        raise TQError(TQ_ERR_INVALID_ARG, f"unsupported dtype {dtype}")
+    nq, nd = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.tq_launch_counts(ctypes.byref(cache.struct), dt, T, Hq, T_len, ctypes.byref(nq),
+                                ctypes.byref(nd)))
+    return nq.value, nd.value
 
 
 def tq_decode_workspace_bytes(cache: TQCache, Hq: int, T_len: int) -> int:
