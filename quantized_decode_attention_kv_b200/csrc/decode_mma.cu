@@ -111,6 +111,8 @@ __global__ void __launch_bounds__(kD) qprep_kernel(const void *q, int dtype, flo
   __shared__ float red[4];
   const int i = threadIdx.x;
   const size_t bq = blockIdx.x;
+  pdl_wait(); // q may come from the kernel before
+  pdl_trigger();
   float x = load_scalar(q, dtype, bq * kD + i);
   if (sign_is_neg(seed, i)) x = -x;
   v[i] = x;
@@ -189,6 +191,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
   const uint32_t lut_base = static_cast<uint32_t>(__cvta_generic_to_shared(lut));
   const uint32_t one = a.one; // 1, opaque to the compiler so the add stays an IMAD
   __syncthreads();
+  pdl_wait(); // the prepared queries and the cache are written by earlier kernels
+  pdl_trigger();
 
   const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
   const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
@@ -514,51 +518,82 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
 }
 
 // Merge the partial records of one (b, q-head) (log2-domain maxima), apply the inverse
-// rotation D H / d once and divide by the softmax sum.
-__global__ void __launch_bounds__(kD) combine_fast_kernel(const float *part, int Hkv, int G,
-                                                          int tiles_per_bh, int tiles_per_cta,
-                                                          int slots, int stride, uint64_t seed,
-                                                          float *out) {
-  __shared__ float o[kD];
-  const int i = threadIdx.x;
-  const int hq = blockIdx.x, b = blockIdx.y;
+// rotation D H / d once and divide by the softmax sum. One warp per (b, q-head): lane k reads
+// the maximum and sum of partial k, so the merge weights need one round of loads; lane l then
+// owns output coordinates [4 l, 4 l + 4) and the Walsh-Hadamard butterflies of span >= 4 run
+// across lanes with shuffles.
+__global__ void __launch_bounds__(128) combine_fast_kernel(const float *part, int B, int Hkv, int G,
+                                                           int tiles_per_bh, int tiles_per_cta,
+                                                           int slots, int stride, uint64_t seed,
+                                                           float *out) {
+  const int lane = threadIdx.x & 31;
   const int Hq = Hkv * G;
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5); // (b, q-head) of this warp
+  pdl_wait(); // the partials come from the decode kernel
+  if (gw >= B * Hq) return;
+  const int b = gw / Hq, hq = gw - b * Hq;
   const int h = hq / G, g = hq - h * G;
   const long long bh = static_cast<long long>(b) * Hkv + h;
   const long long first = bh * tiles_per_bh, last = first + tiles_per_bh - 1;
   const int cta0 = static_cast<int>(first / tiles_per_cta), cta1 = static_cast<int>(last / tiles_per_cta);
+  auto rec = [&](int cta) {
+    const long long bh0 = static_cast<long long>(cta) * tiles_per_cta / tiles_per_bh;
+    return part + ((static_cast<size_t>(cta) * slots + (bh - bh0)) * G + g) * stride;
+  };
   float M = -INFINITY;
-  for (int cta = cta0; cta <= cta1; ++cta) {
-    const long long bh0 = static_cast<long long>(cta) * tiles_per_cta / tiles_per_bh;
-    const float *p = part + ((static_cast<size_t>(cta) * slots + (bh - bh0)) * G + g) * stride;
-    M = fmaxf(M, p[0]);
-  }
-  float L = 0.f, acc = 0.f;
-  for (int cta = cta0; cta <= cta1; ++cta) {
-    const long long bh0 = static_cast<long long>(cta) * tiles_per_cta / tiles_per_bh;
-    const float *p = part + ((static_cast<size_t>(cta) * slots + (bh - bh0)) * G + g) * stride;
-    const float e = exp2f(p[0] - M);
-    L = fmaf(e, p[1], L);
-    acc = fmaf(e, p[2 + i], acc);
-  }
-  o[i] = acc;
-  __syncthreads();
-  for (int hs = 1; hs < kD; hs <<= 1) {
-    float x0 = 0.f, x1 = 0.f;
-    const bool lower = (i & hs) == 0;
-    if (lower) {
-      x0 = o[i];
-      x1 = o[i + hs];
+  for (int c = cta0 + lane; c <= cta1; c += 32) M = fmaxf(M, rec(c)[0]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int c0 = cta0; c0 <= cta1; c0 += 32) {
+    const int c = c0 + lane;
+    float e = 0.f;
+    if (c <= cta1) {
+      const float *p = rec(c);
+      e = exp2f(p[0] - M);
+      L = fmaf(e, p[1], L);
     }
-    __syncthreads();
-    if (lower) {
-      o[i] = x0 + x1;
-      o[i + hs] = x0 - x1;
+    const int n = min(32, cta1 - c0 + 1);
+    for (int k = 0; k < n; ++k) {
+      const float ek = __shfl_sync(0xffffffffu, e, k);
+      const float2 *src = reinterpret_cast<const float2 *>(rec(c0 + k) + 2 + 4 * lane);
+      const float2 u0 = src[0], u1 = src[1];
+      acc[0] = fmaf(ek, u0.x, acc[0]);
+      acc[1] = fmaf(ek, u0.y, acc[1]);
+      acc[2] = fmaf(ek, u1.x, acc[2]);
+      acc[3] = fmaf(ek, u1.y, acc[3]);
     }
-    __syncthreads();
   }
-  const float v = o[i] / (static_cast<float>(kD) * L);
-  out[(static_cast<size_t>(b) * Hq + hq) * kD + i] = sign_is_neg(seed, i) ? -v : v;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  // inverse rotation: butterflies within the lane, then across lanes
+  {
+    const float a0 = acc[0] + acc[1], a1 = acc[0] - acc[1];
+    const float a2 = acc[2] + acc[3], a3 = acc[2] - acc[3];
+    acc[0] = a0 + a2;
+    acc[2] = a0 - a2;
+    acc[1] = a1 + a3;
+    acc[3] = a1 - a3;
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, acc[e], m);
+      acc[e] = upper ? o - acc[e] : acc[e] + o;
+    }
+  }
+  const float sc = 1.0f / (static_cast<float>(kD) * L);
+  const uint64_t sw = dev_splitmix64(seed, static_cast<uint64_t>(lane >> 4)); // coordinates 64 k ..
+  const int sb = (4 * lane) & 63;
+  float4 r;
+  r.x = ((sw >> sb) & 1ull) ? -acc[0] * sc : acc[0] * sc;
+  r.y = ((sw >> (sb + 1)) & 1ull) ? -acc[1] * sc : acc[1] * sc;
+  r.z = ((sw >> (sb + 2)) & 1ull) ? -acc[2] * sc : acc[2] * sc;
+  r.w = ((sw >> (sb + 3)) & 1ull) ? -acc[3] * sc : acc[3] * sc;
+  reinterpret_cast<float4 *>(out + (static_cast<size_t>(b) * Hq + hq) * kD)[lane] = r;
 }
 
 int fast_ctas_per_sm() {
@@ -612,8 +647,8 @@ void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p) {
 cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   const DecodePlan &p = a.plan;
   QPrep *qp = reinterpret_cast<QPrep *>(reinterpret_cast<uint8_t *>(a.ws) + p.part_bytes);
-  qprep_kernel<<<a.B * a.Hq, kD, 0, s>>>(a.q, a.q_dtype, a.scale, a.seed, qp);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(qprep_kernel, dim3(a.B * a.Hq), dim3(kD), 0, s, a.q, a.q_dtype, a.scale,
+                             a.seed, qp);
   if (e != cudaSuccess) return e;
   FastArgs f;
   f.kc = a.k.codes;
@@ -637,16 +672,12 @@ cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   f.one = 1u;
   const int smem = kLutBytes + (kWarps * 8 + 16 + 8 * kD) * 4;
   (void)fast_ctas_per_sm();
-  if (f.G <= 4)
-    decode_k4v2_kernel<1><<<p.ctas, kThreads, smem, s>>>(f);
-  else
-    decode_k4v2_kernel<2><<<p.ctas, kThreads, smem, s>>>(f);
-  e = cudaGetLastError();
+  e = launch_pdl(f.G <= 4 ? decode_k4v2_kernel<1> : decode_k4v2_kernel<2>, dim3(p.ctas),
+                 dim3(kThreads), smem, s, f);
   if (e != cudaSuccess) return e;
-  combine_fast_kernel<<<dim3(a.Hq, a.B), kD, 0, s>>>(a.ws, a.Hkv, f.G, p.tiles_per_bh,
-                                                      p.tiles_per_cta, p.slots, p.ws_stride, a.seed,
-                                                      a.out);
-  return cudaGetLastError();
+  return launch_pdl(combine_fast_kernel, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
+                    static_cast<const float *>(a.ws), a.B, a.Hkv, f.G, p.tiles_per_bh,
+                    p.tiles_per_cta, p.slots, p.ws_stride, a.seed, a.out);
 }
 
 } // namespace tq

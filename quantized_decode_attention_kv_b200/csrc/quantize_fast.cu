@@ -242,6 +242,8 @@ __global__ void __launch_bounds__(kQThreads, 3) quantize_fast_kernel(const FastQ
     }
   };
 
+  pdl_wait(); // K/V may come from the kernel before; the cache may still be read by it
+  pdl_trigger();
   long long g = blockIdx.x;
   int buf = 0;
   if (g < a.nbatch_total) issue(g, 0);
@@ -286,6 +288,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_small_kernel(const FastQua
   const int ti = gv < nv0 ? 0 : 1;
   const FastTensor &t = a.t[ti];
   const unsigned v = gv - (ti ? nv0 : 0u);
+  pdl_wait(); // K/V may come from the kernel before; the cache may still be read by it
+  pdl_trigger();
   if (ti == 1 && (a.nbatch_total == a.t[0].nbatch || v >= t.nvec)) return;
 
   float x[E];
@@ -367,16 +371,15 @@ cudaError_t run_fast(const FastQuantArgs &f, int sms, cudaStream_t s) {
   const unsigned nvec = f.t[0].nvec + (f.nbatch_total > f.t[0].nbatch ? f.t[1].nvec : 0u);
   if (f.nbatch_total < sms) { // fewer than one 128-vector batch per SM
     const unsigned blocks = (nvec + kQThreads / 32 - 1) / (kQThreads / 32);
-    quantize_small_kernel<D, BF16><<<blocks, kQThreads, 0, s>>>(f);
-    return cudaGetLastError();
+    return launch_pdl(quantize_small_kernel<D, BF16>, dim3(blocks), dim3(kQThreads), 0, s, f);
   }
   const int smem = 2048 + 2 * kCells * 8 + 2 * kQThreads * (2 * D + 16); // 2048: alignment slack
   cudaError_t e = cudaFuncSetAttribute(quantize_fast_kernel<D, BF16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long grid = std::min<long long>(f.nbatch_total, 3ll * sms);
-  quantize_fast_kernel<D, BF16><<<static_cast<unsigned>(grid), kQThreads, smem, s>>>(f);
-  return cudaGetLastError();
+  return launch_pdl(quantize_fast_kernel<D, BF16>, dim3(static_cast<unsigned>(grid)), dim3(kQThreads),
+                    smem, s, f);
 }
 
 } // namespace
