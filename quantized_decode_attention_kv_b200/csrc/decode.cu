@@ -570,10 +570,10 @@ cudaError_t run_decode_bf16(const DecodeBf16Args &a, cudaStream_t s) {
 } // namespace
 
 DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count, bool bf16,
-                       bool fast) {
+                       int fast) {
   DecodePlan p{};
   if (fast && !bf16) {
-    plan_fast(B, Hq, Hkv, T_len, sm_count, &p);
+    plan_fast(B, Hq, Hkv, T_len, sm_count, fast >> 4, fast & 15, &p);
     return p;
   }
   p.path = 0;

@@ -37,7 +37,6 @@ constexpr int kD = 128;
 constexpr float kLoScale = 4096.0f; // residual scaling 2^12 (keeps residuals normal in fp16)
 constexpr float kLoInv = 1.0f / 4096.0f;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kLutBytes = 256 * 32 * 8; // [code byte][hi, lo][lane] fp16x2
 #ifndef TQ_DECODE_PREFETCH
 #define TQ_DECODE_PREFETCH 2
 #endif
@@ -63,12 +62,6 @@ __device__ __forceinline__ uint32_t lds32(uint32_t smem_addr) {
   return v;
 }
 
-__device__ __forceinline__ uint2 lds64(uint32_t smem_addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr));
-  return v;
-}
-
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -84,12 +77,35 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Per-tile registers of one warp lane.
+// Per-tile registers of one warp lane for KB-bit keys and VB-bit values (d = 128).
+//  keys: the lane's slice [32c, 32c+32) of the coordinates = KB words of each of tokens r, r+8
+//  values: the lane's run [16r, 16r+16) of the coordinates of tokens 2c, 2c+1, 2c+8, 2c+9:
+//          VB = 2: one word; VB = 3: the two words that hold its 48 bits; VB = 4: two words
+template <int KB, int VB>
 struct Tile {
-  uint4 k0, k1;   // key bytes [16c, 16c+16) of tokens r and r+8
-  uint32_t v[4];  // value word r of tokens 2c, 2c+1, 2c+8, 2c+9
+  static constexpr int VW = VB == 2 ? 1 : 2;
+  uint32_t k[2][KB];
+  uint32_t v[4][VW];
   uint16_t kn[2]; // key norms (fp16 bits) of tokens r, r+8
   uint16_t vn[2]; // value norms (fp16 bits) of tokens r, r+8
+};
+
+// Shared-memory tables of one configuration. Key rows: one code-pair index (4-bit keys: a
+// byte of two codes, 256 rows; 3-bit keys: 6 bits, 64 rows) x {32 lane copies of the fp16x2
+// hi pair, 32 of the lo pair} = 256 bytes. Value rows (VB >= 3): one index (code of the first
+// token | code of the second << VB) x 32 lane copies of the fp16x2 pair = 128 bytes. The
+// 3-bit key table and the value tables sit at addresses aligned to their size so that an
+// index OR-ed above the lane offset is already the address.
+template <int KB, int VB>
+struct Lut {
+  static constexpr int kRows = KB == 4 ? 256 : 64;
+  static constexpr int kBytes = kRows * 256;
+  static constexpr int kAlign = KB == 4 ? 16 : kBytes;
+  static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : 0;
+  static constexpr int vBytes = vRows * 128;
+  static constexpr int vAlign = VB >= 3 ? vBytes : 16;
+  static constexpr int kMergeBytes = (4 * 8 + 16 + 8 * 128) * 4;
+  static constexpr int kSmem = kBytes + kAlign - 16 + vBytes + vAlign - 16 + kMergeBytes;
 };
 
 } // namespace
@@ -159,15 +175,40 @@ struct FastArgs {
   int tiles_per_bh, tiles_per_cta, slots, stride;
   long long total_tiles;
   float kcent[16];
-  float vcent[4];
+  float vcent[16];
   uint32_t one;
 };
 
-template <int NT>
-__global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs a) {
+// Bits [o, o + n) of the little-endian bit string w[0..NWD) moved to bit DST (other bits
+// of the result are unspecified above DST + n and zero below DST when o >= DST).
+template <int NWD>
+__device__ __forceinline__ uint32_t bits_at(const uint32_t (&w)[NWD], int o, int dst) {
+  const int sh = o - dst;
+  if (sh < 0) return w[0] << (-sh);
+  const int wi = sh >> 5, bi = sh & 31;
+  if (bi == 0) return w[wi];
+  const uint32_t hi = wi + 1 < NWD ? w[wi + 1] : 0u;
+  return __funnelshift_r(w[wi], hi, bi);
+}
+
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(c)); // (a & mask) | c
+  return d;
+}
+
+template <int KB, int VB, int NT>
+__global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs a) {
+  using L = Lut<KB, VB>;
+  using TileT = Tile<KB, VB>;
+  constexpr int KR = KB * 16, VR = VB * 16; // record bytes
   extern __shared__ __align__(16) uint8_t smem[];
-  uint2 *lut = reinterpret_cast<uint2 *>(smem);
-  float *mst = reinterpret_cast<float *>(smem + kLutBytes); // [kWarps][8] running max
+  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const uint32_t klut = (sbase + L::kAlign - 1) & ~static_cast<uint32_t>(L::kAlign - 1);
+  const uint32_t vlut = (klut + L::kBytes + L::vAlign - 1) & ~static_cast<uint32_t>(L::vAlign - 1);
+  uint8_t *const kl_p = smem + (klut - sbase);
+  uint8_t *const vl_p = smem + (vlut - sbase);
+  float *mst = reinterpret_cast<float *>(vl_p + L::vBytes); // [kWarps][8] running max
   float *gmx = mst + kWarps * 8;                            // [8] merged max
   float *lsum = gmx + 8;                                    // [8] merged sum
   float *obuf = lsum + 8;                                   // [G][128] merged accumulator
@@ -175,20 +216,26 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
 
-  // Row e (one code byte) = 32 lane copies of the hi pair, then 32 lane copies of the lo pair
-  // (256 bytes); a lane reads word `lane` of each half, so lookups never share a bank.
-  uint32_t *lutw = reinterpret_cast<uint32_t *>(smem);
-  for (int idx = tid; idx < 256 * 32; idx += kThreads) {
-    const int e = idx >> 5, l = idx & 31;
-    const float c0 = a.kcent[e & 15], c1 = a.kcent[e >> 4];
-    const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
-    lutw[e * 64 + l] = pack_h2(c0, c1);
-    lutw[e * 64 + 32 + l] = pack_h2((c0 - h0) * kLoScale, (c1 - h1) * kLoScale);
+  {
+    uint32_t *kw = reinterpret_cast<uint32_t *>(kl_p);
+    for (int idx = tid; idx < L::kRows * 32; idx += kThreads) {
+      const int e = idx >> 5, l = idx & 31;
+      const float c0 = a.kcent[e & (KB == 4 ? 15 : 7)], c1 = a.kcent[KB == 4 ? e >> 4 : e >> 3];
+      const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
+      kw[e * 64 + l] = pack_h2(c0, c1);
+      kw[e * 64 + 32 + l] = pack_h2((c0 - h0) * kLoScale, (c1 - h1) * kLoScale);
+    }
+    uint32_t *vw = reinterpret_cast<uint32_t *>(vl_p);
+    for (int idx = tid; idx < L::vRows * 32; idx += kThreads) {
+      const int e = idx >> 5;
+      vw[idx] = pack_h2(a.vcent[e & ((1 << VB) - 1)], a.vcent[e >> VB]);
+    }
   }
   const uint32_t vt0 = pack_h2(a.vcent[0], a.vcent[1]);
   const uint32_t vt1 = pack_h2(a.vcent[2], a.vcent[3]);
   const uint32_t lanebase = static_cast<uint32_t>(lane) << 2;
-  const uint32_t lut_base = static_cast<uint32_t>(__cvta_generic_to_shared(lut));
+  const uint32_t klb = klut | lanebase; // 3-bit keys: table base with the lane offset
+  const uint32_t vlb = vlut | lanebase;
   const uint32_t one = a.one; // 1, opaque to the compiler so the add stays an IMAD
   __syncthreads();
   pdl_wait(); // the prepared queries and the cache are written by earlier kernels
@@ -244,78 +291,100 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
 
     const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
     const int tlast = a.T_len - 1;
+    // word offset of this lane's value run within a record (3-bit runs start mid-word for odd r)
+    constexpr int kVWordOff = 0;
+    const int vwo = VB == 2 ? r : (VB == 4 ? 2 * r : (3 * r) >> 1);
+    const int vsh = VB == 3 ? 16 * (r & 1) : kVWordOff;
     // Lane pointers of the next tile this warp loads; a warp advances 4 tiles (64 tokens).
     int jl = warp;
     const int tw0 = (tile0 + warp) * 16;
-    const uint8_t *kp = a.kc + (rec0 + tw0 + r) * 64 + 16 * c;
-    const uint8_t *vp = a.vc + (rec0 + tw0 + 2 * c) * 32 + 4 * r;
+    const uint8_t *kp = a.kc + (rec0 + tw0 + r) * KR + 4 * KB * c;
+    const uint8_t *vp = a.vc + (rec0 + tw0 + 2 * c) * VR + 4 * vwo;
     const uint16_t *knp = a.kn + rec0 + tw0 + r;
     const uint16_t *vnp = a.vn + rec0 + tw0 + r;
 
-    // Full tiles load at fixed offsets from the lane pointers; the ragged last tile of a
-    // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
-    // L2 prefetch lanes: 0-7 the eight 128-byte lines of the key codes of a tile, 8-11 the
-    // four lines of its value codes, 12 and 13 its key and value norms.
+    // L2 prefetch lanes: the 128-byte lines of a tile's key codes, then of its value codes,
+    // then one lane each for its key and value norms.
+    constexpr int KL = 16 * KR / 128, VL = 16 * VR / 128;
     const int tp0 = tw0 + kPrefetchSteps * kWarps * 16;
     const char *pfp;
     size_t pfstep;
-    if (lane < 8) {
-      pfp = reinterpret_cast<const char *>(a.kc + (rec0 + tp0) * 64 + 128 * lane);
-      pfstep = 64 * 64;
-    } else if (lane < 12) {
-      pfp = reinterpret_cast<const char *>(a.vc + (rec0 + tp0) * 32 + 128 * (lane - 8));
-      pfstep = 64 * 32;
+    if (lane < KL) {
+      pfp = reinterpret_cast<const char *>(a.kc + (rec0 + tp0) * KR + 128 * lane);
+      pfstep = 64 * KR;
+    } else if (lane < KL + VL) {
+      pfp = reinterpret_cast<const char *>(a.vc + (rec0 + tp0) * VR + 128 * (lane - KL));
+      pfstep = 64 * VR;
     } else {
-      pfp = reinterpret_cast<const char *>((lane == 12 ? a.kn : a.vn) + rec0 + tp0);
+      pfp = reinterpret_cast<const char *>((lane == KL + VL ? a.kn : a.vn) + rec0 + tp0);
       pfstep = 64 * 2;
     }
     int tpf = tp0;
 
-    auto load_next = [&](Tile &T) {
+    auto load_k = [&](uint32_t (&dst)[KB], const uint8_t *p) {
+      if constexpr (KB == 4) {
+        const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
+        dst[0] = q.x;
+        dst[1] = q.y;
+        dst[2] = q.z;
+        dst[3] = q.w;
+      } else {
+#pragma unroll
+        for (int k = 0; k < KB; ++k) dst[k] = __ldcs(reinterpret_cast<const uint32_t *>(p) + k);
+      }
+    };
+    auto load_v = [&](uint32_t (&dst)[TileT::VW], const uint8_t *p) {
+#pragma unroll
+      for (int k = 0; k < TileT::VW; ++k) dst[k] = __ldcs(reinterpret_cast<const uint32_t *>(p) + k);
+    };
+
+    // Full tiles load at fixed offsets from the lane pointers; the ragged last tile of a
+    // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
+    auto load_next = [&](TileT &T) {
       if (kPrefetchSteps > 0) {
-        if (lane < 14 && tpf + 16 <= a.T_len && tpf < (tile0 + ntiles) * 16)
+        if (lane < KL + VL + 2 && tpf + 16 <= a.T_len && tpf < (tile0 + ntiles) * 16)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
         pfp += pfstep;
         tpf += kWarps * 16;
       }
       const int t0 = (tile0 + jl) * 16;
       if (t0 + 16 <= a.T_len) {
-        T.k0 = __ldcs(reinterpret_cast<const uint4 *>(kp));
-        T.k1 = __ldcs(reinterpret_cast<const uint4 *>(kp + 8 * 64));
-        const uint32_t *vq = reinterpret_cast<const uint32_t *>(vp);
-        T.v[0] = __ldcs(vq);
-        T.v[1] = __ldcs(vq + 8);
-        T.v[2] = __ldcs(vq + 64);
-        T.v[3] = __ldcs(vq + 72);
+        load_k(T.k[0], kp);
+        load_k(T.k[1], kp + 8 * KR);
+        load_v(T.v[0], vp);
+        load_v(T.v[1], vp + VR);
+        load_v(T.v[2], vp + 8 * VR);
+        load_v(T.v[3], vp + 9 * VR);
         T.kn[0] = __ldcs(knp);
         T.kn[1] = __ldcs(knp + 8);
         T.vn[0] = __ldcs(vnp);
         T.vn[1] = __ldcs(vnp + 8);
       } else {
         const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
-        const uint8_t *kb = a.kc + rec0 * 64 + 16 * c;
-        T.k0 = __ldcs(reinterpret_cast<const uint4 *>(kb + static_cast<size_t>(tr) * 64));
-        T.k1 = __ldcs(reinterpret_cast<const uint4 *>(kb + static_cast<size_t>(tr8) * 64));
-        const uint8_t *vb = a.vc + rec0 * 32 + 4 * r;
+        const uint8_t *kb = a.kc + rec0 * KR + 4 * KB * c;
+        load_k(T.k[0], kb + static_cast<size_t>(tr) * KR);
+        load_k(T.k[1], kb + static_cast<size_t>(tr8) * KR);
+        const uint8_t *vb = a.vc + rec0 * VR + 4 * vwo;
         const int tv = t0 + 2 * c;
-        T.v[0] = __ldcs(reinterpret_cast<const uint32_t *>(vb + static_cast<size_t>(min(tv, tlast)) * 32));
-        T.v[1] = __ldcs(reinterpret_cast<const uint32_t *>(vb + static_cast<size_t>(min(tv + 1, tlast)) * 32));
-        T.v[2] = __ldcs(reinterpret_cast<const uint32_t *>(vb + static_cast<size_t>(min(tv + 8, tlast)) * 32));
-        T.v[3] = __ldcs(reinterpret_cast<const uint32_t *>(vb + static_cast<size_t>(min(tv + 9, tlast)) * 32));
+        load_v(T.v[0], vb + static_cast<size_t>(min(tv, tlast)) * VR);
+        load_v(T.v[1], vb + static_cast<size_t>(min(tv + 1, tlast)) * VR);
+        load_v(T.v[2], vb + static_cast<size_t>(min(tv + 8, tlast)) * VR);
+        load_v(T.v[3], vb + static_cast<size_t>(min(tv + 9, tlast)) * VR);
         T.kn[0] = __ldcs(a.kn + rec0 + tr);
         T.kn[1] = __ldcs(a.kn + rec0 + tr8);
         T.vn[0] = __ldcs(a.vn + rec0 + tr);
         T.vn[1] = __ldcs(a.vn + rec0 + tr8);
       }
-      kp += 64 * 64;
-      vp += 64 * 32;
+      kp += 64 * KR;
+      vp += 64 * VR;
       knp += 64;
       vnp += 64;
       jl += kWarps;
     };
 
-    auto compute = [&](const Tile &T, int t0) {
-      // ---- scores: two MMAs per k-step (centroid hi and residual) per n-tile
+    auto compute = [&](const TileT &T, int t0) {
+      // ---- scores: two MMAs per k-step (centroid hi and residual) per n-tile. k-step s
+      //      takes the lane's coordinate pairs 2s (a0, a1) and 2s + 1 (a2, a3).
       constexpr int SPL = NT == 1 ? 2 : 1; // independent accumulator chains
       float c1[SPL][NT][4], c2[SPL][NT][4];
 #pragma unroll
@@ -324,18 +393,24 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) c1[u][nt][e] = c2[u][nt][e] = 0.f;
-      const uint32_t w0[4] = {T.k0.x, T.k0.y, T.k0.z, T.k0.w};
-      const uint32_t w1[4] = {T.k1.x, T.k1.y, T.k1.z, T.k1.w};
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        const uint32_t sel0 = 0x7604u | (static_cast<uint32_t>((2 * s) & 3) << 4);
-        const uint32_t sel1 = 0x7604u | (static_cast<uint32_t>((2 * s + 1) & 3) << 4);
-        // LUT row (code byte << 8) + lane word; the table base is added on the IMAD pipe. The
-        // four lookups land directly in the A-operand registers of the hi and lo MMAs.
-        const uint32_t ad0 = imad(prmt(w0[s >> 1], lanebase, sel0), one, lut_base); // token r
-        const uint32_t ad1 = imad(prmt(w1[s >> 1], lanebase, sel0), one, lut_base); // token r+8
-        const uint32_t ad2 = imad(prmt(w0[s >> 1], lanebase, sel1), one, lut_base);
-        const uint32_t ad3 = imad(prmt(w1[s >> 1], lanebase, sel1), one, lut_base);
+        uint32_t ad0, ad1, ad2, ad3;
+        if constexpr (KB == 4) {
+          // LUT row (code byte << 8) + lane word; the table base is added on the IMAD pipe
+          const uint32_t sel0 = 0x7604u | (static_cast<uint32_t>((2 * s) & 3) << 4);
+          const uint32_t sel1 = 0x7604u | (static_cast<uint32_t>((2 * s + 1) & 3) << 4);
+          ad0 = imad(prmt(T.k[0][s >> 1], lanebase, sel0), one, klut); // token r
+          ad1 = imad(prmt(T.k[1][s >> 1], lanebase, sel0), one, klut); // token r+8
+          ad2 = imad(prmt(T.k[0][s >> 1], lanebase, sel1), one, klut);
+          ad3 = imad(prmt(T.k[1][s >> 1], lanebase, sel1), one, klut);
+        } else {
+          // the 6-bit pair index lands at bits 8..13 above the lane offset of the aligned table
+          ad0 = lop_and_or(bits_at(T.k[0], 12 * s, 8), 0x3F00u, klb);
+          ad1 = lop_and_or(bits_at(T.k[1], 12 * s, 8), 0x3F00u, klb);
+          ad2 = lop_and_or(bits_at(T.k[0], 12 * s + 6, 8), 0x3F00u, klb);
+          ad3 = lop_and_or(bits_at(T.k[1], 12 * s + 6, 8), 0x3F00u, klb);
+        }
         uint32_t ah[4], al[4];
         ah[0] = lds32(ad0);
         ah[1] = lds32(ad1);
@@ -422,34 +497,64 @@ __global__ void __launch_bounds__(kThreads, 3) decode_k4v2_kernel(const FastArgs
       const uint32_t pb0 = prmt(x0, x1, 0x5410u); // tokens 2c, 2c+1
       const uint32_t pb1 = prmt(x0, x1, 0x7632u); // tokens 2c+8, 2c+9
 
-      // ---- values: pair-of-token PRMT lookups straight into the A operand, then P'.V
+      // ---- values. m-tile m covers the lane's run coordinates 2m (rows r) and 2m + 1
+      //      (rows r+8); operand quad (a0, a1, a2, a3) = (2m, 2m+1) x tokens (2c, 2c+1) then
+      //      (2c+8, 2c+9).
+      if constexpr (VB == 2) {
+        // pair-of-token PRMT lookups into a 4-entry fp16 table held in two registers
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint32_t xsel = half ? 0x7362u : 0x5140u;
-        const uint32_t xa = prmt(T.v[0], T.v[1], xsel); // tokens 2c, 2c+1: codes 8half..+7
-        const uint32_t xb = prmt(T.v[2], T.v[3], xsel); // tokens 2c+8, 2c+9
-        // operand quads of the four m-tiles of this half: codes 2m (rows r) and 2m+1 (rows
-        // r+8), tokens (2c, 2c+1) and (2c+8, 2c+9)
-        uint32_t aq[4][4];
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t xsel = half ? 0x7362u : 0x5140u;
+          const uint32_t xa = prmt(T.v[0][0], T.v[1][0], xsel); // tokens 2c, 2c+1: codes 8half..+7
+          const uint32_t xb = prmt(T.v[2][0], T.v[3][0], xsel); // tokens 2c+8, 2c+9
+          uint32_t aq[4][4];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t ya = (xa >> (2 * kk)) & 0x03030303u;
-          const uint32_t yb = (xb >> (2 * kk)) & 0x03030303u;
-          const uint32_t za = imad(ya, 0x22u, 0x10101010u);
-          const uint32_t zb = imad(yb, 0x22u, 0x10101010u);
-          aq[kk >> 1][kk & 1] = prmt(vt0, vt1, za);
-          aq[kk >> 1][2 + (kk & 1)] = prmt(vt0, vt1, zb);
-          aq[2 + (kk >> 1)][kk & 1] = prmt(vt0, vt1, za >> 16);
-          aq[2 + (kk >> 1)][2 + (kk & 1)] = prmt(vt0, vt1, zb >> 16);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t ya = (xa >> (2 * kk)) & 0x03030303u;
+            const uint32_t yb = (xb >> (2 * kk)) & 0x03030303u;
+            const uint32_t za = imad(ya, 0x22u, 0x10101010u);
+            const uint32_t zb = imad(yb, 0x22u, 0x10101010u);
+            aq[kk >> 1][kk & 1] = prmt(vt0, vt1, za);
+            aq[kk >> 1][2 + (kk & 1)] = prmt(vt0, vt1, zb);
+            aq[2 + (kk >> 1)][kk & 1] = prmt(vt0, vt1, za >> 16);
+            aq[2 + (kk >> 1)][2 + (kk & 1)] = prmt(vt0, vt1, zb >> 16);
+          }
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm)
+            mma16816(o[4 * half + mm], aq[mm][0], aq[mm][1], aq[mm][2], aq[mm][3], pb0, pb1);
         }
+      } else {
+        // each operand register is one lane-replicated table word indexed by the two tokens'
+        // codes at that coordinate
+        uint32_t run[4][2];
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm)
-          mma16816(o[4 * half + mm], aq[mm][0], aq[mm][1], aq[mm][2], aq[mm][3], pb0, pb1);
+        for (int t = 0; t < 4; ++t) {
+          if constexpr (VB == 3) {
+            run[t][0] = __funnelshift_r(T.v[t][0], T.v[t][1], vsh);
+            run[t][1] = T.v[t][1] >> vsh;
+          } else {
+            run[t][0] = T.v[t][0];
+            run[t][1] = T.v[t][1];
+          }
+        }
+        constexpr uint32_t MA = ((1u << VB) - 1u) << 7, MB = MA << VB;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          uint32_t q[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 2 * m + (e & 1), tp = e >> 1;
+            const uint32_t ta = bits_at(run[2 * tp], VB * i, 7);
+            const uint32_t tb = bits_at(run[2 * tp + 1], VB * i, 7 + VB);
+            q[e] = lds32(lop_and_or(tb, MB, lop_and_or(ta, MA, vlb)));
+          }
+          mma16816(o[m], q[0], q[1], q[2], q[3], pb0, pb1);
+        }
       }
     };
 
     // Two tile buffers in turn: the next tile loads while the current one computes.
-    Tile ta, tb;
+    TileT ta, tb;
     int jt = warp;
     if (jl < ntiles) load_next(ta);
     while (jt < ntiles) {
@@ -596,34 +701,34 @@ __global__ void __launch_bounds__(128) combine_fast_kernel(const float *part, in
   reinterpret_cast<float4 *>(out + (static_cast<size_t>(b) * Hq + hq) * kD)[lane] = r;
 }
 
-int fast_ctas_per_sm() {
-  static std::once_flag once;
-  static int n = 0;
-  std::call_once(once, [] {
-    int v = 0;
-    const int smem = kLutBytes + (kWarps * 8 + 16 + 8 * kD) * 4;
-    if (cudaFuncSetAttribute(decode_k4v2_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) == cudaSuccess &&
-        cudaFuncSetAttribute(decode_k4v2_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) == cudaSuccess &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, decode_k4v2_kernel<2>, kThreads, smem) ==
-            cudaSuccess)
-      n = std::max(1, v);
-    else
-      n = 1;
-  });
-  return n;
+constexpr int kSmemPerSm = 228 * 1024;
+
+// CTAs of the tensor-core decode kernel that fit on one SM (3 at most: 168 registers each).
+int mse_ctas_per_sm(int kb, int vb) {
+  int smem = 0;
+  if (kb == 4) smem = vb == 2 ? Lut<4, 2>::kSmem : vb == 3 ? Lut<4, 3>::kSmem : Lut<4, 4>::kSmem;
+  else smem = vb == 2 ? Lut<3, 2>::kSmem : vb == 3 ? Lut<3, 3>::kSmem : Lut<3, 4>::kSmem;
+  return std::max(1, std::min(3, kSmemPerSm / (smem + 1024)));
+}
+
+template <int KB, int VB>
+cudaError_t run_mse(const FastArgs &f, int ctas, cudaStream_t s) {
+  constexpr int smem = Lut<KB, VB>::kSmem;
+  auto kern = f.G <= 4 ? decode_mse_kernel<KB, VB, 1> : decode_mse_kernel<KB, VB, 2>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(ctas), dim3(kThreads), smem, s, f);
 }
 
 } // namespace
 
 bool fast_decode_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G) {
-  return d == kD && k_mode == TQ_MSE && k_wbits == 4 && v_mode == TQ_MSE && v_wbits == 2 &&
-         G >= 1 && G <= 8;
+  return d == kD && k_mode == TQ_MSE && (k_wbits == 3 || k_wbits == 4) && v_mode == TQ_MSE &&
+         v_wbits >= 2 && v_wbits <= 4 && G >= 1 && G <= 8;
 }
 
 // Layout of the fast path's workspace: [partials][query prep].
-void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p) {
+void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, DecodePlan *p) {
   const int G = Hq / Hkv;
   p->path = 1;
   p->tile = 16;
@@ -631,7 +736,7 @@ void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p) {
   p->ws_stride = 2 + kD + 2; // 132 floats
   p->tiles_per_bh = (T_len + 15) / 16;
   const long long total = static_cast<long long>(B) * Hkv * p->tiles_per_bh;
-  long long ctas = static_cast<long long>(sm_count) * 3;
+  long long ctas = static_cast<long long>(sm_count) * mse_ctas_per_sm(kb, vb);
   ctas = std::min<long long>(ctas, (total + 7) / 8); // at least 8 tiles per CTA
   ctas = std::max<long long>(ctas, 1);
   p->tiles_per_cta = static_cast<int>((total + ctas - 1) / ctas);
@@ -668,12 +773,13 @@ cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   f.stride = p.ws_stride;
   f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
   for (int j = 0; j < 16; ++j) f.kcent[j] = a.k.cb.c[j];
-  for (int j = 0; j < 4; ++j) f.vcent[j] = a.v.cb.c[j];
+  for (int j = 0; j < 16; ++j) f.vcent[j] = a.v.cb.c[j];
   f.one = 1u;
-  const int smem = kLutBytes + (kWarps * 8 + 16 + 8 * kD) * 4;
-  (void)fast_ctas_per_sm();
-  e = launch_pdl(f.G <= 4 ? decode_k4v2_kernel<1> : decode_k4v2_kernel<2>, dim3(p.ctas),
-                 dim3(kThreads), smem, s, f);
+  const int kb = a.k.wbits, vb = a.v.wbits;
+  if (kb == 4) e = vb == 2 ? run_mse<4, 2>(f, p.ctas, s) : vb == 3 ? run_mse<4, 3>(f, p.ctas, s)
+                                                                 : run_mse<4, 4>(f, p.ctas, s);
+  else e = vb == 2 ? run_mse<3, 2>(f, p.ctas, s) : vb == 3 ? run_mse<3, 3>(f, p.ctas, s)
+                                                          : run_mse<3, 4>(f, p.ctas, s);
   if (e != cudaSuccess) return e;
   return launch_pdl(combine_fast_kernel, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
                     static_cast<const float *>(a.ws), a.B, a.Hkv, f.G, p.tiles_per_bh,

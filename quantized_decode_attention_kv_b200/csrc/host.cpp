@@ -193,11 +193,13 @@ int cuda_status(cudaError_t e, const char *what) {
 
 bool dtype_ok(int dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
 
-// Whether the cache's bit-widths and shape take the tensor-core decode kernel.
-bool fast_path(const tq_cache &c, int Hq) {
+// Whether the cache's bit-widths and shape take the tensor-core decode kernel: 0 if not,
+// else (key bits << 4) | value bits.
+int fast_path(const tq_cache &c, int Hq) {
   const int kw = c.kc.mode == TQ_MSE ? c.kc.bits : c.kc.bits - 1;
   const int vw = c.vc.mode == TQ_MSE ? c.vc.bits : c.vc.bits - 1;
-  return tq::fast_decode_supported(c.d, c.kc.mode, kw, c.vc.mode, vw, Hq / c.Hkv);
+  return tq::fast_decode_supported(c.d, c.kc.mode, kw, c.vc.mode, vw, Hq / c.Hkv) ? (kw << 4) | vw
+                                                                                    : 0;
 }
 
 } // namespace
@@ -458,7 +460,7 @@ int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,
     else ++nq;
   }
   if (quantize_launches) *quantize_launches = nq + (any_fast ? 1 : 0);
-  if (decode_launches) *decode_launches = fast_path(*cache, Hq) ? 3 : 2; // (query prep,) split-K, combine
+  if (decode_launches) *decode_launches = fast_path(*cache, Hq) != 0 ? 3 : 2; // (query prep,) split-K, combine
   return TQ_OK;
 }
 

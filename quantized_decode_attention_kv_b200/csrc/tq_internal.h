@@ -103,14 +103,14 @@ cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s);
 cudaError_t fixed_scratch(float **ptr, size_t *bytes);
 
 // Split-K plan for the compressed and bf16 decode kernels (decode.cu). `fast` selects the
-// tensor-core kernel (see fast_decode_supported).
+// tensor-core kernel: 0, or (key bits << 4) | value bits (see fast_decode_supported).
 DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count,
-                       bool bf16, bool fast = false);
+                       bool bf16, int fast = 0);
 
-// Tensor-core decode (decode_mma.cu): head_dim 128, 4-bit MSE keys, 2-bit MSE values,
-// 1..8 query heads per KV head.
+// Tensor-core decode (decode_mma.cu): head_dim 128, MSE keys of 3 or 4 bits, MSE values of
+// 2, 3 or 4 bits, 1..8 query heads per KV head.
 bool fast_decode_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G);
-void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p);
+void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, DecodePlan *p);
 cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s);
 
 } // namespace tq

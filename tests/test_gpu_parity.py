@@ -131,6 +131,10 @@ DECODE_CASES = [
     (256, 3, 1, (2, O.PROD), (4, O.MSE), 128, 128, 128),
     (128, 32, 1, (4, O.MSE), (2, O.MSE), 0, 64, 64),
     (128, 4, 2, (4, O.MSE), (2, O.MSE), 0, 1, 10),
+    # the other key/value bit-widths of the tensor-core kernel, ragged tails
+    (128, 2, 3, (3, O.MSE), (2, O.MSE), 0, 613, 640),
+    (128, 6, 1, (4, O.MSE), (3, O.MSE), 0, 450, 450),
+    (128, 3, 2, (3, O.MSE), (4, O.MSE), 0, 95, 100),
 ]
 
 
