@@ -572,6 +572,10 @@ cudaError_t run_decode_bf16(const DecodeBf16Args &a, cudaStream_t s) {
 DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count, bool bf16,
                        int fast) {
   DecodePlan p{};
+  if (fast == kProdFast && !bf16) {
+    plan_prod(B, Hq, Hkv, T_len, sm_count, &p);
+    return p;
+  }
   if (fast && !bf16) {
     plan_fast(B, Hq, Hkv, T_len, sm_count, fast >> 4, fast & 15, &p);
     return p;
@@ -599,6 +603,7 @@ DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
   if (a.plan.path == 1) return launch_fast_decode(a, s);
+  if (a.plan.path == 2) return launch_prod_decode(a, s);
   TQ_DISPATCH_DEC(run_decode)
 }
 

@@ -23,13 +23,14 @@
 // one (batch, KV head) is a segment, its tiles dealt round-robin to the warps, each warp
 // keeping its own online-softmax state (log2 domain); the warps merge through shared memory
 // at the end of the segment and write one partial record per query head.
-#include "tq_device.cuh"
+#include "mma_ops.cuh"
 
 #include <algorithm>
 #include <mutex>
 
 namespace tq {
 namespace {
+using namespace mma_ops;
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
@@ -43,39 +44,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 // A warp asks L2 for the tile it will load this many of its own steps later (0: no prefetch):
 // loads one step ahead in registers only cover part of the DRAM latency.
 constexpr int kPrefetchSteps = TQ_DECODE_PREFETCH;
-
-__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&h);
-}
-
-// a * b + c on the IMAD pipe (keeps adds and small multiplies off the integer ALU pipe)
-__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t lds32(uint32_t smem_addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // Per-tile registers of one warp lane for KB-bit keys and VB-bit values (d = 128).
 //  keys: the lane's slice [32c, 32c+32) of the coordinates = KB words of each of tokens r, r+8

@@ -1,0 +1,493 @@
+// Tensor-core decode attention over TurboQuant_prod records of head_dim 64 with 2-bit keys
+// and values (1-bit Lloyd-Max codes + a 64-row QJL sign sketch of the residual + the
+// residual norm), one or two query heads per KV head ("Closing - The Three-Step Summary",
+// Step 3; "What the Paper Doesn't Tell You", Finding 2: the GPT-2 low-bit path).
+//
+// Every stored bit of a record is a +-1 factor: the 1-bit code selects -c1 or +c1, the QJL
+// bit the sign of one projection. So per token the 128 bits (64 codes, then 64 signs) form
+// one +-1 vector, exact in fp16, and both products of decode attention are tensor-core MMAs
+// (mma.sync m16n8k16, fp16 x fp16 -> fp32) whose +-1 operand is built from the record bits
+// with one shift and one mask per register (an A register pairs bits j and j + 16 of one
+// record word, which lands them on the two fp16 sign bits; bit set = -1):
+//
+//   scores  S[16 tokens x 8] = A[16 x 128] . B[128 x 8]; per head four columns: the
+//           code part (-c1 q~) and the sketch part (s^ = scale sqrt(pi/2)/(m sqrt(d)) S H D q),
+//           each as an fp16 hi and a 2^12-scaled fp16 residual, in the record-bit order the
+//           A registers use. score_t = ||k_t|| (code part + gamma_t * sketch part).
+//   values  O^T[128 x heads] += A^T[128 x 16 tokens] . P'[16 tokens x heads], code rows with
+//           P' = p ||v||, sketch rows with P' = p ||v|| gamma; the combine forms
+//           u' = -c1 u (the codes' centroids), adds sqrt(d) sqrt(pi/2)/m S^T w, applies the
+//           inverse rotation D H / d once and divides by the softmax sum.
+//
+// The work split, online softmax and partial records follow the MSE tensor-core kernel.
+#include "mma_ops.cuh"
+
+#include <algorithm>
+
+namespace tq {
+namespace {
+using namespace mma_ops;
+
+constexpr int kPW = 4;            // warps per CTA
+constexpr int kPThreads = kPW * 32;
+constexpr int kPD = 64;           // head_dim
+constexpr int kPM = 64;           // QJL rows
+constexpr float kPLoScale = 4096.0f;
+constexpr float kPLoInv = 1.0f / 4096.0f;
+constexpr float kPLog2e = 1.4426950408889634f;
+constexpr float kPSqrtHalfPi = 1.2533141373155003f;
+
+// Prepared query of one (b, q-head): the B operand of the score MMA in fragment order.
+// Word 16 c + 2 s (+1) holds the values at record bits 32 c + 2 s (+1) and 32 c + 2 s + 16
+// (+1) of lane group c, k-step s; bits 0..63 are code bits (value -c1 q~_i), 64..127 sketch
+// bits (value s^_j). inv[t] undoes the power-of-two normalisation of part t (codes, sketch).
+struct QPrepP {
+  uint32_t hi[64];
+  uint32_t lo[64];
+  float inv[2];
+  float pad[2];
+};
+
+__global__ void __launch_bounds__(kPD) qprep_prod_kernel(const void *q, int dtype, float scale,
+                                                         uint64_t seed, const float *Sk, float c1,
+                                                         QPrepP *out) {
+  __shared__ float v[kPD];
+  __shared__ float val[kPD + kPM];
+  __shared__ float red[4];
+  const int i = threadIdx.x;
+  const size_t bq = blockIdx.x;
+  pdl_wait(); // q may come from the kernel before
+  pdl_trigger();
+  float x = load_scalar(q, dtype, bq * kPD + i);
+  if (sign_is_neg(seed, i)) x = -x;
+  v[i] = x;
+  __syncthreads();
+  for (int hs = 1; hs < kPD; hs <<= 1) {
+    float a = 0.f, b = 0.f;
+    const bool lower = (i & hs) == 0;
+    if (lower) {
+      a = v[i];
+      b = v[i + hs];
+    }
+    __syncthreads();
+    if (lower) {
+      v[i] = a + b;
+      v[i + hs] = a - b;
+    }
+    __syncthreads();
+  }
+  // v = H D q; code part -c1 scale v / d, sketch part scale sqrt(pi/2) / (m sqrt(d)) S v
+  const float sk_scale = scale * kPSqrtHalfPi / (static_cast<float>(kPM) * sqrtf(static_cast<float>(kPD)));
+  float sacc = 0.f;
+  const float *srow = Sk + static_cast<size_t>(i) * kPD;
+  for (int k = 0; k < kPD; ++k) sacc = fmaf(__ldg(srow + k), v[k], sacc);
+  val[i] = -c1 * v[i] * (scale / static_cast<float>(kPD));
+  val[kPD + i] = sk_scale * sacc;
+  // power-of-two normalisation per part so that max |value| lands in [1, 2)
+  float m0 = warp_max(fabsf(val[i])), m1 = warp_max(fabsf(val[kPD + i]));
+  if ((i & 31) == 0) {
+    red[i >> 5] = m0;
+    red[2 + (i >> 5)] = m1;
+  }
+  __syncthreads();
+  float f[2];
+  for (int t = 0; t < 2; ++t) {
+    const float mx = fmaxf(red[2 * t], red[2 * t + 1]);
+    f[t] = 1.0f;
+    if (mx > 0.f && isfinite(mx)) {
+      int ex;
+      frexpf(mx, &ex);
+      f[t] = ldexpf(1.0f, 1 - ex);
+    }
+  }
+  // thread i writes fragment word i: lane group c, k-step s, second half of the pair if odd
+  const int c = i >> 4, w = i & 15, s = w >> 1, odd = w & 1;
+  const int e0 = 32 * c + 2 * s + odd, e1 = e0 + 16;
+  const float y0 = val[e0] * f[e0 >> 6], y1 = val[e1] * f[e1 >> 6];
+  const __half h0 = __float2half_rn(y0), h1 = __float2half_rn(y1);
+  const __half l0 = __float2half_rn((y0 - __half2float(h0)) * kPLoScale);
+  const __half l1 = __float2half_rn((y1 - __half2float(h1)) * kPLoScale);
+  out[bq].hi[i] = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
+  out[bq].lo[i] = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+  if (i == 0) {
+    out[bq].inv[0] = 1.0f / f[0];
+    out[bq].inv[1] = 1.0f / f[1];
+  }
+}
+
+struct ProdArgs {
+  const uint8_t *kc, *ks, *vc, *vs;       // codes and sign sketches, 8 bytes per record each
+  const uint16_t *kn, *kg, *vn, *vg;      // norms and residual norms (fp16 bits)
+  const QPrepP *qp;
+  float *part; // partial records [cta][slot][G][stride]
+  int Hq, Hkv, G, T_len, T_cap;
+  int tiles_per_bh, tiles_per_cta, slots, stride;
+  long long total_tiles;
+};
+
+// +-1 fp16 pair from bits (j, j + 16) of w moved to the sign bits by a left shift of `sh`
+// (sh = 15 - j): bit set = -1.
+__device__ __forceinline__ uint32_t pm1(uint32_t w, int sh) {
+  return ((w << sh) & 0x80008000u) | 0x3C003C00u;
+}
+
+struct ProdTile {
+  uint32_t kw[2];  // record word c (codes 0-1, signs 2-3) of tokens r, r + 8
+  uint32_t vm[4];  // code word r / 4 of tokens 2c, 2c+1, 2c+8, 2c+9
+  uint32_t vq[4];  // sign word r / 4 of the same tokens
+  uint16_t kn[2], kg[2], vn[2], vg[2]; // norms and residual norms of tokens r, r + 8
+};
+
+__global__ void __launch_bounds__(kPThreads, 4) decode_prod_kernel(const ProdArgs a) {
+  __shared__ float mst[kPW * 8];
+  __shared__ float gmx[8];
+  __shared__ float lsum[8];
+  __shared__ float obuf[2][kPD + kPM];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = lane >> 2, c = lane & 3;
+  const int gh = c >> 1, part = c & 1; // head and part of this lane's score columns
+  pdl_wait(); // the prepared queries and the cache are written by earlier kernels
+  pdl_trigger();
+
+  const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
+  const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
+  int slot = 0;
+  for (long long seg = range0; seg < range1; ++slot) {
+    const long long bh = seg / a.tiles_per_bh;
+    const long long seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
+    const int tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+    const int ntiles = static_cast<int>(seg_end - seg);
+    seg = seg_end;
+    const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
+
+    // B operand of the score MMA: column r = head r / 4, part (r / 2) & 1, hi/lo r & 1; only
+    // record words of that part (codes: c < 2, sketch: c >= 2) are non-zero.
+    uint32_t qb[16];
+    {
+      const int g = r >> 2, t = (r >> 1) & 1;
+      if (g < a.G && (c >= 2) == (t == 1)) {
+        const QPrepP *p = a.qp + static_cast<size_t>(b) * a.Hq + h * a.G + g;
+        const uint4 *src = reinterpret_cast<const uint4 *>(((r & 1) ? p->lo : p->hi) + 16 * c);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 w = __ldg(src + k);
+          qb[4 * k] = w.x;
+          qb[4 * k + 1] = w.y;
+          qb[4 * k + 2] = w.z;
+          qb[4 * k + 3] = w.w;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) qb[k] = 0u;
+      }
+    }
+    const float pinv = gh < a.G ? __ldg(&a.qp[static_cast<size_t>(b) * a.Hq + h * a.G + gh].inv[part]) : 0.f;
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[8][4];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+
+    const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
+    const int tlast = a.T_len - 1;
+    const uint8_t *kbase = (c < 2 ? a.kc : a.ks) + 4 * (c & 1);
+    const int vwo = 4 * (r >> 2);
+    const uint32_t selx = static_cast<uint32_t>(r & 3) | (static_cast<uint32_t>(4 + (r & 3)) << 8);
+    int jl = warp;
+
+    auto load_next = [&](ProdTile &T) {
+      const int t0 = (tile0 + jl) * 16;
+      const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
+      const int tv = t0 + 2 * c;
+      const int tvs[4] = {min(tv, tlast), min(tv + 1, tlast), min(tv + 8, tlast), min(tv + 9, tlast)};
+      T.kw[0] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (rec0 + tr) * 8));
+      T.kw[1] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (rec0 + tr8) * 8));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        T.vm[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (rec0 + tvs[e]) * 8 + vwo));
+        T.vq[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (rec0 + tvs[e]) * 8 + vwo));
+      }
+      T.kn[0] = __ldcs(a.kn + rec0 + tr);
+      T.kn[1] = __ldcs(a.kn + rec0 + tr8);
+      T.kg[0] = __ldcs(a.kg + rec0 + tr);
+      T.kg[1] = __ldcs(a.kg + rec0 + tr8);
+      T.vn[0] = __ldcs(a.vn + rec0 + tr);
+      T.vn[1] = __ldcs(a.vn + rec0 + tr8);
+      T.vg[0] = __ldcs(a.vg + rec0 + tr);
+      T.vg[1] = __ldcs(a.vg + rec0 + tr8);
+      jl += kPW;
+    };
+
+    auto compute = [&](const ProdTile &T, int t0) {
+      // ---- scores: one MMA per k-step; lane (r, c) gets part c & 1 of head c >> 1 for
+      //      tokens r, r + 8 (hi in even columns, residual in odd columns)
+      float acc[2][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        mma16816(acc[s & 1], pm1(T.kw[0], 15 - 2 * s), pm1(T.kw[1], 15 - 2 * s),
+                 pm1(T.kw[0], 14 - 2 * s), pm1(T.kw[1], 14 - 2 * s), qb[2 * s], qb[2 * s + 1]);
+      const float mine0 = fmaf(acc[0][1] + acc[1][1], kPLoInv, acc[0][0] + acc[1][0]) * pinv;
+      const float mine1 = fmaf(acc[0][3] + acc[1][3], kPLoInv, acc[0][2] + acc[1][2]) * pinv;
+      const float oth0 = __shfl_xor_sync(0xffffffffu, mine0, 1);
+      const float oth1 = __shfl_xor_sync(0xffffffffu, mine1, 1);
+      const float code0 = part ? oth0 : mine0, sk0 = part ? mine0 : oth0;
+      const float code1 = part ? oth1 : mine1, sk1 = part ? mine1 : oth1;
+      const float kn0 = f16_bits_to_f32(T.kn[0]), kn1 = f16_bits_to_f32(T.kn[1]);
+      const float kg0 = f16_bits_to_f32(T.kg[0]), kg1 = f16_bits_to_f32(T.kg[1]);
+      const float vn0 = f16_bits_to_f32(T.vn[0]), vn1 = f16_bits_to_f32(T.vn[1]);
+      const float vg0 = f16_bits_to_f32(T.vg[0]), vg1 = f16_bits_to_f32(T.vg[1]);
+      const bool ok0 = t0 + r < a.T_len, ok1 = t0 + r + 8 < a.T_len;
+      const float s0 = ok0 ? kn0 * fmaf(kg0, sk0, code0) * kPLog2e : -INFINITY;
+      const float s1 = ok1 ? kn1 * fmaf(kg1, sk1, code1) * kPLog2e : -INFINITY;
+
+      // ---- online softmax (log2 domain) over the lane's head
+      float mx = fmaxf(s0, s1);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mn = fmaxf(m_run, mx);
+      const float alpha = exp2f(m_run - mn);
+      const bool moved = mn != m_run;
+      m_run = mn;
+      const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
+      l_run = fmaf(l_run, alpha, p0 + p1);
+      const uint32_t pkc = pack_h2(p0 * vn0, p1 * vn1);
+      const uint32_t pks = pack_h2(p0 * vn0 * vg0, p1 * vn1 * vg1);
+      if (__any_sync(0xffffffffu, moved)) {
+        // lane (r, c) accumulates heads 2c, 2c + 1: head 0 lives on lanes c = 0, head 1 on c = 2
+        const float al0 = __shfl_sync(0xffffffffu, alpha, lane & ~3);
+        const float al1 = __shfl_sync(0xffffffffu, alpha, (lane & ~3) | 2);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          o[m][0] *= al0;
+          o[m][1] *= al1;
+          o[m][2] *= al0;
+          o[m][3] *= al1;
+        }
+      }
+
+      // ---- P' operands (column r = head r): tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1)
+      const int srca = 8 * c + 2 * (r & 1), srcb = srca + 4;
+      uint32_t xc0 = __shfl_sync(0xffffffffu, pkc, srca), xc1 = __shfl_sync(0xffffffffu, pkc, srcb);
+      uint32_t xs0 = __shfl_sync(0xffffffffu, pks, srca), xs1 = __shfl_sync(0xffffffffu, pks, srcb);
+      if (r >= a.G) xc0 = xc1 = xs0 = xs1 = 0u;
+      const uint32_t pbc0 = prmt(xc0, xc1, 0x5410u), pbc1 = prmt(xc0, xc1, 0x7632u);
+      const uint32_t pbs0 = prmt(xs0, xs1, 0x5410u), pbs1 = prmt(xs0, xs1, 0x7632u);
+
+      // ---- values: byte r & 3 of the lane's record word, first token in byte 0, second in
+      //      byte 2, so bit i of the byte pair shifts onto the fp16 sign bits
+      const uint32_t xm0 = prmt(T.vm[0], T.vm[1], selx), xm1 = prmt(T.vm[2], T.vm[3], selx);
+      const uint32_t xq0 = prmt(T.vq[0], T.vq[1], selx), xq1 = prmt(T.vq[2], T.vq[3], selx);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int sh0 = 15 - 2 * m, sh1 = 14 - 2 * m;
+        mma16816(o[m], pm1(xm0, sh0), pm1(xm0, sh1), pm1(xm1, sh0), pm1(xm1, sh1), pbc0, pbc1);
+        mma16816(o[4 + m], pm1(xq0, sh0), pm1(xq0, sh1), pm1(xq1, sh0), pm1(xq1, sh1), pbs0, pbs1);
+      }
+    };
+
+    ProdTile ta, tb;
+    int jt = warp;
+    if (jl < ntiles) load_next(ta);
+    while (jt < ntiles) {
+      if (jl < ntiles) load_next(tb);
+      compute(ta, (tile0 + jt) * 16);
+      jt += kPW;
+      if (jt >= ntiles) break;
+      if (jl < ntiles) load_next(ta);
+      compute(tb, (tile0 + jt) * 16);
+      jt += kPW;
+    }
+
+    // ---- merge the warps: common max per head, rescale, accumulate in shared memory
+    float l = l_run;
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
+    l += __shfl_xor_sync(0xffffffffu, l, 8);
+    l += __shfl_xor_sync(0xffffffffu, l, 16);
+    if (r == 0 && part == 0) mst[warp * 8 + gh] = m_run;
+    for (int idx = tid; idx < 2 * (kPD + kPM); idx += kPThreads) (&obuf[0][0])[idx] = 0.f;
+    if (tid < 8) lsum[tid] = 0.f;
+    __syncthreads();
+    if (tid < 2) {
+      float M = -INFINITY;
+      for (int w = 0; w < kPW; ++w) M = fmaxf(M, mst[w * 8 + tid]);
+      gmx[tid] = M;
+    }
+    __syncthreads();
+    if (r == 0 && part == 0 && gh < a.G) atomicAdd(&lsum[gh], l * exp2f(m_run - gmx[gh]));
+    if (c == 0) {
+      const float f0 = exp2f(mst[warp * 8] - gmx[0]);
+      const float f1 = a.G > 1 ? exp2f(mst[warp * 8 + 1] - gmx[1]) : 0.f;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int i0 = (m < 4 ? 0 : kPD) + 8 * r + 2 * (m & 3);
+        atomicAdd(&obuf[0][i0], o[m][0] * f0);
+        atomicAdd(&obuf[0][i0 + 1], o[m][2] * f0);
+        if (a.G > 1) {
+          atomicAdd(&obuf[1][i0], o[m][1] * f1);
+          atomicAdd(&obuf[1][i0 + 1], o[m][3] * f1);
+        }
+      }
+    }
+    __syncthreads();
+    float *dst = a.part + (static_cast<size_t>(blockIdx.x) * a.slots + slot) * a.G * a.stride;
+    for (int idx = tid; idx < a.G * (kPD + kPM); idx += kPThreads) {
+      const int g = idx / (kPD + kPM), i = idx - g * (kPD + kPM);
+      dst[static_cast<size_t>(g) * a.stride + 2 + i] = obuf[g][i];
+    }
+    if (tid < a.G) {
+      dst[static_cast<size_t>(tid) * a.stride] = gmx[tid];
+      dst[static_cast<size_t>(tid) * a.stride + 1] = lsum[tid];
+    }
+    __syncthreads();
+  }
+}
+
+// Merge the partial records of one (b, q-head); u' = -c1 u, add sqrt(d) sqrt(pi/2)/m S^T w,
+// apply the inverse rotation D H / d and divide by the softmax sum. One warp per (b, q-head);
+// lane l owns coordinates 2 l, 2 l + 1 and sketch rows 2 l, 2 l + 1.
+__global__ void __launch_bounds__(128) combine_prod_kernel(const float *part, int B, int Hkv, int G,
+                                                           int tiles_per_bh, int tiles_per_cta,
+                                                           int slots, int stride, uint64_t seed,
+                                                           const float *Sv, float c1v, float *out) {
+  const int lane = threadIdx.x & 31;
+  const int Hq = Hkv * G;
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  pdl_wait(); // the partials come from the decode kernel
+  if (gw >= B * Hq) return;
+  const int b = gw / Hq, hq = gw - b * Hq;
+  const int h = hq / G, g = hq - h * G;
+  const long long bh = static_cast<long long>(b) * Hkv + h;
+  const long long first = bh * tiles_per_bh, last = first + tiles_per_bh - 1;
+  const int cta0 = static_cast<int>(first / tiles_per_cta), cta1 = static_cast<int>(last / tiles_per_cta);
+  auto rec = [&](int cta) {
+    const long long bh0 = static_cast<long long>(cta) * tiles_per_cta / tiles_per_bh;
+    return part + ((static_cast<size_t>(cta) * slots + (bh - bh0)) * G + g) * stride;
+  };
+  float M = -INFINITY;
+  for (int c = cta0 + lane; c <= cta1; c += 32) M = fmaxf(M, rec(c)[0]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f, u0 = 0.f, u1 = 0.f, w0 = 0.f, w1 = 0.f;
+  for (int c0 = cta0; c0 <= cta1; c0 += 32) {
+    const int c = c0 + lane;
+    float e = 0.f;
+    if (c <= cta1) {
+      const float *p = rec(c);
+      e = exp2f(p[0] - M);
+      L = fmaf(e, p[1], L);
+    }
+    const int n = min(32, cta1 - c0 + 1);
+    for (int k = 0; k < n; ++k) {
+      const float ek = __shfl_sync(0xffffffffu, e, k);
+      const float *p = rec(c0 + k) + 2;
+      const float2 uu = *reinterpret_cast<const float2 *>(p + 2 * lane);
+      const float2 ww = *reinterpret_cast<const float2 *>(p + kPD + 2 * lane);
+      u0 = fmaf(ek, uu.x, u0);
+      u1 = fmaf(ek, uu.y, u1);
+      w0 = fmaf(ek, ww.x, w0);
+      w1 = fmaf(ek, ww.y, w1);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  // y = S^T w for this lane's two coordinates
+  float y0 = 0.f, y1 = 0.f;
+#pragma unroll 8
+  for (int j = 0; j < kPM; ++j) {
+    const float wj = __shfl_sync(0xffffffffu, (j & 1) ? w1 : w0, j >> 1);
+    const float2 sj = __ldg(reinterpret_cast<const float2 *>(Sv + static_cast<size_t>(j) * kPD) + lane);
+    y0 = fmaf(sj.x, wj, y0);
+    y1 = fmaf(sj.y, wj, y1);
+  }
+  const float kap = sqrtf(static_cast<float>(kPD)) * kPSqrtHalfPi / static_cast<float>(kPM);
+  float x0 = fmaf(kap, y0, -c1v * u0), x1 = fmaf(kap, y1, -c1v * u1);
+  // inverse rotation: the span-1 butterfly in the lane, spans 2..32 across lanes
+  {
+    const float a0 = x0 + x1, a1 = x0 - x1;
+    x0 = a0;
+    x1 = a1;
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+    const float o0 = __shfl_xor_sync(0xffffffffu, x0, m);
+    const float o1 = __shfl_xor_sync(0xffffffffu, x1, m);
+    x0 = upper ? o0 - x0 : x0 + o0;
+    x1 = upper ? o1 - x1 : x1 + o1;
+  }
+  const float sc = 1.0f / (static_cast<float>(kPD) * L);
+  const uint64_t sw = dev_splitmix64(seed, 0);
+  float2 res;
+  res.x = ((sw >> (2 * lane)) & 1ull) ? -x0 * sc : x0 * sc;
+  res.y = ((sw >> (2 * lane + 1)) & 1ull) ? -x1 * sc : x1 * sc;
+  reinterpret_cast<float2 *>(out + (static_cast<size_t>(b) * Hq + hq) * kPD)[lane] = res;
+}
+
+} // namespace
+
+bool prod_decode_supported(int d, int k_mode, int k_bits, int k_m, int v_mode, int v_bits, int v_m,
+                           int G) {
+  return d == kPD && k_mode == TQ_PROD && k_bits == 2 && k_m == kPM && v_mode == TQ_PROD &&
+         v_bits == 2 && v_m == kPM && G >= 1 && G <= 2;
+}
+
+void plan_prod(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p) {
+  const int G = Hq / Hkv;
+  p->path = 2;
+  p->tile = 16;
+  p->gc = G;
+  p->ws_stride = 2 + kPD + kPM + 2; // 132 floats
+  p->tiles_per_bh = (T_len + 15) / 16;
+  const long long total = static_cast<long long>(B) * Hkv * p->tiles_per_bh;
+  long long ctas = static_cast<long long>(sm_count) * 4;
+  ctas = std::min<long long>(ctas, (total + 7) / 8); // at least 8 tiles per CTA
+  ctas = std::max<long long>(ctas, 1);
+  p->tiles_per_cta = static_cast<int>((total + ctas - 1) / ctas);
+  p->ctas = static_cast<int>((total + p->tiles_per_cta - 1) / p->tiles_per_cta);
+  p->slots = (p->tiles_per_cta + p->tiles_per_bh - 1) / p->tiles_per_bh + 1;
+  p->splits = 0;
+  p->chunk = 0;
+  p->part_bytes = static_cast<size_t>(p->ctas) * p->slots * G * p->ws_stride * sizeof(float);
+  p->part_bytes = (p->part_bytes + 255) / 256 * 256;
+  p->ws_bytes = p->part_bytes + static_cast<size_t>(B) * Hq * sizeof(QPrepP);
+}
+
+cudaError_t launch_prod_decode(const DecodeArgs &a, cudaStream_t s) {
+  const DecodePlan &p = a.plan;
+  QPrepP *qp = reinterpret_cast<QPrepP *>(reinterpret_cast<uint8_t *>(a.ws) + p.part_bytes);
+  cudaError_t e = launch_pdl(qprep_prod_kernel, dim3(a.B * a.Hq), dim3(kPD), 0, s, a.q, a.q_dtype,
+                             a.scale, a.seed, a.k.S, a.k.cb.c[1], qp);
+  if (e != cudaSuccess) return e;
+  ProdArgs f;
+  f.kc = a.k.codes;
+  f.ks = a.k.signs;
+  f.vc = a.v.codes;
+  f.vs = a.v.signs;
+  f.kn = a.k.norm;
+  f.kg = a.k.rnorm;
+  f.vn = a.v.norm;
+  f.vg = a.v.rnorm;
+  f.qp = qp;
+  f.part = a.ws;
+  f.Hq = a.Hq;
+  f.Hkv = a.Hkv;
+  f.G = a.Hq / a.Hkv;
+  f.T_len = a.T_len;
+  f.T_cap = a.T_cap;
+  f.tiles_per_bh = p.tiles_per_bh;
+  f.tiles_per_cta = p.tiles_per_cta;
+  f.slots = p.slots;
+  f.stride = p.ws_stride;
+  f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
+  e = launch_pdl(decode_prod_kernel, dim3(p.ctas), dim3(kPThreads), 0, s, f);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(combine_prod_kernel, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
+                    static_cast<const float *>(a.ws), a.B, a.Hkv, f.G, p.tiles_per_bh,
+                    p.tiles_per_cta, p.slots, p.ws_stride, a.seed, a.v.S, a.v.cb.c[1], a.out);
+}
+
+} // namespace tq

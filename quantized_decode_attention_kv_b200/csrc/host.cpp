@@ -193,11 +193,14 @@ int cuda_status(cudaError_t e, const char *what) {
 
 bool dtype_ok(int dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
 
-// Whether the cache's bit-widths and shape take the tensor-core decode kernel: 0 if not,
-// else (key bits << 4) | value bits.
+// Whether the cache's bit-widths and shape take a tensor-core decode kernel: 0 if not,
+// kProdFast for the TurboQuant_prod kernel, else (key bits << 4) | value bits.
 int fast_path(const tq_cache &c, int Hq) {
   const int kw = c.kc.mode == TQ_MSE ? c.kc.bits : c.kc.bits - 1;
   const int vw = c.vc.mode == TQ_MSE ? c.vc.bits : c.vc.bits - 1;
+  const int km = c.kc.qjl_m ? c.kc.qjl_m : c.d, vm = c.vc.qjl_m ? c.vc.qjl_m : c.d;
+  if (tq::prod_decode_supported(c.d, c.kc.mode, c.kc.bits, km, c.vc.mode, c.vc.bits, vm, Hq / c.Hkv))
+    return tq::kProdFast;
   return tq::fast_decode_supported(c.d, c.kc.mode, kw, c.vc.mode, vw, Hq / c.Hkv) ? (kw << 4) | vw
                                                                                     : 0;
 }

@@ -51,7 +51,8 @@ struct DequantArgs {
 };
 
 struct DecodePlan {
-  int path;      // 0: generic split-K kernel; 1: tensor-core kernel (decode_mma.cu)
+  int path;      // 0: generic split-K kernel; 1: tensor-core MSE kernel (decode_mma.cu);
+                 // 2: tensor-core PROD kernel (decode_prod.cu)
   int tile;      // tokens per pipeline tile
   int splits;    // context splits per (b, KV head) (path 0)
   int chunk;     // tokens per split (a multiple of tile) (path 0)
@@ -102,8 +103,9 @@ cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s);
 // with that device current; later calls return the cached address.
 cudaError_t fixed_scratch(float **ptr, size_t *bytes);
 
-// Split-K plan for the compressed and bf16 decode kernels (decode.cu). `fast` selects the
-// tensor-core kernel: 0, or (key bits << 4) | value bits (see fast_decode_supported).
+// Split-K plan for the compressed and bf16 decode kernels (decode.cu). `fast` selects a
+// tensor-core kernel: 0 (none), (key bits << 4) | value bits (MSE, see
+// fast_decode_supported) or kProdFast (see prod_decode_supported).
 DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count,
                        bool bf16, int fast = 0);
 
@@ -112,5 +114,13 @@ DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm
 bool fast_decode_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G);
 void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, DecodePlan *p);
 cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s);
+
+// Tensor-core decode of TurboQuant_prod records (decode_prod.cu): head_dim 64, 2-bit keys and
+// values with 64 QJL rows each, 1..2 query heads per KV head. Plan code kProdFast.
+constexpr int kProdFast = 0x200;
+bool prod_decode_supported(int d, int k_mode, int k_bits, int k_m, int v_mode, int v_bits, int v_m,
+                           int G);
+void plan_prod(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p);
+cudaError_t launch_prod_decode(const DecodeArgs &a, cudaStream_t s);
 
 } // namespace tq

@@ -135,6 +135,8 @@ DECODE_CASES = [
     (128, 2, 3, (3, O.MSE), (2, O.MSE), 0, 613, 640),
     (128, 6, 1, (4, O.MSE), (3, O.MSE), 0, 450, 450),
     (128, 3, 2, (3, O.MSE), (4, O.MSE), 0, 95, 100),
+    # the tensor-core TurboQuant_prod kernel with two query heads per KV head
+    (64, 2, 2, (2, O.PROD), (2, O.PROD), 64, 333, 340),
 ]
 
 
