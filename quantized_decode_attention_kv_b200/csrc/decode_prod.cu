@@ -36,6 +36,10 @@ constexpr float kPLoScale = 4096.0f;
 constexpr float kPLoInv = 1.0f / 4096.0f;
 constexpr float kPLog2e = 1.4426950408889634f;
 constexpr float kPSqrtHalfPi = 1.2533141373155003f;
+#ifndef TQ_PROD_PREFETCH
+#define TQ_PROD_PREFETCH 3
+#endif
+constexpr int kPPrefetch = TQ_PROD_PREFETCH; // L2 prefetch distance in warp steps
 
 // Prepared query of one (b, q-head): the B operand of the score MMA in fragment order.
 // Word 16 c + 2 s (+1) holds the values at record bits 32 c + 2 s (+1) and 32 c + 2 s + 16
@@ -123,12 +127,16 @@ struct ProdArgs {
   int Hq, Hkv, G, T_len, T_cap;
   int tiles_per_bh, tiles_per_cta, slots, stride;
   long long total_tiles;
+  uint32_t one2; // fp16 (1, 1): 0x3C003C00
 };
 
 // +-1 fp16 pair from bits (j, j + 16) of w moved to the sign bits by a left shift of `sh`
-// (sh = 15 - j): bit set = -1.
-__device__ __forceinline__ uint32_t pm1(uint32_t w, int sh) {
-  return ((w << sh) & 0x80008000u) | 0x3C003C00u;
+// (sh = 15 - j): bit set = -1. `one2` holds fp16 (1, 1) in a register so that the mask and
+// the OR are one LOP3.
+__device__ __forceinline__ uint32_t pm1(uint32_t w, int sh, uint32_t one2) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, 0x80008000, %2, 0xEA;" : "=r"(d) : "r"(w << sh), "r"(one2));
+  return d;
 }
 
 struct ProdTile {
@@ -138,7 +146,7 @@ struct ProdTile {
   uint16_t kn[2], kg[2], vn[2], vg[2]; // norms and residual norms of tokens r, r + 8
 };
 
-__global__ void __launch_bounds__(kPThreads, 4) decode_prod_kernel(const ProdArgs a) {
+__global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArgs a) {
   __shared__ float mst[kPW * 8];
   __shared__ float gmx[8];
   __shared__ float lsum[8];
@@ -147,6 +155,7 @@ __global__ void __launch_bounds__(kPThreads, 4) decode_prod_kernel(const ProdArg
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
   const int gh = c >> 1, part = c & 1; // head and part of this lane's score columns
+  const uint32_t one2 = a.one2;
   pdl_wait(); // the prepared queries and the cache are written by earlier kernels
   pdl_trigger();
 
@@ -195,27 +204,81 @@ __global__ void __launch_bounds__(kPThreads, 4) decode_prod_kernel(const ProdArg
     const int vwo = 4 * (r >> 2);
     const uint32_t selx = static_cast<uint32_t>(r & 3) | (static_cast<uint32_t>(4 + (r & 3)) << 8);
     int jl = warp;
+    // L2 prefetch, kPrefetchSteps warp steps ahead: lanes 0-3 the 128-byte lines of a tile's
+    // key codes, key signs, value codes and value signs; lanes 4-7 its four norm arrays.
+    const int tp0 = (tile0 + warp) * 16 + kPPrefetch * kPW * 16;
+    const char *pfp = nullptr;
+    int pfstep = 0;
+    {
+      const int q = lane & 3;
+      if (lane < 4) {
+        const uint8_t *base = q == 0 ? a.kc : q == 1 ? a.ks : q == 2 ? a.vc : a.vs;
+        pfp = reinterpret_cast<const char *>(base + (rec0 + tp0) * 8);
+        pfstep = kPW * 16 * 8;
+      } else if (lane < 8) {
+        const uint16_t *base = q == 0 ? a.kn : q == 1 ? a.kg : q == 2 ? a.vn : a.vg;
+        pfp = reinterpret_cast<const char *>(base + rec0 + tp0);
+        pfstep = kPW * 16 * 2;
+      }
+    }
+    int tpf = tp0;
+
+    // lane pointers of the next full tile this warp loads (a warp advances 64 tokens)
+    const int tw0 = (tile0 + warp) * 16;
+    const uint8_t *kp = kbase + (rec0 + tw0 + r) * 8;
+    const uint8_t *vcp = a.vc + (rec0 + tw0 + 2 * c) * 8 + vwo;
+    const uint8_t *vsp = a.vs + (rec0 + tw0 + 2 * c) * 8 + vwo;
+    const uint16_t *np[4] = {a.kn + rec0 + tw0 + r, a.kg + rec0 + tw0 + r, a.vn + rec0 + tw0 + r,
+                             a.vg + rec0 + tw0 + r};
 
     auto load_next = [&](ProdTile &T) {
+      if (lane < 8 && tpf + 16 <= a.T_len && tpf < (tile0 + ntiles) * 16)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
+      pfp += pfstep;
+      tpf += kPW * 16;
       const int t0 = (tile0 + jl) * 16;
-      const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
-      const int tv = t0 + 2 * c;
-      const int tvs[4] = {min(tv, tlast), min(tv + 1, tlast), min(tv + 8, tlast), min(tv + 9, tlast)};
-      T.kw[0] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (rec0 + tr) * 8));
-      T.kw[1] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (rec0 + tr8) * 8));
+      if (t0 + 16 <= a.T_len) {
+        T.kw[0] = __ldcs(reinterpret_cast<const uint32_t *>(kp));
+        T.kw[1] = __ldcs(reinterpret_cast<const uint32_t *>(kp + 64));
+        const int toff[4] = {0, 8, 64, 72};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        T.vm[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (rec0 + tvs[e]) * 8 + vwo));
-        T.vq[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (rec0 + tvs[e]) * 8 + vwo));
+        for (int e = 0; e < 4; ++e) {
+          T.vm[e] = __ldcs(reinterpret_cast<const uint32_t *>(vcp + toff[e]));
+          T.vq[e] = __ldcs(reinterpret_cast<const uint32_t *>(vsp + toff[e]));
+        }
+        T.kn[0] = __ldcs(np[0]);
+        T.kn[1] = __ldcs(np[0] + 8);
+        T.kg[0] = __ldcs(np[1]);
+        T.kg[1] = __ldcs(np[1] + 8);
+        T.vn[0] = __ldcs(np[2]);
+        T.vn[1] = __ldcs(np[2] + 8);
+        T.vg[0] = __ldcs(np[3]);
+        T.vg[1] = __ldcs(np[3] + 8);
+      } else {
+        const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
+        const int tv = t0 + 2 * c;
+        const int tvs[4] = {min(tv, tlast), min(tv + 1, tlast), min(tv + 8, tlast), min(tv + 9, tlast)};
+        T.kw[0] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (rec0 + tr) * 8));
+        T.kw[1] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (rec0 + tr8) * 8));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          T.vm[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (rec0 + tvs[e]) * 8 + vwo));
+          T.vq[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (rec0 + tvs[e]) * 8 + vwo));
+        }
+        T.kn[0] = __ldcs(a.kn + rec0 + tr);
+        T.kn[1] = __ldcs(a.kn + rec0 + tr8);
+        T.kg[0] = __ldcs(a.kg + rec0 + tr);
+        T.kg[1] = __ldcs(a.kg + rec0 + tr8);
+        T.vn[0] = __ldcs(a.vn + rec0 + tr);
+        T.vn[1] = __ldcs(a.vn + rec0 + tr8);
+        T.vg[0] = __ldcs(a.vg + rec0 + tr);
+        T.vg[1] = __ldcs(a.vg + rec0 + tr8);
       }
-      T.kn[0] = __ldcs(a.kn + rec0 + tr);
-      T.kn[1] = __ldcs(a.kn + rec0 + tr8);
-      T.kg[0] = __ldcs(a.kg + rec0 + tr);
-      T.kg[1] = __ldcs(a.kg + rec0 + tr8);
-      T.vn[0] = __ldcs(a.vn + rec0 + tr);
-      T.vn[1] = __ldcs(a.vn + rec0 + tr8);
-      T.vg[0] = __ldcs(a.vg + rec0 + tr);
-      T.vg[1] = __ldcs(a.vg + rec0 + tr8);
+      kp += kPW * 16 * 8;
+      vcp += kPW * 16 * 8;
+      vsp += kPW * 16 * 8;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) np[e] += kPW * 16;
       jl += kPW;
     };
 
@@ -227,8 +290,8 @@ __global__ void __launch_bounds__(kPThreads, 4) decode_prod_kernel(const ProdArg
       for (int u = 0; u < 2; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
 #pragma unroll
       for (int s = 0; s < 8; ++s)
-        mma16816(acc[s & 1], pm1(T.kw[0], 15 - 2 * s), pm1(T.kw[1], 15 - 2 * s),
-                 pm1(T.kw[0], 14 - 2 * s), pm1(T.kw[1], 14 - 2 * s), qb[2 * s], qb[2 * s + 1]);
+        mma16816(acc[s & 1], pm1(T.kw[0], 15 - 2 * s, one2), pm1(T.kw[1], 15 - 2 * s, one2),
+                 pm1(T.kw[0], 14 - 2 * s, one2), pm1(T.kw[1], 14 - 2 * s, one2), qb[2 * s], qb[2 * s + 1]);
       const float mine0 = fmaf(acc[0][1] + acc[1][1], kPLoInv, acc[0][0] + acc[1][0]) * pinv;
       const float mine1 = fmaf(acc[0][3] + acc[1][3], kPLoInv, acc[0][2] + acc[1][2]) * pinv;
       const float oth0 = __shfl_xor_sync(0xffffffffu, mine0, 1);
@@ -284,8 +347,10 @@ __global__ void __launch_bounds__(kPThreads, 4) decode_prod_kernel(const ProdArg
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int sh0 = 15 - 2 * m, sh1 = 14 - 2 * m;
-        mma16816(o[m], pm1(xm0, sh0), pm1(xm0, sh1), pm1(xm1, sh0), pm1(xm1, sh1), pbc0, pbc1);
-        mma16816(o[4 + m], pm1(xq0, sh0), pm1(xq0, sh1), pm1(xq1, sh0), pm1(xq1, sh1), pbs0, pbs1);
+        mma16816(o[m], pm1(xm0, sh0, one2), pm1(xm0, sh1, one2), pm1(xm1, sh0, one2),
+                 pm1(xm1, sh1, one2), pbc0, pbc1);
+        mma16816(o[4 + m], pm1(xq0, sh0, one2), pm1(xq0, sh1, one2), pm1(xq1, sh0, one2),
+                 pm1(xq1, sh1, one2), pbs0, pbs1);
       }
     };
 
@@ -443,7 +508,7 @@ void plan_prod(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p) {
   p->ws_stride = 2 + kPD + kPM + 2; // 132 floats
   p->tiles_per_bh = (T_len + 15) / 16;
   const long long total = static_cast<long long>(B) * Hkv * p->tiles_per_bh;
-  long long ctas = static_cast<long long>(sm_count) * 4;
+  long long ctas = static_cast<long long>(sm_count) * 3;
   ctas = std::min<long long>(ctas, (total + 7) / 8); // at least 8 tiles per CTA
   ctas = std::max<long long>(ctas, 1);
   p->tiles_per_cta = static_cast<int>((total + ctas - 1) / ctas);
@@ -483,6 +548,7 @@ cudaError_t launch_prod_decode(const DecodeArgs &a, cudaStream_t s) {
   f.slots = p.slots;
   f.stride = p.ws_stride;
   f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
+  f.one2 = 0x3C003C00u;
   e = launch_pdl(decode_prod_kernel, dim3(p.ctas), dim3(kPThreads), 0, s, f);
   if (e != cudaSuccess) return e;
   return launch_pdl(combine_prod_kernel, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
