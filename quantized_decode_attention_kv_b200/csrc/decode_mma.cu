@@ -27,6 +27,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 namespace tq {
 namespace {
@@ -44,6 +45,17 @@ constexpr float kLog2e = 1.4426950408889634f;
 // A warp asks L2 for the tile it will load this many of its own steps later (0: no prefetch):
 // loads one step ahead in registers only cover part of the DRAM latency.
 constexpr int kPrefetchSteps = TQ_DECODE_PREFETCH;
+
+// The first dynamic shared address of a kernel without static shared memory on sm_100 (the
+// 1 KB below it is reserved by the hardware); the kernel checks it before relying on it.
+constexpr uint32_t kFixedBase = 1024;
+
+template <uint32_t OFF>
+__device__ __forceinline__ uint32_t lds32_off(uint32_t smem_addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(smem_addr), "n"(OFF));
+  return v;
+}
 
 // Per-tile registers of one warp lane for KB-bit keys and VB-bit values (d = 128).
 //  keys: the lane's slice [32c, 32c+32) of the coordinates = KB words of each of tokens r, r+8
@@ -209,385 +221,415 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
   pdl_wait(); // the prepared queries and the cache are written by earlier kernels
   pdl_trigger();
 
-  const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
-  const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
-  int slot = 0;
-  for (long long seg = range0; seg < range1; ++slot) {
-    const long long bh = seg / a.tiles_per_bh;
-    const long long seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
-    const int tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
-    const int ntiles = static_cast<int>(seg_end - seg);
-    seg = seg_end;
-    const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
+  // Two copies of the persistent loop: when the 4-bit key table starts at the usual first
+  // dynamic shared address (kFixedBase), the table base is an immediate offset of the shared
+  // loads and the PRMT that places the code byte above the lane offset is the whole address
+  // computation; otherwise an IMAD adds the base.
+  auto run = [&](auto fixed_tag) {
+    constexpr bool kFixed = decltype(fixed_tag)::value;
+    const uint32_t klane = lanebase;
+    const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
+    const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
+    int slot = 0;
+    for (long long seg = range0; seg < range1; ++slot) {
+      const long long bh = seg / a.tiles_per_bh;
+      const long long seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
+      const int tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+      const int ntiles = static_cast<int>(seg_end - seg);
+      seg = seg_end;
+      const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
 
-    // ---- B operands of the score MMA: column n = r of n-tile nt is head g = 4 nt + r/2,
-    //      hi (r even) or residual (r odd); thread c holds coordinates [32c, 32c+32).
-    uint32_t qb[NT][16];
-    float qscale[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int g = nt * 4 + (r >> 1);
-      if (g < a.G) {
-        const QPrep *p = a.qp + static_cast<size_t>(b) * a.Hq + h * a.G + g;
-        const uint4 *src = reinterpret_cast<const uint4 *>(((r & 1) ? p->lo : p->hi) + 32 * c);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint4 w = __ldg(src + k);
-          qb[nt][4 * k] = w.x;
-          qb[nt][4 * k + 1] = w.y;
-          qb[nt][4 * k + 2] = w.z;
-          qb[nt][4 * k + 3] = w.w;
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) qb[nt][k] = 0u;
-      }
-      const int gs = nt * 4 + c; // head of this lane's score columns
-      qscale[nt] = gs < a.G ? __ldg(&a.qp[static_cast<size_t>(b) * a.Hq + h * a.G + gs].inv) * kLog2e
-                            : 0.f;
-    }
-
-    float m_run[NT], l_run[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      m_run[nt] = -INFINITY;
-      l_run[nt] = 0.f;
-    }
-    float o[8][4];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
-
-    const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
-    const int tlast = a.T_len - 1;
-    // word offset of this lane's value run within a record (3-bit runs start mid-word for odd r)
-    constexpr int kVWordOff = 0;
-    const int vwo = VB == 2 ? r : (VB == 4 ? 2 * r : (3 * r) >> 1);
-    const int vsh = VB == 3 ? 16 * (r & 1) : kVWordOff;
-    // Lane pointers of the next tile this warp loads; a warp advances 4 tiles (64 tokens).
-    int jl = warp;
-    const int tw0 = (tile0 + warp) * 16;
-    const uint8_t *kp = a.kc + (rec0 + tw0 + r) * KR + 4 * KB * c;
-    const uint8_t *vp = a.vc + (rec0 + tw0 + 2 * c) * VR + 4 * vwo;
-    const uint16_t *knp = a.kn + rec0 + tw0 + r;
-    const uint16_t *vnp = a.vn + rec0 + tw0 + r;
-
-    // L2 prefetch lanes: the 128-byte lines of a tile's key codes, then of its value codes,
-    // then one lane each for its key and value norms.
-    constexpr int KL = 16 * KR / 128, VL = 16 * VR / 128;
-    const int tp0 = tw0 + kPrefetchSteps * kWarps * 16;
-    const char *pfp;
-    size_t pfstep;
-    if (lane < KL) {
-      pfp = reinterpret_cast<const char *>(a.kc + (rec0 + tp0) * KR + 128 * lane);
-      pfstep = 64 * KR;
-    } else if (lane < KL + VL) {
-      pfp = reinterpret_cast<const char *>(a.vc + (rec0 + tp0) * VR + 128 * (lane - KL));
-      pfstep = 64 * VR;
-    } else {
-      pfp = reinterpret_cast<const char *>((lane == KL + VL ? a.kn : a.vn) + rec0 + tp0);
-      pfstep = 64 * 2;
-    }
-    int tpf = tp0;
-
-    auto load_k = [&](uint32_t (&dst)[KB], const uint8_t *p) {
-      if constexpr (KB == 4) {
-        const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
-        dst[0] = q.x;
-        dst[1] = q.y;
-        dst[2] = q.z;
-        dst[3] = q.w;
-      } else {
-#pragma unroll
-        for (int k = 0; k < KB; ++k) dst[k] = __ldcs(reinterpret_cast<const uint32_t *>(p) + k);
-      }
-    };
-    auto load_v = [&](uint32_t (&dst)[TileT::VW], const uint8_t *p) {
-#pragma unroll
-      for (int k = 0; k < TileT::VW; ++k) dst[k] = __ldcs(reinterpret_cast<const uint32_t *>(p) + k);
-    };
-
-    // Full tiles load at fixed offsets from the lane pointers; the ragged last tile of a
-    // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
-    auto load_next = [&](TileT &T) {
-      if (kPrefetchSteps > 0) {
-        if (lane < KL + VL + 2 && tpf + 16 <= a.T_len && tpf < (tile0 + ntiles) * 16)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
-        pfp += pfstep;
-        tpf += kWarps * 16;
-      }
-      const int t0 = (tile0 + jl) * 16;
-      if (t0 + 16 <= a.T_len) {
-        load_k(T.k[0], kp);
-        load_k(T.k[1], kp + 8 * KR);
-        load_v(T.v[0], vp);
-        load_v(T.v[1], vp + VR);
-        load_v(T.v[2], vp + 8 * VR);
-        load_v(T.v[3], vp + 9 * VR);
-        T.kn[0] = __ldcs(knp);
-        T.kn[1] = __ldcs(knp + 8);
-        T.vn[0] = __ldcs(vnp);
-        T.vn[1] = __ldcs(vnp + 8);
-      } else {
-        const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
-        const uint8_t *kb = a.kc + rec0 * KR + 4 * KB * c;
-        load_k(T.k[0], kb + static_cast<size_t>(tr) * KR);
-        load_k(T.k[1], kb + static_cast<size_t>(tr8) * KR);
-        const uint8_t *vb = a.vc + rec0 * VR + 4 * vwo;
-        const int tv = t0 + 2 * c;
-        load_v(T.v[0], vb + static_cast<size_t>(min(tv, tlast)) * VR);
-        load_v(T.v[1], vb + static_cast<size_t>(min(tv + 1, tlast)) * VR);
-        load_v(T.v[2], vb + static_cast<size_t>(min(tv + 8, tlast)) * VR);
-        load_v(T.v[3], vb + static_cast<size_t>(min(tv + 9, tlast)) * VR);
-        T.kn[0] = __ldcs(a.kn + rec0 + tr);
-        T.kn[1] = __ldcs(a.kn + rec0 + tr8);
-        T.vn[0] = __ldcs(a.vn + rec0 + tr);
-        T.vn[1] = __ldcs(a.vn + rec0 + tr8);
-      }
-      kp += 64 * KR;
-      vp += 64 * VR;
-      knp += 64;
-      vnp += 64;
-      jl += kWarps;
-    };
-
-    auto compute = [&](const TileT &T, int t0) {
-      // ---- scores: two MMAs per k-step (centroid hi and residual) per n-tile. k-step s
-      //      takes the lane's coordinate pairs 2s (a0, a1) and 2s + 1 (a2, a3).
-      constexpr int SPL = NT == 1 ? 2 : 1; // independent accumulator chains
-      float c1[SPL][NT][4], c2[SPL][NT][4];
-#pragma unroll
-      for (int u = 0; u < SPL; ++u)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) c1[u][nt][e] = c2[u][nt][e] = 0.f;
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        uint32_t ad0, ad1, ad2, ad3;
-        if constexpr (KB == 4) {
-          // LUT row (code byte << 8) + lane word; the table base is added on the IMAD pipe
-          const uint32_t sel0 = 0x7604u | (static_cast<uint32_t>((2 * s) & 3) << 4);
-          const uint32_t sel1 = 0x7604u | (static_cast<uint32_t>((2 * s + 1) & 3) << 4);
-          ad0 = imad(prmt(T.k[0][s >> 1], lanebase, sel0), one, klut); // token r
-          ad1 = imad(prmt(T.k[1][s >> 1], lanebase, sel0), one, klut); // token r+8
-          ad2 = imad(prmt(T.k[0][s >> 1], lanebase, sel1), one, klut);
-          ad3 = imad(prmt(T.k[1][s >> 1], lanebase, sel1), one, klut);
-        } else {
-          // the 6-bit pair index lands at bits 8..13 above the lane offset of the aligned table
-          ad0 = lop_and_or(bits_at(T.k[0], 12 * s, 8), 0x3F00u, klb);
-          ad1 = lop_and_or(bits_at(T.k[1], 12 * s, 8), 0x3F00u, klb);
-          ad2 = lop_and_or(bits_at(T.k[0], 12 * s + 6, 8), 0x3F00u, klb);
-          ad3 = lop_and_or(bits_at(T.k[1], 12 * s + 6, 8), 0x3F00u, klb);
-        }
-        uint32_t ah[4], al[4];
-        ah[0] = lds32(ad0);
-        ah[1] = lds32(ad1);
-        ah[2] = lds32(ad2);
-        ah[3] = lds32(ad3);
-        al[0] = lds32(ad0 + 128);
-        al[1] = lds32(ad1 + 128);
-        al[2] = lds32(ad2 + 128);
-        al[3] = lds32(ad3 + 128);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma16816(c1[s % SPL][nt], ah[0], ah[1], ah[2], ah[3], qb[nt][2 * s], qb[nt][2 * s + 1]);
-          mma16816(c2[s % SPL][nt], al[0], al[1], al[2], al[3], qb[nt][2 * s], qb[nt][2 * s + 1]);
-        }
-      }
-
-      // ---- online softmax (log2 domain); lane (r, c) owns head 4 nt + c, tokens r, r+8
-      const float kn0 = f16_bits_to_f32(T.kn[0]);
-      const float kn1 = f16_bits_to_f32(T.kn[1]);
-      const float vn0 = f16_bits_to_f32(T.vn[0]);
-      const float vn1 = f16_bits_to_f32(T.vn[1]);
-      const bool ok0 = t0 + r < a.T_len, ok1 = t0 + r + 8 < a.T_len;
-      uint32_t pk[NT];
-      float alpha[NT];
-      bool rescale = false;
+      // ---- B operands of the score MMA: column n = r of n-tile nt is head g = 4 nt + r/2,
+      //      hi (r even) or residual (r odd); thread c holds coordinates [32c, 32c+32).
+      uint32_t qb[NT][16];
+      float qscale[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float hh0 = c1[0][nt][0], hl0 = c1[0][nt][1], lh0 = c2[0][nt][0];
-        float hh1 = c1[0][nt][2], hl1 = c1[0][nt][3], lh1 = c2[0][nt][2];
-        if (SPL == 2) {
-          hh0 += c1[SPL - 1][nt][0];
-          hl0 += c1[SPL - 1][nt][1];
-          lh0 += c2[SPL - 1][nt][0];
-          hh1 += c1[SPL - 1][nt][2];
-          hl1 += c1[SPL - 1][nt][3];
-          lh1 += c2[SPL - 1][nt][2];
+        const int g = nt * 4 + (r >> 1);
+        if (g < a.G) {
+          const QPrep *p = a.qp + static_cast<size_t>(b) * a.Hq + h * a.G + g;
+          const uint4 *src = reinterpret_cast<const uint4 *>(((r & 1) ? p->lo : p->hi) + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 w = __ldg(src + k);
+            qb[nt][4 * k] = w.x;
+            qb[nt][4 * k + 1] = w.y;
+            qb[nt][4 * k + 2] = w.z;
+            qb[nt][4 * k + 3] = w.w;
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) qb[nt][k] = 0u;
         }
-        const float s0 = ok0 ? kn0 * qscale[nt] * fmaf(hl0 + lh0, kLoInv, hh0) : -INFINITY;
-        const float s1 = ok1 ? kn1 * qscale[nt] * fmaf(hl1 + lh1, kLoInv, hh1) : -INFINITY;
-        float mx = fmaxf(s0, s1);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float mn = fmaxf(m_run[nt], mx);
-        alpha[nt] = exp2f(m_run[nt] - mn);
-        rescale |= mn != m_run[nt];
-        m_run[nt] = mn;
-        const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
-        l_run[nt] = fmaf(l_run[nt], alpha[nt], p0 + p1);
-        pk[nt] = pack_h2(p0 * vn0, p1 * vn1);
+        const int gs = nt * 4 + c; // head of this lane's score columns
+        qscale[nt] = gs < a.G ? __ldg(&a.qp[static_cast<size_t>(b) * a.Hq + h * a.G + gs].inv) * kLog2e
+                              : 0.f;
       }
-      // rescale the value accumulators (lane owns heads 2c, 2c+1) when any max moved
-      if (__any_sync(0xffffffffu, rescale)) {
-        float a0[NT], a1[NT];
+
+      float m_run[NT], l_run[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        m_run[nt] = -INFINITY;
+        l_run[nt] = 0.f;
+      }
+      float o[8][4];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+
+      const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
+      const int tlast = a.T_len - 1;
+      // word offset of this lane's value run within a record (3-bit runs start mid-word for odd r)
+      constexpr int kVWordOff = 0;
+      const int vwo = VB == 2 ? r : (VB == 4 ? 2 * r : (3 * r) >> 1);
+      const int vsh = VB == 3 ? 16 * (r & 1) : kVWordOff;
+      // Lane pointers of the next tile this warp loads; a warp advances 4 tiles (64 tokens).
+      int jl = warp;
+      const int tw0 = (tile0 + warp) * 16;
+      const uint8_t *kp = a.kc + (rec0 + tw0 + r) * KR + 4 * KB * c;
+      const uint8_t *vp = a.vc + (rec0 + tw0 + 2 * c) * VR + 4 * vwo;
+      const uint16_t *knp = a.kn + rec0 + tw0 + r;
+      const uint16_t *vnp = a.vn + rec0 + tw0 + r;
+
+      // L2 prefetch lanes: the 128-byte lines of a tile's key codes, then of its value codes,
+      // then one lane each for its key and value norms.
+      constexpr int KL = 16 * KR / 128, VL = 16 * VR / 128;
+      const int tp0 = tw0 + kPrefetchSteps * kWarps * 16;
+      const char *pfp;
+      size_t pfstep;
+      if (lane < KL) {
+        pfp = reinterpret_cast<const char *>(a.kc + (rec0 + tp0) * KR + 128 * lane);
+        pfstep = 64 * KR;
+      } else if (lane < KL + VL) {
+        pfp = reinterpret_cast<const char *>(a.vc + (rec0 + tp0) * VR + 128 * (lane - KL));
+        pfstep = 64 * VR;
+      } else {
+        pfp = reinterpret_cast<const char *>((lane == KL + VL ? a.kn : a.vn) + rec0 + tp0);
+        pfstep = 64 * 2;
+      }
+      int tpf = tp0;
+
+      auto load_k = [&](uint32_t (&dst)[KB], const uint8_t *p) {
+        if constexpr (KB == 4) {
+          const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
+          dst[0] = q.x;
+          dst[1] = q.y;
+          dst[2] = q.z;
+          dst[3] = q.w;
+        } else {
+#pragma unroll
+          for (int k = 0; k < KB; ++k) dst[k] = __ldcs(reinterpret_cast<const uint32_t *>(p) + k);
+        }
+      };
+      auto load_v = [&](uint32_t (&dst)[TileT::VW], const uint8_t *p) {
+#pragma unroll
+        for (int k = 0; k < TileT::VW; ++k) dst[k] = __ldcs(reinterpret_cast<const uint32_t *>(p) + k);
+      };
+
+      // Full tiles load at fixed offsets from the lane pointers; the ragged last tile of a
+      // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
+      auto load_next = [&](TileT &T) {
+        if (kPrefetchSteps > 0) {
+          if (lane < KL + VL + 2 && tpf + 16 <= a.T_len && tpf < (tile0 + ntiles) * 16)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
+          pfp += pfstep;
+          tpf += kWarps * 16;
+        }
+        const int t0 = (tile0 + jl) * 16;
+        if (t0 + 16 <= a.T_len) {
+          load_k(T.k[0], kp);
+          load_k(T.k[1], kp + 8 * KR);
+          load_v(T.v[0], vp);
+          load_v(T.v[1], vp + VR);
+          load_v(T.v[2], vp + 8 * VR);
+          load_v(T.v[3], vp + 9 * VR);
+          T.kn[0] = __ldcs(knp);
+          T.kn[1] = __ldcs(knp + 8);
+          T.vn[0] = __ldcs(vnp);
+          T.vn[1] = __ldcs(vnp + 8);
+        } else {
+          const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
+          const uint8_t *kb = a.kc + rec0 * KR + 4 * KB * c;
+          load_k(T.k[0], kb + static_cast<size_t>(tr) * KR);
+          load_k(T.k[1], kb + static_cast<size_t>(tr8) * KR);
+          const uint8_t *vb = a.vc + rec0 * VR + 4 * vwo;
+          const int tv = t0 + 2 * c;
+          load_v(T.v[0], vb + static_cast<size_t>(min(tv, tlast)) * VR);
+          load_v(T.v[1], vb + static_cast<size_t>(min(tv + 1, tlast)) * VR);
+          load_v(T.v[2], vb + static_cast<size_t>(min(tv + 8, tlast)) * VR);
+          load_v(T.v[3], vb + static_cast<size_t>(min(tv + 9, tlast)) * VR);
+          T.kn[0] = __ldcs(a.kn + rec0 + tr);
+          T.kn[1] = __ldcs(a.kn + rec0 + tr8);
+          T.vn[0] = __ldcs(a.vn + rec0 + tr);
+          T.vn[1] = __ldcs(a.vn + rec0 + tr8);
+        }
+        kp += 64 * KR;
+        vp += 64 * VR;
+        knp += 64;
+        vnp += 64;
+        jl += kWarps;
+      };
+
+      auto compute = [&](const TileT &T, int t0) {
+        // ---- scores: two MMAs per k-step (centroid hi and residual) per n-tile. k-step s
+        //      takes the lane's coordinate pairs 2s (a0, a1) and 2s + 1 (a2, a3).
+        constexpr int SPL = NT == 1 ? 2 : 1; // independent accumulator chains
+        float c1[SPL][NT][4], c2[SPL][NT][4];
+#pragma unroll
+        for (int u = 0; u < SPL; ++u)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c1[u][nt][e] = c2[u][nt][e] = 0.f;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          uint32_t ad0, ad1, ad2, ad3;
+          if constexpr (KB == 4) {
+            // LUT row (code byte << 8) + lane word; the table base is added on the IMAD pipe
+            const uint32_t sel0 = 0x7604u | (static_cast<uint32_t>((2 * s) & 3) << 4);
+            const uint32_t sel1 = 0x7604u | (static_cast<uint32_t>((2 * s + 1) & 3) << 4);
+            if constexpr (kFixed) {
+              ad0 = prmt(T.k[0][s >> 1], klane, sel0); // token r
+              ad1 = prmt(T.k[1][s >> 1], klane, sel0); // token r+8
+              ad2 = prmt(T.k[0][s >> 1], klane, sel1);
+              ad3 = prmt(T.k[1][s >> 1], klane, sel1);
+            } else {
+              ad0 = imad(prmt(T.k[0][s >> 1], klane, sel0), one, klut); // token r
+              ad1 = imad(prmt(T.k[1][s >> 1], klane, sel0), one, klut); // token r+8
+              ad2 = imad(prmt(T.k[0][s >> 1], klane, sel1), one, klut);
+              ad3 = imad(prmt(T.k[1][s >> 1], klane, sel1), one, klut);
+            }
+          } else {
+            // the 6-bit pair index lands at bits 8..13 above the lane offset of the aligned table
+            ad0 = lop_and_or(bits_at(T.k[0], 12 * s, 8), 0x3F00u, klb);
+            ad1 = lop_and_or(bits_at(T.k[1], 12 * s, 8), 0x3F00u, klb);
+            ad2 = lop_and_or(bits_at(T.k[0], 12 * s + 6, 8), 0x3F00u, klb);
+            ad3 = lop_and_or(bits_at(T.k[1], 12 * s + 6, 8), 0x3F00u, klb);
+          }
+          uint32_t ah[4], al[4];
+          if constexpr (KB == 4 && kFixed) {
+            ah[0] = lds32_off<kFixedBase>(ad0);
+            ah[1] = lds32_off<kFixedBase>(ad1);
+            ah[2] = lds32_off<kFixedBase>(ad2);
+            ah[3] = lds32_off<kFixedBase>(ad3);
+            al[0] = lds32_off<kFixedBase + 128>(ad0);
+            al[1] = lds32_off<kFixedBase + 128>(ad1);
+            al[2] = lds32_off<kFixedBase + 128>(ad2);
+            al[3] = lds32_off<kFixedBase + 128>(ad3);
+          } else {
+            ah[0] = lds32(ad0);
+            ah[1] = lds32(ad1);
+            ah[2] = lds32(ad2);
+            ah[3] = lds32(ad3);
+            al[0] = lds32(ad0 + 128);
+            al[1] = lds32(ad1 + 128);
+            al[2] = lds32(ad2 + 128);
+            al[3] = lds32(ad3 + 128);
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma16816(c1[s % SPL][nt], ah[0], ah[1], ah[2], ah[3], qb[nt][2 * s], qb[nt][2 * s + 1]);
+            mma16816(c2[s % SPL][nt], al[0], al[1], al[2], al[3], qb[nt][2 * s], qb[nt][2 * s + 1]);
+          }
+        }
+
+        // ---- online softmax (log2 domain); lane (r, c) owns head 4 nt + c, tokens r, r+8
+        const float kn0 = f16_bits_to_f32(T.kn[0]);
+        const float kn1 = f16_bits_to_f32(T.kn[1]);
+        const float vn0 = f16_bits_to_f32(T.vn[0]);
+        const float vn1 = f16_bits_to_f32(T.vn[1]);
+        const bool ok0 = t0 + r < a.T_len, ok1 = t0 + r + 8 < a.T_len;
+        uint32_t pk[NT];
+        float alpha[NT];
+        bool rescale = false;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          a0[nt] = __shfl_sync(0xffffffffu, alpha[nt], (2 * c) & 3);
-          a1[nt] = __shfl_sync(0xffffffffu, alpha[nt], (2 * c + 1) & 3);
-        }
-        const float al0 = NT == 2 && c >= 2 ? a0[NT - 1] : a0[0];
-        const float al1 = NT == 2 && c >= 2 ? a1[NT - 1] : a1[0];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          o[m][0] *= al0;
-          o[m][1] *= al1;
-          o[m][2] *= al0;
-          o[m][3] *= al1;
-        }
-      }
-
-      // ---- P'^T as the B operand: lane (r, c) needs head g = r at tokens 2c, 2c+1, 2c+8, 2c+9
-      const int src0 = 8 * c + (r & 3);
-      uint32_t x0 = __shfl_sync(0xffffffffu, pk[0], src0);
-      uint32_t x1 = __shfl_sync(0xffffffffu, pk[0], src0 + 4);
-      if (NT == 2) {
-        const uint32_t y0 = __shfl_sync(0xffffffffu, pk[NT - 1], src0);
-        const uint32_t y1 = __shfl_sync(0xffffffffu, pk[NT - 1], src0 + 4);
-        if (r >= 4) {
-          x0 = y0;
-          x1 = y1;
-        }
-      }
-      if (r >= a.G) x0 = x1 = 0u;
-      const uint32_t pb0 = prmt(x0, x1, 0x5410u); // tokens 2c, 2c+1
-      const uint32_t pb1 = prmt(x0, x1, 0x7632u); // tokens 2c+8, 2c+9
-
-      // ---- values. m-tile m covers the lane's run coordinates 2m (rows r) and 2m + 1
-      //      (rows r+8); operand quad (a0, a1, a2, a3) = (2m, 2m+1) x tokens (2c, 2c+1) then
-      //      (2c+8, 2c+9).
-      if constexpr (VB == 2) {
-        // pair-of-token PRMT lookups into a 4-entry fp16 table held in two registers
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t xsel = half ? 0x7362u : 0x5140u;
-          const uint32_t xa = prmt(T.v[0][0], T.v[1][0], xsel); // tokens 2c, 2c+1: codes 8half..+7
-          const uint32_t xb = prmt(T.v[2][0], T.v[3][0], xsel); // tokens 2c+8, 2c+9
-          uint32_t aq[4][4];
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t ya = (xa >> (2 * kk)) & 0x03030303u;
-            const uint32_t yb = (xb >> (2 * kk)) & 0x03030303u;
-            const uint32_t za = imad(ya, 0x22u, 0x10101010u);
-            const uint32_t zb = imad(yb, 0x22u, 0x10101010u);
-            aq[kk >> 1][kk & 1] = prmt(vt0, vt1, za);
-            aq[kk >> 1][2 + (kk & 1)] = prmt(vt0, vt1, zb);
-            aq[2 + (kk >> 1)][kk & 1] = prmt(vt0, vt1, za >> 16);
-            aq[2 + (kk >> 1)][2 + (kk & 1)] = prmt(vt0, vt1, zb >> 16);
+          float hh0 = c1[0][nt][0], hl0 = c1[0][nt][1], lh0 = c2[0][nt][0];
+          float hh1 = c1[0][nt][2], hl1 = c1[0][nt][3], lh1 = c2[0][nt][2];
+          if (SPL == 2) {
+            hh0 += c1[SPL - 1][nt][0];
+            hl0 += c1[SPL - 1][nt][1];
+            lh0 += c2[SPL - 1][nt][0];
+            hh1 += c1[SPL - 1][nt][2];
+            hl1 += c1[SPL - 1][nt][3];
+            lh1 += c2[SPL - 1][nt][2];
           }
-#pragma unroll
-          for (int mm = 0; mm < 4; ++mm)
-            mma16816(o[4 * half + mm], aq[mm][0], aq[mm][1], aq[mm][2], aq[mm][3], pb0, pb1);
+          const float s0 = ok0 ? kn0 * qscale[nt] * fmaf(hl0 + lh0, kLoInv, hh0) : -INFINITY;
+          const float s1 = ok1 ? kn1 * qscale[nt] * fmaf(hl1 + lh1, kLoInv, hh1) : -INFINITY;
+          float mx = fmaxf(s0, s1);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float mn = fmaxf(m_run[nt], mx);
+          alpha[nt] = exp2f(m_run[nt] - mn);
+          rescale |= mn != m_run[nt];
+          m_run[nt] = mn;
+          const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
+          l_run[nt] = fmaf(l_run[nt], alpha[nt], p0 + p1);
+          pk[nt] = pack_h2(p0 * vn0, p1 * vn1);
         }
-      } else {
-        // each operand register is one lane-replicated table word indexed by the two tokens'
-        // codes at that coordinate
-        uint32_t run[4][2];
+        // rescale the value accumulators (lane owns heads 2c, 2c+1) when any max moved
+        if (__any_sync(0xffffffffu, rescale)) {
+          float a0[NT], a1[NT];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          if constexpr (VB == 3) {
-            run[t][0] = __funnelshift_r(T.v[t][0], T.v[t][1], vsh);
-            run[t][1] = T.v[t][1] >> vsh;
-          } else {
-            run[t][0] = T.v[t][0];
-            run[t][1] = T.v[t][1];
+          for (int nt = 0; nt < NT; ++nt) {
+            a0[nt] = __shfl_sync(0xffffffffu, alpha[nt], (2 * c) & 3);
+            a1[nt] = __shfl_sync(0xffffffffu, alpha[nt], (2 * c + 1) & 3);
+          }
+          const float al0 = NT == 2 && c >= 2 ? a0[NT - 1] : a0[0];
+          const float al1 = NT == 2 && c >= 2 ? a1[NT - 1] : a1[0];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            o[m][0] *= al0;
+            o[m][1] *= al1;
+            o[m][2] *= al0;
+            o[m][3] *= al1;
           }
         }
-        constexpr uint32_t MA = ((1u << VB) - 1u) << 7, MB = MA << VB;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          uint32_t q[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 2 * m + (e & 1), tp = e >> 1;
-            const uint32_t ta = bits_at(run[2 * tp], VB * i, 7);
-            const uint32_t tb = bits_at(run[2 * tp + 1], VB * i, 7 + VB);
-            q[e] = lds32(lop_and_or(tb, MB, lop_and_or(ta, MA, vlb)));
-          }
-          mma16816(o[m], q[0], q[1], q[2], q[3], pb0, pb1);
-        }
-      }
-    };
 
-    // Two tile buffers in turn: the next tile loads while the current one computes.
-    TileT ta, tb;
-    int jt = warp;
-    if (jl < ntiles) load_next(ta);
-    while (jt < ntiles) {
-      if (jl < ntiles) load_next(tb);
-      compute(ta, (tile0 + jt) * 16);
-      jt += kWarps;
-      if (jt >= ntiles) break;
+        // ---- P'^T as the B operand: lane (r, c) needs head g = r at tokens 2c, 2c+1, 2c+8, 2c+9
+        const int src0 = 8 * c + (r & 3);
+        uint32_t x0 = __shfl_sync(0xffffffffu, pk[0], src0);
+        uint32_t x1 = __shfl_sync(0xffffffffu, pk[0], src0 + 4);
+        if (NT == 2) {
+          const uint32_t y0 = __shfl_sync(0xffffffffu, pk[NT - 1], src0);
+          const uint32_t y1 = __shfl_sync(0xffffffffu, pk[NT - 1], src0 + 4);
+          if (r >= 4) {
+            x0 = y0;
+            x1 = y1;
+          }
+        }
+        if (r >= a.G) x0 = x1 = 0u;
+        const uint32_t pb0 = prmt(x0, x1, 0x5410u); // tokens 2c, 2c+1
+        const uint32_t pb1 = prmt(x0, x1, 0x7632u); // tokens 2c+8, 2c+9
+
+        // ---- values. m-tile m covers the lane's run coordinates 2m (rows r) and 2m + 1
+        //      (rows r+8); operand quad (a0, a1, a2, a3) = (2m, 2m+1) x tokens (2c, 2c+1) then
+        //      (2c+8, 2c+9).
+        if constexpr (VB == 2) {
+          // pair-of-token PRMT lookups into a 4-entry fp16 table held in two registers
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t xsel = half ? 0x7362u : 0x5140u;
+            const uint32_t xa = prmt(T.v[0][0], T.v[1][0], xsel); // tokens 2c, 2c+1: codes 8half..+7
+            const uint32_t xb = prmt(T.v[2][0], T.v[3][0], xsel); // tokens 2c+8, 2c+9
+            uint32_t aq[4][4];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t ya = (xa >> (2 * kk)) & 0x03030303u;
+              const uint32_t yb = (xb >> (2 * kk)) & 0x03030303u;
+              const uint32_t za = imad(ya, 0x22u, 0x10101010u);
+              const uint32_t zb = imad(yb, 0x22u, 0x10101010u);
+              aq[kk >> 1][kk & 1] = prmt(vt0, vt1, za);
+              aq[kk >> 1][2 + (kk & 1)] = prmt(vt0, vt1, zb);
+              aq[2 + (kk >> 1)][kk & 1] = prmt(vt0, vt1, za >> 16);
+              aq[2 + (kk >> 1)][2 + (kk & 1)] = prmt(vt0, vt1, zb >> 16);
+            }
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm)
+              mma16816(o[4 * half + mm], aq[mm][0], aq[mm][1], aq[mm][2], aq[mm][3], pb0, pb1);
+          }
+        } else {
+          // each operand register is one lane-replicated table word indexed by the two tokens'
+          // codes at that coordinate
+          uint32_t run[4][2];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            if constexpr (VB == 3) {
+              run[t][0] = __funnelshift_r(T.v[t][0], T.v[t][1], vsh);
+              run[t][1] = T.v[t][1] >> vsh;
+            } else {
+              run[t][0] = T.v[t][0];
+              run[t][1] = T.v[t][1];
+            }
+          }
+          constexpr uint32_t MA = ((1u << VB) - 1u) << 7, MB = MA << VB;
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            uint32_t q[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 2 * m + (e & 1), tp = e >> 1;
+              const uint32_t ta = bits_at(run[2 * tp], VB * i, 7);
+              const uint32_t tb = bits_at(run[2 * tp + 1], VB * i, 7 + VB);
+              q[e] = lds32(lop_and_or(tb, MB, lop_and_or(ta, MA, vlb)));
+            }
+            mma16816(o[m], q[0], q[1], q[2], q[3], pb0, pb1);
+          }
+        }
+      };
+
+      // Two tile buffers in turn: the next tile loads while the current one computes.
+      TileT ta, tb;
+      int jt = warp;
       if (jl < ntiles) load_next(ta);
-      compute(tb, (tile0 + jt) * 16);
-      jt += kWarps;
-    }
+      while (jt < ntiles) {
+        if (jl < ntiles) load_next(tb);
+        compute(ta, (tile0 + jt) * 16);
+        jt += kWarps;
+        if (jt >= ntiles) break;
+        if (jl < ntiles) load_next(ta);
+        compute(tb, (tile0 + jt) * 16);
+        jt += kWarps;
+      }
 
-    // ---- merge the warps: common max per head, rescale, accumulate in shared memory
+      // ---- merge the warps: common max per head, rescale, accumulate in shared memory
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float l = l_run[nt];
-      l += __shfl_xor_sync(0xffffffffu, l, 4);
-      l += __shfl_xor_sync(0xffffffffu, l, 8);
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
-      l_run[nt] = l;
-      if (r == 0) mst[warp * 8 + nt * 4 + c] = m_run[nt];
-    }
-    for (int idx = tid; idx < a.G * kD; idx += kThreads) obuf[idx] = 0.f;
-    if (tid < 8) lsum[tid] = 0.f;
-    __syncthreads();
-    if (tid < 8) {
-      float M = -INFINITY;
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mst[w * 8 + tid]);
-      gmx[tid] = M;
-    }
-    __syncthreads();
+      for (int nt = 0; nt < NT; ++nt) {
+        float l = l_run[nt];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        l_run[nt] = l;
+        if (r == 0) mst[warp * 8 + nt * 4 + c] = m_run[nt];
+      }
+      for (int idx = tid; idx < a.G * kD; idx += kThreads) obuf[idx] = 0.f;
+      if (tid < 8) lsum[tid] = 0.f;
+      __syncthreads();
+      if (tid < 8) {
+        float M = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mst[w * 8 + tid]);
+        gmx[tid] = M;
+      }
+      __syncthreads();
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int g = nt * 4 + c;
-      if (r == 0 && g < a.G) atomicAdd(&lsum[g], l_run[nt] * exp2f(m_run[nt] - gmx[g]));
-    }
-    {
-      const int g0 = 2 * c, g1 = 2 * c + 1;
-      const float f0 = g0 < a.G ? exp2f(mst[warp * 8 + g0] - gmx[g0]) : 0.f;
-      const float f1 = g1 < a.G ? exp2f(mst[warp * 8 + g1] - gmx[g1]) : 0.f;
+      for (int nt = 0; nt < NT; ++nt) {
+        const int g = nt * 4 + c;
+        if (r == 0 && g < a.G) atomicAdd(&lsum[g], l_run[nt] * exp2f(m_run[nt] - gmx[g]));
+      }
+      {
+        const int g0 = 2 * c, g1 = 2 * c + 1;
+        const float f0 = g0 < a.G ? exp2f(mst[warp * 8 + g0] - gmx[g0]) : 0.f;
+        const float f1 = g1 < a.G ? exp2f(mst[warp * 8 + g1] - gmx[g1]) : 0.f;
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int i0 = 16 * r + 2 * m;
-        if (g0 < a.G) {
-          atomicAdd(&obuf[g0 * kD + i0], o[m][0] * f0);
-          atomicAdd(&obuf[g0 * kD + i0 + 1], o[m][2] * f0);
-        }
-        if (g1 < a.G) {
-          atomicAdd(&obuf[g1 * kD + i0], o[m][1] * f1);
-          atomicAdd(&obuf[g1 * kD + i0 + 1], o[m][3] * f1);
+        for (int m = 0; m < 8; ++m) {
+          const int i0 = 16 * r + 2 * m;
+          if (g0 < a.G) {
+            atomicAdd(&obuf[g0 * kD + i0], o[m][0] * f0);
+            atomicAdd(&obuf[g0 * kD + i0 + 1], o[m][2] * f0);
+          }
+          if (g1 < a.G) {
+            atomicAdd(&obuf[g1 * kD + i0], o[m][1] * f1);
+            atomicAdd(&obuf[g1 * kD + i0 + 1], o[m][3] * f1);
+          }
         }
       }
+      __syncthreads();
+      float *dst = a.part + (static_cast<size_t>(blockIdx.x) * a.slots + slot) * a.G * a.stride;
+      for (int idx = tid; idx < a.G * kD; idx += kThreads) {
+        const int g = idx / kD, i = idx - g * kD;
+        dst[static_cast<size_t>(g) * a.stride + 2 + i] = obuf[idx];
+      }
+      if (tid < a.G) {
+        dst[static_cast<size_t>(tid) * a.stride] = gmx[tid];
+        dst[static_cast<size_t>(tid) * a.stride + 1] = lsum[tid];
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    float *dst = a.part + (static_cast<size_t>(blockIdx.x) * a.slots + slot) * a.G * a.stride;
-    for (int idx = tid; idx < a.G * kD; idx += kThreads) {
-      const int g = idx / kD, i = idx - g * kD;
-      dst[static_cast<size_t>(g) * a.stride + 2 + i] = obuf[idx];
-    }
-    if (tid < a.G) {
-      dst[static_cast<size_t>(tid) * a.stride] = gmx[tid];
-      dst[static_cast<size_t>(tid) * a.stride + 1] = lsum[tid];
-    }
-    __syncthreads();
-  }
+  };
+  if (KB == 4 && klut == kFixedBase)
+    run(std::true_type{});
+  else
+    run(std::false_type{});
 }
 
 // Merge the partial records of one (b, q-head) (log2-domain maxima), apply the inverse
