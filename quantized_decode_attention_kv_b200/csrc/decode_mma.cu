@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
   // computation; otherwise an IMAD adds the base.
   auto run = [&](auto fixed_tag) {
     constexpr bool kFixed = decltype(fixed_tag)::value;
-    const uint32_t klane = lanebase;
+    [[maybe_unused]] const uint32_t klane = lanebase;
     const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
     const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
     int slot = 0;
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
       // word offset of this lane's value run within a record (3-bit runs start mid-word for odd r)
       constexpr int kVWordOff = 0;
       const int vwo = VB == 2 ? r : (VB == 4 ? 2 * r : (3 * r) >> 1);
-      const int vsh = VB == 3 ? 16 * (r & 1) : kVWordOff;
+      [[maybe_unused]] const int vsh = VB == 3 ? 16 * (r & 1) : kVWordOff;
       // Lane pointers of the next tile this warp loads; a warp advances 4 tiles (64 tokens).
       int jl = warp;
       const int tw0 = (tile0 + warp) * 16;

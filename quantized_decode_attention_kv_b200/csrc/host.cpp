@@ -304,23 +304,33 @@ int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
     q.seed = cache->seed;
     for (int k = 0; k < 4; ++k) q.sign_words[k] = splitmix64_at(cache->seed, static_cast<uint64_t>(k));
   }
-  // 16-bit MSE tensors take the streaming kernel (both in one launch); the rest, the
-  // per-vector kernel.
-  const tq::QuantArgs *fast[2] = {nullptr, nullptr};
+  // 16-bit MSE tensors take the streaming kernel, 16-bit d=64 TurboQuant_prod tensors the
+  // tensor-core sketch kernel (each with K and V in one launch); the rest, the per-vector
+  // kernel.
+  const tq::QuantArgs *fast[2] = {nullptr, nullptr}, *prod[2] = {nullptr, nullptr};
   for (int which = 0; which < 2; ++which) {
     const void *x = which == 0 ? K : V;
-    if (x && tq::quantize_fast_supported(a[which])) fast[which] = &a[which];
+    if (!x) continue;
+    if (tq::quantize_fast_supported(a[which])) fast[which] = &a[which];
+    else if (tq::quantize_prod_supported(a[which])) prod[which] = &a[which];
   }
-  if (fast[0] || fast[1]) {
+  if (fast[0] || fast[1] || prod[0] || prod[1]) {
     const int sms = sm_count();
     if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
-    st = cuda_status(tq::launch_quantize_fast(fast[0], fast[1], sms, static_cast<cudaStream_t>(stream)),
-                     "quantize launch");
-    if (st) return st;
+    if (fast[0] || fast[1]) {
+      st = cuda_status(tq::launch_quantize_fast(fast[0], fast[1], sms, static_cast<cudaStream_t>(stream)),
+                       "quantize launch");
+      if (st) return st;
+    }
+    if (prod[0] || prod[1]) {
+      st = cuda_status(tq::launch_quantize_prod(prod[0], prod[1], sms, static_cast<cudaStream_t>(stream)),
+                       "quantize launch");
+      if (st) return st;
+    }
   }
   for (int which = 0; which < 2; ++which) {
     const void *x = which == 0 ? K : V;
-    if (!x || fast[which]) continue;
+    if (!x || fast[which] || prod[which]) continue;
     st = cuda_status(tq::launch_quantize(a[which], static_cast<cudaStream_t>(stream)), "quantize launch");
     if (st) return st;
   }
@@ -449,7 +459,7 @@ int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,
   if (Hq < 1 || Hq % cache->Hkv || Hq > 65535 || T_len < 1 || T_len > cache->T_cap)
     return fail(TQ_ERR_INVALID_ARG, "bad Hq=%d or T_len=%d", Hq, T_len);
   int nq = 0;
-  bool any_fast = false;
+  bool any_fast = false, any_prod = false;
   for (int which = 0; which < 2 && T > 0; ++which) {
     tq::QuantArgs q{};
     st = resolve_tensor(*cache, which, &q.t);
@@ -460,9 +470,10 @@ int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,
     q.T = T;
     q.d = cache->d;
     if (tq::quantize_fast_supported(q)) any_fast = true;
+    else if (tq::quantize_prod_supported(q)) any_prod = true;
     else ++nq;
   }
-  if (quantize_launches) *quantize_launches = nq + (any_fast ? 1 : 0);
+  if (quantize_launches) *quantize_launches = nq + (any_fast ? 1 : 0) + (any_prod ? 1 : 0);
   if (decode_launches) *decode_launches = fast_path(*cache, Hq) != 0 ? 3 : 2; // (query prep,) split-K, combine
   return TQ_OK;
 }

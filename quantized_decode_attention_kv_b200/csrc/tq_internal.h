@@ -94,6 +94,12 @@ cudaError_t launch_quantize(const QuantArgs &a, cudaStream_t s);
 bool quantize_fast_supported(const QuantArgs &a);
 cudaError_t launch_quantize_fast(const QuantArgs *k, const QuantArgs *v, int sm_count,
                                  cudaStream_t s);
+
+// TurboQuant_prod quantiser with the QJL sketch on the tensor cores (quantize_prod.cu):
+// head_dim 64, 64 sketch rows, 1- or 2-bit records, bf16/f16 input; K and V in one launch.
+bool quantize_prod_supported(const QuantArgs &a);
+cudaError_t launch_quantize_prod(const QuantArgs *k, const QuantArgs *v, int sm_count,
+                                 cudaStream_t s);
 cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s);

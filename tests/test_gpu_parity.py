@@ -39,6 +39,7 @@ QUANT_CASES = [
     (128, (1, O.MSE), (4, O.MSE), 0),
     (64, (2, O.PROD), (2, O.PROD), 64),
     (64, (1, O.PROD), (3, O.PROD), 32),
+    (64, (1, O.PROD), (2, O.PROD), 64),
     (16, (3, O.MSE), (1, O.MSE), 0),
     (16, (2, O.PROD), (4, O.PROD), 8),
     (32, (4, O.MSE), (2, O.PROD), 0),
