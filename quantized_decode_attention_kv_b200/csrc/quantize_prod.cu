@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kRWarps * 32) quantize_prod_kernel(const ProdQ
   for (long long gi = static_cast<long long>(blockIdx.x) * kRWarps + warp; gi < total;
        gi += static_cast<long long>(gridDim.x) * kRWarps) {
     const int ti = gi < a.groups[0] ? 0 : 1;
-    const ProdQuantTensor &t = a.t[ti];
+    const ProdQuantTensor t = a.t[ti]; // one copy of the tensor's fields per group
     const unsigned v0 = static_cast<unsigned>((gi - (ti ? a.groups[0] : 0)) * 16);
     const unsigned va = v0 + r, vb = v0 + r + 8;
     const unsigned la = min(va, t.nvec - 1), lb = min(vb, t.nvec - 1);
@@ -128,14 +128,15 @@ __global__ void __launch_bounds__(kRWarps * 32) quantize_prod_kernel(const ProdQ
           }
 #pragma unroll
       for (int m = 1; m < 4; m <<= 1) {
-        const bool upper = (c & m) != 0;
+        const float sgnm = (c & m) ? -1.0f : 1.0f; // upper lane keeps partner - own
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float o = __shfl_xor_sync(0xffffffffu, x[u][e], m);
-          x[u][e] = upper ? o - x[u][e] : x[u][e] + o;
+          x[u][e] = fmaf(x[u][e], sgnm, o);
         }
       }
     }
+    const bool wb1 = t.wbits == 1;
     // ---- z, 1-bit codes, unit-domain residual r = (z - c[code]) / sqrt(d) and its norm
     uint32_t code_bits[2] = {0u, 0u}; // bit e: code of coordinate 16 c + e
     float nrm[2], gam[2];
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(kRWarps * 32) quantize_prod_kernel(const ProdQ
       for (int e = 0; e < 16; ++e) {
         const float z = x[u][e] * inv;
         float chat = 0.f;
-        if (t.wbits == 1) {
+        if (wb1) {
           const bool up = z > 0.f;
           code_bits[u] |= (up ? 1u : 0u) << e;
           chat = up ? t.c1 : -t.c1;
@@ -180,8 +181,9 @@ __global__ void __launch_bounds__(kRWarps * 32) quantize_prod_kernel(const ProdQ
       const int j = 8 * nt + 2 * c, wi = j >> 5, sh = j & 31;
       const float p00 = fmaf(m1[0], kRLoInv, m0[0]), p01 = fmaf(m1[1], kRLoInv, m0[1]);
       const float p10 = fmaf(m1[2], kRLoInv, m0[2]), p11 = fmaf(m1[3], kRLoInv, m0[3]);
-      sg[0][wi] |= ((p00 < 0.f ? 1u : 0u) | (p01 < 0.f ? 2u : 0u)) << sh;
-      sg[1][wi] |= ((p10 < 0.f ? 1u : 0u) | (p11 < 0.f ? 2u : 0u)) << sh;
+      // sign bit = (p < 0): the accumulators start at +0, so an exact zero is +0 (bit 0)
+      sg[0][wi] |= ((__float_as_uint(p00) >> 31) | ((__float_as_uint(p01) >> 31) << 1)) << sh;
+      sg[1][wi] |= ((__float_as_uint(p10) >> 31) | ((__float_as_uint(p11) >> 31) << 1)) << sh;
     }
     // gather the four lanes of the row: signs, codes
 #pragma unroll
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kRWarps * 32) quantize_prod_kernel(const ProdQ
         const unsigned tt = v - bh * static_cast<unsigned>(t.T);
         const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
         reinterpret_cast<uint2 *>(t.signs)[rec] = make_uint2(sg[u][0], sg[u][1]);
-        if (t.wbits == 1) reinterpret_cast<uint2 *>(t.codes)[rec] = make_uint2(code_bits[u], cw1[u]);
+        if (wb1) reinterpret_cast<uint2 *>(t.codes)[rec] = make_uint2(code_bits[u], cw1[u]);
         t.norm[rec] = f32_to_f16_bits(nrm[u]);
         t.rnorm[rec] = f32_to_f16_bits(gam[u]);
       }
