@@ -33,8 +33,12 @@ namespace tq {
 namespace {
 using namespace mma_ops;
 
-constexpr int kWarps = 4;
+#ifndef TQ_MSE_WARPS
+#define TQ_MSE_WARPS 4
+#endif
+constexpr int kWarps = TQ_MSE_WARPS; // warps per CTA of the MSE kernel
 constexpr int kThreads = kWarps * 32;
+constexpr int kStep = kWarps * 16;  // tokens a warp advances per step
 constexpr int kD = 128;
 constexpr float kLoScale = 4096.0f; // residual scaling 2^12 (keeps residuals normal in fp16)
 constexpr float kLoInv = 1.0f / 4096.0f;
@@ -50,10 +54,14 @@ constexpr int kPrefetchSteps = TQ_DECODE_PREFETCH;
 // 1 KB below it is reserved by the hardware); the kernel checks it before relying on it.
 constexpr uint32_t kFixedBase = 1024;
 
+#ifndef TQ_MSE_CTAS
+#define TQ_MSE_CTAS 3
+#endif
+
 template <uint32_t OFF>
-__device__ __forceinline__ uint32_t lds32_off(uint32_t smem_addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(smem_addr), "n"(OFF));
+__device__ __forceinline__ uint2 lds64_off(uint32_t smem_addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr), "n"(OFF));
   return v;
 }
 
@@ -84,7 +92,7 @@ struct Lut {
   static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : 0;
   static constexpr int vBytes = vRows * 128;
   static constexpr int vAlign = VB >= 3 ? vBytes : 16;
-  static constexpr int kMergeBytes = (4 * 8 + 16 + 8 * 128) * 4;
+  static constexpr int kMergeBytes = (kWarps * 8 + 16 + 8 * 128) * 4;
   static constexpr int kSmem = kBytes + kAlign - 16 + vBytes + vAlign - 16 + kMergeBytes;
 };
 
@@ -178,7 +186,7 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32
 }
 
 template <int KB, int VB, int NT>
-__global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs a) {
+__global__ void __launch_bounds__(kThreads, TQ_MSE_CTAS) decode_mse_kernel(const FastArgs a) {
   using L = Lut<KB, VB>;
   using TileT = Tile<KB, VB>;
   constexpr int KR = KB * 16, VR = VB * 16; // record bytes
@@ -202,8 +210,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
       const int e = idx >> 5, l = idx & 31;
       const float c0 = a.kcent[e & (KB == 4 ? 15 : 7)], c1 = a.kcent[KB == 4 ? e >> 4 : e >> 3];
       const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
-      kw[e * 64 + l] = pack_h2(c0, c1);
-      kw[e * 64 + 32 + l] = pack_h2((c0 - h0) * kLoScale, (c1 - h1) * kLoScale);
+      kw[e * 64 + 2 * l] = pack_h2(c0, c1);
+      kw[e * 64 + 2 * l + 1] = pack_h2((c0 - h0) * kLoScale, (c1 - h1) * kLoScale);
     }
     uint32_t *vw = reinterpret_cast<uint32_t *>(vl_p);
     for (int idx = tid; idx < L::vRows * 32; idx += kThreads) {
@@ -214,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
   const uint32_t vt0 = pack_h2(a.vcent[0], a.vcent[1]);
   const uint32_t vt1 = pack_h2(a.vcent[2], a.vcent[3]);
   const uint32_t lanebase = static_cast<uint32_t>(lane) << 2;
-  const uint32_t klb = klut | lanebase; // 3-bit keys: table base with the lane offset
+  const uint32_t klane8 = static_cast<uint32_t>(lane) << 3; // lane's 8-byte {hi, lo} entry
+  const uint32_t klb = klut | klane8;                          // 3-bit keys: base + lane offset
   const uint32_t vlb = vlut | lanebase;
   const uint32_t one = a.one; // 1, opaque to the compiler so the add stays an IMAD
   __syncthreads();
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
   // computation; otherwise an IMAD adds the base.
   auto run = [&](auto fixed_tag) {
     constexpr bool kFixed = decltype(fixed_tag)::value;
-    [[maybe_unused]] const uint32_t klane = lanebase;
+    const uint32_t klane = klane8;
     const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
     const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
     int slot = 0;
@@ -282,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
       constexpr int kVWordOff = 0;
       const int vwo = VB == 2 ? r : (VB == 4 ? 2 * r : (3 * r) >> 1);
       [[maybe_unused]] const int vsh = VB == 3 ? 16 * (r & 1) : kVWordOff;
-      // Lane pointers of the next tile this warp loads; a warp advances 4 tiles (64 tokens).
+      // Lane pointers of the next tile this warp loads; a warp advances kWarps tiles per step.
       int jl = warp;
       const int tw0 = (tile0 + warp) * 16;
       const uint8_t *kp = a.kc + (rec0 + tw0 + r) * KR + 4 * KB * c;
@@ -298,13 +307,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
       size_t pfstep;
       if (lane < KL) {
         pfp = reinterpret_cast<const char *>(a.kc + (rec0 + tp0) * KR + 128 * lane);
-        pfstep = 64 * KR;
+        pfstep = kStep * KR;
       } else if (lane < KL + VL) {
         pfp = reinterpret_cast<const char *>(a.vc + (rec0 + tp0) * VR + 128 * (lane - KL));
-        pfstep = 64 * VR;
+        pfstep = kStep * VR;
       } else {
         pfp = reinterpret_cast<const char *>((lane == KL + VL ? a.kn : a.vn) + rec0 + tp0);
-        pfstep = 64 * 2;
+        pfstep = kStep * 2;
       }
       int tpf = tp0;
 
@@ -362,29 +371,29 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
           T.vn[0] = __ldcs(a.vn + rec0 + tr);
           T.vn[1] = __ldcs(a.vn + rec0 + tr8);
         }
-        kp += 64 * KR;
-        vp += 64 * VR;
-        knp += 64;
-        vnp += 64;
+        kp += kStep * KR;
+        vp += kStep * VR;
+        knp += kStep;
+        vnp += kStep;
         jl += kWarps;
       };
 
       auto compute = [&](const TileT &T, int t0) {
-        // ---- scores: two MMAs per k-step (centroid hi and residual) per n-tile. k-step s
-        //      takes the lane's coordinate pairs 2s (a0, a1) and 2s + 1 (a2, a3).
-        constexpr int SPL = NT == 1 ? 2 : 1; // independent accumulator chains
-        float c1[SPL][NT][4], c2[SPL][NT][4];
+        // ---- scores. MMA A takes tokens r (its rows 0-7 hold the centroid hi, rows 8-15 the
+        //      residual lo of the same tokens), MMA B tokens r + 8, so one 64-bit table load
+        //      {hi, lo} fills an adjacent pair of A registers. k-step s takes the lane's
+        //      coordinate pairs 2s (a0, a1) and 2s + 1 (a2, a3).
+        float cA[NT][4], cB[NT][4];
 #pragma unroll
-        for (int u = 0; u < SPL; ++u)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) c1[u][nt][e] = c2[u][nt][e] = 0.f;
+          for (int e = 0; e < 4; ++e) cA[nt][e] = cB[nt][e] = 0.f;
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           uint32_t ad0, ad1, ad2, ad3;
           if constexpr (KB == 4) {
-            // LUT row (code byte << 8) + lane word; the table base is added on the IMAD pipe
+            // table row (code byte << 8) + the lane's 8-byte entry; the base is an immediate
+            // offset of the load or is added on the IMAD pipe
             const uint32_t sel0 = 0x7604u | (static_cast<uint32_t>((2 * s) & 3) << 4);
             const uint32_t sel1 = 0x7604u | (static_cast<uint32_t>((2 * s + 1) & 3) << 4);
             if constexpr (kFixed) {
@@ -405,30 +414,22 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
             ad2 = lop_and_or(bits_at(T.k[0], 12 * s + 6, 8), 0x3F00u, klb);
             ad3 = lop_and_or(bits_at(T.k[1], 12 * s + 6, 8), 0x3F00u, klb);
           }
-          uint32_t ah[4], al[4];
+          uint2 e0, e1, e2, e3;
           if constexpr (KB == 4 && kFixed) {
-            ah[0] = lds32_off<kFixedBase>(ad0);
-            ah[1] = lds32_off<kFixedBase>(ad1);
-            ah[2] = lds32_off<kFixedBase>(ad2);
-            ah[3] = lds32_off<kFixedBase>(ad3);
-            al[0] = lds32_off<kFixedBase + 128>(ad0);
-            al[1] = lds32_off<kFixedBase + 128>(ad1);
-            al[2] = lds32_off<kFixedBase + 128>(ad2);
-            al[3] = lds32_off<kFixedBase + 128>(ad3);
+            e0 = lds64_off<kFixedBase>(ad0);
+            e1 = lds64_off<kFixedBase>(ad1);
+            e2 = lds64_off<kFixedBase>(ad2);
+            e3 = lds64_off<kFixedBase>(ad3);
           } else {
-            ah[0] = lds32(ad0);
-            ah[1] = lds32(ad1);
-            ah[2] = lds32(ad2);
-            ah[3] = lds32(ad3);
-            al[0] = lds32(ad0 + 128);
-            al[1] = lds32(ad1 + 128);
-            al[2] = lds32(ad2 + 128);
-            al[3] = lds32(ad3 + 128);
+            e0 = lds64_off<0>(ad0);
+            e1 = lds64_off<0>(ad1);
+            e2 = lds64_off<0>(ad2);
+            e3 = lds64_off<0>(ad3);
           }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            mma16816(c1[s % SPL][nt], ah[0], ah[1], ah[2], ah[3], qb[nt][2 * s], qb[nt][2 * s + 1]);
-            mma16816(c2[s % SPL][nt], al[0], al[1], al[2], al[3], qb[nt][2 * s], qb[nt][2 * s + 1]);
+            mma16816(cA[nt], e0.x, e0.y, e2.x, e2.y, qb[nt][2 * s], qb[nt][2 * s + 1]);
+            mma16816(cB[nt], e1.x, e1.y, e3.x, e3.y, qb[nt][2 * s], qb[nt][2 * s + 1]);
           }
         }
 
@@ -443,16 +444,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mse_kernel(const FastArgs 
         bool rescale = false;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          float hh0 = c1[0][nt][0], hl0 = c1[0][nt][1], lh0 = c2[0][nt][0];
-          float hh1 = c1[0][nt][2], hl1 = c1[0][nt][3], lh1 = c2[0][nt][2];
-          if (SPL == 2) {
-            hh0 += c1[SPL - 1][nt][0];
-            hl0 += c1[SPL - 1][nt][1];
-            lh0 += c2[SPL - 1][nt][0];
-            hh1 += c1[SPL - 1][nt][2];
-            hl1 += c1[SPL - 1][nt][3];
-            lh1 += c2[SPL - 1][nt][2];
-          }
+          // token r: hi x q_hi, hi x q_lo, lo x q_hi from MMA A; token r + 8 from MMA B
+          const float hh0 = cA[nt][0], hl0 = cA[nt][1], lh0 = cA[nt][2];
+          const float hh1 = cB[nt][0], hl1 = cB[nt][1], lh1 = cB[nt][2];
           const float s0 = ok0 ? kn0 * qscale[nt] * fmaf(hl0 + lh0, kLoInv, hh0) : -INFINITY;
           const float s1 = ok1 ? kn1 * qscale[nt] * fmaf(hl1 + lh1, kLoInv, hh1) : -INFINITY;
           float mx = fmaxf(s0, s1);
@@ -718,7 +712,7 @@ int mse_ctas_per_sm(int kb, int vb) {
   int smem = 0;
   if (kb == 4) smem = vb == 2 ? Lut<4, 2>::kSmem : vb == 3 ? Lut<4, 3>::kSmem : Lut<4, 4>::kSmem;
   else smem = vb == 2 ? Lut<3, 2>::kSmem : vb == 3 ? Lut<3, 3>::kSmem : Lut<3, 4>::kSmem;
-  return std::max(1, std::min(3, kSmemPerSm / (smem + 1024)));
+  return std::max(1, std::min(TQ_MSE_CTAS, kSmemPerSm / (smem + 1024)));
 }
 
 template <int KB, int VB>
