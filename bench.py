@@ -20,7 +20,6 @@ from __future__ import annotations
 import argparse
 import csv
 import dataclasses
-import datetime
 import hashlib
 import io
 import json
@@ -215,29 +214,24 @@ def run_reference(args):
 # ------------------------------------------------------------------ CUDA arm
 def run_ours(args):
     import torch
-    import torch.distributed as dist
 
+    from quantized_decode_attention_kv_b200 import replicas as R
     from quantized_decode_attention_kv_b200 import tq
     from quantized_decode_attention_kv_b200.workloads import WORKLOADS, make_inputs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, local, world = R.env_ranks()
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
-                                device_id=torch.device("cuda", local))
+    R.init("nccl", world, torch.device("cuda", local))
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        R.barrier(world)
 
     w = WORKLOADS[args.workload]
     if args.T:
         w = dataclasses.replace(w, T=args.T)
-    K, V, q = make_inputs(w, device="cuda", layer=rank)
+    K, V, q = make_inputs(w, device="cuda", layer=R.replica_layer(rank))
     cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, w.k_mode, w.v_mode, w.qjl_m,
                        w.qjl_m, seed=w.seed, qjl_seed=w.qjl_seed)
     tq.tq_quantize_kv(K, V, cache)  # prefill the whole context
@@ -267,21 +261,16 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * packed / (ms * 1e-3) / 1e9
+    ms = R.max_over_ranks(e0.elapsed_time(e1) / args.steps, world, device="cuda")
+    value = R.job_throughput(packed, world, ms * 1e-3) / 1e9
     nq, nd = tq.tq_launch_counts(cache, k_new.dtype, 1, w.Hq, w.T)
     launches_per_step = nq + nd
 
     side = {}
     if rank == 0 and not args.no_side:
         side = side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new, packed, stream)
-    if world > 1:
-        barrier()
-        dist.destroy_process_group()
+    barrier()
+    R.finish(world)
     if rank != 0:
         return
     hbm, hbm_src = peaks()
