@@ -572,6 +572,10 @@ cudaError_t run_decode_bf16(const DecodeBf16Args &a, cudaStream_t s) {
 DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm_count, bool bf16,
                        int fast) {
   DecodePlan p{};
+  if (bf16 && bf16_decode_supported(d, Hq / Hkv)) {
+    plan_bf16_mma(B, Hq, Hkv, T_len, sm_count, &p);
+    return p;
+  }
   if (fast == kProdFast && !bf16) {
     plan_prod(B, Hq, Hkv, T_len, sm_count, &p);
     return p;
@@ -608,6 +612,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
 }
 
 cudaError_t launch_decode_bf16(const DecodeBf16Args &a, cudaStream_t s) {
+  if (a.plan.path == 3) return launch_bf16_mma(a, s);
   TQ_DISPATCH_DEC(run_decode_bf16)
 }
 

@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, TQ_MSE_CTAS) decode_mse_kernel(const
   // computation; otherwise an IMAD adds the base.
   auto run = [&](auto fixed_tag) {
     constexpr bool kFixed = decltype(fixed_tag)::value;
-    const uint32_t klane = klane8;
+    [[maybe_unused]] const uint32_t klane = klane8;
     const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
     const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
     int slot = 0;

@@ -52,7 +52,8 @@ struct DequantArgs {
 
 struct DecodePlan {
   int path;      // 0: generic split-K kernel; 1: tensor-core MSE kernel (decode_mma.cu);
-                 // 2: tensor-core PROD kernel (decode_prod.cu)
+                 // 2: tensor-core PROD kernel (decode_prod.cu); 3: tensor-core bf16 kernel
+                 // (decode_bf16.cu)
   int tile;      // tokens per pipeline tile
   int splits;    // context splits per (b, KV head) (path 0)
   int chunk;     // tokens per split (a multiple of tile) (path 0)
@@ -128,5 +129,10 @@ bool prod_decode_supported(int d, int k_mode, int k_bits, int k_m, int v_mode, i
                            int G);
 void plan_prod(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p);
 cudaError_t launch_prod_decode(const DecodeArgs &a, cudaStream_t s);
+
+// Tensor-core bf16 decode (decode_bf16.cu): head_dim 128, 1..8 query heads per KV head.
+bool bf16_decode_supported(int d, int G);
+void plan_bf16_mma(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p);
+cudaError_t launch_bf16_mma(const DecodeBf16Args &a, cudaStream_t s);
 
 } // namespace tq

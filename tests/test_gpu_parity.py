@@ -240,7 +240,9 @@ def test_decode_rejects_small_workspace_and_empty_context():
 
 # ------------------------------------------------------------------ bf16 comparator
 @pytest.mark.parametrize("d,G,Hkv,T_len,T_cap", [(128, 4, 2, 1000, 1024), (64, 1, 3, 129, 140),
-                                                  (256, 8, 1, 300, 300), (16, 2, 2, 1, 4)])
+                                                  (256, 8, 1, 300, 300), (16, 2, 2, 1, 4),
+                                                  (128, 8, 1, 777, 800), (128, 1, 3, 33, 40),
+                                                  (128, 3, 2, 1, 5), (128, 16, 1, 100, 100)])
 def test_bf16_decode_matches_oracle(d, G, Hkv, T_len, T_cap):
     B, Hq = 2, G * Hkv
     K, V = _inputs(B, Hkv, T_cap, d, torch.bfloat16, seed=d + G, outliers=True)
