@@ -73,9 +73,9 @@ def kernel_traffic():
 
 
 def decode_sources_digest() -> str:
-    """sha256 over the decode kernels' sources (the split-K and tensor-core decode files)."""
+    """sha256 over the sources of the bench's dominant kernel (the tensor-core decode)."""
     h = hashlib.sha256()
-    for name in ("decode.cu", "decode_mma.cu"):
+    for name in ("decode_mma.cu", "mma_ops.cuh"):
         with open(os.path.join(ROOT, "quantized_decode_attention_kv_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
