@@ -153,3 +153,46 @@ def test_binding_refuses_host_tensors():
     cache = type("C", (), {})()
     with pytest.raises(tq.TQError):
         tq.tq_quantize_kv(torch.zeros(1, 1, 4, 128), None, cache)
+
+
+def _fake_cache(B, Hkv, T_cap, d, kb, km, vb, vm, m=0):
+    """A tq_cache whose pointers are aligned placeholders: tq_launch_counts inspects shapes and
+    bit-widths only and never touches device memory."""
+    c = tq.tq_cache()
+    c.B, c.Hkv, c.T_cap, c.d, c.seed = B, Hkv, T_cap, d, 0
+    c.kc = tq.tq_qcfg(kb, km, m)
+    c.vc = tq.tq_qcfg(vb, vm, m)
+    for i, f in enumerate(("k_codes", "v_codes", "k_norm", "v_norm", "k_signs", "v_signs",
+                           "k_rnorm", "v_rnorm", "k_qjl", "v_qjl")):
+        setattr(c, f, 0x10000 * (i + 1))
+    return c
+
+
+@pytest.mark.parametrize("cfg,dtype,Hq,want", [
+    # 16-bit MSE write: one streaming launch for K and V; MSE d=128 decode: prep, decode, combine
+    ((16, 8, 32768, 128, 4, O.MSE, 2, O.MSE), 1, 32, (1, 3)),
+    ((4, 8, 1024, 128, 3, O.MSE, 3, O.MSE), 2, 32, (1, 3)),
+    # fp32 input takes the per-vector kernel, one launch per tensor
+    ((1, 1, 1024, 128, 4, O.MSE, 4, O.MSE), 0, 1, (2, 3)),
+    # d = 64 TurboQuant_prod with 64 sketch rows: tensor-core write and decode (G <= 2)
+    ((64, 12, 8192, 64, 2, O.PROD, 2, O.PROD, 64), 1, 12, (1, 3)),
+    ((64, 12, 8192, 64, 2, O.PROD, 2, O.PROD, 64), 1, 48, (1, 2)),
+    # shapes without a tensor-core kernel: per-vector write, split-K decode + combine
+    ((2, 2, 100, 256, 4, O.MSE, 2, O.MSE), 1, 4, (2, 2)),
+    ((2, 2, 100, 128, 4, O.MSE, 2, O.MSE), 1, 2 * 32, (1, 2)),
+])
+def test_launch_counts_follow_the_kernel_selection(cfg, dtype, Hq, want):
+    c = _fake_cache(*cfg)
+    nq, nd = ctypes.c_int(-1), ctypes.c_int(-1)
+    st = tq.lib.tq_launch_counts(ctypes.byref(c), dtype, 1, Hq, min(c.T_cap, 100), ctypes.byref(nq),
+                                 ctypes.byref(nd))
+    assert st == tq.TQ_OK, tq.last_error()
+    assert (nq.value, nd.value) == want
+
+
+def test_launch_counts_reject_bad_arguments():
+    c = _fake_cache(1, 2, 10, 128, 4, O.MSE, 2, O.MSE)
+    n = ctypes.c_int(0)
+    assert tq.lib.tq_launch_counts(ctypes.byref(c), 7, 1, 2, 5, ctypes.byref(n), None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_launch_counts(ctypes.byref(c), 1, 1, 3, 5, ctypes.byref(n), None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_launch_counts(ctypes.byref(c), 1, 1, 2, 11, ctypes.byref(n), None) == tq.TQ_ERR_INVALID_ARG
