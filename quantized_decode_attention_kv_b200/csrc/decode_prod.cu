@@ -50,6 +50,9 @@ struct QPrepP {
   uint32_t lo[64];
   float inv[2];
   float pad[2];
+  float val[128]; // the per-bit values in record order (code part, then sketch part)
+  float sum[2];   // sum of the code-part and of the sketch-part values
+  float pad2[2];
 };
 
 __global__ void __launch_bounds__(kPD) qprep_prod_kernel(const void *q, int dtype, float scale,
@@ -116,6 +119,24 @@ __global__ void __launch_bounds__(kPD) qprep_prod_kernel(const void *q, int dtyp
   if (i == 0) {
     out[bq].inv[0] = 1.0f / f[0];
     out[bq].inv[1] = 1.0f / f[1];
+  }
+  out[bq].val[i] = val[i];
+  out[bq].val[kPD + i] = val[kPD + i];
+  float s0 = val[i], s1 = val[kPD + i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+  }
+  __syncthreads(); // every thread has read the normalisation maxima from red
+  if ((i & 31) == 0) {
+    red[i >> 5] = s0;
+    red[2 + (i >> 5)] = s1;
+  }
+  __syncthreads();
+  if (i == 0) {
+    out[bq].sum[0] = red[0] + red[1];
+    out[bq].sum[1] = red[2] + red[3];
   }
 }
 
@@ -411,6 +432,195 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
   }
 }
 
+// One query head per KV head (multi-head attention): the score of a token is a dot product of
+// one query with 128 +-1 factors, so it is computed on the CUDA cores, one token per lane, from
+// per-query tables T_p[byte] = -2 * (sum of the values of the set bits of byte p of a record):
+// sum_k v_k (1 - 2 bit_k) = sum_k v_k + sum_p T_p[byte_p], 16 table reads per token instead of
+// an MMA whose score columns would be 3/4 empty. The values keep the tensor-core path above.
+struct LutTile {
+  uint2 kc, ks;                // key codes and sketch of token `lane` of the group
+  uint16_t kn, kg, vn, vg;     // its norms
+  uint32_t vm[2][4], vq[2][4]; // value code / sketch word r/4 of tokens 16 h + {2c, 2c+1, 2c+8, 2c+9}
+};
+
+__global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const ProdArgs a) {
+  __shared__ float tab[16 * 256];
+  __shared__ float mst[kPW];
+  __shared__ float gmx, lsum;
+  __shared__ float obuf[kPD + kPM];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = lane >> 2, c = lane & 3;
+  const uint32_t one2 = a.one2;
+  pdl_wait(); // the prepared queries and the cache are written by earlier kernels
+  pdl_trigger();
+
+  const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
+  const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
+  int slot = 0;
+  for (long long seg = range0; seg < range1; ++slot) {
+    const long long bh = seg / a.tiles_per_bh;
+    const long long seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
+    const int tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+    const int ntiles = static_cast<int>(seg_end - seg);
+    seg = seg_end;
+    const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
+
+    // ---- the query's tables (one query head: q-head h of sequence b)
+    const QPrepP *qp = a.qp + static_cast<size_t>(b) * a.Hq + h;
+    __syncthreads(); // the previous segment's readers are done with tab
+    for (int e = tid; e < 16 * 256; e += kPThreads) {
+      const float *v = qp->val + 8 * (e >> 8);
+      const int byte = e & 255;
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc += ((byte >> k) & 1) ? __ldg(v + k) : 0.f;
+      tab[e] = -2.0f * acc;
+    }
+    const float csum = __ldg(&qp->sum[0]), ssum = __ldg(&qp->sum[1]);
+    __syncthreads();
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[8][4];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+
+    const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
+    const int ts = tile0 * 16, te = min((tile0 + ntiles) * 16, a.T_len); // segment tokens
+    const int ngroups = (te - ts + 31) / 32;
+    const int vwo = 4 * (r >> 2);
+    const uint32_t selx = static_cast<uint32_t>(r & 3) | (static_cast<uint32_t>(4 + (r & 3)) << 8);
+    int jl = warp;
+
+    auto load_next = [&](LutTile &T) {
+      const int t0 = ts + 32 * jl;
+      const size_t tk = rec0 + min(t0 + lane, te - 1);
+      T.kc = __ldcs(reinterpret_cast<const uint2 *>(a.kc) + tk);
+      T.ks = __ldcs(reinterpret_cast<const uint2 *>(a.ks) + tk);
+      T.kn = __ldcs(a.kn + tk);
+      T.kg = __ldcs(a.kg + tk);
+      T.vn = __ldcs(a.vn + tk);
+      T.vg = __ldcs(a.vg + tk);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int tv = t0 + 16 * hh + 2 * c;
+        const int tvs[4] = {min(tv, te - 1), min(tv + 1, te - 1), min(tv + 8, te - 1), min(tv + 9, te - 1)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          T.vm[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (rec0 + tvs[e]) * 8 + vwo));
+          T.vq[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (rec0 + tvs[e]) * 8 + vwo));
+        }
+      }
+      jl += kPW;
+    };
+
+    // table offset (bytes) of byte k of a record word, for table block p: ((w >> 8k) & 255) * 4
+    auto tab_at = [&](uint32_t w, int k, int p) -> float {
+      const uint32_t off = (k == 0 ? (w << 2) : (w >> (8 * k - 2))) & 0x3FCu;
+      return *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(tab) + p * 1024 + off);
+    };
+
+    auto compute = [&](const LutTile &T, int t0) {
+      // ---- scores: one token per lane
+      float sc = 0.f, sk = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        sc += tab_at(T.kc.x, k, k) + tab_at(T.kc.y, k, 4 + k);
+        sk += tab_at(T.ks.x, k, 8 + k) + tab_at(T.ks.y, k, 12 + k);
+      }
+      const float kn = f16_bits_to_f32(T.kn), kg = f16_bits_to_f32(T.kg);
+      const float s = t0 + lane < te ? kn * (csum + sc + kg * (ssum + sk)) * kPLog2e : -INFINITY;
+      // ---- online softmax over the 32 tokens of the group (one head: the max is warp-uniform)
+      float mx = s;
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+      const float mn = fmaxf(m_run, mx);
+      if (mn != m_run) {
+        const float alpha = exp2f(m_run - mn);
+        l_run *= alpha;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          o[m][0] *= alpha;
+          o[m][1] *= alpha;
+          o[m][2] *= alpha;
+          o[m][3] *= alpha;
+        }
+        m_run = mn;
+      }
+      const float pr = exp2f(s - mn);
+      l_run += pr;
+      const float vn = f16_bits_to_f32(T.vn), vg = f16_bits_to_f32(T.vg);
+      const uint32_t pk = pack_h2(pr * vn, pr * vn * vg); // (code rows, sketch rows)
+
+      // ---- values: two 16-token MMA groups; P' column 0 = the head (other columns zero)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int base = 16 * hh + 2 * c;
+        const uint32_t x0 = __shfl_sync(0xffffffffu, pk, base), x1 = __shfl_sync(0xffffffffu, pk, base + 1);
+        const uint32_t x8 = __shfl_sync(0xffffffffu, pk, base + 8), x9 = __shfl_sync(0xffffffffu, pk, base + 9);
+        uint32_t pbc0 = prmt(x0, x1, 0x5410u), pbc1 = prmt(x8, x9, 0x5410u);
+        uint32_t pbs0 = prmt(x0, x1, 0x7632u), pbs1 = prmt(x8, x9, 0x7632u);
+        if (r != 0) pbc0 = pbc1 = pbs0 = pbs1 = 0u;
+        const uint32_t xm0 = prmt(T.vm[hh][0], T.vm[hh][1], selx), xm1 = prmt(T.vm[hh][2], T.vm[hh][3], selx);
+        const uint32_t xq0 = prmt(T.vq[hh][0], T.vq[hh][1], selx), xq1 = prmt(T.vq[hh][2], T.vq[hh][3], selx);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int sh0 = 15 - 2 * m, sh1 = 14 - 2 * m;
+          mma16816(o[m], pm1(xm0, sh0, one2), pm1(xm0, sh1, one2), pm1(xm1, sh0, one2),
+                   pm1(xm1, sh1, one2), pbc0, pbc1);
+          mma16816(o[4 + m], pm1(xq0, sh0, one2), pm1(xq0, sh1, one2), pm1(xq1, sh0, one2),
+                   pm1(xq1, sh1, one2), pbs0, pbs1);
+        }
+      }
+    };
+
+    LutTile ta, tb;
+    int jt = warp;
+    if (jl < ngroups) load_next(ta);
+    while (jt < ngroups) {
+      if (jl < ngroups) load_next(tb);
+      compute(ta, ts + 32 * jt);
+      jt += kPW;
+      if (jt >= ngroups) break;
+      if (jl < ngroups) load_next(ta);
+      compute(tb, ts + 32 * jt);
+      jt += kPW;
+    }
+
+    // ---- merge the warps (one head)
+    float l = l_run;
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o2);
+    if (lane == 0) mst[warp] = m_run;
+    for (int idx = tid; idx < kPD + kPM; idx += kPThreads) obuf[idx] = 0.f;
+    if (tid == 0) lsum = 0.f;
+    __syncthreads();
+    if (tid == 0) {
+      float M = -INFINITY;
+      for (int w = 0; w < kPW; ++w) M = fmaxf(M, mst[w]);
+      gmx = M;
+    }
+    __syncthreads();
+    const float f = exp2f(m_run - gmx);
+    if (lane == 0) atomicAdd(&lsum, l * f);
+    if (c == 0) {
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int i0 = (m < 4 ? 0 : kPD) + 8 * r + 2 * (m & 3);
+        atomicAdd(&obuf[i0], o[m][0] * f);
+        atomicAdd(&obuf[i0 + 1], o[m][2] * f);
+      }
+    }
+    __syncthreads();
+    float *dst = a.part + (static_cast<size_t>(blockIdx.x) * a.slots + slot) * a.stride;
+    for (int idx = tid; idx < kPD + kPM; idx += kPThreads) dst[2 + idx] = obuf[idx];
+    if (tid == 0) {
+      dst[0] = gmx;
+      dst[1] = lsum;
+    }
+  }
+}
+
 // Merge the partial records of one (b, q-head); u' = -c1 u, add sqrt(d) sqrt(pi/2)/m S^T w,
 // apply the inverse rotation D H / d and divide by the softmax sum. One warp per (b, q-head);
 // lane l owns coordinates 2 l, 2 l + 1 and sketch rows 2 l, 2 l + 1.
@@ -549,7 +759,8 @@ cudaError_t launch_prod_decode(const DecodeArgs &a, cudaStream_t s) {
   f.stride = p.ws_stride;
   f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
   f.one2 = 0x3C003C00u;
-  e = launch_pdl(decode_prod_kernel, dim3(p.ctas), dim3(kPThreads), 0, s, f);
+  e = launch_pdl(f.G == 1 ? decode_prod_lut_kernel : decode_prod_kernel, dim3(p.ctas),
+                 dim3(kPThreads), 0, s, f);
   if (e != cudaSuccess) return e;
   return launch_pdl(combine_prod_kernel, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
                     static_cast<const float *>(a.ws), a.B, a.Hkv, f.G, p.tiles_per_bh,
