@@ -492,25 +492,56 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
     const uint32_t selx = static_cast<uint32_t>(r & 3) | (static_cast<uint32_t>(4 + (r & 3)) << 8);
     int jl = warp;
 
+    // lane pointers of the next full group this warp loads (a warp advances kPW groups)
+    const size_t tw0 = rec0 + ts + 32 * warp;
+    const uint2 *kcp = reinterpret_cast<const uint2 *>(a.kc) + tw0 + lane;
+    const uint2 *ksp = reinterpret_cast<const uint2 *>(a.ks) + tw0 + lane;
+    const uint16_t *np[4] = {a.kn + tw0 + lane, a.kg + tw0 + lane, a.vn + tw0 + lane, a.vg + tw0 + lane};
+    const uint8_t *vcp = a.vc + (tw0 + 2 * c) * 8 + vwo;
+    const uint8_t *vsp = a.vs + (tw0 + 2 * c) * 8 + vwo;
+
     auto load_next = [&](LutTile &T) {
       const int t0 = ts + 32 * jl;
-      const size_t tk = rec0 + min(t0 + lane, te - 1);
-      T.kc = __ldcs(reinterpret_cast<const uint2 *>(a.kc) + tk);
-      T.ks = __ldcs(reinterpret_cast<const uint2 *>(a.ks) + tk);
-      T.kn = __ldcs(a.kn + tk);
-      T.kg = __ldcs(a.kg + tk);
-      T.vn = __ldcs(a.vn + tk);
-      T.vg = __ldcs(a.vg + tk);
+      if (t0 + 32 <= te) {
+        T.kc = __ldcs(kcp);
+        T.ks = __ldcs(ksp);
+        T.kn = __ldcs(np[0]);
+        T.kg = __ldcs(np[1]);
+        T.vn = __ldcs(np[2]);
+        T.vg = __ldcs(np[3]);
+        const int toff[4] = {0, 8, 64, 72}; // tokens 2c, 2c+1, 2c+8, 2c+9 (bytes)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int tv = t0 + 16 * hh + 2 * c;
-        const int tvs[4] = {min(tv, te - 1), min(tv + 1, te - 1), min(tv + 8, te - 1), min(tv + 9, te - 1)};
+        for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          T.vm[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (rec0 + tvs[e]) * 8 + vwo));
-          T.vq[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (rec0 + tvs[e]) * 8 + vwo));
+          for (int e = 0; e < 4; ++e) {
+            T.vm[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(vcp + 128 * hh + toff[e]));
+            T.vq[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(vsp + 128 * hh + toff[e]));
+          }
+      } else {
+        const size_t tk = rec0 + min(t0 + lane, te - 1);
+        T.kc = __ldcs(reinterpret_cast<const uint2 *>(a.kc) + tk);
+        T.ks = __ldcs(reinterpret_cast<const uint2 *>(a.ks) + tk);
+        T.kn = __ldcs(a.kn + tk);
+        T.kg = __ldcs(a.kg + tk);
+        T.vn = __ldcs(a.vn + tk);
+        T.vg = __ldcs(a.vg + tk);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int tv = t0 + 16 * hh + 2 * c;
+          const int tvs[4] = {min(tv, te - 1), min(tv + 1, te - 1), min(tv + 8, te - 1), min(tv + 9, te - 1)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            T.vm[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (rec0 + tvs[e]) * 8 + vwo));
+            T.vq[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (rec0 + tvs[e]) * 8 + vwo));
+          }
         }
       }
+      kcp += kPW * 32;
+      ksp += kPW * 32;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) np[e] += kPW * 32;
+      vcp += kPW * 32 * 8;
+      vsp += kPW * 32 * 8;
       jl += kPW;
     };
 
