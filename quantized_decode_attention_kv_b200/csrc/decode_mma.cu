@@ -33,12 +33,6 @@ namespace tq {
 namespace {
 using namespace mma_ops;
 
-#ifndef TQ_MSE_WARPS
-#define TQ_MSE_WARPS 4
-#endif
-constexpr int kWarps = TQ_MSE_WARPS; // warps per CTA of the MSE kernel
-constexpr int kThreads = kWarps * 32;
-constexpr int kStep = kWarps * 16;  // tokens a warp advances per step
 constexpr int kD = 128;
 constexpr float kLoScale = 4096.0f; // residual scaling 2^12 (keeps residuals normal in fp16)
 constexpr float kLoInv = 1.0f / 4096.0f;
@@ -54,14 +48,24 @@ constexpr int kPrefetchSteps = TQ_DECODE_PREFETCH;
 // 1 KB below it is reserved by the hardware); the kernel checks it before relying on it.
 constexpr uint32_t kFixedBase = 1024;
 
-#ifndef TQ_MSE_CTAS
-#define TQ_MSE_CTAS 3
-#endif
+// Warps per CTA and CTAs per SM. 2-bit values use a 64 KB value table beside the 64 KB key
+// table, so one CTA of 12 warps per SM shares both; other configurations run three CTAs of 4
+// warps (12 warps of up to 168 registers per SM either way; 16 warps of 128 registers were
+// measured slower).
+template <int KB, int VB>
+struct Cfg {
+  static constexpr int kWarps = VB == 2 ? 12 : 4;
+  static constexpr int kCtas = VB == 2 ? 1 : 3;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kStep = kWarps * 16; // tokens a warp advances per step
+};
 
 template <uint32_t OFF>
 __device__ __forceinline__ uint2 lds64_off(uint32_t smem_addr) {
   uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr), "n"(OFF));
+  // not volatile: the tables are read-only after the fill barrier, and leaving the loads free
+  // lets the compiler hoist them ahead of the MMAs that consume them
+  asm("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr), "n"(OFF));
   return v;
 }
 
@@ -80,19 +84,23 @@ struct Tile {
 
 // Shared-memory tables of one configuration. Key rows: one code-pair index (4-bit keys: a
 // byte of two codes, 256 rows; 3-bit keys: 6 bits, 64 rows) x {32 lane copies of the fp16x2
-// hi pair, 32 of the lo pair} = 256 bytes. Value rows (VB >= 3): one index (code of the first
-// token | code of the second << VB) x 32 lane copies of the fp16x2 pair = 128 bytes. The
-// 3-bit key table and the value tables sit at addresses aligned to their size so that an
-// index OR-ed above the lane offset is already the address.
+// hi pair, 32 of the lo pair} = 256 bytes. Value rows, 2-bit values: one byte holding the
+// codes of two adjacent coordinates of two tokens (low nibble the first token) x 32 lane
+// copies of the two fp16x2 operand words = 256 bytes; 3/4-bit values: one index (code of the
+// first token | code of the second << VB) x 32 lane copies of the fp16x2 pair = 128 bytes.
+// The 3-bit key table and the 3/4-bit value tables sit at addresses aligned to their size so
+// that an index OR-ed above the lane offset is already the address.
 template <int KB, int VB>
 struct Lut {
   static constexpr int kRows = KB == 4 ? 256 : 64;
   static constexpr int kBytes = kRows * 256;
   static constexpr int kAlign = KB == 4 ? 16 : kBytes;
-  static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : 0;
-  static constexpr int vBytes = vRows * 128;
+  static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : 256;
+  static constexpr int vBytes = vRows * (VB >= 3 ? 128 : 256);
   static constexpr int vAlign = VB >= 3 ? vBytes : 16;
-  static constexpr int kMergeBytes = (kWarps * 8 + 16 + 8 * 128) * 4;
+  // merge area: per-warp maxima and sums [warps][8] each, merged [8] each, then the per-warp
+  // value accumulators [warps][8 m-tiles][32 lanes] float4
+  static constexpr int kMergeBytes = (2 * Cfg<KB, VB>::kWarps * 8 + 16) * 4 + Cfg<KB, VB>::kWarps * 256 * 16;
   static constexpr int kSmem = kBytes + kAlign - 16 + vBytes + vAlign - 16 + kMergeBytes;
 };
 
@@ -186,8 +194,11 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32
 }
 
 template <int KB, int VB, int NT>
-__global__ void __launch_bounds__(kThreads, TQ_MSE_CTAS) decode_mse_kernel(const FastArgs a) {
+__global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
+    decode_mse_kernel(const FastArgs a) {
   using L = Lut<KB, VB>;
+  using C = Cfg<KB, VB>;
+  constexpr int kWarps = C::kWarps, kThreads = C::kThreads, kStep = C::kStep;
   using TileT = Tile<KB, VB>;
   constexpr int KR = KB * 16, VR = VB * 16; // record bytes
   extern __shared__ __align__(16) uint8_t smem[];
@@ -197,9 +208,10 @@ __global__ void __launch_bounds__(kThreads, TQ_MSE_CTAS) decode_mse_kernel(const
   uint8_t *const kl_p = smem + (klut - sbase);
   uint8_t *const vl_p = smem + (vlut - sbase);
   float *mst = reinterpret_cast<float *>(vl_p + L::vBytes); // [kWarps][8] running max
-  float *gmx = mst + kWarps * 8;                            // [8] merged max
+  float *lst = mst + kWarps * 8;                            // [kWarps][8] running sum
+  float *gmx = lst + kWarps * 8;                            // [8] merged max
   float *lsum = gmx + 8;                                    // [8] merged sum
-  float *obuf = lsum + 8;                                   // [G][128] merged accumulator
+  float4 *obw = reinterpret_cast<float4 *>(lsum + 8);       // [kWarps][8][32] accumulators
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
@@ -216,11 +228,17 @@ __global__ void __launch_bounds__(kThreads, TQ_MSE_CTAS) decode_mse_kernel(const
     uint32_t *vw = reinterpret_cast<uint32_t *>(vl_p);
     for (int idx = tid; idx < L::vRows * 32; idx += kThreads) {
       const int e = idx >> 5;
-      vw[idx] = pack_h2(a.vcent[e & ((1 << VB) - 1)], a.vcent[e >> VB]);
+      if constexpr (VB == 2) {
+        // byte e: first token's codes at coordinates j, j+1 in bits 0-1, 2-3, the second
+        // token's in bits 4-5, 6-7; words: coordinate j, coordinate j+1 (tokens in halves)
+        const int l = idx & 31;
+        vw[e * 64 + 2 * l] = pack_h2(a.vcent[e & 3], a.vcent[(e >> 4) & 3]);
+        vw[e * 64 + 2 * l + 1] = pack_h2(a.vcent[(e >> 2) & 3], a.vcent[(e >> 6) & 3]);
+      } else {
+        vw[idx] = pack_h2(a.vcent[e & ((1 << VB) - 1)], a.vcent[e >> VB]);
+      }
     }
   }
-  const uint32_t vt0 = pack_h2(a.vcent[0], a.vcent[1]);
-  const uint32_t vt1 = pack_h2(a.vcent[2], a.vcent[3]);
   const uint32_t lanebase = static_cast<uint32_t>(lane) << 2;
   const uint32_t klane8 = static_cast<uint32_t>(lane) << 3; // lane's 8-byte {hi, lo} entry
   const uint32_t klb = klut | klane8;                          // 3-bit keys: base + lane offset
@@ -500,27 +518,27 @@ __global__ void __launch_bounds__(kThreads, TQ_MSE_CTAS) decode_mse_kernel(const
         //      (rows r+8); operand quad (a0, a1, a2, a3) = (2m, 2m+1) x tokens (2c, 2c+1) then
         //      (2c+8, 2c+9).
         if constexpr (VB == 2) {
-          // pair-of-token PRMT lookups into a 4-entry fp16 table held in two registers
+          // Interleave the nibbles of the two tokens of each k pair: byte k of u holds both
+          // tokens' codes at run coordinates 4k, 4k+1 (m-tile 2k), byte k of w those at 4k+2,
+          // 4k+3 (m-tile 2k+1); one 64-bit table load per byte is the operand pair (a0, a1)
+          // or (a2, a3) of that m-tile.
+          const uint32_t u01 = (T.v[0][0] & 0x0F0F0F0Fu) | ((T.v[1][0] << 4) & 0xF0F0F0F0u);
+          const uint32_t w01 = ((T.v[0][0] >> 4) & 0x0F0F0F0Fu) | (T.v[1][0] & 0xF0F0F0F0u);
+          const uint32_t u23 = (T.v[2][0] & 0x0F0F0F0Fu) | ((T.v[3][0] << 4) & 0xF0F0F0F0u);
+          const uint32_t w23 = ((T.v[2][0] >> 4) & 0x0F0F0F0Fu) | (T.v[3][0] & 0xF0F0F0F0u);
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint32_t xsel = half ? 0x7362u : 0x5140u;
-            const uint32_t xa = prmt(T.v[0][0], T.v[1][0], xsel); // tokens 2c, 2c+1: codes 8half..+7
-            const uint32_t xb = prmt(T.v[2][0], T.v[3][0], xsel); // tokens 2c+8, 2c+9
-            uint32_t aq[4][4];
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t ya = (xa >> (2 * kk)) & 0x03030303u;
-              const uint32_t yb = (xb >> (2 * kk)) & 0x03030303u;
-              const uint32_t za = imad(ya, 0x22u, 0x10101010u);
-              const uint32_t zb = imad(yb, 0x22u, 0x10101010u);
-              aq[kk >> 1][kk & 1] = prmt(vt0, vt1, za);
-              aq[kk >> 1][2 + (kk & 1)] = prmt(vt0, vt1, zb);
-              aq[2 + (kk >> 1)][kk & 1] = prmt(vt0, vt1, za >> 16);
-              aq[2 + (kk >> 1)][2 + (kk & 1)] = prmt(vt0, vt1, zb >> 16);
+          for (int m = 0; m < 8; ++m) {
+            const uint32_t sel = 0x7604u | (static_cast<uint32_t>(m >> 1) << 4);
+            const uint32_t x01 = (m & 1) ? w01 : u01, x23 = (m & 1) ? w23 : u23;
+            uint2 e01, e23;
+            if constexpr (kFixed) {
+              e01 = lds64_off<kFixedBase + L::kBytes>(prmt(x01, klane, sel));
+              e23 = lds64_off<kFixedBase + L::kBytes>(prmt(x23, klane, sel));
+            } else {
+              e01 = lds64_off<0>(imad(prmt(x01, klane, sel), one, vlut));
+              e23 = lds64_off<0>(imad(prmt(x23, klane, sel), one, vlut));
             }
-#pragma unroll
-            for (int mm = 0; mm < 4; ++mm)
-              mma16816(o[4 * half + mm], aq[mm][0], aq[mm][1], aq[mm][2], aq[mm][3], pb0, pb1);
+            mma16816(o[m], e01.x, e01.y, e23.x, e23.y, pb0, pb1);
           }
         } else {
           // each operand register is one lane-replicated table word indexed by the two tokens'
@@ -566,52 +584,62 @@ __global__ void __launch_bounds__(kThreads, TQ_MSE_CTAS) decode_mse_kernel(const
         jt += kWarps;
       }
 
-      // ---- merge the warps: common max per head, rescale, accumulate in shared memory
+      // ---- merge the warps: common max and sum per head, then each warp stores its rescaled
+      //      accumulators in its own slots ([m-tile][lane] float4, conflict-free) and the
+      //      threads sum them over the warps into the partial record
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         float l = l_run[nt];
         l += __shfl_xor_sync(0xffffffffu, l, 4);
         l += __shfl_xor_sync(0xffffffffu, l, 8);
         l += __shfl_xor_sync(0xffffffffu, l, 16);
-        l_run[nt] = l;
-        if (r == 0) mst[warp * 8 + nt * 4 + c] = m_run[nt];
+        if (r == 0) {
+          mst[warp * 8 + nt * 4 + c] = m_run[nt];
+          lst[warp * 8 + nt * 4 + c] = l;
+        }
       }
-      for (int idx = tid; idx < a.G * kD; idx += kThreads) obuf[idx] = 0.f;
-      if (tid < 8) lsum[tid] = 0.f;
       __syncthreads();
       if (tid < 8) {
         float M = -INFINITY;
         for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mst[w * 8 + tid]);
+        float Ls = 0.f;
+        for (int w = 0; w < kWarps; ++w) {
+          const float mw = mst[w * 8 + tid];
+          if (mw != -INFINITY) Ls = fmaf(lst[w * 8 + tid], exp2f(mw - M), Ls);
+        }
         gmx[tid] = M;
+        lsum[tid] = Ls;
       }
       __syncthreads();
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int g = nt * 4 + c;
-        if (r == 0 && g < a.G) atomicAdd(&lsum[g], l_run[nt] * exp2f(m_run[nt] - gmx[g]));
-      }
       {
         const int g0 = 2 * c, g1 = 2 * c + 1;
         const float f0 = g0 < a.G ? exp2f(mst[warp * 8 + g0] - gmx[g0]) : 0.f;
         const float f1 = g1 < a.G ? exp2f(mst[warp * 8 + g1] - gmx[g1]) : 0.f;
+        float4 *ow = obw + warp * 256 + lane;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int i0 = 16 * r + 2 * m;
-          if (g0 < a.G) {
-            atomicAdd(&obuf[g0 * kD + i0], o[m][0] * f0);
-            atomicAdd(&obuf[g0 * kD + i0 + 1], o[m][2] * f0);
-          }
-          if (g1 < a.G) {
-            atomicAdd(&obuf[g1 * kD + i0], o[m][1] * f1);
-            atomicAdd(&obuf[g1 * kD + i0 + 1], o[m][3] * f1);
-          }
-        }
+        for (int m = 0; m < 8; ++m)
+          ow[32 * m] = make_float4(o[m][0] * f0, o[m][1] * f1, o[m][2] * f0, o[m][3] * f1);
       }
       __syncthreads();
       float *dst = a.part + (static_cast<size_t>(blockIdx.x) * a.slots + slot) * a.G * a.stride;
-      for (int idx = tid; idx < a.G * kD; idx += kThreads) {
-        const int g = idx / kD, i = idx - g * kD;
-        dst[static_cast<size_t>(g) * a.stride + 2 + i] = obuf[idx];
+      for (int idx = tid; idx < 256; idx += kThreads) {
+        float4 acc = obw[idx];
+        for (int w = 1; w < kWarps; ++w) {
+          const float4 x = obw[w * 256 + idx];
+          acc.x += x.x;
+          acc.y += x.y;
+          acc.z += x.z;
+          acc.w += x.w;
+        }
+        // slot (m, lane (rr, cc)): coordinates 16 rr + 2m, +1 of heads 2 cc, 2 cc + 1
+        const int m = idx >> 5, rr = (idx >> 2) & 7, cc = idx & 3;
+        const int i0 = 16 * rr + 2 * m;
+        if (2 * cc < a.G)
+          *reinterpret_cast<float2 *>(dst + static_cast<size_t>(2 * cc) * a.stride + 2 + i0) =
+              make_float2(acc.x, acc.z);
+        if (2 * cc + 1 < a.G)
+          *reinterpret_cast<float2 *>(dst + static_cast<size_t>(2 * cc + 1) * a.stride + 2 + i0) =
+              make_float2(acc.y, acc.w);
       }
       if (tid < a.G) {
         dst[static_cast<size_t>(tid) * a.stride] = gmx[tid];
@@ -707,12 +735,15 @@ __global__ void __launch_bounds__(128) combine_fast_kernel(const float *part, in
 
 constexpr int kSmemPerSm = 228 * 1024;
 
-// CTAs of the tensor-core decode kernel that fit on one SM (3 at most: 168 registers each).
+template <int KB, int VB>
+int ctas_per_sm() {
+  return std::max(1, std::min(Cfg<KB, VB>::kCtas, kSmemPerSm / (Lut<KB, VB>::kSmem + 1024)));
+}
+
+// CTAs of the tensor-core decode kernel that fit on one SM.
 int mse_ctas_per_sm(int kb, int vb) {
-  int smem = 0;
-  if (kb == 4) smem = vb == 2 ? Lut<4, 2>::kSmem : vb == 3 ? Lut<4, 3>::kSmem : Lut<4, 4>::kSmem;
-  else smem = vb == 2 ? Lut<3, 2>::kSmem : vb == 3 ? Lut<3, 3>::kSmem : Lut<3, 4>::kSmem;
-  return std::max(1, std::min(TQ_MSE_CTAS, kSmemPerSm / (smem + 1024)));
+  if (kb == 4) return vb == 2 ? ctas_per_sm<4, 2>() : vb == 3 ? ctas_per_sm<4, 3>() : ctas_per_sm<4, 4>();
+  return vb == 2 ? ctas_per_sm<3, 2>() : vb == 3 ? ctas_per_sm<3, 3>() : ctas_per_sm<3, 4>();
 }
 
 template <int KB, int VB>
@@ -721,7 +752,7 @@ cudaError_t run_mse(const FastArgs &f, int ctas, cudaStream_t s) {
   auto kern = f.G <= 4 ? decode_mse_kernel<KB, VB, 1> : decode_mse_kernel<KB, VB, 2>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(ctas), dim3(kThreads), smem, s, f);
+  return launch_pdl(kern, dim3(ctas), dim3(Cfg<KB, VB>::kThreads), smem, s, f);
 }
 
 } // namespace
