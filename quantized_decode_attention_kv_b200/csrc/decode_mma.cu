@@ -52,10 +52,13 @@ constexpr uint32_t kFixedBase = 1024;
 // table, so one CTA of 12 warps per SM shares both; other configurations run three CTAs of 4
 // warps (12 warps of up to 168 registers per SM either way; 16 warps of 128 registers were
 // measured slower).
+#ifndef TQ_VTAB_M
+#define TQ_VTAB_M 8
+#endif
 template <int KB, int VB>
 struct Cfg {
-  static constexpr int kWarps = VB == 2 ? 12 : 4;
-  static constexpr int kCtas = VB == 2 ? 1 : 3;
+  static constexpr int kWarps = VB == 2 && TQ_VTAB_M > 0 ? 12 : 4;
+  static constexpr int kCtas = VB == 2 && TQ_VTAB_M > 0 ? 1 : 3;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kStep = kWarps * 16; // tokens a warp advances per step
 };
@@ -71,7 +74,8 @@ __device__ __forceinline__ uint2 lds64_off(uint32_t smem_addr) {
 
 // Per-tile registers of one warp lane for KB-bit keys and VB-bit values (d = 128).
 //  keys: the lane's slice [32c, 32c+32) of the coordinates = KB words of each of tokens r, r+8
-//  values: the lane's run [16r, 16r+16) of the coordinates of tokens 2c, 2c+1, 2c+8, 2c+9:
+//  values: the lane's run [16r, 16r+16) of the coordinates of tokens c, c+4, c+8, c+12 (the
+//          value MMA's k order, so that each load instruction reads four consecutive records):
 //          VB = 2: one word; VB = 3: the two words that hold its 48 bits; VB = 4: two words
 template <int KB, int VB>
 struct Tile {
@@ -95,7 +99,7 @@ struct Lut {
   static constexpr int kRows = KB == 4 ? 256 : 64;
   static constexpr int kBytes = kRows * 256;
   static constexpr int kAlign = KB == 4 ? 16 : kBytes;
-  static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : 256;
+  static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : TQ_VTAB_M > 0 ? 256 : 0;
   static constexpr int vBytes = vRows * (VB >= 3 ? 128 : 256);
   static constexpr int vAlign = VB >= 3 ? vBytes : 16;
   // merge area: per-warp maxima and sums [warps][8] each, merged [8] each, then the per-warp
@@ -239,6 +243,8 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       }
     }
   }
+  [[maybe_unused]] const uint32_t vt0 = pack_h2(a.vcent[0], a.vcent[1]);
+  [[maybe_unused]] const uint32_t vt1 = pack_h2(a.vcent[2], a.vcent[3]);
   const uint32_t lanebase = static_cast<uint32_t>(lane) << 2;
   const uint32_t klane8 = static_cast<uint32_t>(lane) << 3; // lane's 8-byte {hi, lo} entry
   const uint32_t klb = klut | klane8;                          // 3-bit keys: base + lane offset
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       int jl = warp;
       const int tw0 = (tile0 + warp) * 16;
       const uint8_t *kp = a.kc + (rec0 + tw0 + r) * KR + 4 * KB * c;
-      const uint8_t *vp = a.vc + (rec0 + tw0 + 2 * c) * VR + 4 * vwo;
+      const uint8_t *vp = a.vc + (rec0 + tw0 + c) * VR + 4 * vwo;
       const uint16_t *knp = a.kn + rec0 + tw0 + r;
       const uint16_t *vnp = a.vn + rec0 + tw0 + r;
 
@@ -366,9 +372,9 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           load_k(T.k[0], kp);
           load_k(T.k[1], kp + 8 * KR);
           load_v(T.v[0], vp);
-          load_v(T.v[1], vp + VR);
+          load_v(T.v[1], vp + 4 * VR);
           load_v(T.v[2], vp + 8 * VR);
-          load_v(T.v[3], vp + 9 * VR);
+          load_v(T.v[3], vp + 12 * VR);
           T.kn[0] = __ldcs(knp);
           T.kn[1] = __ldcs(knp + 8);
           T.vn[0] = __ldcs(vnp);
@@ -379,11 +385,11 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           load_k(T.k[0], kb + static_cast<size_t>(tr) * KR);
           load_k(T.k[1], kb + static_cast<size_t>(tr8) * KR);
           const uint8_t *vb = a.vc + rec0 * VR + 4 * vwo;
-          const int tv = t0 + 2 * c;
+          const int tv = t0 + c;
           load_v(T.v[0], vb + static_cast<size_t>(min(tv, tlast)) * VR);
-          load_v(T.v[1], vb + static_cast<size_t>(min(tv + 1, tlast)) * VR);
+          load_v(T.v[1], vb + static_cast<size_t>(min(tv + 4, tlast)) * VR);
           load_v(T.v[2], vb + static_cast<size_t>(min(tv + 8, tlast)) * VR);
-          load_v(T.v[3], vb + static_cast<size_t>(min(tv + 9, tlast)) * VR);
+          load_v(T.v[3], vb + static_cast<size_t>(min(tv + 12, tlast)) * VR);
           T.kn[0] = __ldcs(a.kn + rec0 + tr);
           T.kn[1] = __ldcs(a.kn + rec0 + tr8);
           T.vn[0] = __ldcs(a.vn + rec0 + tr);
@@ -498,25 +504,26 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           }
         }
 
-        // ---- P'^T as the B operand: lane (r, c) needs head g = r at tokens 2c, 2c+1, 2c+8, 2c+9
-        const int src0 = 8 * c + (r & 3);
+        // ---- P'^T as the B operand: lane (r, c) needs head g = r at k rows 2c, 2c+1, 2c+8, 2c+9,
+        //      which hold tokens c, c+4, c+8, c+12
+        const int src0 = 4 * c + (r & 3);
         uint32_t x0 = __shfl_sync(0xffffffffu, pk[0], src0);
-        uint32_t x1 = __shfl_sync(0xffffffffu, pk[0], src0 + 4);
+        uint32_t x1 = __shfl_sync(0xffffffffu, pk[0], src0 + 16);
         if (NT == 2) {
           const uint32_t y0 = __shfl_sync(0xffffffffu, pk[NT - 1], src0);
-          const uint32_t y1 = __shfl_sync(0xffffffffu, pk[NT - 1], src0 + 4);
+          const uint32_t y1 = __shfl_sync(0xffffffffu, pk[NT - 1], src0 + 16);
           if (r >= 4) {
             x0 = y0;
             x1 = y1;
           }
         }
         if (r >= a.G) x0 = x1 = 0u;
-        const uint32_t pb0 = prmt(x0, x1, 0x5410u); // tokens 2c, 2c+1
-        const uint32_t pb1 = prmt(x0, x1, 0x7632u); // tokens 2c+8, 2c+9
+        const uint32_t pb0 = prmt(x0, x1, 0x5410u); // tokens c, c+4
+        const uint32_t pb1 = prmt(x0, x1, 0x7632u); // tokens c+8, c+12
 
         // ---- values. m-tile m covers the lane's run coordinates 2m (rows r) and 2m + 1
-        //      (rows r+8); operand quad (a0, a1, a2, a3) = (2m, 2m+1) x tokens (2c, 2c+1) then
-        //      (2c+8, 2c+9).
+        //      (rows r+8); operand quad (a0, a1, a2, a3) = (2m, 2m+1) x tokens (c, c+4) then
+        //      (c+8, c+12).
         if constexpr (VB == 2) {
           // Interleave the nibbles of the two tokens of each k pair: byte k of u holds both
           // tokens' codes at run coordinates 4k, 4k+1 (m-tile 2k), byte k of w those at 4k+2,
@@ -527,7 +534,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           const uint32_t u23 = (T.v[2][0] & 0x0F0F0F0Fu) | ((T.v[3][0] << 4) & 0xF0F0F0F0u);
           const uint32_t w23 = ((T.v[2][0] >> 4) & 0x0F0F0F0Fu) | (T.v[3][0] & 0xF0F0F0F0u);
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
+          for (int m = 0; m < TQ_VTAB_M; ++m) {
             const uint32_t sel = 0x7604u | (static_cast<uint32_t>(m >> 1) << 4);
             const uint32_t x01 = (m & 1) ? w01 : u01, x23 = (m & 1) ? w23 : u23;
             uint2 e01, e23;
@@ -539,6 +546,27 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
               e23 = lds64_off<0>(imad(prmt(x23, klane, sel), one, vlut));
             }
             mma16816(o[m], e01.x, e01.y, e23.x, e23.y, pb0, pb1);
+          }
+#pragma unroll
+          for (int half = TQ_VTAB_M / 4; half < 2; ++half) {
+            const uint32_t xsel = half ? 0x7362u : 0x5140u;
+            const uint32_t xa = prmt(T.v[0][0], T.v[1][0], xsel);
+            const uint32_t xb = prmt(T.v[2][0], T.v[3][0], xsel);
+            uint32_t aq[4][4];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t ya = (xa >> (2 * kk)) & 0x03030303u;
+              const uint32_t yb = (xb >> (2 * kk)) & 0x03030303u;
+              const uint32_t za = imad(ya, 0x22u, 0x10101010u);
+              const uint32_t zb = imad(yb, 0x22u, 0x10101010u);
+              aq[kk >> 1][kk & 1] = prmt(vt0, vt1, za);
+              aq[kk >> 1][2 + (kk & 1)] = prmt(vt0, vt1, zb);
+              aq[2 + (kk >> 1)][kk & 1] = prmt(vt0, vt1, za >> 16);
+              aq[2 + (kk >> 1)][2 + (kk & 1)] = prmt(vt0, vt1, zb >> 16);
+            }
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm)
+              mma16816(o[4 * half + mm], aq[mm][0], aq[mm][1], aq[mm][2], aq[mm][3], pb0, pb1);
           }
         } else {
           // each operand register is one lane-replicated table word indexed by the two tokens'
