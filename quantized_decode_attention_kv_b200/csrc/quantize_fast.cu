@@ -21,6 +21,8 @@
 //    to z = 0, whose cell holds the boundary 0, and gets the lower code as a tie should.
 #include "tq_device.cuh"
 
+#include <type_traits>
+
 namespace tq {
 namespace {
 
@@ -44,6 +46,7 @@ struct FastQuantArgs {
   long long nbatch_total;
   // bit 31 set where D flips coordinate 2p (lo) / 2p + 1 (hi) of 16-bit pair p
   uint32_t sgn_lo[64], sgn_hi[64];
+  uint32_t sbits[4]; // D's sign bits of coordinates 0..127 (bit j % 32 of word j / 32)
 };
 
 typedef unsigned long long f2_t; // two fp32 lanes in one 64-bit register pair
@@ -366,6 +369,275 @@ __global__ void __launch_bounds__(kQThreads) quantize_small_kernel(const FastQua
   if (lane == 0) t.norm[rec] = f32_to_f16_bits(n);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Tensor-core variant for d = 128: one warp quantises 16 vectors at a time.
+//
+// The unnormalised Sylvester Hadamard matrix factors over the bits of the coordinate index,
+// H_128 = H_S (x) H_T with S = bits 3..6 and T = bits 0..2. For each value j_T of the low bits
+// (a "block" of 16 input coordinates 8 m + j_T, m = 0..15) one m16n8k16 MMA pair applies H_S:
+// A = 16 vectors x the block's 16 coordinates (the 16-bit inputs with D's signs flipped),
+// B = the 16 x 16 matrix of +-1. The 8-point transform over T then runs in registers.
+// Lane (r, c) loads 16-byte chunks c, c+4, c+8, c+12 of vectors r and r+8 (k index
+// k = 2c' + e + 8t' holds chunk c' + 4e + 8t'), and the output column n of its accumulators
+// is mapped to coordinate bits so that after the 8-point stage the lane holds output
+// coordinates [32c, 32c+32) of both vectors: packing and the record store stay lane-local.
+template <bool BF16>
+__device__ __forceinline__ void mma_pm1(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (BF16)
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+                 "{%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+                 : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+  else
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+                 "{%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+                 : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Codes of one vector's 32 coordinates held by this lane (local index o = o_T + 8 e + 16 t),
+// packed LSB-first into WB words, then stored at the lane's place in the record.
+template <int WB>
+__device__ __forceinline__ void mma_codes_store(const float (&acc)[8][2][4], int rho, float inv,
+                                                uint32_t cells, uint8_t *dst) {
+  uint32_t words[WB];
+#pragma unroll
+  for (int k = 0; k < WB; ++k) words[k] = 0u;
+  const f2_t inv2 = f2(inv, inv);
+  const f2_t cs2 = f2(kCellScale, kCellScale), cm2 = f2(kCellMagic, kCellMagic);
+#pragma unroll
+  for (int ot = 0; ot < 8; ++ot) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const f2_t z2 = mul2(f2(acc[ot][t][2 * rho], acc[ot][t][2 * rho + 1]), inv2);
+      const f2_t u2 = fma2(z2, cs2, cm2);
+      float z0, z1, u0, u1;
+      f2_split(z2, z0, z1);
+      f2_split(u2, u0, u1);
+      const uint2 e0 = cell_entry(u0, cells);
+      const uint2 e1 = cell_entry(u1, cells);
+      put_code<WB>(words, ot + 16 * t, e0.y + (z0 > __uint_as_float(e0.x) ? 1u : 0u));
+      put_code<WB>(words, ot + 8 + 16 * t, e1.y + (z1 > __uint_as_float(e1.x) ? 1u : 0u));
+    }
+  }
+  if constexpr (WB == 4) {
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
+  } else if constexpr (WB == 2) {
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(words[0], words[1]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < WB; ++k) reinterpret_cast<uint32_t *>(dst)[k] = words[k];
+  }
+}
+
+constexpr int kMmaWarps = 4;
+#ifndef TQ_QUANT_MMA
+#define TQ_QUANT_MMA 1
+#endif
+
+template <bool BF16>
+__global__ void __launch_bounds__(kMmaWarps * 32, 3) quantize_mma_kernel(const FastQuantArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const uint32_t pad = ((sbase + 2047u) & ~2047u) - sbase;
+  uint8_t *cells = smem + pad;
+  const uint32_t cells_s = sbase + pad;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = lane >> 2, c = lane & 3;
+
+  // cell tables, as in the streaming kernel
+  for (int idx = tid; idx < 2 * kCells; idx += kMmaWarps * 32) {
+    const FastTensor &t = a.t[idx / kCells];
+    const int k = idx % kCells;
+    const float lo = (8.0f * k - 1024.5f) / 32.0f, hi = lo + 0.25f;
+    uint32_t base = 0;
+    float inner = INFINITY;
+    for (int j = 0; j < t.nbeta; ++j) {
+      const float b = t.beta[j];
+      if (b <= lo) ++base;
+      else if (b < hi) inner = b;
+    }
+    reinterpret_cast<uint2 *>(cells)[idx] = make_uint2(__float_as_uint(inner), base);
+  }
+
+  // B fragments of H_S: element (k, n) = (-1)^popc(kappa(k) & sigma(n)), kappa(k) = the chunk
+  // held at k, sigma(n) = output coordinate bits 3..6 of column n (bit 3 = n0, bit 4 = n3,
+  // bit 5 = n1, bit 6 = n2)
+  const uint32_t one = BF16 ? 0x3F80u : 0x3C00u;
+  uint32_t hb[2][2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int n = 8 * t + r;
+    const int sigma = (n & 1) | (((n >> 3) & 1) << 1) | (((n >> 1) & 1) << 2) | (((n >> 2) & 1) << 3);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int k = 8 * h + 2 * c + e;
+        const int kappa = ((k >> 1) & 3) | ((k & 1) << 2) | ((k >> 3) << 3);
+        const uint32_t v = one | ((__popc(kappa & sigma) & 1) ? 0x8000u : 0u);
+        w |= v << (16 * e);
+      }
+      hb[t][h] = w;
+    }
+  }
+  // D's sign flips for the 16-bit pairs p of chunks c + 4 i (bit 15 / 31 of the XOR mask)
+  uint32_t sg[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = c + 4 * i; // chunk: coordinates 8 m .. 8 m + 7
+    const uint32_t byte = (a.sbits[m >> 2] >> (8 * (m & 3))) & 0xFFu;
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      sg[i][p] = (((byte >> (2 * p)) & 1u) << 15) | (((byte >> (2 * p + 1)) & 1u) << 31);
+  }
+  __syncthreads();
+  pdl_wait(); // K/V may come from the kernel before; the cache may still be read by it
+  pdl_trigger();
+
+  const long long ng0 = (a.t[0].nvec + 15) / 16;
+  const bool two = a.nbatch_total > a.t[0].nbatch;
+  const long long ngt = ng0 + (two ? (a.t[1].nvec + 15) / 16 : 0);
+  const long long stride = static_cast<long long>(gridDim.x) * kMmaWarps;
+  long long g = static_cast<long long>(blockIdx.x) * kMmaWarps + warp;
+
+  uint4 R[2][4]; // [row r / r+8][chunk c + 4 i]
+  auto load = [&](long long gg) {
+    const int ti = gg < ng0 ? 0 : 1;
+    const FastTensor &t = a.t[ti];
+    const unsigned v0 = static_cast<unsigned>((gg - (ti ? ng0 : 0)) * 16);
+#pragma unroll
+    for (int rho = 0; rho < 2; ++rho) {
+      const unsigned v = min(v0 + r + 8 * rho, t.nvec - 1);
+      const uint4 *src = reinterpret_cast<const uint4 *>(t.x + static_cast<size_t>(v) * 256) + c;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) R[rho][i] = __ldcs(src + 4 * i);
+    }
+  };
+
+  // One phase per tensor (K, then V) with its bit width fixed at compile time; the next
+  // group's loads are issued after this group's MMAs (they may belong to the next phase).
+  auto phase = [&](auto ti_tag, auto wb_tag, long long gend) {
+    constexpr int TI = decltype(ti_tag)::value, WB = decltype(wb_tag)::value;
+    const FastTensor &t = a.t[TI];
+    const uint32_t cl = cells_s + TI * kCells * 8;
+    const unsigned T = static_cast<unsigned>(t.T);
+    for (; g < gend; g += stride) {
+      const unsigned v0 = static_cast<unsigned>((g - (TI ? ng0 : 0)) * 16);
+
+      // ---- H_S on the tensor cores, one block j_T per MMA pair
+      uint32_t X[2][4][4];
+#pragma unroll
+      for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          X[rho][i][0] = R[rho][i].x ^ sg[i][0];
+          X[rho][i][1] = R[rho][i].y ^ sg[i][1];
+          X[rho][i][2] = R[rho][i].z ^ sg[i][2];
+          X[rho][i][3] = R[rho][i].w ^ sg[i][3];
+        }
+      float acc[8][2][4];
+#pragma unroll
+      for (int jt = 0; jt < 8; ++jt) {
+        const int p = jt >> 1;
+        const uint32_t sel = (jt & 1) ? 0x7632u : 0x5410u;
+        const uint32_t a0 = prmt_b32(X[0][0][p], X[0][1][p], sel);
+        const uint32_t a1 = prmt_b32(X[1][0][p], X[1][1][p], sel);
+        const uint32_t a2 = prmt_b32(X[0][2][p], X[0][3][p], sel);
+        const uint32_t a3 = prmt_b32(X[1][2][p], X[1][3][p], sel);
+        mma_pm1<BF16>(acc[jt][0], a0, a1, a2, a3, hb[0][0], hb[0][1]);
+        mma_pm1<BF16>(acc[jt][1], a0, a1, a2, a3, hb[1][0], hb[1][1]);
+      }
+      if (g + stride < ngt) load(g + stride);
+
+      // ---- H_T: 8-point butterflies over the blocks, per (n-tile, accumulator pair)
+#pragma unroll
+      for (int t2 = 0; t2 < 2; ++t2)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          f2_t y[8];
+#pragma unroll
+          for (int jt = 0; jt < 8; ++jt) y[jt] = f2(acc[jt][t2][2 * q], acc[jt][t2][2 * q + 1]);
+#pragma unroll
+          for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+            for (int jt = 0; jt < 8; ++jt)
+              if ((jt & h) == 0) {
+                const f2_t u = y[jt], w = y[jt + h];
+                y[jt] = add2(u, w);
+                y[jt + h] = sub2(u, w);
+              }
+#pragma unroll
+          for (int jt = 0; jt < 8; ++jt) f2_split(y[jt], acc[jt][t2][2 * q], acc[jt][t2][2 * q + 1]);
+        }
+
+      // ---- norms: ||H D x||^2 = 128 ||x||^2, summed over the 4 lanes of each vector
+      f2_t s2a = 0ull, s2b = 0ull;
+#pragma unroll
+      for (int jt = 0; jt < 8; ++jt)
+#pragma unroll
+        for (int t2 = 0; t2 < 2; ++t2) {
+          const f2_t ya = f2(acc[jt][t2][0], acc[jt][t2][1]);
+          const f2_t yb = f2(acc[jt][t2][2], acc[jt][t2][3]);
+          s2a = fma2(ya, ya, s2a);
+          s2b = fma2(yb, yb, s2b);
+        }
+      float sa0, sa1, sb0, sb1;
+      f2_split(s2a, sa0, sa1);
+      f2_split(s2b, sb0, sb1);
+      float sa = sa0 + sa1, sb = sb0 + sb1;
+      sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+      sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+      sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+      sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+
+      // record of vector v0 (the group's first), then of this lane's rows
+      const unsigned bh0 = v0 / T, tt0 = v0 - bh0 * T;
+#pragma unroll
+      for (int rho = 0; rho < 2; ++rho) {
+        const unsigned v = v0 + r + 8 * rho;
+        unsigned bh = bh0, tt = tt0 + r + 8 * rho;
+        while (tt >= T) { // T < 16 wraps more than once
+          tt -= T;
+          ++bh;
+        }
+        const float n = sqrtf((rho ? sb : sa) * (1.0f / 128.0f));
+        const float inv = n > 0.f ? __frcp_rn(n) : 0.0f;
+        if (v < t.nvec) {
+          const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
+          mma_codes_store<WB>(acc, rho, inv, cl, t.codes + rec * (16 * WB) + c * (4 * WB));
+          if (c == 0) t.norm[rec] = f32_to_f16_bits(n);
+        }
+      }
+    }
+  };
+  using I0 = std::integral_constant<int, 0>;
+  using I1 = std::integral_constant<int, 1>;
+  if (g < ngt) load(g);
+  switch (a.t[0].wbits) {
+  case 1: phase(I0{}, std::integral_constant<int, 1>{}, ng0); break;
+  case 2: phase(I0{}, std::integral_constant<int, 2>{}, ng0); break;
+  case 3: phase(I0{}, std::integral_constant<int, 3>{}, ng0); break;
+  default: phase(I0{}, std::integral_constant<int, 4>{}, ng0); break;
+  }
+  if (two) {
+    switch (a.t[1].wbits) {
+    case 1: phase(I1{}, std::integral_constant<int, 1>{}, ngt); break;
+    case 2: phase(I1{}, std::integral_constant<int, 2>{}, ngt); break;
+    case 3: phase(I1{}, std::integral_constant<int, 3>{}, ngt); break;
+    default: phase(I1{}, std::integral_constant<int, 4>{}, ngt); break;
+    }
+  }
+}
+
 template <int D, bool BF16>
 cudaError_t run_fast(const FastQuantArgs &f, int sms, cudaStream_t s) {
   const unsigned nvec = f.t[0].nvec + (f.nbatch_total > f.t[0].nbatch ? f.t[1].nvec : 0u);
@@ -373,6 +645,16 @@ cudaError_t run_fast(const FastQuantArgs &f, int sms, cudaStream_t s) {
     const unsigned blocks = (nvec + kQThreads / 32 - 1) / (kQThreads / 32);
     return launch_pdl(quantize_small_kernel<D, BF16>, dim3(blocks), dim3(kQThreads), 0, s, f);
   }
+#if TQ_QUANT_MMA
+  if constexpr (D == 128) {
+    const unsigned ngt = (f.t[0].nvec + 15) / 16 +
+                         (f.nbatch_total > f.t[0].nbatch ? (f.t[1].nvec + 15) / 16 : 0u);
+    const int msmem = 2048 + 2 * kCells * 8;
+    const long long grid = std::min<long long>((ngt + kMmaWarps - 1) / kMmaWarps, 3ll * sms);
+    return launch_pdl(quantize_mma_kernel<BF16>, dim3(static_cast<unsigned>(grid)),
+                      dim3(kMmaWarps * 32), msmem, s, f);
+  }
+#endif
   const int smem = 2048 + 2 * kCells * 8 + 2 * kQThreads * (2 * D + 16); // 2048: alignment slack
   cudaError_t e = cudaFuncSetAttribute(quantize_fast_kernel<D, BF16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -427,6 +709,8 @@ cudaError_t launch_quantize_fast(const QuantArgs *k, const QuantArgs *v, int sms
     f.sgn_lo[p] = ((first->sign_words[(2 * p) / 64] >> ((2 * p) % 64)) & 1ull) ? 0x80000000u : 0u;
     f.sgn_hi[p] = ((first->sign_words[(2 * p + 1) / 64] >> ((2 * p + 1) % 64)) & 1ull) ? 0x80000000u : 0u;
   }
+  for (int k = 0; k < 4; ++k)
+    f.sbits[k] = static_cast<uint32_t>(first->sign_words[k / 2] >> (32 * (k & 1)));
   const bool bf16 = first->dtype == TQ_BF16;
   if (d == 128) return bf16 ? run_fast<128, true>(f, sms, s) : run_fast<128, false>(f, sms, s);
   return bf16 ? run_fast<64, true>(f, sms, s) : run_fast<64, false>(f, sms, s);
