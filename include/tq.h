@@ -183,6 +183,13 @@ int tq_decode_attention_bf16(const void *q, int Hq, const void *K, const void *V
                              int Hkv, int T_cap, int T_len, int d, float scale, float *out,
                              void *ws, size_t ws_bytes, void *stream);
 
+/* Device-side faults recorded since the last call, as bits: bit 0 = a tensor-core kernel
+ * (tcgen05 write path of TurboQuant_prod records) gave up waiting for its MMAs after about a
+ * second, recorded a fault, freed its tensor memory and returned without writing the rest of
+ * its records. Reading synchronises the device and clears the bits. Writes *flags; returns
+ * TQ_OK or TQ_ERR_CUDA. The pages have no counterpart to this call. */
+int tq_device_faults(unsigned *flags);
+
 #ifdef __cplusplus
 }
 #endif

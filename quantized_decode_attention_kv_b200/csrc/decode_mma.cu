@@ -11,18 +11,20 @@
 //     (lo); two MMAs (hi, lo) give scores good to ~2^-21 relative, as fp32 scoring would.
 //     The query side is split the same way by the query-prep kernel.
 //   values  O^T[128 x heads] += V^T[128 x 16 tokens] . P'^T[16 tokens x heads]
-//     V^ comes from a 4-entry fp16 table held in two registers and indexed with PRMT, one
-//     PRMT per pair of tokens; P' = p * ||v_t|| in fp16.
+//     2-bit V^: one byte of nibble-interleaved codes (two tokens, two coordinates) indexes a
+//     lane-replicated shared table whose 8-byte entry is a pair of operand registers;
+//     3/4-bit V^: one table word per operand register. P' = p * ||v_t|| in fp16.
 //
 // The contraction order is free along k, so each thread owns a contiguous 16-byte slice of
 // every key record and one 32-bit word of every value record: all loads are 16- or 4-byte,
 // and the permutation is undone when the partial accumulators are written.
 //
 // Work split: the (batch, KV head, 16-token tile) space is flattened and cut into equal
-// contiguous ranges, one per persistent CTA of 4 warps; within a range each maximal run of
-// one (batch, KV head) is a segment, its tiles dealt round-robin to the warps, each warp
-// keeping its own online-softmax state (log2 domain); the warps merge through shared memory
-// at the end of the segment and write one partial record per query head.
+// contiguous ranges, one per persistent CTA (12 warps with 2-bit values, else 4); within a
+// range each maximal run of one (batch, KV head) is a segment, its tiles dealt round-robin to
+// the warps, each warp keeping its own online-softmax state (log2 domain); at the end of the
+// segment the warps store their rescaled accumulators in their own shared-memory slots, which
+// are summed into one partial record per query head.
 #include "mma_ops.cuh"
 
 #include <algorithm>
@@ -52,13 +54,10 @@ constexpr uint32_t kFixedBase = 1024;
 // table, so one CTA of 12 warps per SM shares both; other configurations run three CTAs of 4
 // warps (12 warps of up to 168 registers per SM either way; 16 warps of 128 registers were
 // measured slower).
-#ifndef TQ_VTAB_M
-#define TQ_VTAB_M 8
-#endif
 template <int KB, int VB>
 struct Cfg {
-  static constexpr int kWarps = VB == 2 && TQ_VTAB_M > 0 ? 12 : 4;
-  static constexpr int kCtas = VB == 2 && TQ_VTAB_M > 0 ? 1 : 3;
+  static constexpr int kWarps = VB == 2 ? 12 : 4;
+  static constexpr int kCtas = VB == 2 ? 1 : 3;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kStep = kWarps * 16; // tokens a warp advances per step
 };
@@ -99,7 +98,7 @@ struct Lut {
   static constexpr int kRows = KB == 4 ? 256 : 64;
   static constexpr int kBytes = kRows * 256;
   static constexpr int kAlign = KB == 4 ? 16 : kBytes;
-  static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : TQ_VTAB_M > 0 ? 256 : 0;
+  static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : 256;
   static constexpr int vBytes = vRows * (VB >= 3 ? 128 : 256);
   static constexpr int vAlign = VB >= 3 ? vBytes : 16;
   // merge area: per-warp maxima and sums [warps][8] each, merged [8] each, then the per-warp
@@ -243,8 +242,6 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       }
     }
   }
-  [[maybe_unused]] const uint32_t vt0 = pack_h2(a.vcent[0], a.vcent[1]);
-  [[maybe_unused]] const uint32_t vt1 = pack_h2(a.vcent[2], a.vcent[3]);
   const uint32_t lanebase = static_cast<uint32_t>(lane) << 2;
   const uint32_t klane8 = static_cast<uint32_t>(lane) << 3; // lane's 8-byte {hi, lo} entry
   const uint32_t klb = klut | klane8;                          // 3-bit keys: base + lane offset
@@ -534,7 +531,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           const uint32_t u23 = (T.v[2][0] & 0x0F0F0F0Fu) | ((T.v[3][0] << 4) & 0xF0F0F0F0u);
           const uint32_t w23 = ((T.v[2][0] >> 4) & 0x0F0F0F0Fu) | (T.v[3][0] & 0xF0F0F0F0u);
 #pragma unroll
-          for (int m = 0; m < TQ_VTAB_M; ++m) {
+          for (int m = 0; m < 8; ++m) {
             const uint32_t sel = 0x7604u | (static_cast<uint32_t>(m >> 1) << 4);
             const uint32_t x01 = (m & 1) ? w01 : u01, x23 = (m & 1) ? w23 : u23;
             uint2 e01, e23;
@@ -546,27 +543,6 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
               e23 = lds64_off<0>(imad(prmt(x23, klane, sel), one, vlut));
             }
             mma16816(o[m], e01.x, e01.y, e23.x, e23.y, pb0, pb1);
-          }
-#pragma unroll
-          for (int half = TQ_VTAB_M / 4; half < 2; ++half) {
-            const uint32_t xsel = half ? 0x7362u : 0x5140u;
-            const uint32_t xa = prmt(T.v[0][0], T.v[1][0], xsel);
-            const uint32_t xb = prmt(T.v[2][0], T.v[3][0], xsel);
-            uint32_t aq[4][4];
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t ya = (xa >> (2 * kk)) & 0x03030303u;
-              const uint32_t yb = (xb >> (2 * kk)) & 0x03030303u;
-              const uint32_t za = imad(ya, 0x22u, 0x10101010u);
-              const uint32_t zb = imad(yb, 0x22u, 0x10101010u);
-              aq[kk >> 1][kk & 1] = prmt(vt0, vt1, za);
-              aq[kk >> 1][2 + (kk & 1)] = prmt(vt0, vt1, zb);
-              aq[2 + (kk >> 1)][kk & 1] = prmt(vt0, vt1, za >> 16);
-              aq[2 + (kk >> 1)][2 + (kk & 1)] = prmt(vt0, vt1, zb >> 16);
-            }
-#pragma unroll
-            for (int mm = 0; mm < 4; ++mm)
-              mma16816(o[4 * half + mm], aq[mm][0], aq[mm][1], aq[mm][2], aq[mm][3], pb0, pb1);
           }
         } else {
           // each operand register is one lane-replicated table word indexed by the two tokens'

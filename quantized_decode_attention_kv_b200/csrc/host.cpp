@@ -450,6 +450,11 @@ int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, flo
                      "decode (fixed scratch) launch");
 }
 
+int tq_device_faults(unsigned *flags) {
+  if (!flags) return fail(TQ_ERR_INVALID_ARG, "flags is NULL");
+  return cuda_status(tq::read_and_clear_prod_faults(flags), "tq_device_faults");
+}
+
 int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,
                      int *quantize_launches, int *decode_launches) {
   int st = check_cache(cache);

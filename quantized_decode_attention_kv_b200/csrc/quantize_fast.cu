@@ -1,24 +1,28 @@
-// Streaming quantise-on-write for MSE records of 16-bit K/V ("Closing - The Three-Step
-// Summary", Steps 1-3; the spec write path: norm, seeded-sign Walsh-Hadamard rotation,
-// Lloyd-Max codes, LSB-first packing).
+// Quantise-on-write for MSE records of 16-bit K/V ("Closing - The Three-Step Summary",
+// Steps 1-3: norm, seeded-sign Walsh-Hadamard rotation, Lloyd-Max codes, LSB-first packing).
 //
 // Design (B200):
-//  * Persistent CTAs of 128 threads walk 128-vector batches of K and then V in one launch.
-//    Each batch (128 x d 16-bit elements, contiguous in memory) is copied into shared memory
-//    with coalesced 16-byte cp.async copies, double-buffered so the next batch is in flight
-//    while this one is computed. Rows are padded by 16 bytes so that the 16-byte row reads of
-//    one thread per vector never share a bank.
-//  * One thread owns one vector: the whole transform stays in registers. Coordinates are
+//  * head_dim 128 (quantize_mma_kernel): one warp quantises 16 vectors; the 16-point factor
+//    of the Hadamard transform runs on the tensor cores, the 8-point factor in registers
+//    (the kernel's own comment block below gives the index mapping).
+//  * head_dim 64 (quantize_fast_kernel): persistent CTAs of 128 threads walk 128-vector
+//    batches of K and then V in one launch. Each batch (128 x d 16-bit elements, contiguous
+//    in memory) is copied into shared memory with coalesced 16-byte cp.async copies,
+//    double-buffered so the next batch is in flight while this one is computed. Rows are
+//    padded by 16 bytes so that the 16-byte row reads of one thread per vector never share a
+//    bank. One thread owns one vector: the whole transform stays in registers. Coordinates are
 //    held as packed fp32 pairs (x_j, x_{j+d/2}); the sum of squares and all but one of the
 //    log2(d) butterfly stages run as Blackwell f32x2 instructions (two lanes of work per
 //    instruction). Signs are applied while widening the 16-bit inputs (an add of 2^31 to the
 //    fp32 bit pattern flips its sign).
-//  * Code search: z is mapped to one of 256 cells of width 1/4 on the N(0,1) scale with one
-//    fused multiply-add (the cell index lands in the low mantissa bits of a float offset by
-//    1.5 * 2^23); a shared-memory table gives, per cell, the number of decision boundaries
-//    below it and the single boundary inside it (Lloyd-Max boundaries of <= 4 bits are more
-//    than 1/4 apart), so every code costs one table read and one compare. A zero vector maps
-//    to z = 0, whose cell holds the boundary 0, and gets the lower code as a tie should.
+//  * A few vectors (a decode step's new token): quantize_small_kernel, one warp per vector.
+//  * Code search (all three): z is mapped to one of 256 cells of width 1/4 on the N(0,1)
+//    scale with one fused multiply-add (the cell index lands in the low mantissa bits of a
+//    float offset by 1.5 * 2^23); a shared-memory table gives, per cell, the number of
+//    decision boundaries below it and the single boundary inside it (Lloyd-Max boundaries of
+//    <= 4 bits are more than 1/4 apart), so every code costs one table read and one compare.
+//    A zero vector maps to z = 0, whose cell holds the boundary 0, and gets the lower code as
+//    a tie should.
 #include "tq_device.cuh"
 
 #include <type_traits>
@@ -438,9 +442,6 @@ __device__ __forceinline__ void mma_codes_store(const float (&acc)[8][2][4], int
 }
 
 constexpr int kMmaWarps = 4;
-#ifndef TQ_QUANT_MMA
-#define TQ_QUANT_MMA 1
-#endif
 
 template <bool BF16>
 __global__ void __launch_bounds__(kMmaWarps * 32, 3) quantize_mma_kernel(const FastQuantArgs a) {
@@ -645,7 +646,6 @@ cudaError_t run_fast(const FastQuantArgs &f, int sms, cudaStream_t s) {
     const unsigned blocks = (nvec + kQThreads / 32 - 1) / (kQThreads / 32);
     return launch_pdl(quantize_small_kernel<D, BF16>, dim3(blocks), dim3(kQThreads), 0, s, f);
   }
-#if TQ_QUANT_MMA
   if constexpr (D == 128) {
     const unsigned ngt = (f.t[0].nvec + 15) / 16 +
                          (f.nbatch_total > f.t[0].nbatch ? (f.t[1].nvec + 15) / 16 : 0u);
@@ -654,7 +654,6 @@ cudaError_t run_fast(const FastQuantArgs &f, int sms, cudaStream_t s) {
     return launch_pdl(quantize_mma_kernel<BF16>, dim3(static_cast<unsigned>(grid)),
                       dim3(kMmaWarps * 32), msmem, s, f);
   }
-#endif
   const int smem = 2048 + 2 * kCells * 8 + 2 * kQThreads * (2 * D + 16); // 2048: alignment slack
   cudaError_t e = cudaFuncSetAttribute(quantize_fast_kernel<D, BF16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

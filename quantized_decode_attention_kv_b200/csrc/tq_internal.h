@@ -99,6 +99,7 @@ cudaError_t launch_quantize_fast(const QuantArgs *k, const QuantArgs *v, int sm_
 // TurboQuant_prod quantiser with the QJL sketch on the tensor cores (quantize_prod.cu):
 // head_dim 64, 64 sketch rows, 1- or 2-bit records, bf16/f16 input; K and V in one launch.
 bool quantize_prod_supported(const QuantArgs &a);
+cudaError_t read_and_clear_prod_faults(unsigned *flags);
 cudaError_t launch_quantize_prod(const QuantArgs *k, const QuantArgs *v, int sm_count,
                                  cudaStream_t s);
 cudaError_t launch_dequantize(const DequantArgs &a, cudaStream_t s);

@@ -56,6 +56,7 @@ EXPORTS = {
     "tq_record_bytes": (ctypes.c_size_t, [ctypes.c_int, tq_qcfg]),
     "tq_quantize_kv": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ctypes.POINTER(tq_cache), ctypes.c_void_p]),
+    "tq_device_faults": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint)]),
     "tq_launch_counts": (ctypes.c_int, [ctypes.POINTER(tq_cache), ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "tq_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -231,6 +232,14 @@ def tq_launch_counts(cache: TQCache, dtype: torch.dtype, T: int, Hq: int, T_len:
     _check(lib.tq_launch_counts(ctypes.byref(cache.struct), dt, T, Hq, T_len, ctypes.byref(nq),
                                 ctypes.byref(nd)))
     return nq.value, nd.value
+
+
+def tq_device_faults() -> int:
+    """Device-side fault bits recorded since the last call (bit 0: a tensor-core write kernel
+    timed out waiting for its MMAs); synchronises the device and clears them."""
+    v = ctypes.c_uint(0)
+    _check(lib.tq_device_faults(ctypes.byref(v)))
+    return v.value
 
 
 def tq_decode_workspace_bytes(cache: TQCache, Hq: int, T_len: int) -> int:

@@ -255,18 +255,21 @@ def test_bf16_decode_matches_oracle(d, G, Hkv, T_len, T_cap):
     P.assert_attention_close(P.to_np(out), want)
 
 
-@pytest.mark.parametrize("d,kcfg,vcfg,m", [
-    (128, (4, O.MSE), (2, O.MSE), 0),       # streaming quantiser, 128-vector batches
-    (64, (3, O.MSE), (1, O.MSE), 0),
-    (64, (2, O.PROD), (2, O.PROD), 64),     # tensor-core sketch quantiser, 16-vector groups
-    (64, (1, O.PROD), (2, O.PROD), 64),
+@pytest.mark.parametrize("d,kcfg,vcfg,m,dtype", [
+    (128, (4, O.MSE), (2, O.MSE), 0, torch.bfloat16),   # tensor-core Hadamard, 16-vector groups
+    (128, (3, O.MSE), (2, O.MSE), 0, torch.float16),
+    (64, (3, O.MSE), (1, O.MSE), 0, torch.bfloat16),    # streaming quantiser, 128-vector batches
+    (64, (2, O.PROD), (2, O.PROD), 64, torch.bfloat16),  # tcgen05 sketch quantiser, 128-vector tiles
+    (64, (1, O.PROD), (2, O.PROD), 64, torch.bfloat16),
+    (64, (2, O.PROD), (1, O.PROD), 64, torch.float16),
 ])
-def test_bulk_quantize_with_ragged_batches_and_offset(d, kcfg, vcfg, m):
+def test_bulk_quantize_with_ragged_batches_and_offset(d, kcfg, vcfg, m, dtype):
     # 3 x 7 x 1000 = 21000 vectors per tensor: above the few-token path, and neither a whole
-    # number of 128-vector batches nor of 16-vector groups; written at offset 5 of T_cap 1010
+    # number of 128-vector batches or tiles nor of 16-vector groups; written at offset 5 of
+    # T_cap 1010
     B, Hkv, T, T_cap, t_off = 3, 7, 1000, 1010, 5
     (kb, km), (vb, vm) = kcfg, vcfg
-    K, V = _inputs(B, Hkv, T, d, torch.bfloat16, seed=d + kb + vb, outliers=True, zero_at=17)
+    K, V = _inputs(B, Hkv, T, d, dtype, seed=d + kb + vb, outliers=True, zero_at=17)
     cache = tq.TQCache(B, Hkv, T_cap, d, kb, vb, km, vm, m, m, seed=13, qjl_seed=7)
     tq.tq_quantize_kv(K.cuda(), V.cuda(), cache, t_offset=t_off)
     torch.cuda.synchronize()
@@ -277,3 +280,4 @@ def test_bulk_quantize_with_ragged_batches_and_offset(d, kcfg, vcfg, m):
         P.compare_records(cache, side, recs, t_offset=t_off, heads=heads)
     assert int(cache["k_norm"][:, :, :t_off].abs().sum()) == 0
     assert int(cache["v_norm"][:, :, t_off + T:].abs().sum()) == 0
+    assert tq.tq_device_faults() == 0
