@@ -370,119 +370,137 @@ __global__ void __launch_bounds__(kTcRows, 3) quantize_prod_tc_kernel(const Prod
   long long tile = blockIdx.x;
   uint32_t ph = 0;
   bool fault = false;
-  int cur_ti = 0;
-  if (tile < ntt) issue(tile);
-  for (; tile < ntt; tile += gridDim.x) {
-    const int ti = tile < nt0 ? 0 : 1;
-    if (ti != cur_ti) { // the sketch of the second tensor (all MMAs on the first are complete)
-      build_s(ti);
-      cur_ti = ti;
-    }
-    const ProdQuantTensor &t = a.t[ti];
-    const unsigned v0 = static_cast<unsigned>((tile - (ti ? nt0 : 0)) * kTcRows);
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    tc::fence_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    // ---- z = X (H D)^T
-    if (tid == 0) {
-#pragma unroll
-      for (int s = 0; s < 4; ++s) tc::mma_ss(tmem, dsc(kTcX, s), dsc(kTcHB, s), id_z, s > 0);
-      tc::commit(mbar0);
-    }
-    bool ok = tc::mbar_wait(mbar0, ph, kTcWaitCycles);
-    if (__syncthreads_or(!ok)) {
-      fault = true;
-      break;
-    }
-    tc::fence_after_sync();
-    if (tile + gridDim.x < ntt) issue(tile + gridDim.x); // X is free again
-    float z[64];
-    {
-      float h0[32], h1[32];
-      tc::tmem_ld32(tlane, h0);
-      tc::tmem_ld32(tlane + 32, h1);
-      tc::tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        z[i] = h0[i];
-        z[32 + i] = h1[i];
-      }
-    }
-    // ---- norm, codes (bit k = z_k > 0), residual r = (z - c^) / 8, its norm, hi/lo split
-    float ss = 0.f;
-#pragma unroll
-    for (int k = 0; k < 64; ++k) ss = fmaf(z[k], z[k], ss);
-    const float nrm = sqrtf(ss * (1.0f / 64.0f)); // ||H D x||^2 = 64 ||x||^2
-    const float inv = nrm > 0.f ? __frcp_rn(nrm) : 0.0f;
-    const float inv8 = inv * 0.125f;
+  // One phase per tensor, the record bit width a compile-time constant.
+  auto phase = [&](auto ti_tag, auto wb_tag, long long tend) {
+    constexpr int TI = decltype(ti_tag)::value, WB = decltype(wb_tag)::value;
+    const ProdQuantTensor &t = a.t[TI];
+    const unsigned T = static_cast<unsigned>(t.T);
     const uint32_t c18 = __float_as_uint(t.c1 * 0.125f);
-    const bool wb1 = t.wbits == 1;
-    uint32_t cw[2] = {0u, 0u}, rh[32], rl[32];
-    float rr = 0.f;
+    for (; tile < tend; tile += gridDim.x) {
+      const unsigned v0 = static_cast<unsigned>((tile - (TI ? nt0 : 0)) * kTcRows);
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+      // ---- z = X (H D)^T
+      if (tid == 0) {
 #pragma unroll
-    for (int k = 63; k >= 0; --k) {
-      // sign of z inv - 2^-149 is clear exactly when z inv > 0 (inv >= 0)
-      const float zs = fmaf(z[k], inv, -0x1p-149f);
-      cw[k >> 5] = __funnelshift_l(__float_as_uint(zs), cw[k >> 5], 1);
-      const float negc = wb1 ? __uint_as_float(c18 | (~__float_as_uint(zs) & 0x80000000u)) : 0.0f;
-      z[k] = fmaf(z[k], inv8, negc); // residual, unit-domain / sqrt(64)
-      rr = fmaf(z[k], z[k], rr);
-    }
+        for (int s = 0; s < 4; ++s) tc::mma_ss(tmem, dsc(kTcX, s), dsc(kTcHB, s), id_z, s > 0);
+        tc::commit(mbar0);
+      }
+      bool ok = tc::mbar_wait(mbar0, ph, kTcWaitCycles);
+      if (__syncthreads_or(!ok)) {
+        fault = true;
+        return;
+      }
+      tc::fence_after_sync();
+      if (tile + gridDim.x < ntt) issue(tile + gridDim.x); // X is free again
+      f2_t z[32];
+      {
+        float h0[32], h1[32];
+        tc::tmem_ld32(tlane, h0);
+        tc::tmem_ld32(tlane + 32, h1);
+        tc::tmem_wait_ld();
 #pragma unroll
-    for (int p = 0; p < 32; ++p) split2(z[2 * p], z[2 * p + 1], rh[p], rl[p]);
+        for (int p = 0; p < 16; ++p) {
+          z[p] = f2(h0[2 * p], h0[2 * p + 1]);
+          z[16 + p] = f2(h1[2 * p], h1[2 * p + 1]);
+        }
+      }
+      // ---- norm, codes (bit k = z_k > 0), residual r = (z - c^) / 8, its norm, hi/lo split
+      f2_t ss2 = 0ull;
 #pragma unroll
-    for (int kc = 0; kc < 8; ++kc) {
-      const uint32_t off = tc::kmajor_offset(tid, 8 * kc, kRD);
-      *reinterpret_cast<uint4 *>(sm + kTcAH + off) = make_uint4(rh[4 * kc], rh[4 * kc + 1], rh[4 * kc + 2], rh[4 * kc + 3]);
-      *reinterpret_cast<uint4 *>(sm + kTcAL + off) = make_uint4(rl[4 * kc], rl[4 * kc + 1], rl[4 * kc + 2], rl[4 * kc + 3]);
-    }
-    tc::fence_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    // ---- S r: lo terms, then hi x hi with the lo terms scaled by 2^-12
-    if (tid == 0) {
+      for (int p = 0; p < 32; ++p) ss2 = fma2(z[p], z[p], ss2);
+      float s0, s1;
+      f2_split(ss2, s0, s1);
+      const float nrm = sqrtf((s0 + s1) * (1.0f / 64.0f)); // ||H D x||^2 = 64 ||x||^2
+      const float inv = nrm > 0.f ? __frcp_rn(nrm) : 0.0f;
+      const f2_t inv2 = f2(inv, inv), inv82 = f2(inv * 0.125f, inv * 0.125f);
+      const f2_t tiny2 = f2(-0x1p-149f, -0x1p-149f);
+      uint32_t cw[2] = {0u, 0u}, rh[32], rl[32];
+      f2_t rr2 = 0ull;
 #pragma unroll
-      for (int s = 0; s < 4; ++s) tc::mma_ss(tmem, dsc(kTcAL, s), dsc(kTcSH, s), id_s, s > 0);
+      for (int p = 31; p >= 0; --p) {
+        f2_t negc2 = 0ull;
+        if constexpr (WB == 1) {
+          // the sign of z inv - 2^-149 is clear exactly when z inv > 0 (inv >= 0)
+          float za, zb;
+          f2_split(fma2(z[p], inv2, tiny2), za, zb);
+          cw[p >> 4] = __funnelshift_l(__float_as_uint(zb), cw[p >> 4], 1);
+          cw[p >> 4] = __funnelshift_l(__float_as_uint(za), cw[p >> 4], 1);
+          negc2 = f2(__uint_as_float(c18 | (~__float_as_uint(za) & 0x80000000u)),
+                     __uint_as_float(c18 | (~__float_as_uint(zb) & 0x80000000u)));
+        }
+        const f2_t r2 = fma2(z[p], inv82, negc2); // unit-domain residual / sqrt(64)
+        rr2 = fma2(r2, r2, rr2);
+        float ra, rb;
+        f2_split(r2, ra, rb);
+        split2(ra, rb, rh[p], rl[p]);
+      }
 #pragma unroll
-      for (int s = 0; s < 4; ++s) tc::mma_ss(tmem, dsc(kTcAH, s), dsc(kTcSL, s), id_s, 1);
-      tc::mma_ss_scaled<12>(tmem, dsc(kTcAH, 0), dsc(kTcSH, 0), id_s);
+      for (int kc = 0; kc < 8; ++kc) {
+        const uint32_t off = tc::kmajor_offset(tid, 8 * kc, kRD);
+        *reinterpret_cast<uint4 *>(sm + kTcAH + off) = make_uint4(rh[4 * kc], rh[4 * kc + 1], rh[4 * kc + 2], rh[4 * kc + 3]);
+        *reinterpret_cast<uint4 *>(sm + kTcAL + off) = make_uint4(rl[4 * kc], rl[4 * kc + 1], rl[4 * kc + 2], rl[4 * kc + 3]);
+      }
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+      // ---- S r: lo terms, then hi x hi with the lo terms scaled by 2^-12
+      if (tid == 0) {
 #pragma unroll
-      for (int s = 1; s < 4; ++s) tc::mma_ss(tmem, dsc(kTcAH, s), dsc(kTcSH, s), id_s, 1);
-      tc::commit(mbar1);
-    }
-    ok = tc::mbar_wait(mbar1, ph, kTcWaitCycles);
-    if (__syncthreads_or(!ok)) {
-      fault = true;
-      break;
-    }
-    tc::fence_after_sync();
-    ph ^= 1u;
-    uint32_t sg[2] = {0u, 0u};
-    {
-      float p0[32], p1[32];
-      tc::tmem_ld32(tlane, p0);
-      tc::tmem_ld32(tlane + 32, p1);
-      tc::tmem_wait_ld();
-      // bit j = (S r)_j < 0 (sign bit; an exact zero of a sum of products is +0)
+        for (int s = 0; s < 4; ++s) tc::mma_ss(tmem, dsc(kTcAL, s), dsc(kTcSH, s), id_s, s > 0);
 #pragma unroll
-      for (int j = 31; j >= 0; --j) {
-        sg[0] = __funnelshift_l(__float_as_uint(p0[j]), sg[0], 1);
-        sg[1] = __funnelshift_l(__float_as_uint(p1[j]), sg[1], 1);
+        for (int s = 0; s < 4; ++s) tc::mma_ss(tmem, dsc(kTcAH, s), dsc(kTcSL, s), id_s, 1);
+        tc::mma_ss_scaled<12>(tmem, dsc(kTcAH, 0), dsc(kTcSH, 0), id_s);
+#pragma unroll
+        for (int s = 1; s < 4; ++s) tc::mma_ss(tmem, dsc(kTcAH, s), dsc(kTcSH, s), id_s, 1);
+        tc::commit(mbar1);
+      }
+      ok = tc::mbar_wait(mbar1, ph, kTcWaitCycles);
+      if (__syncthreads_or(!ok)) {
+        fault = true;
+        return;
+      }
+      tc::fence_after_sync();
+      ph ^= 1u;
+      uint32_t sg[2] = {0u, 0u};
+      {
+        float p0[32], p1[32];
+        tc::tmem_ld32(tlane, p0);
+        tc::tmem_ld32(tlane + 32, p1);
+        tc::tmem_wait_ld();
+        // bit j = (S r)_j < 0 (sign bit; an exact zero of a sum of products is +0)
+#pragma unroll
+        for (int j = 31; j >= 0; --j) {
+          sg[0] = __funnelshift_l(__float_as_uint(p0[j]), sg[0], 1);
+          sg[1] = __funnelshift_l(__float_as_uint(p1[j]), sg[1], 1);
+        }
+      }
+      float q0, q1;
+      f2_split(rr2, q0, q1);
+      const unsigned v = v0 + tid;
+      if (v < t.nvec) {
+        const unsigned bh = v / T, tt = v - bh * T;
+        const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
+        reinterpret_cast<uint2 *>(t.signs)[rec] = make_uint2(sg[0], sg[1]);
+        if constexpr (WB == 1) reinterpret_cast<uint2 *>(t.codes)[rec] = make_uint2(~cw[0], ~cw[1]);
+        t.norm[rec] = f32_to_f16_bits(nrm);
+        t.rnorm[rec] = f32_to_f16_bits(sqrtf(q0 + q1));
       }
     }
-    const unsigned v = v0 + tid;
-    if (v < t.nvec) {
-      const unsigned T = static_cast<unsigned>(t.T);
-      const unsigned bh = v / T, tt = v - bh * T;
-      const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
-      reinterpret_cast<uint2 *>(t.signs)[rec] = make_uint2(sg[0], sg[1]);
-      if (wb1) reinterpret_cast<uint2 *>(t.codes)[rec] = make_uint2(~cw[0], ~cw[1]);
-      t.norm[rec] = f32_to_f16_bits(nrm);
-      t.rnorm[rec] = f32_to_f16_bits(sqrtf(rr));
-    }
+  };
+  using I0 = std::integral_constant<int, 0>;
+  using I1 = std::integral_constant<int, 1>;
+  if (tile < ntt) issue(tile);
+  if (a.t[0].wbits == 1) phase(I0{}, I1{}, nt0);
+  else phase(I0{}, I0{}, nt0);
+  if (!fault && a.ntensors > 1) {
+    build_s(1); // every MMA on the first tensor's sketch has completed
+    if (a.t[1].wbits == 1) phase(I1{}, I1{}, ntt);
+    else phase(I1{}, I0{}, ntt);
   }
   if (fault && tid == 0) atomicOr(&g_prod_tc_fault, 1u);
   asm volatile("cp.async.wait_all;" ::: "memory"); // own copies in flight
