@@ -109,8 +109,9 @@ struct Lut {
 
 } // namespace
 
-// Query prep: rotate once (q'' = H D q), scale (q~ = scale q'' / d), normalise by a power of
-// two so max|q^| is in [1, 2), split into fp16 hi and 2^12-scaled fp16 residual.
+// A prepared query: rotated once (q'' = H D q), scaled (q~ = scale q'' / d), normalised by a
+// power of two so max|q^| is in [1, 2), split into fp16 hi and 2^12-scaled fp16 residual. The
+// decode kernel builds one per query head of a segment in shared memory.
 struct QPrep {
   uint16_t hi[kD];
   uint16_t lo[kD];
@@ -120,55 +121,72 @@ struct QPrep {
 
 namespace {
 
-__global__ void __launch_bounds__(kD) qprep_kernel(const void *q, int dtype, float scale,
-                                                   uint64_t seed, QPrep *out) {
-  __shared__ float v[kD];
-  __shared__ float red[4];
-  const int i = threadIdx.x;
-  const size_t bq = blockIdx.x;
-  pdl_wait(); // q may come from the kernel before
-  pdl_trigger();
-  float x = load_scalar(q, dtype, bq * kD + i);
-  if (sign_is_neg(seed, i)) x = -x;
-  v[i] = x;
-  __syncthreads();
-  for (int hs = 1; hs < kD; hs <<= 1) {
-    float a = 0.f, b = 0.f;
-    const bool lower = (i & hs) == 0;
-    if (lower) {
-      a = v[i];
-      b = v[i + hs];
-    }
-    __syncthreads();
-    if (lower) {
-      v[i] = a + b;
-      v[i + hs] = a - b;
-    }
-    __syncthreads();
+// Query prep of one query by one warp: rotate (q'' = H D q), scale (q~ = scale q'' / d),
+// normalise by a power of two so max|q^| is in [1, 2), split into fp16 hi and 2^12-scaled fp16
+// residual. Lane l holds coordinates 4 l .. 4 l + 3; the butterflies of span 1, 2 run in the
+// lane, those of span 4 .. 64 across lanes (the lane with the span bit set keeps
+// partner - own).
+__device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, float scale,
+                                           uint64_t seed, QPrep *out, int lane) {
+  float x[4];
+  const uint64_t sw = dev_splitmix64(seed, static_cast<uint64_t>(lane >> 4)); // coordinates 64 k ..
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int i = 4 * lane + e;
+    x[e] = load_scalar(q, dtype, bq * kD + i);
+    if ((sw >> (i & 63)) & 1ull) x[e] = -x[e];
   }
-  const float qt = v[i] * (scale / static_cast<float>(kD));
-  float mx = warp_max(fabsf(qt));
-  if ((i & 31) == 0) red[i >> 5] = mx;
-  __syncthreads();
-  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  {
+    const float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
+    x[0] = a0 + a2;
+    x[2] = a0 - a2;
+    x[1] = a1 + a3;
+    x[3] = a1 - a3;
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
+      x[e] = upper ? o - x[e] : x[e] + o;
+    }
+  }
+  float mx = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    x[e] *= scale / static_cast<float>(kD);
+    mx = fmaxf(mx, fabsf(x[e]));
+  }
+  mx = warp_max(mx);
   float factor = 1.0f;
   if (mx > 0.f && isfinite(mx)) {
     int ex;
-    frexpf(mx, &ex);             // mx = f * 2^ex, f in [0.5, 1)
+    frexpf(mx, &ex);               // mx = f * 2^ex, f in [0.5, 1)
     factor = ldexpf(1.0f, 1 - ex); // mx * factor in [1, 2)
   }
-  const float qh = qt * factor;
-  const __half hi = __float2half_rn(qh);
-  const __half lo = __float2half_rn((qh - __half2float(hi)) * kLoScale);
-  out[bq].hi[i] = __half_as_ushort(hi);
-  out[bq].lo[i] = __half_as_ushort(lo);
-  if (i == 0) out[bq].inv = 1.0f / factor;
+  uint32_t hw[2], lw[2];
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const float q0 = x[2 * p] * factor, q1 = x[2 * p + 1] * factor;
+    const __half h0 = __float2half_rn(q0), h1 = __float2half_rn(q1);
+    const __half l0 = __float2half_rn((q0 - __half2float(h0)) * kLoScale);
+    const __half l1 = __float2half_rn((q1 - __half2float(h1)) * kLoScale);
+    hw[p] = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
+    lw[p] = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+  }
+  reinterpret_cast<uint2 *>(out->hi)[lane] = make_uint2(hw[0], hw[1]);
+  reinterpret_cast<uint2 *>(out->lo)[lane] = make_uint2(lw[0], lw[1]);
+  if (lane == 0) out->inv = 1.0f / factor;
 }
 
 struct FastArgs {
   const uint8_t *kc, *vc;
   const uint16_t *kn, *vn;
-  const QPrep *qp;
+  const void *q; // queries [B][Hq][128] of q_dtype, rotated by the kernel itself
+  int q_dtype;
+  float scale;
+  uint64_t seed;
   float *part; // partial records [cta][slot][G][stride]
   int Hq, Hkv, G, T_len, T_cap;
   int tiles_per_bh, tiles_per_cta, slots, stride;
@@ -271,17 +289,23 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
 
       // ---- B operands of the score MMA: column n = r of n-tile nt is head g = 4 nt + r/2,
       //      hi (r even) or residual (r odd); thread c holds coordinates [32c, 32c+32).
+      // ---- the segment's queries, rotated and split by warps 0 .. G-1 into the merge area
+      //      (free between segments), then read as fragments by every warp
+      QPrep *qs = reinterpret_cast<QPrep *>(obw);
+      for (int g = warp; g < a.G; g += kWarps)
+        prep_query(a.q, a.q_dtype, static_cast<size_t>(b) * a.Hq + h * a.G + g, a.scale, a.seed, qs + g, lane);
+      __syncthreads();
       uint32_t qb[NT][16];
       float qscale[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int g = nt * 4 + (r >> 1);
         if (g < a.G) {
-          const QPrep *p = a.qp + static_cast<size_t>(b) * a.Hq + h * a.G + g;
+          const QPrep *p = qs + g;
           const uint4 *src = reinterpret_cast<const uint4 *>(((r & 1) ? p->lo : p->hi) + 32 * c);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint4 w = __ldg(src + k);
+            const uint4 w = src[k];
             qb[nt][4 * k] = w.x;
             qb[nt][4 * k + 1] = w.y;
             qb[nt][4 * k + 2] = w.z;
@@ -292,8 +316,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           for (int k = 0; k < 16; ++k) qb[nt][k] = 0u;
         }
         const int gs = nt * 4 + c; // head of this lane's score columns
-        qscale[nt] = gs < a.G ? __ldg(&a.qp[static_cast<size_t>(b) * a.Hq + h * a.G + gs].inv) * kLog2e
-                              : 0.f;
+        qscale[nt] = gs < a.G ? qs[gs].inv * kLog2e : 0.f;
       }
 
       float m_run[NT], l_run[NT];
@@ -766,7 +789,8 @@ bool fast_decode_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbi
          v_wbits >= 2 && v_wbits <= 4 && G >= 1 && G <= 8;
 }
 
-// Layout of the fast path's workspace: [partials][query prep].
+// Layout of the fast path's workspace: the partial records (the kernel prepares its queries in
+// shared memory).
 void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, DecodePlan *p) {
   const int G = Hq / Hkv;
   p->path = 1;
@@ -785,21 +809,20 @@ void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, 
   p->chunk = 0;
   p->part_bytes = static_cast<size_t>(p->ctas) * p->slots * G * p->ws_stride * sizeof(float);
   p->part_bytes = (p->part_bytes + 255) / 256 * 256;
-  p->ws_bytes = p->part_bytes + static_cast<size_t>(B) * Hq * sizeof(QPrep);
+  p->ws_bytes = p->part_bytes; // the decode kernel prepares the queries in shared memory
 }
 
 cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   const DecodePlan &p = a.plan;
-  QPrep *qp = reinterpret_cast<QPrep *>(reinterpret_cast<uint8_t *>(a.ws) + p.part_bytes);
-  cudaError_t e = launch_pdl(qprep_kernel, dim3(a.B * a.Hq), dim3(kD), 0, s, a.q, a.q_dtype, a.scale,
-                             a.seed, qp);
-  if (e != cudaSuccess) return e;
   FastArgs f;
   f.kc = a.k.codes;
   f.vc = a.v.codes;
   f.kn = a.k.norm;
   f.vn = a.v.norm;
-  f.qp = qp;
+  f.q = a.q;
+  f.q_dtype = a.q_dtype;
+  f.scale = a.scale;
+  f.seed = a.seed;
   f.part = a.ws;
   f.Hq = a.Hq;
   f.Hkv = a.Hkv;
@@ -815,6 +838,7 @@ cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   for (int j = 0; j < 16; ++j) f.vcent[j] = a.v.cb.c[j];
   f.one = 1u;
   const int kb = a.k.wbits, vb = a.v.wbits;
+  cudaError_t e;
   if (kb == 4) e = vb == 2 ? run_mse<4, 2>(f, p.ctas, s) : vb == 3 ? run_mse<4, 3>(f, p.ctas, s)
                                                                  : run_mse<4, 4>(f, p.ctas, s);
   else e = vb == 2 ? run_mse<3, 2>(f, p.ctas, s) : vb == 3 ? run_mse<3, 3>(f, p.ctas, s)

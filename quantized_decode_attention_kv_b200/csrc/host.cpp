@@ -479,7 +479,9 @@ int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,
     else ++nq;
   }
   if (quantize_launches) *quantize_launches = nq + (any_fast ? 1 : 0) + (any_prod ? 1 : 0);
-  if (decode_launches) *decode_launches = fast_path(*cache, Hq) != 0 ? 3 : 2; // (query prep,) split-K, combine
+  // split-K kernel and combine; the TurboQuant_prod kernels add a query-prep kernel (the MSE
+  // tensor-core kernel and the generic kernel prepare their queries themselves)
+  if (decode_launches) *decode_launches = fast_path(*cache, Hq) == tq::kProdFast ? 3 : 2;
   return TQ_OK;
 }
 

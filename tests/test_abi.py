@@ -169,11 +169,12 @@ def _fake_cache(B, Hkv, T_cap, d, kb, km, vb, vm, m=0):
 
 
 @pytest.mark.parametrize("cfg,dtype,Hq,want", [
-    # 16-bit MSE write: one streaming launch for K and V; MSE d=128 decode: prep, decode, combine
-    ((16, 8, 32768, 128, 4, O.MSE, 2, O.MSE), 1, 32, (1, 3)),
-    ((4, 8, 1024, 128, 3, O.MSE, 3, O.MSE), 2, 32, (1, 3)),
+    # 16-bit MSE write: one launch for K and V; MSE d=128 decode: decode (which prepares its
+    # queries itself) and combine
+    ((16, 8, 32768, 128, 4, O.MSE, 2, O.MSE), 1, 32, (1, 2)),
+    ((4, 8, 1024, 128, 3, O.MSE, 3, O.MSE), 2, 32, (1, 2)),
     # fp32 input takes the per-vector kernel, one launch per tensor
-    ((1, 1, 1024, 128, 4, O.MSE, 4, O.MSE), 0, 1, (2, 3)),
+    ((1, 1, 1024, 128, 4, O.MSE, 4, O.MSE), 0, 1, (2, 2)),
     # d = 64 TurboQuant_prod with 64 sketch rows: tensor-core write and decode (G <= 2)
     ((64, 12, 8192, 64, 2, O.PROD, 2, O.PROD, 64), 1, 12, (1, 3)),
     ((64, 12, 8192, 64, 2, O.PROD, 2, O.PROD, 64), 1, 48, (1, 2)),
