@@ -40,7 +40,7 @@ constexpr float kLoScale = 4096.0f; // residual scaling 2^12 (keeps residuals no
 constexpr float kLoInv = 1.0f / 4096.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 #ifndef TQ_DECODE_PREFETCH
-#define TQ_DECODE_PREFETCH 2
+#define TQ_DECODE_PREFETCH 1
 #endif
 // A warp asks L2 for the tile it will load this many of its own steps later (0: no prefetch):
 // loads one step ahead in registers only cover part of the DRAM latency.
