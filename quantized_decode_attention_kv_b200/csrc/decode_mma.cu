@@ -13,7 +13,8 @@
 //   values  O^T[128 x heads] += V^T[128 x 16 tokens] . P'^T[16 tokens x heads]
 //     2-bit V^: one byte of nibble-interleaved codes (two tokens, two coordinates) indexes a
 //     lane-replicated shared table whose 8-byte entry is a pair of operand registers;
-//     3/4-bit V^: one table word per operand register. P' = p * ||v_t|| in fp16.
+//     3/4-bit V^: one table word per token and pair of adjacent coordinates, two PRMTs per
+//     pair of operand registers. P' = p * ||v_t|| in fp16.
 //
 // The contraction order is free along k, so each thread owns a contiguous 16-byte slice of
 // every key record and one 32-bit word of every value record: all loads are 16- or 4-byte,
@@ -89,8 +90,9 @@ struct Tile {
 // byte of two codes, 256 rows; 3-bit keys: 6 bits, 64 rows) x {32 lane copies of the fp16x2
 // hi pair, 32 of the lo pair} = 256 bytes. Value rows, 2-bit values: one byte holding the
 // codes of two adjacent coordinates of two tokens (low nibble the first token) x 32 lane
-// copies of the two fp16x2 operand words = 256 bytes; 3/4-bit values: one index (code of the
-// first token | code of the second << VB) x 32 lane copies of the fp16x2 pair = 128 bytes.
+// copies of the two fp16x2 operand words = 256 bytes; 3/4-bit values: one index (the codes of
+// two adjacent coordinates of one token, the first in the low bits) x 32 lane copies of the
+// fp16x2 pair of their centroids = 128 bytes.
 // The 3-bit key table and the 3/4-bit value tables sit at addresses aligned to their size so
 // that an index OR-ed above the lane offset is already the address.
 template <int KB, int VB>
@@ -568,8 +570,10 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
             mma16816(o[m], e01.x, e01.y, e23.x, e23.y, pb0, pb1);
           }
         } else {
-          // each operand register is one lane-replicated table word indexed by the two tokens'
-          // codes at that coordinate
+          // one lane-replicated table word per token and coordinate pair: the word indexed by a
+          // token's codes at run coordinates 2m, 2m+1 holds both centroids (fp16x2); two PRMTs
+          // turn the words of the two tokens of a k pair into the operand registers of
+          // coordinates 2m and 2m+1
           uint32_t run[4][2];
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
@@ -581,18 +585,14 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
               run[t][1] = T.v[t][1];
             }
           }
-          constexpr uint32_t MA = ((1u << VB) - 1u) << 7, MB = MA << VB;
+          constexpr uint32_t MI = ((1u << (2 * VB)) - 1u) << 7;
 #pragma unroll
           for (int m = 0; m < 8; ++m) {
-            uint32_t q[4];
+            uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i = 2 * m + (e & 1), tp = e >> 1;
-              const uint32_t ta = bits_at(run[2 * tp], VB * i, 7);
-              const uint32_t tb = bits_at(run[2 * tp + 1], VB * i, 7 + VB);
-              q[e] = lds32(lop_and_or(tb, MB, lop_and_or(ta, MA, vlb)));
-            }
-            mma16816(o[m], q[0], q[1], q[2], q[3], pb0, pb1);
+            for (int t = 0; t < 4; ++t) w[t] = lds32(lop_and_or(bits_at(run[t], 2 * VB * m, 7), MI, vlb));
+            mma16816(o[m], prmt(w[0], w[1], 0x5410u), prmt(w[0], w[1], 0x7632u), prmt(w[2], w[3], 0x5410u),
+                     prmt(w[2], w[3], 0x7632u), pb0, pb1);
           }
         }
       };
