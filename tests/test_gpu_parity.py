@@ -281,3 +281,26 @@ def test_bulk_quantize_with_ragged_batches_and_offset(d, kcfg, vcfg, m, dtype):
     assert int(cache["k_norm"][:, :, :t_off].abs().sum()) == 0
     assert int(cache["v_norm"][:, :, t_off + T:].abs().sum()) == 0
     assert tq.tq_device_faults() == 0
+
+
+@pytest.mark.parametrize("d,kcfg,vcfg,m", [
+    (128, (4, O.MSE), (2, O.MSE), 0),        # tensor-core writer, 16-vector groups
+    (64, (2, O.PROD), (1, O.PROD), 64),      # tcgen05 writer, 128-vector tiles
+])
+def test_bulk_quantize_short_context_wraps_records(d, kcfg, vcfg, m):
+    # T = 5 < 16: one 16-vector group spans several (batch, KV head) slices, so the record
+    # index wraps inside a group; 600 x 8 x 5 = 24000 vectors per tensor keeps the bulk kernels
+    B, Hkv, T, T_cap, t_off = 600, 8, 5, 9, 3
+    (kb, km), (vb, vm) = kcfg, vcfg
+    K, V = _inputs(B, Hkv, T, d, torch.bfloat16, seed=77 + d, outliers=True)
+    cache = tq.TQCache(B, Hkv, T_cap, d, kb, vb, km, vm, m, m, seed=17, qjl_seed=9)
+    tq.tq_quantize_kv(K.cuda(), V.cuda(), cache, t_offset=t_off)
+    torch.cuda.synchronize()
+    heads = [(0, 0), (0, 7), (1, 2), (299, 4), (599, 7)]
+    for side, X, bits, mode in (("k", K, kb, km), ("v", V, vb, vm)):
+        Xn = P.to_np(X)
+        recs = [P.oracle_records(Xn[b:b + 1, h:h + 1], bits, mode, 17, 9, m or None)[0] for b, h in heads]
+        P.compare_records(cache, side, recs, t_offset=t_off, heads=heads)
+    assert int(cache["k_norm"][:, :, :t_off].abs().sum()) == 0
+    assert int(cache["v_norm"][:, :, t_off + T:].abs().sum()) == 0
+    assert tq.tq_device_faults() == 0
