@@ -160,6 +160,22 @@ int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale
 int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, float scale,
                                 const tq_cache *cache, float *out, void *stream);
 
+/* Ragged decode (the sequences of one batch have different context lengths): like
+ * tq_decode_attention, but sequence b attends to its first T_lens[b] cached
+ * positions. T_lens is a HOST array of B = cache->B ints, each in 1..T_cap; it is read during
+ * the call only (the lengths travel to the kernels as launch parameters, so a captured graph
+ * keeps the values of the capture). The work is split evenly over the ragged (sequence, KV
+ * head, 16-token tile) space. Supported for the tensor-core MSE configuration (d = 128, MSE
+ * keys of 3/4 bits, MSE values of 2..4 bits, at most 8 query heads per KV head) with
+ * B <= 512; other configurations return TQ_ERR_UNSUPPORTED. Workspace size from
+ * tq_decode_varlen_workspace_bytes (0 on invalid arguments). Errors as tq_decode_attention.
+ * This extends the pages' decode ("Where This Fits in the Inference Stack": real serving
+ * batches sequences of different lengths). */
+size_t tq_decode_varlen_workspace_bytes(int Hq, const tq_cache *cache, const int *T_lens);
+int tq_decode_attention_varlen(const void *q, int dtype, int Hq, const int *T_lens, float scale,
+                               const tq_cache *cache, float *out, void *ws, size_t ws_bytes,
+                               void *stream);
+
 /* How many kernels tq_quantize_kv (K and V both given, `dtype` input, T new positions) and
  * tq_decode_attention (Hq query heads over T_len positions) launch for this cache on the
  * current device. The pages have no counterpart to this call; benchmarks use it to count the

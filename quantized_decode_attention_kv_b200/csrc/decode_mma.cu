@@ -29,6 +29,7 @@
 #include "mma_ops.cuh"
 
 #include <algorithm>
+#include <vector>
 #include <mutex>
 #include <type_traits>
 
@@ -196,7 +197,18 @@ struct FastArgs {
   float kcent[16];
   float vcent[16];
   uint32_t one;
+  int B;
 };
+
+// A ragged call's launch parameters: the common ones and the per-sequence lengths (kept out of
+// the uniform kernels' parameters, which travel with every launch).
+struct FastArgsV {
+  FastArgs a;
+  VarLen vl;
+};
+struct NoVarLen {};
+__device__ __forceinline__ const FastArgs &base_args(const FastArgs &a) { return a; }
+__device__ __forceinline__ const FastArgs &base_args(const FastArgsV &a) { return a.a; }
 
 // Bits [o, o + n) of the little-endian bit string w[0..NWD) moved to bit DST (other bits
 // of the result are unspecified above DST + n and zero below DST when o >= DST).
@@ -216,9 +228,10 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32
   return d;
 }
 
-template <int KB, int VB, int NT>
+template <int KB, int VB, int NT, bool RAG>
 __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
-    decode_mse_kernel(const FastArgs a) {
+    decode_mse_kernel(const std::conditional_t<RAG, FastArgsV, FastArgs> args) {
+  const FastArgs &a = base_args(args);
   using L = Lut<KB, VB>;
   using C = Cfg<KB, VB>;
   constexpr int kWarps = C::kWarps, kThreads = C::kThreads, kStep = C::kStep;
@@ -281,10 +294,27 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
     const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
     const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
     int slot = 0;
+    [[maybe_unused]] int vb = 0; // ragged calls: the sequence of the current segment
+    if constexpr (RAG)
+      while (vb + 1 < a.B && args.vl.boff[vb + 1] <= range0) ++vb;
     for (long long seg = range0; seg < range1; ++slot) {
-      const long long bh = seg / a.tiles_per_bh;
-      const long long seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
-      const int tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+      long long bh, seg_end;
+      int tile0, T_len;
+      if constexpr (RAG) {
+        while (vb + 1 < a.B && args.vl.boff[vb + 1] <= seg) ++vb;
+        T_len = args.vl.blen[vb];
+        const int tpb = (T_len + 15) >> 4;
+        const long long local = seg - args.vl.boff[vb];
+        const int hh = static_cast<int>(local / tpb);
+        tile0 = static_cast<int>(local - static_cast<long long>(hh) * tpb);
+        bh = static_cast<long long>(vb) * a.Hkv + hh;
+        seg_end = min(range1, args.vl.boff[vb] + static_cast<long long>(hh + 1) * tpb);
+      } else {
+        T_len = a.T_len;
+        bh = seg / a.tiles_per_bh;
+        seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
+        tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+      }
       const int ntiles = static_cast<int>(seg_end - seg);
       seg = seg_end;
       const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
@@ -332,7 +362,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
 
       const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
-      const int tlast = a.T_len - 1;
+      const int tlast = T_len - 1;
       // word offset of this lane's value run within a record (3-bit runs start mid-word for odd r)
       constexpr int kVWordOff = 0;
       const int vwo = VB == 2 ? r : (VB == 4 ? 2 * r : (3 * r) >> 1);
@@ -384,13 +414,13 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
       auto load_next = [&](TileT &T) {
         if (kPrefetchSteps > 0) {
-          if (lane < KL + VL + 2 && tpf + 16 <= a.T_len && tpf < (tile0 + ntiles) * 16)
+          if (lane < KL + VL + 2 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16)
             asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
           pfp += pfstep;
           tpf += kWarps * 16;
         }
         const int t0 = (tile0 + jl) * 16;
-        if (t0 + 16 <= a.T_len) {
+        if (t0 + 16 <= T_len) {
           load_k(T.k[0], kp);
           load_k(T.k[1], kp + 8 * KR);
           load_v(T.v[0], vp);
@@ -484,7 +514,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
         const float kn1 = f16_bits_to_f32(T.kn[1]);
         const float vn0 = f16_bits_to_f32(T.vn[0]);
         const float vn1 = f16_bits_to_f32(T.vn[1]);
-        const bool ok0 = t0 + r < a.T_len, ok1 = t0 + r + 8 < a.T_len;
+        const bool ok0 = t0 + r < T_len, ok1 = t0 + r + 8 < T_len;
         uint32_t pk[NT];
         float alpha[NT];
         bool rescale = false;
@@ -686,10 +716,12 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
 // the maximum and sum of partial k, so the merge weights need one round of loads; lane l then
 // owns output coordinates [4 l, 4 l + 4) and the Walsh-Hadamard butterflies of span >= 4 run
 // across lanes with shuffles.
+template <bool RAG>
 __global__ void __launch_bounds__(128) combine_fast_kernel(const float *part, int B, int Hkv, int G,
                                                            int tiles_per_bh, int tiles_per_cta,
                                                            int slots, int stride, uint64_t seed,
-                                                           float *out) {
+                                                           float *out,
+                                                           const std::conditional_t<RAG, VarLen, NoVarLen> vl) {
   const int lane = threadIdx.x & 31;
   const int Hq = Hkv * G;
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5); // (b, q-head) of this warp
@@ -698,10 +730,31 @@ __global__ void __launch_bounds__(128) combine_fast_kernel(const float *part, in
   const int b = gw / Hq, hq = gw - b * Hq;
   const int h = hq / G, g = hq - h * G;
   const long long bh = static_cast<long long>(b) * Hkv + h;
-  const long long first = bh * tiles_per_bh, last = first + tiles_per_bh - 1;
+  // the (b, KV head) of flattened tile f (ragged calls: sequence by binary search)
+  auto bh_of = [&](long long f) -> long long {
+    if constexpr (!RAG) {
+      return f / tiles_per_bh;
+    } else {
+      int lo = 0, hi = B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (vl.boff[mid] <= f) lo = mid;
+        else hi = mid - 1;
+      }
+      const int tpb = (vl.blen[lo] + 15) >> 4;
+      return static_cast<long long>(lo) * Hkv + (f - vl.boff[lo]) / tpb;
+    }
+  };
+  int tpb = tiles_per_bh;
+  long long first = bh * tiles_per_bh;
+  if constexpr (RAG) {
+    tpb = (vl.blen[b] + 15) >> 4;
+    first = vl.boff[b] + static_cast<long long>(h) * tpb;
+  }
+  const long long last = first + tpb - 1;
   const int cta0 = static_cast<int>(first / tiles_per_cta), cta1 = static_cast<int>(last / tiles_per_cta);
   auto rec = [&](int cta) {
-    const long long bh0 = static_cast<long long>(cta) * tiles_per_cta / tiles_per_bh;
+    const long long bh0 = bh_of(static_cast<long long>(cta) * tiles_per_cta);
     return part + ((static_cast<size_t>(cta) * slots + (bh - bh0)) * G + g) * stride;
   };
   float M = -INFINITY;
@@ -774,10 +827,20 @@ int mse_ctas_per_sm(int kb, int vb) {
 }
 
 template <int KB, int VB>
-cudaError_t run_mse(const FastArgs &f, int ctas, cudaStream_t s) {
+cudaError_t run_mse(const FastArgs &f, const VarLen *vl, int ctas, cudaStream_t s) {
   constexpr int smem = Lut<KB, VB>::kSmem;
-  auto kern = f.G <= 4 ? decode_mse_kernel<KB, VB, 1> : decode_mse_kernel<KB, VB, 2>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e;
+  if (vl) {
+    auto kern = f.G <= 4 ? decode_mse_kernel<KB, VB, 1, true> : decode_mse_kernel<KB, VB, 2, true>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    FastArgsV fv;
+    fv.a = f;
+    fv.vl = *vl;
+    return launch_pdl(kern, dim3(ctas), dim3(Cfg<KB, VB>::kThreads), smem, s, fv);
+  }
+  auto kern = f.G <= 4 ? decode_mse_kernel<KB, VB, 1, false> : decode_mse_kernel<KB, VB, 2, false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(ctas), dim3(Cfg<KB, VB>::kThreads), smem, s, f);
 }
@@ -791,20 +854,38 @@ bool fast_decode_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbi
 
 // Layout of the fast path's workspace: the partial records (the kernel prepares its queries in
 // shared memory).
-void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, DecodePlan *p) {
+void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, DecodePlan *p,
+               const int *T_lens) {
   const int G = Hq / Hkv;
   p->path = 1;
   p->tile = 16;
   p->gc = G;
   p->ws_stride = 2 + kD + 2; // 132 floats
   p->tiles_per_bh = (T_len + 15) / 16;
-  const long long total = static_cast<long long>(B) * Hkv * p->tiles_per_bh;
+  long long total = static_cast<long long>(B) * Hkv * p->tiles_per_bh;
+  if (T_lens) {
+    total = 0;
+    for (int b = 0; b < B; ++b) total += static_cast<long long>(Hkv) * ((T_lens[b] + 15) / 16);
+  }
   long long ctas = static_cast<long long>(sm_count) * mse_ctas_per_sm(kb, vb);
   ctas = std::min<long long>(ctas, (total + 7) / 8); // at least 8 tiles per CTA
   ctas = std::max<long long>(ctas, 1);
   p->tiles_per_cta = static_cast<int>((total + ctas - 1) / ctas);
   p->ctas = static_cast<int>((total + p->tiles_per_cta - 1) / p->tiles_per_cta);
   p->slots = (p->tiles_per_cta + p->tiles_per_bh - 1) / p->tiles_per_bh + 1;
+  if (T_lens) { // the most (b, KV head) segments any CTA's range touches
+    std::vector<int> nseg(p->ctas, 0);
+    long long off = 0;
+    for (int b = 0; b < B; ++b) {
+      const int tpb = (T_lens[b] + 15) / 16;
+      for (int h = 0; h < Hkv; ++h, off += tpb) {
+        const int c0 = static_cast<int>(off / p->tiles_per_cta);
+        const int c1 = static_cast<int>((off + tpb - 1) / p->tiles_per_cta);
+        for (int c = c0; c <= c1; ++c) ++nseg[c];
+      }
+    }
+    p->slots = *std::max_element(nseg.begin(), nseg.end());
+  }
   p->splits = 0;
   p->chunk = 0;
   p->part_bytes = static_cast<size_t>(p->ctas) * p->slots * G * p->ws_stride * sizeof(float);
@@ -837,16 +918,32 @@ cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   for (int j = 0; j < 16; ++j) f.kcent[j] = a.k.cb.c[j];
   for (int j = 0; j < 16; ++j) f.vcent[j] = a.v.cb.c[j];
   f.one = 1u;
+  f.B = a.B;
+  VarLen vl;
+  const VarLen *vlp = nullptr;
+  if (a.T_lens) {
+    vl.on = 1;
+    vl.boff[0] = 0;
+    for (int b = 0; b < a.B; ++b) {
+      vl.blen[b] = a.T_lens[b];
+      vl.boff[b + 1] = vl.boff[b] + a.Hkv * ((a.T_lens[b] + 15) / 16);
+    }
+    vlp = &vl;
+  }
   const int kb = a.k.wbits, vb = a.v.wbits;
   cudaError_t e;
-  if (kb == 4) e = vb == 2 ? run_mse<4, 2>(f, p.ctas, s) : vb == 3 ? run_mse<4, 3>(f, p.ctas, s)
-                                                                 : run_mse<4, 4>(f, p.ctas, s);
-  else e = vb == 2 ? run_mse<3, 2>(f, p.ctas, s) : vb == 3 ? run_mse<3, 3>(f, p.ctas, s)
-                                                          : run_mse<3, 4>(f, p.ctas, s);
+  if (kb == 4) e = vb == 2 ? run_mse<4, 2>(f, vlp, p.ctas, s) : vb == 3 ? run_mse<4, 3>(f, vlp, p.ctas, s)
+                                                                      : run_mse<4, 4>(f, vlp, p.ctas, s);
+  else e = vb == 2 ? run_mse<3, 2>(f, vlp, p.ctas, s) : vb == 3 ? run_mse<3, 3>(f, vlp, p.ctas, s)
+                                                               : run_mse<3, 4>(f, vlp, p.ctas, s);
   if (e != cudaSuccess) return e;
-  return launch_pdl(combine_fast_kernel, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
+  if (vlp)
+    return launch_pdl(combine_fast_kernel<true>, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
+                      static_cast<const float *>(a.ws), a.B, a.Hkv, f.G, p.tiles_per_bh,
+                      p.tiles_per_cta, p.slots, p.ws_stride, a.seed, a.out, vl);
+  return launch_pdl(combine_fast_kernel<false>, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
                     static_cast<const float *>(a.ws), a.B, a.Hkv, f.G, p.tiles_per_bh,
-                    p.tiles_per_cta, p.slots, p.ws_stride, a.seed, a.out);
+                    p.tiles_per_cta, p.slots, p.ws_stride, a.seed, a.out, NoVarLen{});
 }
 
 } // namespace tq

@@ -400,6 +400,84 @@ int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale
   return cuda_status(tq::launch_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
 }
 
+// Ragged decode: validation shared by the size query and the call. Returns TQ_OK and the
+// longest length, or an error.
+static int check_varlen(const tq_cache *cache, int Hq, const int *T_lens, int *T_max) {
+  int st = check_cache(cache);
+  if (st) return st;
+  if (Hq < 1 || Hq % cache->Hkv || Hq > 65535)
+    return fail(TQ_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d (<= 65535)", Hq,
+                cache->Hkv);
+  if (!T_lens) return fail(TQ_ERR_INVALID_ARG, "T_lens is NULL");
+  if (cache->B > tq::kMaxVarlenB)
+    return fail(TQ_ERR_UNSUPPORTED, "ragged decode supports B <= %d, got %d", tq::kMaxVarlenB, cache->B);
+  int mx = 0;
+  for (int b = 0; b < cache->B; ++b) {
+    if (T_lens[b] < 1 || T_lens[b] > cache->T_cap)
+      return fail(TQ_ERR_INVALID_ARG, "T_lens[%d]=%d must be in 1..T_cap=%d", b, T_lens[b], cache->T_cap);
+    mx = std::max(mx, T_lens[b]);
+  }
+  const int fp = fast_path(*cache, Hq);
+  if (fp == 0 || fp == tq::kProdFast)
+    return fail(TQ_ERR_UNSUPPORTED, "ragged decode needs the tensor-core MSE configuration "
+                                    "(d = 128, MSE, 3/4-bit K, 2..4-bit V, <= 8 query heads per KV head)");
+  *T_max = mx;
+  return TQ_OK;
+}
+
+size_t tq_decode_varlen_workspace_bytes(int Hq, const tq_cache *cache, const int *T_lens) {
+  int mx = 0;
+  if (check_varlen(cache, Hq, T_lens, &mx)) return 0;
+  int sms = sm_count();
+  if (sms <= 0) {
+    fail(TQ_ERR_CUDA, "cannot query the device's SM count");
+    return 0;
+  }
+  tq::DecodePlan p{};
+  const int fp = fast_path(*cache, Hq);
+  tq::plan_fast(cache->B, Hq, cache->Hkv, mx, sms, fp >> 4, fp & 15, &p, T_lens);
+  return p.ws_bytes;
+}
+
+int tq_decode_attention_varlen(const void *q, int dtype, int Hq, const int *T_lens, float scale,
+                               const tq_cache *cache, float *out, void *ws, size_t ws_bytes,
+                               void *stream) {
+  int mx = 0;
+  int st = check_varlen(cache, Hq, T_lens, &mx);
+  if (st) return st;
+  if (!dtype_ok(dtype)) return fail(TQ_ERR_INVALID_ARG, "dtype=%d is not F32/BF16/F16", dtype);
+  if (!q || !out || !aligned16(q) || !aligned16(out))
+    return fail(TQ_ERR_INVALID_ARG, "q/out must be non-NULL and 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale is not finite");
+  tq::DecodeArgs a;
+  std::memset(&a, 0, sizeof a);
+  st = resolve_tensor(*cache, 0, &a.k);
+  if (st) return st;
+  st = resolve_tensor(*cache, 1, &a.v);
+  if (st) return st;
+  int sms = sm_count();
+  if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
+  const int fp = fast_path(*cache, Hq);
+  tq::plan_fast(cache->B, Hq, cache->Hkv, mx, sms, fp >> 4, fp & 15, &a.plan, T_lens);
+  if (!ws || !aligned16(ws) || ws_bytes < a.plan.ws_bytes)
+    return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
+                a.plan.ws_bytes, ws ? ws_bytes : 0);
+  a.T_lens = T_lens;
+  a.q = q;
+  a.q_dtype = dtype;
+  a.B = cache->B;
+  a.Hq = Hq;
+  a.Hkv = cache->Hkv;
+  a.d = cache->d;
+  a.T_len = mx;
+  a.T_cap = cache->T_cap;
+  a.scale = scale;
+  a.seed = cache->seed;
+  a.out = out;
+  a.ws = static_cast<float *>(ws);
+  return cuda_status(tq::launch_fast_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
+}
+
 int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, float scale,
                                 const tq_cache *cache, float *out, void *stream) {
   // Same arguments and checks as tq_decode_attention, minus the workspace: the split-K

@@ -65,7 +65,18 @@ struct DecodePlan {
   size_t ws_bytes;
 };
 
+// Per-sequence context lengths of a ragged decode call, passed by value to the kernels: the
+// flattened (b, KV head, 16-token tile) space gives sequence b ceil(len[b] / 16) tiles per KV
+// head, starting at tile boff[b].
+constexpr int kMaxVarlenB = 512;
+struct VarLen {
+  int on; // 0: every sequence has the call's T_len
+  int boff[kMaxVarlenB + 1];
+  int blen[kMaxVarlenB];
+};
+
 struct DecodeArgs {
+  const int *T_lens; // host array of B per-sequence lengths, or NULL (uniform T_len)
   const void *q;
   int q_dtype;
   int B, Hq, Hkv, d, T_len, T_cap;
@@ -120,7 +131,9 @@ DecodePlan plan_decode(int B, int Hq, int Hkv, int d, int T_len, int v_m, int sm
 // Tensor-core decode (decode_mma.cu): head_dim 128, MSE keys of 3 or 4 bits, MSE values of
 // 2, 3 or 4 bits, 1..8 query heads per KV head.
 bool fast_decode_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G);
-void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, DecodePlan *p);
+// T_lens: NULL (every sequence T_len long) or B per-sequence lengths (ragged call).
+void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, DecodePlan *p,
+               const int *T_lens = nullptr);
 cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s);
 
 // Tensor-core decode of TurboQuant_prod records (decode_prod.cu): head_dim 64, 2-bit keys and

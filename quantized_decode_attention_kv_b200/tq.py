@@ -64,6 +64,12 @@ EXPORTS = {
     "tq_decode_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_float, ctypes.POINTER(tq_cache), ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tq_decode_varlen_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.POINTER(tq_cache),
+                                                           ctypes.c_void_p]),
+    "tq_decode_attention_varlen": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_void_p, ctypes.c_float, ctypes.POINTER(tq_cache),
+                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                                  ctypes.c_void_p]),
     "tq_decode_attention_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, ctypes.c_float, ctypes.POINTER(tq_cache),
                                                    ctypes.c_void_p, ctypes.c_void_p]),
@@ -257,6 +263,32 @@ def tq_decode_attention(q: torch.Tensor, cache: TQCache, T_len: int, scale: floa
     _check(lib.tq_decode_attention(_dev(q, "q"), dt, q.shape[1], T_len, scale, ctypes.byref(cache.struct),
                                    _dev(out, "out"), _dev(ws, "ws"), ws.numel() * ws.element_size(),
                                    _stream(stream)))
+
+
+def _lens(T_lens) -> ctypes.Array:
+    vals = [int(t) for t in T_lens]
+    return (ctypes.c_int * len(vals))(*vals)
+
+
+def tq_decode_varlen_workspace_bytes(cache: TQCache, Hq: int, T_lens) -> int:
+    """Workspace bytes of a ragged decode call (T_lens: B per-sequence context lengths)."""
+    lens = _lens(T_lens)
+    n = int(lib.tq_decode_varlen_workspace_bytes(Hq, ctypes.byref(cache.struct), ctypes.cast(lens, ctypes.c_void_p)))
+    if n == 0:
+        raise TQError(TQ_ERR_INVALID_ARG, last_error())
+    return n
+
+
+def tq_decode_attention_varlen(q: torch.Tensor, cache: TQCache, T_lens, scale: float, out: torch.Tensor,
+                               ws: torch.Tensor, stream=None) -> None:
+    """Decode attention where sequence b attends to its first T_lens[b] cached positions."""
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise TQError(TQ_ERR_INVALID_ARG, f"unsupported dtype {q.dtype}")
+    lens = _lens(T_lens)
+    _check(lib.tq_decode_attention_varlen(_dev(q, "q"), dt, q.shape[1], ctypes.cast(lens, ctypes.c_void_p),
+                                          scale, ctypes.byref(cache.struct), _dev(out, "out"), _dev(ws, "ws"),
+                                          ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def tq_decode_attention_noalloc(q: torch.Tensor, cache: TQCache, T_len: int, scale: float,

@@ -197,3 +197,28 @@ def test_launch_counts_reject_bad_arguments():
     assert tq.lib.tq_launch_counts(ctypes.byref(c), 7, 1, 2, 5, ctypes.byref(n), None) == tq.TQ_ERR_INVALID_ARG
     assert tq.lib.tq_launch_counts(ctypes.byref(c), 1, 1, 3, 5, ctypes.byref(n), None) == tq.TQ_ERR_INVALID_ARG
     assert tq.lib.tq_launch_counts(ctypes.byref(c), 1, 1, 2, 11, ctypes.byref(n), None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_varlen_decode_validates_before_any_device_work():
+    c = _fake_cache(3, 2, 64, 128, 4, O.MSE, 2, O.MSE)
+    lens = (ctypes.c_int * 3)(10, 0, 5)
+    out = ctypes.c_void_p(0x100000)
+    st = tq.lib.tq_decode_attention_varlen(out, 1, 8, ctypes.cast(lens, ctypes.c_void_p), 0.1,
+                                           ctypes.byref(c), out, out, 1 << 20, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "T_lens[1]" in tq.last_error()
+    lens[1] = 65  # above T_cap
+    assert tq.lib.tq_decode_attention_varlen(out, 1, 8, ctypes.cast(lens, ctypes.c_void_p), 0.1,
+                                             ctypes.byref(c), out, out, 1 << 20, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_decode_attention_varlen(out, 1, 8, None, 0.1, ctypes.byref(c), out, out, 1 << 20,
+                                             None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_decode_varlen_workspace_bytes(8, ctypes.byref(c), None) == 0
+    # TurboQuant_prod records and head_dim 64 have no ragged kernel
+    p = _fake_cache(3, 2, 64, 64, 2, O.PROD, 2, O.PROD, 64)
+    lens[1] = 7
+    assert tq.lib.tq_decode_attention_varlen(out, 1, 4, ctypes.cast(lens, ctypes.c_void_p), 0.1,
+                                             ctypes.byref(p), out, out, 1 << 20, None) == tq.TQ_ERR_UNSUPPORTED
+    # more sequences than one launch's parameters carry
+    big = _fake_cache(513, 1, 16, 128, 4, O.MSE, 2, O.MSE)
+    many = (ctypes.c_int * 513)(*([4] * 513))
+    assert tq.lib.tq_decode_attention_varlen(out, 1, 4, ctypes.cast(many, ctypes.c_void_p), 0.1,
+                                             ctypes.byref(big), out, out, 1 << 20, None) == tq.TQ_ERR_UNSUPPORTED
