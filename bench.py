@@ -302,6 +302,8 @@ def run_ours(args):
         line["quantize"] = side["quantize"]
         line["bf16_decode"] = side["bf16"]
         line["speedup_vs_bf16"] = side["bf16"]["us"] / (side["decode_s"] * 1e6)
+        if "ragged" in side:
+            line["ragged_decode"] = side["ragged"]
     print(json.dumps(line), flush=True)
 
 
@@ -341,6 +343,25 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
                        "bytes": bbytes}
     else:
         res["bf16"] = {"us": float("nan")}
+    # ragged batch of the same shape: sequence b attends to its first T_lens[b] positions
+    # (seeded lengths in [T/4, T]); bytes are the packed records actually read. The padded
+    # alternative is the uniform call at the longest length, masking nothing.
+    if w.d == 128 and w.k_mode == 0 and w.v_mode == 0 and w.B <= 512:
+        import random
+        rnd = random.Random(1234)
+        lens = [rnd.randint(w.T // 4, w.T) for _ in range(w.B)]
+        per_tok = packed // (w.B * w.T)
+        rbytes = sum(lens) * per_tok
+        wsr = tq.workspace(tq.tq_decode_varlen_workspace_bytes(cache, w.Hq, lens))
+        rs = _time(lambda: tq.tq_decode_attention_varlen(q, cache, lens, w.scale, out, wsr, stream=stream),
+                   stream, max(args.steps // 4, 20), torch)
+        wsp = tq.workspace(tq.tq_decode_workspace_bytes(cache, w.Hq, max(lens)))
+        ps = _time(lambda: tq.tq_decode_attention(q, cache, max(lens), w.scale, out, wsp, stream=stream),
+                   stream, max(args.steps // 4, 20), torch)
+        res["ragged"] = {"us": rs * 1e6, "gbs": rbytes / rs / 1e9, "frac": rbytes / rs / 1e9 / hbm,
+                         "bytes": rbytes, "lengths": f"{w.B} sequences, seeded uniform in [T/4, T], "
+                                                    f"min {min(lens)}, max {max(lens)}, sum {sum(lens)}",
+                         "padded_uniform_us": ps * 1e6}
     # end to end through the C ABI from pinned host buffers, as a serving loop runs it: every
     # step copies its inputs (query, the new token's K and V) in from pinned memory, runs the
     # two calls and reads its attention output back; the copies run on their own streams and
