@@ -86,6 +86,25 @@ typedef struct {
   const float *k_qjl, *v_qjl;
 } tq_cache;
 
+/* A paged compressed KV cache (one layer): records live in pages of page_size positions
+ * (a power of two, >= 16) drawn from a pool the caller manages; row b of the block table
+ * maps sequence b's logical page j (positions [j page_size, (j+1) page_size)) to a physical
+ * page. All pointers are device pointers owned by the caller. Per tensor:
+ *   codes  [num_pages][Hkv][page_size][tq_code_bytes]  uint8   Lloyd-Max codes
+ *   norm   [num_pages][Hkv][page_size]                 uint16  fp16 bits of ||x||
+ *   block_table [B][max_pages]                         int32   physical page of each logical
+ *                                                              page (entries in 0..num_pages-1)
+ * Supported: head_dim 128, TurboQuant_mse keys and values (3/4-bit keys, 2..4-bit values for
+ * decode). A sequence may hold at most max_pages * page_size positions. */
+typedef struct {
+  int B, Hkv, d, page_size, num_pages, max_pages;
+  uint64_t seed;
+  tq_qcfg kc, vc;
+  uint8_t *k_codes, *v_codes;
+  uint16_t *k_norm, *v_norm;
+  const int32_t *block_table;
+} tq_paged_cache;
+
 /* Message for the last failure on the calling thread ("" if none). */
 const char *tq_last_error(void);
 
@@ -198,6 +217,22 @@ size_t tq_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int T_len, int d);
 int tq_decode_attention_bf16(const void *q, int Hq, const void *K, const void *V, int B,
                              int Hkv, int T_cap, int T_len, int d, float scale, float *out,
                              void *ws, size_t ws_bytes, void *stream);
+
+/* Paged counterparts of tq_quantize_kv and tq_decode_attention_varlen: the same
+ * computation, with record (b, h, t) at page block_table[b][t / page_size], head h, slot
+ * t % page_size. tq_quantize_kv_paged takes 16-bit K, V [B][Hkv][T][d] and writes positions
+ * t_offset .. t_offset + T - 1 of every sequence (their pages must be mapped). The decode takes
+ * per-sequence lengths (host array, 1..max_pages * page_size). Errors: TQ_ERR_INVALID_ARG
+ * (shapes, pointers, page size, lengths), TQ_ERR_UNSUPPORTED (other d, modes or dtypes),
+ * TQ_ERR_WORKSPACE, TQ_ERR_CUDA; nothing is launched on error. The block-table entries are
+ * read by the kernels and must be valid page indices. These extend the pages' decode
+ * ("Where This Fits in the Inference Stack": PagedAttention allocates the cache this way). */
+int tq_quantize_kv_paged(const void *K, const void *V, int dtype, int T, int t_offset,
+                         const tq_paged_cache *cache, void *stream);
+size_t tq_decode_paged_workspace_bytes(int Hq, const tq_paged_cache *cache, const int *T_lens);
+int tq_decode_attention_paged(const void *q, int dtype, int Hq, const int *T_lens, float scale,
+                              const tq_paged_cache *cache, float *out, void *ws, size_t ws_bytes,
+                              void *stream);
 
 /* Device-side faults recorded since the last call, as bits: bit 0 = a tensor-core kernel
  * (tcgen05 write path of TurboQuant_prod records) gave up waiting for its MMAs after about a

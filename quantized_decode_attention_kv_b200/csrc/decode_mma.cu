@@ -198,6 +198,8 @@ struct FastArgs {
   float vcent[16];
   uint32_t one;
   int B;
+  const int *bt; // paged cache: block table [B][maxp]; record (b, h, t) at page bt[b][t >> pshift]
+  int pshift, maxp;
 };
 
 // A ragged call's launch parameters: the common ones and the per-sequence lengths (kept out of
@@ -228,9 +230,12 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32
   return d;
 }
 
-template <int KB, int VB, int NT, bool RAG>
+// MODE 0: dense cache, one T_len; 1: dense cache, per-sequence lengths; 2: paged cache,
+// per-sequence lengths.
+template <int KB, int VB, int NT, int MODE>
 __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
-    decode_mse_kernel(const std::conditional_t<RAG, FastArgsV, FastArgs> args) {
+    decode_mse_kernel(const std::conditional_t<MODE != 0, FastArgsV, FastArgs> args) {
+  constexpr bool RAG = MODE != 0, PG = MODE == 2;
   const FastArgs &a = base_args(args);
   using L = Lut<KB, VB>;
   using C = Cfg<KB, VB>;
@@ -361,7 +366,16 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
 #pragma unroll
       for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
 
-      const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
+      const size_t rec0 = PG ? 0 : static_cast<size_t>(bh) * a.T_cap;
+      // record index of token t0 (a multiple of 16: a tile never straddles a page)
+      [[maybe_unused]] auto tile_rec = [&](int t0) -> long long {
+        if constexpr (PG) {
+          const int page = __ldg(a.bt + static_cast<size_t>(b) * a.maxp + (t0 >> a.pshift));
+          return ((static_cast<long long>(page) * a.Hkv + h) << a.pshift) + (t0 & ((1 << a.pshift) - 1));
+        } else {
+          return static_cast<long long>(rec0) + t0;
+        }
+      };
       const int tlast = T_len - 1;
       // word offset of this lane's value run within a record (3-bit runs start mid-word for odd r)
       constexpr int kVWordOff = 0;
@@ -414,12 +428,27 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
       auto load_next = [&](TileT &T) {
         if (kPrefetchSteps > 0) {
-          if (lane < KL + VL + 2 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16)
+          if (lane < KL + VL + 2 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16) {
+            if constexpr (PG) {
+              const long long rp = tile_rec(tpf);
+              pfp = lane < KL ? reinterpret_cast<const char *>(a.kc + rp * KR + 128 * lane)
+                    : lane < KL + VL ? reinterpret_cast<const char *>(a.vc + rp * VR + 128 * (lane - KL))
+                                     : reinterpret_cast<const char *>((lane == KL + VL ? a.kn : a.vn) + rp);
+            }
             asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
+          }
           pfp += pfstep;
           tpf += kWarps * 16;
         }
         const int t0 = (tile0 + jl) * 16;
+        [[maybe_unused]] long long rb = 0;
+        if constexpr (PG) {
+          rb = tile_rec(t0);
+          kp = a.kc + (rb + r) * KR + 4 * KB * c;
+          vp = a.vc + (rb + c) * VR + 4 * vwo;
+          knp = a.kn + rb + r;
+          vnp = a.vn + rb + r;
+        }
         if (t0 + 16 <= T_len) {
           load_k(T.k[0], kp);
           load_k(T.k[1], kp + 8 * KR);
@@ -432,20 +461,22 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           T.vn[0] = __ldcs(vnp);
           T.vn[1] = __ldcs(vnp + 8);
         } else {
-          const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
-          const uint8_t *kb = a.kc + rec0 * KR + 4 * KB * c;
-          load_k(T.k[0], kb + static_cast<size_t>(tr) * KR);
-          load_k(T.k[1], kb + static_cast<size_t>(tr8) * KR);
-          const uint8_t *vb = a.vc + rec0 * VR + 4 * vwo;
+          // record of token t (within this tile, so within one page) = base + t
+          const long long base = PG ? rb - t0 : static_cast<long long>(rec0);
+          const long long tr = base + min(t0 + r, tlast), tr8 = base + min(t0 + r + 8, tlast);
+          const uint8_t *kb = a.kc + 4 * KB * c;
+          load_k(T.k[0], kb + tr * KR);
+          load_k(T.k[1], kb + tr8 * KR);
+          const uint8_t *vb = a.vc + 4 * vwo;
           const int tv = t0 + c;
-          load_v(T.v[0], vb + static_cast<size_t>(min(tv, tlast)) * VR);
-          load_v(T.v[1], vb + static_cast<size_t>(min(tv + 4, tlast)) * VR);
-          load_v(T.v[2], vb + static_cast<size_t>(min(tv + 8, tlast)) * VR);
-          load_v(T.v[3], vb + static_cast<size_t>(min(tv + 12, tlast)) * VR);
-          T.kn[0] = __ldcs(a.kn + rec0 + tr);
-          T.kn[1] = __ldcs(a.kn + rec0 + tr8);
-          T.vn[0] = __ldcs(a.vn + rec0 + tr);
-          T.vn[1] = __ldcs(a.vn + rec0 + tr8);
+          load_v(T.v[0], vb + (base + min(tv, tlast)) * VR);
+          load_v(T.v[1], vb + (base + min(tv + 4, tlast)) * VR);
+          load_v(T.v[2], vb + (base + min(tv + 8, tlast)) * VR);
+          load_v(T.v[3], vb + (base + min(tv + 12, tlast)) * VR);
+          T.kn[0] = __ldcs(a.kn + tr);
+          T.kn[1] = __ldcs(a.kn + tr8);
+          T.vn[0] = __ldcs(a.vn + tr);
+          T.vn[1] = __ldcs(a.vn + tr8);
         }
         kp += kStep * KR;
         vp += kStep * VR;
@@ -831,7 +862,8 @@ cudaError_t run_mse(const FastArgs &f, const VarLen *vl, int ctas, cudaStream_t 
   constexpr int smem = Lut<KB, VB>::kSmem;
   cudaError_t e;
   if (vl) {
-    auto kern = f.G <= 4 ? decode_mse_kernel<KB, VB, 1, true> : decode_mse_kernel<KB, VB, 2, true>;
+    auto kern = f.bt ? (f.G <= 4 ? decode_mse_kernel<KB, VB, 1, 2> : decode_mse_kernel<KB, VB, 2, 2>)
+                     : (f.G <= 4 ? decode_mse_kernel<KB, VB, 1, 1> : decode_mse_kernel<KB, VB, 2, 1>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     FastArgsV fv;
@@ -839,7 +871,7 @@ cudaError_t run_mse(const FastArgs &f, const VarLen *vl, int ctas, cudaStream_t 
     fv.vl = *vl;
     return launch_pdl(kern, dim3(ctas), dim3(Cfg<KB, VB>::kThreads), smem, s, fv);
   }
-  auto kern = f.G <= 4 ? decode_mse_kernel<KB, VB, 1, false> : decode_mse_kernel<KB, VB, 2, false>;
+  auto kern = f.G <= 4 ? decode_mse_kernel<KB, VB, 1, 0> : decode_mse_kernel<KB, VB, 2, 0>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(ctas), dim3(Cfg<KB, VB>::kThreads), smem, s, f);
@@ -919,6 +951,9 @@ cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   for (int j = 0; j < 16; ++j) f.vcent[j] = a.v.cb.c[j];
   f.one = 1u;
   f.B = a.B;
+  f.bt = a.pg.bt;
+  f.pshift = a.pg.pshift;
+  f.maxp = a.pg.maxp;
   VarLen vl;
   const VarLen *vlp = nullptr;
   if (a.T_lens) {

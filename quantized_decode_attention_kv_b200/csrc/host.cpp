@@ -270,10 +270,21 @@ size_t tq_record_bytes(int d, tq_qcfg c) {
   return tq_code_bytes(d, c) + tq_sign_bytes(d, c) + (c.mode == TQ_PROD ? 4 : 2);
 }
 
+// Shared body of the dense and paged writes (cache: the dense descriptor or a paged cache's
+// view; pg.bt == nullptr for the dense layout).
+static int quantize_impl(const void *K, const void *V, int dtype, int T, int t_offset,
+                         const tq_cache *cache, const tq::Paging &pg, void *stream);
+
 int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
                    const tq_cache *cache, void *stream) {
   int st = check_cache(cache);
   if (st) return st;
+  return quantize_impl(K, V, dtype, T, t_offset, cache, tq::Paging{nullptr, -1, 0}, stream);
+}
+
+static int quantize_impl(const void *K, const void *V, int dtype, int T, int t_offset,
+                         const tq_cache *cache, const tq::Paging &pg, void *stream) {
+  int st = TQ_OK;
   if (!dtype_ok(dtype)) return fail(TQ_ERR_INVALID_ARG, "dtype=%d is not F32/BF16/F16", dtype);
   if (T < 0 || t_offset < 0 || (long long)t_offset + T > cache->T_cap)
     return fail(TQ_ERR_INVALID_ARG, "positions [%d, %d) fall outside T_cap=%d", t_offset,
@@ -303,6 +314,7 @@ int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
     q.d = cache->d;
     q.seed = cache->seed;
     for (int k = 0; k < 4; ++k) q.sign_words[k] = splitmix64_at(cache->seed, static_cast<uint64_t>(k));
+    q.pg = pg;
   }
   // 16-bit MSE tensors take the streaming kernel, 16-bit d=64 TurboQuant_prod tensors the
   // tensor-core sketch kernel (each with K and V in one launch); the rest, the per-vector
@@ -313,6 +325,8 @@ int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
     if (!x) continue;
     if (tq::quantize_fast_supported(a[which])) fast[which] = &a[which];
     else if (tq::quantize_prod_supported(a[which])) prod[which] = &a[which];
+    if (pg.bt && !fast[which]) // the paged layout is written by the 16-bit MSE kernels only
+      return fail(TQ_ERR_UNSUPPORTED, "paged writes need 16-bit input and TurboQuant_mse records");
   }
   if (fast[0] || fast[1] || prod[0] || prod[1]) {
     const int sms = sm_count();
@@ -439,9 +453,9 @@ size_t tq_decode_varlen_workspace_bytes(int Hq, const tq_cache *cache, const int
   return p.ws_bytes;
 }
 
-int tq_decode_attention_varlen(const void *q, int dtype, int Hq, const int *T_lens, float scale,
-                               const tq_cache *cache, float *out, void *ws, size_t ws_bytes,
-                               void *stream) {
+static int decode_varlen_impl(const void *q, int dtype, int Hq, const int *T_lens, float scale,
+                              const tq_cache *cache, const tq::Paging &pg, float *out, void *ws,
+                              size_t ws_bytes, void *stream) {
   int mx = 0;
   int st = check_varlen(cache, Hq, T_lens, &mx);
   if (st) return st;
@@ -463,6 +477,7 @@ int tq_decode_attention_varlen(const void *q, int dtype, int Hq, const int *T_le
     return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
                 a.plan.ws_bytes, ws ? ws_bytes : 0);
   a.T_lens = T_lens;
+  a.pg = pg;
   a.q = q;
   a.q_dtype = dtype;
   a.B = cache->B;
@@ -476,6 +491,76 @@ int tq_decode_attention_varlen(const void *q, int dtype, int Hq, const int *T_le
   a.out = out;
   a.ws = static_cast<float *>(ws);
   return cuda_status(tq::launch_fast_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
+}
+
+int tq_decode_attention_varlen(const void *q, int dtype, int Hq, const int *T_lens, float scale,
+                               const tq_cache *cache, float *out, void *ws, size_t ws_bytes,
+                               void *stream) {
+  return decode_varlen_impl(q, dtype, Hq, T_lens, scale, cache, tq::Paging{nullptr, -1, 0}, out, ws,
+                            ws_bytes, stream);
+}
+
+// A paged cache seen as the dense descriptor the shared checks and resolvers read (T_cap: one
+// sequence's capacity; the pointers: the page pools), plus its paging.
+static int paged_view(const tq_paged_cache *pc, tq_cache *view, tq::Paging *pg) {
+  if (!pc) return fail(TQ_ERR_INVALID_ARG, "cache is NULL");
+  if (pc->B < 1 || pc->Hkv < 1 || pc->num_pages < 1 || pc->max_pages < 1)
+    return fail(TQ_ERR_INVALID_ARG, "bad paged cache shape B=%d Hkv=%d num_pages=%d max_pages=%d",
+                pc->B, pc->Hkv, pc->num_pages, pc->max_pages);
+  if (pc->page_size < 16 || (pc->page_size & (pc->page_size - 1)))
+    return fail(TQ_ERR_INVALID_ARG, "page_size=%d must be a power of two >= 16", pc->page_size);
+  if (!pc->block_table) return fail(TQ_ERR_INVALID_ARG, "block_table is NULL");
+  if (pc->d != 128) return fail(TQ_ERR_UNSUPPORTED, "paged caches support d = 128, got %d", pc->d);
+  if (pc->kc.mode != TQ_MSE || pc->vc.mode != TQ_MSE)
+    return fail(TQ_ERR_UNSUPPORTED, "paged caches support TurboQuant_mse records only");
+  const long long cap = static_cast<long long>(pc->max_pages) * pc->page_size;
+  const long long recs = static_cast<long long>(pc->num_pages) * pc->Hkv * pc->page_size;
+  if (cap > (1ll << 30) || recs > (1ll << 40))
+    return fail(TQ_ERR_INVALID_ARG, "paged cache too large (capacity %lld positions)", cap);
+  std::memset(view, 0, sizeof *view);
+  view->B = pc->B;
+  view->Hkv = pc->Hkv;
+  view->T_cap = static_cast<int>(cap);
+  view->d = pc->d;
+  view->seed = pc->seed;
+  view->kc = pc->kc;
+  view->vc = pc->vc;
+  view->k_codes = pc->k_codes;
+  view->v_codes = pc->v_codes;
+  view->k_norm = pc->k_norm;
+  view->v_norm = pc->v_norm;
+  int st = check_cache(view);
+  if (st) return st;
+  int shift = 0;
+  while ((1 << shift) < pc->page_size) ++shift;
+  *pg = tq::Paging{pc->block_table, shift, pc->max_pages};
+  return TQ_OK;
+}
+
+int tq_quantize_kv_paged(const void *K, const void *V, int dtype, int T, int t_offset,
+                         const tq_paged_cache *cache, void *stream) {
+  tq_cache view;
+  tq::Paging pg;
+  int st = paged_view(cache, &view, &pg);
+  if (st) return st;
+  return quantize_impl(K, V, dtype, T, t_offset, &view, pg, stream);
+}
+
+size_t tq_decode_paged_workspace_bytes(int Hq, const tq_paged_cache *cache, const int *T_lens) {
+  tq_cache view;
+  tq::Paging pg;
+  if (paged_view(cache, &view, &pg)) return 0;
+  return tq_decode_varlen_workspace_bytes(Hq, &view, T_lens);
+}
+
+int tq_decode_attention_paged(const void *q, int dtype, int Hq, const int *T_lens, float scale,
+                              const tq_paged_cache *cache, float *out, void *ws, size_t ws_bytes,
+                              void *stream) {
+  tq_cache view;
+  tq::Paging pg;
+  int st = paged_view(cache, &view, &pg);
+  if (st) return st;
+  return decode_varlen_impl(q, dtype, Hq, T_lens, scale, &view, pg, out, ws, ws_bytes, stream);
 }
 
 int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, float scale,

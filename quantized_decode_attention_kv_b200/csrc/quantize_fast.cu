@@ -43,7 +43,18 @@ struct FastTensor {
   unsigned nvec;
   int T, T_cap, t_offset, wbits, code_bytes, nbeta;
   float beta[15];
+  const int *bt; // paged cache: block table [B][maxp] (nullptr: dense [B][Hkv][T_cap] layout)
+  int pshift, maxp, Hkv;
 };
+
+// Record index of new position tt of (b, KV head) bh: dense, or through the block table.
+__device__ __forceinline__ size_t rec_index(const FastTensor &t, unsigned bh, unsigned tt) {
+  const unsigned pos = static_cast<unsigned>(t.t_offset) + tt;
+  if (!t.bt) return static_cast<size_t>(bh) * t.T_cap + pos;
+  const unsigned b = bh / static_cast<unsigned>(t.Hkv), h = bh - b * static_cast<unsigned>(t.Hkv);
+  const unsigned page = static_cast<unsigned>(__ldg(t.bt + static_cast<size_t>(b) * t.maxp + (pos >> t.pshift)));
+  return ((static_cast<size_t>(page) * t.Hkv + h) << t.pshift) + (pos & ((1u << t.pshift) - 1u));
+}
 
 struct FastQuantArgs {
   FastTensor t[2];
@@ -151,7 +162,7 @@ __device__ __forceinline__ void quantize_row(const uint8_t *row, uint32_t cells,
 
   const unsigned bh = v / static_cast<unsigned>(t.T);
   const unsigned tt = v - bh * static_cast<unsigned>(t.T);
-  const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
+  const size_t rec = rec_index(t, bh, tt);
   uint8_t *dst = t.codes + rec * (NW * 4);
   if constexpr (NW % 4 == 0) {
 #pragma unroll
@@ -337,7 +348,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_small_kernel(const FastQua
   __syncwarp();
   const unsigned bh = v / static_cast<unsigned>(t.T);
   const unsigned tt = v - bh * static_cast<unsigned>(t.T);
-  const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
+  const size_t rec = rec_index(t, bh, tt);
   if (lane < nw) reinterpret_cast<uint32_t *>(t.codes + rec * (nw * 4))[lane] = rw[lane];
   if (lane == 0) t.norm[rec] = f32_to_f16_bits(n);
 }
@@ -582,7 +593,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 3) quantize_mma_kernel(const F
         const float n = sqrtf((rho ? sb : sa) * (1.0f / 128.0f));
         const float inv = n > 0.f ? __frcp_rn(n) : 0.0f;
         if (v < t.nvec) {
-          const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
+          const size_t rec = rec_index(t, bh, tt);
           mma_codes_store<WB>(acc, rho, inv, cl, t.codes + rec * (16 * WB) + c * (4 * WB));
           if (c == 0) t.norm[rec] = f32_to_f16_bits(n);
         }
@@ -662,6 +673,10 @@ cudaError_t launch_quantize_fast(const QuantArgs *k, const QuantArgs *v, int sms
     t.norm = q.t.norm;
     t.nvec = static_cast<unsigned>(static_cast<long long>(q.B) * q.Hkv * q.T);
     t.nbatch = (t.nvec + kQThreads - 1) / kQThreads;
+    t.bt = q.pg.bt;
+    t.pshift = q.pg.pshift;
+    t.maxp = q.pg.maxp;
+    t.Hkv = q.Hkv;
     t.T = q.T;
     t.T_cap = q.T_cap;
     t.t_offset = q.t_offset;

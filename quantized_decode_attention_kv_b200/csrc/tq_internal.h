@@ -33,6 +33,13 @@ struct TensorArgs {
   Codebook cb;
 };
 
+// Paging of a cache (pshift < 0: the dense [B][Hkv][T_cap] layout): record (b, h, t) sits at
+// page bt[b * maxp + (t >> pshift)], head h, slot t & (2^pshift - 1).
+struct Paging {
+  const int *bt;
+  int pshift, maxp;
+};
+
 struct QuantArgs {
   const void *x;
   int dtype;
@@ -40,6 +47,7 @@ struct QuantArgs {
   uint64_t seed;
   uint64_t sign_words[4]; // SplitMix64 outputs 0..3 of `seed`: bit i set <=> D_ii = -1
   TensorArgs t;
+  Paging pg; // pshift = -1 unless writing a paged cache
 };
 
 struct DequantArgs {
@@ -77,6 +85,7 @@ struct VarLen {
 
 struct DecodeArgs {
   const int *T_lens; // host array of B per-sequence lengths, or NULL (uniform T_len)
+  Paging pg;         // pshift = -1 unless reading a paged cache (then T_lens is set)
   const void *q;
   int q_dtype;
   int B, Hq, Hkv, d, T_len, T_cap;

@@ -45,6 +45,17 @@ class tq_cache(ctypes.Structure):
     ]
 
 
+class tq_paged_cache(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("page_size", ctypes.c_int),
+        ("num_pages", ctypes.c_int), ("max_pages", ctypes.c_int),
+        ("seed", ctypes.c_uint64), ("kc", tq_qcfg), ("vc", tq_qcfg),
+        ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+        ("k_norm", ctypes.c_void_p), ("v_norm", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p),
+    ]
+
+
 EXPORTS = {
     # name: (restype, argtypes)
     "tq_last_error": (ctypes.c_char_p, []),
@@ -70,6 +81,14 @@ EXPORTS = {
                                                   ctypes.c_void_p, ctypes.c_float, ctypes.POINTER(tq_cache),
                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                                   ctypes.c_void_p]),
+    "tq_quantize_kv_paged": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.POINTER(tq_paged_cache), ctypes.c_void_p]),
+    "tq_decode_paged_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.POINTER(tq_paged_cache),
+                                                          ctypes.c_void_p]),
+    "tq_decode_attention_paged": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                                 ctypes.c_float, ctypes.POINTER(tq_paged_cache),
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                                 ctypes.c_void_p]),
     "tq_decode_attention_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, ctypes.c_float, ctypes.POINTER(tq_cache),
                                                    ctypes.c_void_p, ctypes.c_void_p]),
@@ -213,6 +232,36 @@ class TQCache:
         return self.B * self.Hkv * T_len * per
 
 
+class TQPagedCache:
+    """One layer's paged compressed KV cache (TurboQuant_mse, head_dim 128): torch owns the
+    page pools; ``block_table`` is an int32 [B][max_pages] device tensor the caller fills with
+    physical page indices (it may be rewritten between calls). Shapes follow include/tq.h."""
+
+    def __init__(self, B: int, Hkv: int, d: int, page_size: int, num_pages: int, max_pages: int,
+                 k_bits: int, v_bits: int, block_table: torch.Tensor, seed: int = 0, device: str = "cuda"):
+        dev = torch.device(device)
+        self.B, self.Hkv, self.d, self.page_size = B, Hkv, d, page_size
+        self.num_pages, self.max_pages, self.k_bits, self.v_bits, self.seed = num_pages, max_pages, k_bits, v_bits, seed
+        if block_table.dtype != torch.int32 or tuple(block_table.shape) != (B, max_pages) or not block_table.is_cuda:
+            raise TQError(TQ_ERR_INVALID_ARG, "block_table must be an int32 CUDA tensor [B][max_pages]")
+        self.block_table = block_table.contiguous()
+        self.tensors = {}
+        for side, bits in (("k", k_bits), ("v", v_bits)):
+            cb = tq_code_bytes(d, bits, TQ_MSE, 0)
+            shape = (num_pages, Hkv, page_size)
+            self.tensors[f"{side}_codes"] = torch.zeros(shape + (cb,), dtype=torch.uint8, device=dev)
+            self.tensors[f"{side}_norm"] = torch.zeros(shape, dtype=torch.int16, device=dev)
+        t = self.tensors
+        self.struct = tq_paged_cache(B, Hkv, d, page_size, num_pages, max_pages, seed,
+                                     tq_qcfg(k_bits, TQ_MSE, 0), tq_qcfg(v_bits, TQ_MSE, 0),
+                                     t["k_codes"].data_ptr(), t["v_codes"].data_ptr(),
+                                     t["k_norm"].data_ptr(), t["v_norm"].data_ptr(),
+                                     self.block_table.data_ptr())
+
+    def __getitem__(self, key):
+        return self.tensors[key]
+
+
 # ------------------------------------------------------------------ device entry points
 def tq_quantize_kv(K: torch.Tensor | None, V: torch.Tensor | None, cache: TQCache, t_offset: int = 0,
                    stream=None) -> None:
@@ -226,6 +275,41 @@ def tq_quantize_kv(K: torch.Tensor | None, V: torch.Tensor | None, cache: TQCach
     kp = _dev(K, "K") if K is not None else None
     vp = _dev(V, "V") if V is not None else None
     _check(lib.tq_quantize_kv(kp, vp, dt, T, t_offset, ctypes.byref(cache.struct), _stream(stream)))
+
+
+def tq_quantize_kv_paged(K: torch.Tensor | None, V: torch.Tensor | None, cache: TQPagedCache,
+                         t_offset: int = 0, stream=None) -> None:
+    """Write positions t_offset .. t_offset + T - 1 of every sequence into the paged cache."""
+    ref = K if K is not None else V
+    if ref is None:
+        raise TQError(TQ_ERR_INVALID_ARG, "K and V are both None")
+    dt = _DTYPES.get(ref.dtype)
+    if dt is None:
+        raise TQError(TQ_ERR_INVALID_ARG, f"unsupported dtype {ref.dtype}")
+    kp = _dev(K, "K") if K is not None else None
+    vp = _dev(V, "V") if V is not None else None
+    _check(lib.tq_quantize_kv_paged(kp, vp, dt, ref.shape[2], t_offset, ctypes.byref(cache.struct),
+                                    _stream(stream)))
+
+
+def tq_decode_paged_workspace_bytes(cache: TQPagedCache, Hq: int, T_lens) -> int:
+    lens = _lens(T_lens)
+    n = int(lib.tq_decode_paged_workspace_bytes(Hq, ctypes.byref(cache.struct), ctypes.cast(lens, ctypes.c_void_p)))
+    if n == 0:
+        raise TQError(TQ_ERR_INVALID_ARG, last_error())
+    return n
+
+
+def tq_decode_attention_paged(q: torch.Tensor, cache: TQPagedCache, T_lens, scale: float, out: torch.Tensor,
+                              ws: torch.Tensor, stream=None) -> None:
+    """Decode attention over a paged cache; sequence b attends to its first T_lens[b] positions."""
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise TQError(TQ_ERR_INVALID_ARG, f"unsupported dtype {q.dtype}")
+    lens = _lens(T_lens)
+    _check(lib.tq_decode_attention_paged(_dev(q, "q"), dt, q.shape[1], ctypes.cast(lens, ctypes.c_void_p),
+                                         scale, ctypes.byref(cache.struct), _dev(out, "out"), _dev(ws, "ws"),
+                                         ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def tq_launch_counts(cache: TQCache, dtype: torch.dtype, T: int, Hq: int, T_len: int) -> tuple[int, int]:
