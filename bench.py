@@ -304,6 +304,8 @@ def run_ours(args):
         line["speedup_vs_bf16"] = side["bf16"]["us"] / (side["decode_s"] * 1e6)
         if "ragged" in side:
             line["ragged_decode"] = side["ragged"]
+        if "paged" in side:
+            line["paged_decode"] = side["paged"]
     print(json.dumps(line), flush=True)
 
 
@@ -362,6 +364,24 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
                          "bytes": rbytes, "lengths": f"{w.B} sequences, seeded uniform in [T/4, T], "
                                                     f"min {min(lens)}, max {max(lens)}, sum {sum(lens)}",
                          "padded_uniform_us": ps * 1e6}
+    # the same workload in a paged cache (64-position pages scattered over the pool by a
+    # seeded permutation): bulk paged write, then paged decode over the full context
+    if w.d == 128 and w.k_mode == 0 and w.v_mode == 0 and w.B <= 512 and K.dtype != torch.float32:
+        page = 64
+        maxp = (w.T + page - 1) // page
+        npages = w.B * maxp
+        g = torch.Generator().manual_seed(4321)
+        bt = torch.randperm(npages, generator=g).to(torch.int32).reshape(w.B, maxp).cuda()
+        pc = tq.TQPagedCache(w.B, w.Hkv, w.d, page, npages, maxp, w.k_bits, w.v_bits, bt, seed=cache.seed)
+        tq.tq_quantize_kv_paged(K, V, pc, 0, stream=stream)
+        lens = [w.T] * w.B
+        wsp = tq.workspace(tq.tq_decode_paged_workspace_bytes(pc, w.Hq, lens))
+        pgs = _time(lambda: tq.tq_decode_attention_paged(q, pc, lens, w.scale, out, wsp, stream=stream),
+                    stream, max(args.steps // 4, 20), torch)
+        res["paged"] = {"us": pgs * 1e6, "gbs": packed / pgs / 1e9, "frac": packed / pgs / 1e9 / hbm,
+                        "page_size": page, "layout": f"{npages} pages of {page} positions, scattered by a "
+                                                     f"seeded permutation; every sequence at full length"}
+        del pc, bt, wsp
     # end to end through the C ABI from pinned host buffers, as a serving loop runs it: every
     # step copies its inputs (query, the new token's K and V) in from pinned memory, runs the
     # two calls and reads its attention output back; the copies run on their own streams and

@@ -367,14 +367,13 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
 
       const size_t rec0 = PG ? 0 : static_cast<size_t>(bh) * a.T_cap;
-      // record index of token t0 (a multiple of 16: a tile never straddles a page)
-      [[maybe_unused]] auto tile_rec = [&](int t0) -> long long {
-        if constexpr (PG) {
-          const int page = __ldg(a.bt + static_cast<size_t>(b) * a.maxp + (t0 >> a.pshift));
-          return ((static_cast<long long>(page) * a.Hkv + h) << a.pshift) + (t0 & ((1 << a.pshift) - 1));
-        } else {
-          return static_cast<long long>(rec0) + t0;
-        }
+      // paged cache: record index of token t0 (a multiple of 16: a tile never straddles a
+      // page) on a given page, and the page of the warp's tile jj (0 past the segment)
+      [[maybe_unused]] auto page_rec = [&](int page, int t0) -> long long {
+        return ((static_cast<long long>(page) * a.Hkv + h) << a.pshift) + (t0 & ((1 << a.pshift) - 1));
+      };
+      [[maybe_unused]] auto page_of = [&](int jj) -> int {
+        return jj < ntiles ? __ldg(a.bt + static_cast<size_t>(b) * a.maxp + (((tile0 + jj) * 16) >> a.pshift)) : 0;
       };
       const int tlast = T_len - 1;
       // word offset of this lane's value run within a record (3-bit runs start mid-word for odd r)
@@ -406,6 +405,13 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
         pfstep = kStep * 2;
       }
       int tpf = tp0;
+      // page pipeline: pages of the warp's next two tiles, looked up two steps ahead of use
+      [[maybe_unused]] int pg_a = 0, pg_b = 0;
+      if constexpr (PG) {
+        static_assert(kPrefetchSteps <= 1, "the page pipeline serves a prefetch one step ahead");
+        pg_a = page_of(warp);
+        pg_b = page_of(warp + kWarps);
+      }
 
       auto load_k = [&](uint32_t (&dst)[KB], const uint8_t *p) {
         if constexpr (KB == 4) {
@@ -430,7 +436,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
         if (kPrefetchSteps > 0) {
           if (lane < KL + VL + 2 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16) {
             if constexpr (PG) {
-              const long long rp = tile_rec(tpf);
+              const long long rp = page_rec(pg_b, tpf);
               pfp = lane < KL ? reinterpret_cast<const char *>(a.kc + rp * KR + 128 * lane)
                     : lane < KL + VL ? reinterpret_cast<const char *>(a.vc + rp * VR + 128 * (lane - KL))
                                      : reinterpret_cast<const char *>((lane == KL + VL ? a.kn : a.vn) + rp);
@@ -443,7 +449,10 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
         const int t0 = (tile0 + jl) * 16;
         [[maybe_unused]] long long rb = 0;
         if constexpr (PG) {
-          rb = tile_rec(t0);
+          rb = page_rec(pg_a, t0);
+          const int pg_c = page_of(jl + 2 * kWarps);
+          pg_a = pg_b;
+          pg_b = pg_c;
           kp = a.kc + (rb + r) * KR + 4 * KB * c;
           vp = a.vc + (rb + c) * VR + 4 * vwo;
           knp = a.kn + rb + r;
