@@ -54,8 +54,48 @@ def test_decode_step_replays_from_a_cuda_graph(d, G, Hkv, kcfg, vcfg, m, T):
         g.replay()
     torch.cuda.synchronize()
     assert torch.isfinite(out_g).all()
-    # the CTA merge adds warps' partials with shared-memory atomics (order not fixed): equal to
-    # fp32 rounding, not bit for bit
+    # equal to fp32 rounding (the TurboQuant_prod merge adds warps' partials with shared-memory
+    # atomics, whose order is not fixed)
     torch.testing.assert_close(out_g, out_e, rtol=1e-5, atol=1e-6)
     for key in ("k_codes", "v_codes", "k_norm", "v_norm"):
         assert torch.equal(graphed[key], eager[key]), key
+
+
+def test_ragged_and_paged_decode_replay_from_a_cuda_graph():
+    # per-sequence lengths travel as launch parameters: the graph keeps the captured lengths
+    B, Hkv, G, d, T, page = 3, 2, 4, 128, 640, 64
+    Hq, lens = G * Hkv, [640, 17, 300]
+    K, V = random_kv(B, Hkv, T, d, dtype=torch.bfloat16, seed=11)
+    K, V = K.cuda(), V.cuda()
+    q = torch.randn(B, Hq, d, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).cuda()
+    dense = tq.TQCache(B, Hkv, T, d, 4, 2)
+    tq.tq_quantize_kv(K, V, dense)
+    maxp = T // page
+    bt = torch.randperm(B * maxp, generator=torch.Generator().manual_seed(2)).to(torch.int32)
+    paged = tq.TQPagedCache(B, Hkv, d, page, B * maxp, maxp, 4, 2, bt.reshape(B, maxp).cuda())
+    tq.tq_quantize_kv_paged(K, V, paged)
+    ws_r = tq.workspace(tq.tq_decode_varlen_workspace_bytes(dense, Hq, lens))
+    ws_p = tq.workspace(tq.tq_decode_paged_workspace_bytes(paged, Hq, lens))
+    eager_r, eager_p = torch.empty(B, Hq, d, device="cuda"), torch.empty(B, Hq, d, device="cuda")
+    tq.tq_decode_attention_varlen(q, dense, lens, 0.1, eager_r, ws_r)
+    tq.tq_decode_attention_paged(q, paged, lens, 0.1, eager_p, ws_p)
+    out_r = torch.full((B, Hq, d), float("nan"), device="cuda")
+    out_p = torch.full((B, Hq, d), float("nan"), device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        tq.tq_decode_attention_varlen(q, dense, lens, 0.1, out_r, ws_r)
+        tq.tq_decode_attention_paged(q, paged, lens, 0.1, out_p, ws_p)
+    torch.cuda.current_stream().wait_stream(side)
+    out_r.fill_(float("nan"))
+    out_p.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        tq.tq_decode_attention_varlen(q, dense, lens, 0.1, out_r, ws_r)
+        tq.tq_decode_attention_paged(q, paged, lens, 0.1, out_p, ws_p)
+    lens[1] = 600  # the host array may change after capture: the graph keeps its values
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out_r, eager_r, rtol=1e-5, atol=1e-6)
+    torch.testing.assert_close(out_p, eager_p, rtol=1e-5, atol=1e-6)
