@@ -3,13 +3,17 @@
 //
 // "Where This Fits in the Inference Stack", TensorRT-LLM section: dequantise in registers
 // inside the attention kernel. Here the dequantised codes are written straight into the
-// operand registers of warp-level tensor-core MMAs (mma.sync m16n8k16, fp16 x fp16 -> fp32):
+// operand registers of warp-level tensor-core MMAs:
 //
-//   scores  S[16 tokens x (hi, lo) per head] = K^[16 x 128] . [q^_hi | q^_lo]
-//     K^ comes from a shared-memory LUT indexed by one code byte (two 4-bit codes): each entry
-//     holds the two centroids as fp16 (hi) and their fp16 rounding residuals scaled by 2^12
-//     (lo); two MMAs (hi, lo) give scores good to ~2^-21 relative, as fp32 scoring would.
-//     The query side is split the same way by the query-prep kernel.
+//   scores  S[16 tokens x 3 per head] = K^[16 x 2*128] . Q[2*128 x 3 per head]
+//     (mma.sync m16n8k32, int8 x int8 -> int32). Centroids are 16-bit fixed-point numbers
+//     c = 256 c_hi + c_lo, queries 24-bit ones q = 65536 q_hi + 256 q_mid + q_lo, each part an
+//     int8. K^ comes from a shared-memory LUT indexed by one code byte (two 4-bit codes) whose
+//     4-byte entry is {hi, hi, lo, lo} of the two centroids, i.e. four consecutive k slots of
+//     one A row. Per head three columns take {q_hi, 0}, {q_mid, q_hi} and {q_lo, q_mid} at the
+//     {hi, lo} slots, so c.q = 2^24 col0 + 2^16 col1 + 2^8 col2 up to c_lo q_lo (2^-24 of the
+//     scale); the rounding of the centroids to 16 bits, at a scale chosen to make it small, is
+//     the only other error.
 //   values  O^T[128 x heads] += V^T[128 x 16 tokens] . P'^T[16 tokens x heads]
 //     2-bit V^: one byte of nibble-interleaved codes (two tokens, two coordinates) indexes a
 //     lane-replicated shared table whose 8-byte entry is a pair of operand registers;
@@ -38,8 +42,16 @@ namespace {
 using namespace mma_ops;
 
 constexpr int kD = 128;
-constexpr float kLoScale = 4096.0f; // residual scaling 2^12 (keeps residuals normal in fp16)
-constexpr float kLoInv = 1.0f / 4096.0f;
+// Magnitude of the largest 24-bit fixed-point query coordinate: below 127 * 65536 + 127 * 256
+// + 127 = 8355711 with a margin for the float rounding of max|q~| * (8355000 / max|q~|), so the
+// int8 parts stay in [-127, 127] (hi) and [-128, 127] (mid, lo).
+constexpr float kQFixMax = 8355000.0f;
+// Score accumulators start at the bits of 1.5 * 2^23: an int32 sum s with |s| < 2^22 (each
+// column sums 128 products of two int8 parts, one of them <= 127 in magnitude, or two such
+// sums) reads back as the float 1.5 * 2^23 + s exactly. kMagicAdj = 1.5 * 2^23 *
+// (1 + 2^-8 + 2^-16) removes the three offsets of col0 + col1 / 2^8 + col2 / 2^16.
+constexpr int kMagic = 0x4B400000;
+constexpr float kMagicAdj = 12632256.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 #ifndef TQ_DECODE_PREFETCH
 #define TQ_DECODE_PREFETCH 1
@@ -65,6 +77,13 @@ struct Cfg {
 };
 
 template <uint32_t OFF>
+__device__ __forceinline__ uint32_t lds32_off(uint32_t smem_addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(smem_addr), "n"(OFF));
+  return v;
+}
+
+template <uint32_t OFF>
 __device__ __forceinline__ uint2 lds64_off(uint32_t smem_addr) {
   uint2 v;
   // not volatile: the tables are read-only after the fill barrier, and leaving the loads free
@@ -88,8 +107,8 @@ struct Tile {
 };
 
 // Shared-memory tables of one configuration. Key rows: one code-pair index (4-bit keys: a
-// byte of two codes, 256 rows; 3-bit keys: 6 bits, 64 rows) x {32 lane copies of the fp16x2
-// hi pair, 32 of the lo pair} = 256 bytes. Value rows, 2-bit values: one byte holding the
+// byte of two codes, 256 rows; 3-bit keys: 6 bits, 64 rows) x 32 lane copies of the 4-byte
+// int8 entry {hi, hi, lo, lo}, in a 256-byte row (the index lands above bit 8 of the address). Value rows, 2-bit values: one byte holding the
 // codes of two adjacent coordinates of two tokens (low nibble the first token) x 32 lane
 // copies of the two fp16x2 operand words = 256 bytes; 3/4-bit values: one index (the codes of
 // two adjacent coordinates of one token, the first in the low bits) x 32 lane copies of the
@@ -112,25 +131,27 @@ struct Lut {
 
 } // namespace
 
-// A prepared query: rotated once (q'' = H D q), scaled (q~ = scale q'' / d), normalised by a
-// power of two so max|q^| is in [1, 2), split into fp16 hi and 2^12-scaled fp16 residual. The
-// decode kernel builds one per query head of a segment in shared memory.
+// A prepared query: rotated once (q'' = H D q), scaled (q~ = scale q'' / d), as a 24-bit
+// fixed-point vector q_int = rint(q~ * 8355839 / max|q~|) split into int8 parts
+// q_int = 65536 hi + 256 mid + lo. The decode kernel builds one per query head of a segment in
+// shared memory.
 struct QPrep {
-  uint16_t hi[kD];
-  uint16_t lo[kD];
-  float inv; // 1 / (power-of-two factor): score = ||k|| * inv * (K^ . q^)
+  int8_t hi[kD];
+  int8_t mid[kD];
+  int8_t lo[kD];
+  float inv; // score = ||k|| * inv * (col0 + col1 / 2^8 + col2 / 2^16), see the score MMA
   float pad[3];
 };
 
 namespace {
 
 // Query prep of one query by one warp: rotate (q'' = H D q), scale (q~ = scale q'' / d),
-// normalise by a power of two so max|q^| is in [1, 2), split into fp16 hi and 2^12-scaled fp16
-// residual. Lane l holds coordinates 4 l .. 4 l + 3; the butterflies of span 1, 2 run in the
+// round to 24-bit fixed point at the full range and split into int8 hi, mid and lo; csc is
+// the centroids' fixed-point scale. Lane l holds coordinates 4 l .. 4 l + 3; the butterflies of span 1, 2 run in the
 // lane, those of span 4 .. 64 across lanes (the lane with the span bit set keeps
 // partner - own).
 __device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, float scale,
-                                           uint64_t seed, QPrep *out, int lane) {
+                                           uint64_t seed, float csc, QPrep *out, int lane) {
   float x[4];
   const uint64_t sw = dev_splitmix64(seed, static_cast<uint64_t>(lane >> 4)); // coordinates 64 k ..
 #pragma unroll
@@ -162,25 +183,25 @@ __device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, 
     mx = fmaxf(mx, fabsf(x[e]));
   }
   mx = warp_max(mx);
-  float factor = 1.0f;
-  if (mx > 0.f && isfinite(mx)) {
-    int ex;
-    frexpf(mx, &ex);               // mx = f * 2^ex, f in [0.5, 1)
-    factor = ldexpf(1.0f, 1 - ex); // mx * factor in [1, 2)
-  }
-  uint32_t hw[2], lw[2];
+  // all-zero query: zero scores; a non-finite one makes the scores NaN
+  const bool ok = mx > 0.f && isfinite(mx);
+  const float qsc = ok ? kQFixMax / mx : 0.f;
+  uint32_t hw = 0, mw = 0, lw = 0;
 #pragma unroll
-  for (int p = 0; p < 2; ++p) {
-    const float q0 = x[2 * p] * factor, q1 = x[2 * p + 1] * factor;
-    const __half h0 = __float2half_rn(q0), h1 = __float2half_rn(q1);
-    const __half l0 = __float2half_rn((q0 - __half2float(h0)) * kLoScale);
-    const __half l1 = __float2half_rn((q1 - __half2float(h1)) * kLoScale);
-    hw[p] = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
-    lw[p] = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+  for (int e = 0; e < 4; ++e) {
+    const int qi = __float2int_rn(x[e] * qsc);
+    const int lo = ((qi + 128) & 255) - 128;
+    const int q1 = (qi - lo) >> 8;
+    const int mid = ((q1 + 128) & 255) - 128;
+    const int hi = (q1 - mid) >> 8;
+    hw |= static_cast<uint32_t>(hi & 255) << (8 * e);
+    mw |= static_cast<uint32_t>(mid & 255) << (8 * e);
+    lw |= static_cast<uint32_t>(lo & 255) << (8 * e);
   }
-  reinterpret_cast<uint2 *>(out->hi)[lane] = make_uint2(hw[0], hw[1]);
-  reinterpret_cast<uint2 *>(out->lo)[lane] = make_uint2(lw[0], lw[1]);
-  if (lane == 0) out->inv = 1.0f / factor;
+  reinterpret_cast<uint32_t *>(out->hi)[lane] = hw;
+  reinterpret_cast<uint32_t *>(out->mid)[lane] = mw;
+  reinterpret_cast<uint32_t *>(out->lo)[lane] = lw;
+  if (lane == 0) out->inv = ok ? 16777216.0f / (qsc * csc) : (mx == 0.f ? 0.f : __int_as_float(0x7fc00000));
 }
 
 struct FastArgs {
@@ -195,6 +216,7 @@ struct FastArgs {
   int tiles_per_bh, tiles_per_cta, slots, stride;
   long long total_tiles;
   float kcent[16];
+  float kcsc; // 16-bit fixed-point scale of the key centroids
   float vcent[16];
   uint32_t one;
   int B;
@@ -258,13 +280,17 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
   const int r = lane >> 2, c = lane & 3;
 
   {
+    // key row e (256 bytes, the first 128 used): 32 lane copies of {hi(c0), hi(c1), lo(c0),
+    // lo(c1)} for the two codes of index e, the first in the low bits
     uint32_t *kw = reinterpret_cast<uint32_t *>(kl_p);
     for (int idx = tid; idx < L::kRows * 32; idx += kThreads) {
       const int e = idx >> 5, l = idx & 31;
       const float c0 = a.kcent[e & (KB == 4 ? 15 : 7)], c1 = a.kcent[KB == 4 ? e >> 4 : e >> 3];
-      const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
-      kw[e * 64 + 2 * l] = pack_h2(c0, c1);
-      kw[e * 64 + 2 * l + 1] = pack_h2((c0 - h0) * kLoScale, (c1 - h1) * kLoScale);
+      const int i0 = __float2int_rn(c0 * a.kcsc), i1 = __float2int_rn(c1 * a.kcsc);
+      const int l0 = ((i0 + 128) & 255) - 128, l1 = ((i1 + 128) & 255) - 128;
+      const int h0 = (i0 - l0) >> 8, h1 = (i1 - l1) >> 8;
+      kw[e * 64 + l] = static_cast<uint32_t>(h0 & 255) | (static_cast<uint32_t>(h1 & 255) << 8) |
+                       (static_cast<uint32_t>(l0 & 255) << 16) | (static_cast<uint32_t>(l1 & 255) << 24);
     }
     uint32_t *vw = reinterpret_cast<uint32_t *>(vl_p);
     for (int idx = tid; idx < L::vRows * 32; idx += kThreads) {
@@ -281,8 +307,8 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
     }
   }
   const uint32_t lanebase = static_cast<uint32_t>(lane) << 2;
-  const uint32_t klane8 = static_cast<uint32_t>(lane) << 3; // lane's 8-byte {hi, lo} entry
-  const uint32_t klb = klut | klane8;                          // 3-bit keys: base + lane offset
+  const uint32_t klane4 = static_cast<uint32_t>(lane) << 2; // lane's 4-byte key entry
+  const uint32_t klb = klut | klane4;                          // 3-bit keys: base + lane offset
   const uint32_t vlb = vlut | lanebase;
   const uint32_t one = a.one; // 1, opaque to the compiler so the add stays an IMAD
   __syncthreads();
@@ -295,7 +321,8 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
   // computation; otherwise an IMAD adds the base.
   auto run = [&](auto fixed_tag) {
     constexpr bool kFixed = decltype(fixed_tag)::value;
-    [[maybe_unused]] const uint32_t klane = klane8;
+    [[maybe_unused]] const uint32_t klane = klane4;
+    [[maybe_unused]] const uint32_t vlane8 = static_cast<uint32_t>(lane) << 3; // 2-bit values: 8-byte entry
     const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
     const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
     int slot = 0;
@@ -324,36 +351,51 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       seg = seg_end;
       const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
 
-      // ---- B operands of the score MMA: column n = r of n-tile nt is head g = 4 nt + r/2,
-      //      hi (r even) or residual (r odd); thread c holds coordinates [32c, 32c+32).
+      // ---- B operands of the score MMA: column n = r of n-tile nt < NT is head 4 nt + r/2,
+      //      {q_hi, q_hi, 0, 0} (r even) or {q_mid, q_mid, q_hi, q_hi} (r odd) at the k slots
+      //      of each coordinate pair; column r of n-tile NT is head r/2 (r even) or 4 + r/2
+      //      (r odd) with {q_lo, q_lo, q_mid, q_mid}. Thread c holds coordinates [32c, 32c+32),
+      //      k-step s its pairs 2s (b0) and 2s + 1 (b1).
       // ---- the segment's queries, rotated and split by warps 0 .. G-1 into the merge area
       //      (free between segments), then read as fragments by every warp
       QPrep *qs = reinterpret_cast<QPrep *>(obw);
       for (int g = warp; g < a.G; g += kWarps)
-        prep_query(a.q, a.q_dtype, static_cast<size_t>(b) * a.Hq + h * a.G + g, a.scale, a.seed, qs + g, lane);
+        prep_query(a.q, a.q_dtype, static_cast<size_t>(b) * a.Hq + h * a.G + g, a.scale, a.seed, a.kcsc,
+                   qs + g, lane);
       __syncthreads();
-      uint32_t qb[NT][16];
+      uint32_t qb[NT + 1][16];
       float qscale[NT];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int g = nt * 4 + (r >> 1);
+      for (int nt = 0; nt <= NT; ++nt) {
+        const int g = nt < NT ? nt * 4 + (r >> 1) : (r >> 1) + 4 * (r & 1);
         if (g < a.G) {
           const QPrep *p = qs + g;
-          const uint4 *src = reinterpret_cast<const uint4 *>(((r & 1) ? p->lo : p->hi) + 32 * c);
+          // the parts at the hi and the lo k slots of this column
+          const int8_t *xs = nt < NT ? ((r & 1) ? p->mid : p->hi) : p->lo;
+          const int8_t *ys = nt < NT ? p->hi : p->mid;
+          const bool ylo = nt == NT || (r & 1); // the lo slots are used
+          const uint4 *xv4 = reinterpret_cast<const uint4 *>(xs + 32 * c);
+          const uint4 *yv4 = reinterpret_cast<const uint4 *>(ys + 32 * c);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint4 w = src[k];
-            qb[nt][4 * k] = w.x;
-            qb[nt][4 * k + 1] = w.y;
-            qb[nt][4 * k + 2] = w.z;
-            qb[nt][4 * k + 3] = w.w;
+          for (int k = 0; k < 2; ++k) {
+            const uint4 xv = xv4[k];
+            const uint4 yv = ylo ? yv4[k] : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, yw[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int s = 4 * k + j; // word s holds coordinates 32c + 4s .. 32c + 4s + 3
+              qb[nt][2 * s] = prmt(xw[j], yw[j], 0x5410u);
+              qb[nt][2 * s + 1] = prmt(xw[j], yw[j], 0x7632u);
+            }
           }
         } else {
 #pragma unroll
           for (int k = 0; k < 16; ++k) qb[nt][k] = 0u;
         }
-        const int gs = nt * 4 + c; // head of this lane's score columns
-        qscale[nt] = gs < a.G ? qs[gs].inv * kLog2e : 0.f;
+        if (nt < NT) {
+          const int gs = nt * 4 + c; // head of this lane's score columns
+          qscale[nt] = gs < a.G ? qs[gs].inv * kLog2e : 0.f;
+        }
       }
 
       float m_run[NT], l_run[NT];
@@ -495,20 +537,19 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       };
 
       auto compute = [&](const TileT &T, int t0) {
-        // ---- scores. MMA A takes tokens r (its rows 0-7 hold the centroid hi, rows 8-15 the
-        //      residual lo of the same tokens), MMA B tokens r + 8, so one 64-bit table load
-        //      {hi, lo} fills an adjacent pair of A registers. k-step s takes the lane's
-        //      coordinate pairs 2s (a0, a1) and 2s + 1 (a2, a3).
-        float cA[NT][4], cB[NT][4];
+        // ---- scores. A rows r and r + 8 are tokens r and r + 8; k-step s takes the lane's
+        //      coordinate pairs 2s (a0: token r, a1: token r + 8) and 2s + 1 (a2, a3), one
+        //      32-bit table load each.
+        int acc[NT + 1][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt <= NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) cA[nt][e] = cB[nt][e] = 0.f;
+          for (int e = 0; e < 4; ++e) acc[nt][e] = kMagic;
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           uint32_t ad0, ad1, ad2, ad3;
           if constexpr (KB == 4) {
-            // table row (code byte << 8) + the lane's 8-byte entry; the base is an immediate
+            // table row (code byte << 8) + the lane's 4-byte entry; the base is an immediate
             // offset of the load or is added on the IMAD pipe
             const uint32_t sel0 = 0x7604u | (static_cast<uint32_t>((2 * s) & 3) << 4);
             const uint32_t sel1 = 0x7604u | (static_cast<uint32_t>((2 * s + 1) & 3) << 4);
@@ -530,23 +571,20 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
             ad2 = lop_and_or(bits_at(T.k[0], 12 * s + 6, 8), 0x3F00u, klb);
             ad3 = lop_and_or(bits_at(T.k[1], 12 * s + 6, 8), 0x3F00u, klb);
           }
-          uint2 e0, e1, e2, e3;
+          uint32_t e0, e1, e2, e3;
           if constexpr (KB == 4 && kFixed) {
-            e0 = lds64_off<kFixedBase>(ad0);
-            e1 = lds64_off<kFixedBase>(ad1);
-            e2 = lds64_off<kFixedBase>(ad2);
-            e3 = lds64_off<kFixedBase>(ad3);
+            e0 = lds32_off<kFixedBase>(ad0);
+            e1 = lds32_off<kFixedBase>(ad1);
+            e2 = lds32_off<kFixedBase>(ad2);
+            e3 = lds32_off<kFixedBase>(ad3);
           } else {
-            e0 = lds64_off<0>(ad0);
-            e1 = lds64_off<0>(ad1);
-            e2 = lds64_off<0>(ad2);
-            e3 = lds64_off<0>(ad3);
+            e0 = lds32_off<0>(ad0);
+            e1 = lds32_off<0>(ad1);
+            e2 = lds32_off<0>(ad2);
+            e3 = lds32_off<0>(ad3);
           }
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma16816(cA[nt], e0.x, e0.y, e2.x, e2.y, qb[nt][2 * s], qb[nt][2 * s + 1]);
-            mma16816(cB[nt], e1.x, e1.y, e3.x, e3.y, qb[nt][2 * s], qb[nt][2 * s + 1]);
-          }
+          for (int nt = 0; nt <= NT; ++nt) imma16832(acc[nt], e0, e1, e2, e3, qb[nt][2 * s], qb[nt][2 * s + 1]);
         }
 
         // ---- online softmax (log2 domain); lane (r, c) owns head 4 nt + c, tokens r, r+8
@@ -560,11 +598,15 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
         bool rescale = false;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          // token r: hi x q_hi, hi x q_lo, lo x q_hi from MMA A; token r + 8 from MMA B
-          const float hh0 = cA[nt][0], hl0 = cA[nt][1], lh0 = cA[nt][2];
-          const float hh1 = cB[nt][0], hl1 = cB[nt][1], lh1 = cB[nt][2];
-          const float s0 = ok0 ? kn0 * qscale[nt] * fmaf(hl0 + lh0, kLoInv, hh0) : -INFINITY;
-          const float s1 = ok1 ? kn1 * qscale[nt] * fmaf(hl1 + lh1, kLoInv, hh1) : -INFINITY;
+          // token r: columns 2c (2^24 terms) and 2c + 1 (2^16) in acc 0, 1 of n-tile nt and the
+          // 2^8 column of the same head in acc nt of n-tile NT; token r + 8 in acc 2, 3 and
+          // 2 + nt
+          const float d0 = fmaf(__int_as_float(acc[NT][nt]), 1.0f / 65536.0f,
+                                fmaf(__int_as_float(acc[nt][1]), 1.0f / 256.0f, __int_as_float(acc[nt][0]) - kMagicAdj));
+          const float d1 = fmaf(__int_as_float(acc[NT][2 + nt]), 1.0f / 65536.0f,
+                                fmaf(__int_as_float(acc[nt][3]), 1.0f / 256.0f, __int_as_float(acc[nt][2]) - kMagicAdj));
+          const float s0 = ok0 ? kn0 * qscale[nt] * d0 : -INFINITY;
+          const float s1 = ok1 ? kn1 * qscale[nt] * d1 : -INFINITY;
           float mx = fmaxf(s0, s1);
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -631,11 +673,11 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
             const uint32_t x01 = (m & 1) ? w01 : u01, x23 = (m & 1) ? w23 : u23;
             uint2 e01, e23;
             if constexpr (kFixed) {
-              e01 = lds64_off<kFixedBase + L::kBytes>(prmt(x01, klane, sel));
-              e23 = lds64_off<kFixedBase + L::kBytes>(prmt(x23, klane, sel));
+              e01 = lds64_off<kFixedBase + L::kBytes>(prmt(x01, vlane8, sel));
+              e23 = lds64_off<kFixedBase + L::kBytes>(prmt(x23, vlane8, sel));
             } else {
-              e01 = lds64_off<0>(imad(prmt(x01, klane, sel), one, vlut));
-              e23 = lds64_off<0>(imad(prmt(x23, klane, sel), one, vlut));
+              e01 = lds64_off<0>(imad(prmt(x01, vlane8, sel), one, vlut));
+              e23 = lds64_off<0>(imad(prmt(x23, vlane8, sel), one, vlut));
             }
             mma16816(o[m], e01.x, e01.y, e23.x, e23.y, pb0, pb1);
           }
@@ -957,6 +999,7 @@ cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
   f.stride = p.ws_stride;
   f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
   for (int j = 0; j < 16; ++j) f.kcent[j] = a.k.cb.c[j];
+  f.kcsc = a.k.cb.fix_scale;
   for (int j = 0; j < 16; ++j) f.vcent[j] = a.v.cb.c[j];
   f.one = 1u;
   f.B = a.B;

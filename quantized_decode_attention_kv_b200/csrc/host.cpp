@@ -60,7 +60,43 @@ struct DoubleCodebook {
   double c[16], beta[15];
   int levels;
   bool ok;
+  double fix_scale;
 };
+
+// Scale S of the centroids as 16-bit fixed-point integers rint(c_j S), |rint(c_j S)| <= 32639,
+// chosen among 40000 candidates in [0.6, 1] x the largest admissible one to minimise the
+// rounding error sum_j P_j (rint(c_j S) - c_j S)^2 / S^2 (P_j: the probability of level j under
+// N(0, 1)); the products are rounded in float32, as the decode kernel forms them.
+double fixed_point_scale(const double *c, int L) {
+  double cmax = 0.0;
+  for (int j = 0; j < L; ++j) cmax = std::fmax(cmax, std::fabs(c[j]));
+  double prob[16];
+  for (int j = 0; j < L; ++j) {
+    const double lo = j == 0 ? -INFINITY : 0.5 * (c[j - 1] + c[j]);
+    const double hi = j == L - 1 ? INFINITY : 0.5 * (c[j] + c[j + 1]);
+    prob[j] = ncdf(hi) - ncdf(lo);
+  }
+  const double smax = 32639.0 / cmax;
+  double best = smax, best_err = INFINITY;
+  constexpr int kCand = 40000;
+  for (int i = 0; i < kCand; ++i) {
+    const float sf = static_cast<float>(smax * (1.0 - 0.4 * i / kCand));
+    double err = 0.0;
+    bool fits = true;
+    for (int j = 0; j < L; ++j) {
+      const float v = static_cast<float>(c[j]) * sf;
+      const double r = std::nearbyint(static_cast<double>(v));
+      fits = fits && std::fabs(r) <= 32639.0;
+      const double e = (r - c[j] * static_cast<double>(sf)) / sf;
+      err += prob[j] * e * e;
+    }
+    if (fits && err < best_err) {
+      best_err = err;
+      best = sf;
+    }
+  }
+  return best;
+}
 
 DoubleCodebook compute_lloyd_max(int wbits) {
   DoubleCodebook cb{};
@@ -93,6 +129,7 @@ DoubleCodebook compute_lloyd_max(int wbits) {
   }
   for (int j = 0; j < L; ++j) cb.c[j] = c[j];
   for (int j = 0; j + 1 < L; ++j) cb.beta[j] = 0.5 * (c[j] + c[j + 1]);
+  cb.fix_scale = fixed_point_scale(cb.c, L);
   return cb;
 }
 
@@ -161,6 +198,7 @@ int resolve_tensor(const tq_cache &c, int which, tq::TensorArgs *t) {
     cb.levels = d.levels;
     for (int j = 0; j < d.levels; ++j) cb.c[j] = static_cast<float>(d.c[j]);
     for (int j = 0; j + 1 < d.levels; ++j) cb.beta[j] = static_cast<float>(d.beta[j]);
+    cb.fix_scale = static_cast<float>(d.fix_scale);
   }
   return TQ_OK;
 }

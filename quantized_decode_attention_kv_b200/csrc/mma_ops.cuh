@@ -1,5 +1,6 @@
 // Register-level helpers of the tensor-core decode kernels (fp16 packing, PRMT, IMAD,
-// shared loads and the m16n8k16 f16 MMA with fp32 accumulators).
+// shared loads, the m16n8k16 f16 MMA with fp32 accumulators and the m16n8k32 s8 MMA with
+// int32 accumulators).
 #pragma once
 
 #include "tq_device.cuh"
@@ -37,6 +38,17 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A . B + C on int8 operands with int32 accumulators (m16n8k32): A rows 16 x k 32 (four
+// s8 per register), B k 32 x columns 8 (four s8 per register).
+__device__ __forceinline__ void imma16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 

@@ -16,6 +16,7 @@ struct Codebook {
   float c[16];    // centroids, ascending (levels entries used)
   float beta[15]; // decision boundaries, ascending (levels - 1 used)
   int levels;     // 2^wbits; 1 when a PROD record carries no Lloyd-Max codes
+  float fix_scale; // 16-bit fixed-point scale of the centroids (|rint(c * fix_scale)| <= 32639)
 };
 
 // One tensor (K or V) of a cache, resolved from tq_cache + tq_qcfg.
