@@ -81,6 +81,13 @@ def decode_sources_digest() -> str:
     return h.hexdigest()
 
 
+ARITH_MSE = ("u8 packed codes; scores on int8 tensor cores (16-bit fixed-point centroids x 24-bit "
+             "fixed-point queries, int32 accumulation), P.V on f16 tensor cores with f32 "
+             "accumulation; f32 softmax")
+ARITH_PROD = ("u8 packed codes and sign bits as exact +-1 f16 operands; scores and P.V on f16 tensor "
+              "cores with f32 accumulation (hi/lo split query side); f32 softmax")
+
+
 class Clocks:
     """nvidia-smi samples every 100 ms while the timed loop runs."""
 
@@ -277,14 +284,13 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16-mma/f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "i8+f16-mma/f32", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
                    "k": f"{w.k_bits}-bit {'MSE' if w.k_mode == 0 else 'PROD'}",
                    "v": f"{w.v_bits}-bit {'MSE' if w.v_mode == 0 else 'PROD'}",
                    "packed_bytes_per_step": packed,
                    "step": "quantise 1 new token (K,V) + decode attention over T tokens",
-                   "arithmetic": ("u8 packed codes; scores and P.V on f16 tensor cores with f32 "
-                                  "accumulation (hi/lo split centroids and query); f32 softmax"),
+                   "arithmetic": ARITH_MSE if w.k_mode == 0 else ARITH_PROD,
                    "l2": "no flush: packed cache per step larger than the 126 MB L2",
                    "parallelism": f"{world} independent replica(s), one per GPU"},
         "gpu_launches": launches_per_step * args.steps,

@@ -186,19 +186,21 @@ def test_decode_query_dtypes(q_dtype):
     P.assert_attention_close(P.to_np(out), P.oracle_decode(P.to_np(q), k_recs, v_recs, B, Hkv, 0.3, T_len))
 
 
-def test_decode_with_large_key_norms():
+@pytest.mark.parametrize("G,kb,vb,T", [(8, 4, 2, 700), (4, 4, 2, 2000), (3, 3, 3, 1500), (2, 4, 4, 900)])
+def test_decode_with_large_key_norms(G, kb, vb, T):
     # keys 50x the values' norm ("What the Paper Doesn't Tell You", Finding 1): near-one-hot
-    # softmax, where score precision decides the output
-    case = (128, 8, 1, (4, O.MSE), (2, O.MSE), 0, 700, 700)
-    B, Hq, K, V, q = _decode_case(case, torch.bfloat16, k_scale=50.0, seed=3)
-    cache = tq.TQCache(B, 1, 700, 128, 4, 2)
-    k_recs = P.oracle_records(P.to_np(K), 4, O.MSE, 0, 1, None)
-    v_recs = P.oracle_records(P.to_np(V), 2, O.MSE, 0, 1, None)
+    # softmax, where score precision decides the output; every query-group width and key
+    # bit-width of the tensor-core kernel (the last score n-tile full or half used)
+    case = (128, G, 1, (kb, O.MSE), (vb, O.MSE), 0, T, T)
+    B, Hq, K, V, q = _decode_case(case, torch.bfloat16, k_scale=50.0, seed=3 + G)
+    cache = tq.TQCache(B, 1, T, 128, kb, vb)
+    k_recs = P.oracle_records(P.to_np(K), kb, O.MSE, 0, 1, None)
+    v_recs = P.oracle_records(P.to_np(V), vb, O.MSE, 0, 1, None)
     P.upload(cache, "k", k_recs)
     P.upload(cache, "v", v_recs)
     out = torch.empty(B, Hq, 128, device="cuda")
-    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, 700))
-    tq.tq_decode_attention(q.cuda(), cache, 700, 128 ** -0.5, out, ws)
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, T))
+    tq.tq_decode_attention(q.cuda(), cache, T, 128 ** -0.5, out, ws)
     torch.cuda.synchronize()
     P.assert_attention_close(P.to_np(out), P.oracle_decode(P.to_np(q), k_recs, v_recs, B, 1, 128 ** -0.5))
 
@@ -222,6 +224,28 @@ def test_quantize_then_decode_end_to_end(case):
     v_recs = P.oracle_records(P.to_np(Vb[:, :, :T_len]), vb, vm, 6, 3, m or None)
     want = P.oracle_decode(P.to_np(q), k_recs, v_recs, B, Hkv, d ** -0.5)
     P.assert_attention_close(P.to_np(out), want)
+
+
+def test_decode_zero_query_head_attends_uniformly():
+    # an all-zero query has no fixed-point scale: its scores are all zero (uniform weights)
+    # while the other heads of the same KV head decode normally
+    case = (128, 4, 2, (4, O.MSE), (2, O.MSE), 0, 333, 333)
+    B, Hq, K, V, q = _decode_case(case, torch.bfloat16, seed=12)
+    q[0, 1] = 0.0
+    q[1, 6] = 0.0
+    cache = tq.TQCache(B, 2, 333, 128, 4, 2)
+    k_recs = P.oracle_records(P.to_np(K), 4, O.MSE, 0, 1, None)
+    v_recs = P.oracle_records(P.to_np(V), 2, O.MSE, 0, 1, None)
+    P.upload(cache, "k", k_recs)
+    P.upload(cache, "v", v_recs)
+    out = torch.empty(B, Hq, 128, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, 333))
+    tq.tq_decode_attention(q.cuda(), cache, 333, 128 ** -0.5, out, ws)
+    torch.cuda.synchronize()
+    want = P.oracle_decode(P.to_np(q), k_recs, v_recs, B, 2, 128 ** -0.5)
+    P.assert_attention_close(P.to_np(out), want)
+    vh = O.dequantize(v_recs[0])
+    np.testing.assert_allclose(want[0, 1], vh.mean(axis=0), rtol=1e-9, atol=1e-12)
 
 
 def test_decode_rejects_small_workspace_and_empty_context():
