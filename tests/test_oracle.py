@@ -163,6 +163,37 @@ def test_distortion_monte_carlo_and_information_bound(bits):
     assert abs(math.sqrt(3) * math.pi / 2 - 2.72) < 1e-3
 
 
+def _gaussian_mse(levels):
+    """MSE of nearest-level quantisation of N(0,1) by numerical integration over the cells."""
+    levels = np.sort(np.asarray(levels, dtype=np.float64))
+    edges = np.concatenate([[-np.inf], (levels[1:] + levels[:-1]) / 2, [np.inf]])
+    pdf = scipy.stats.norm.pdf
+    return sum(scipy.integrate.quad(lambda t: (t - l) ** 2 * pdf(t), edges[j], edges[j + 1])[0]
+               for j, l in enumerate(levels))
+
+
+def test_e2m1_grid_cannot_hold_the_four_bit_codebook():
+    # The open question of mapping the Lloyd-Max centroids onto Blackwell's FP4 (E2M1) format
+    # ("Where This Fits in the Inference Stack", Blackwell FP4). E2M1 holds 0, 0.5, 1, 1.5, 2,
+    # 3, 4, 6 and their negatives (15 values); a per-block scale s only stretches the grid.
+    c, _, dist = O.lloyd_max_gaussian(4)
+    e2m1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6.0])
+    grid = np.unique(np.concatenate([-e2m1, e2m1]))
+    assert grid.size == 15
+    # (1) as a quantiser, the best stretched grid has a third more MSE than Lloyd-Max
+    scales = np.linspace(0.3, 0.8, 201)
+    mses = np.array([_gaussian_mse(grid * s) for s in scales])
+    best = mses.min()
+    assert abs(_gaussian_mse(c) - dist) < 1e-8
+    assert best > 1.30 * dist and 0.45 < scales[mses.argmin()] < 0.52
+    # (2) keeping the codes and moving each centroid to the nearest stretched E2M1 value merges
+    # two pairs of levels and moves some centroid by more than 0.1 at every scale
+    for s in scales:
+        mapped = (grid * s)[np.abs(c[:, None] - (grid * s)[None, :]).argmin(axis=1)]
+        assert np.unique(mapped).size < 16
+        assert np.abs(mapped - c).max() > 0.1
+
+
 def test_codebook_scales_with_inverse_sqrt_d():
     # "codebook centroids scale with 1/sqrt(d) for your specific head dimension"
     for d in (64, 128):
