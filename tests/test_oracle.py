@@ -186,6 +186,8 @@ def test_e2m1_grid_cannot_hold_the_four_bit_codebook():
     best = mses.min()
     assert abs(_gaussian_mse(c) - dist) < 1e-8
     assert best > 1.30 * dist and 0.45 < scales[mses.argmin()] < 0.52
+    # ... and breaks the pages' guarantee D_b <= (sqrt(3) pi / 2) 4^-b (Three-Step Summary)
+    assert best > (math.sqrt(3) * math.pi / 2) * 4.0 ** -4 > dist
     # (2) keeping the codes and moving each centroid to the nearest stretched E2M1 value merges
     # two pairs of levels and moves some centroid by more than 0.1 at every scale
     for s in scales:
