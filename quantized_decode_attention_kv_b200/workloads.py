@@ -65,6 +65,10 @@ WORKLOADS = {
                  v_bits=3, k_outliers=4, k_jitter=True, layers=32),
         Workload("llama70b_asym_16k", 4, B=32, Hq=64, Hkv=8, d=128, T=16384, k_bits=4, v_bits=2,
                  k_scale=50.0, layers=80, bf16_layers=(0, 1, 78, 79)),
+        # the pages' 3.5-bit operating point read as 4-bit keys and 3-bit values (3.5 bits per
+        # cached coordinate on average) on the Llama-3.1-8B shape
+        Workload("llama3_8b_32k_3p5bit", 5, B=16, Hq=32, Hkv=8, d=128, T=32768, k_bits=4,
+                 v_bits=3, k_outliers=4, k_jitter=True),
     ]
 }
 

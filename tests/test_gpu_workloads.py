@@ -52,7 +52,7 @@ def _check_full(w, layer=0, samples=((0, 0), (-1, -1))):
 
 
 @pytest.mark.parametrize("name", ["tiny_single_head_fp32", "llama3_8b_decode_32k", "gpt2_prod_2bit",
-                                  "llama3_8b_128k_3bit", "llama70b_asym_16k"])
+                                  "llama3_8b_128k_3bit", "llama70b_asym_16k", "llama3_8b_32k_3p5bit"])
 def test_full_size_workload_sampled_parity(name):
     w = WORKLOADS[name]
     stats = _check_full(w)

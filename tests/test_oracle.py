@@ -225,6 +225,18 @@ def test_packing_round_trip(width):
     assert np.array_equal(O.unpack_bits(p, width, 128), v)
 
 
+def test_three_and_a_half_bit_reading_of_the_headline_rate():
+    # "3.5 bits per coordinate ... 4.6x over FP16" (One-Slide Version; Finding 3) read as 4-bit
+    # keys and 3-bit values: 3.5 code bits per cached coordinate, 16 / 3.5 = 4.57x on the codes
+    # alone, 4.41x with the fp16 norms of both records
+    d = 128
+    code_bits = (O.code_bytes(d, 4, O.MSE) + O.code_bytes(d, 3, O.MSE)) * 8
+    assert code_bits / (2 * d) == 3.5
+    assert round(2 * d * 16 / code_bits, 1) == 4.6
+    rec = O.record_bytes(d, 4, O.MSE) + O.record_bytes(d, 3, O.MSE)
+    assert rec == 116 and 4.4 < 2 * d * 2 / rec < 4.42
+
+
 def test_record_sizes_match_published_compression_ratios():
     # "3 bits ... (block_size=128: 5.12x)", "4 bits ... ~4x" (Finding 3): per 128-vector,
     # fp16 costs 256 bytes.
