@@ -72,12 +72,36 @@ def kernel_traffic():
     return rec.get("dram_bytes_per_launch")
 
 
+def _code_only(src: str) -> str:
+    """C++ source without comments and whitespace (string literals kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif src[i] == '"':
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            if not src[i].isspace():
+                out.append(src[i])
+            i += 1
+    return "".join(out)
+
+
 def decode_sources_digest() -> str:
-    """sha256 over the sources of the bench's dominant kernel (the tensor-core decode)."""
+    """sha256 over the code (comments and whitespace removed) of the bench's dominant kernel's
+    sources (the tensor-core decode)."""
     h = hashlib.sha256()
     for name in ("decode_mma.cu", "mma_ops.cuh"):
-        with open(os.path.join(ROOT, "quantized_decode_attention_kv_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "quantized_decode_attention_kv_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

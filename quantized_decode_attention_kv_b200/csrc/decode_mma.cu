@@ -1,5 +1,5 @@
-// Tensor-core decode attention over the compressed cache (head_dim 128, 4-bit keys, 2-bit
-// values, TurboQuant_mse, up to 8 query heads per KV head).
+// Tensor-core decode attention over the compressed cache (head_dim 128, TurboQuant_mse with
+// 3- or 4-bit keys and 2-, 3- or 4-bit values, up to 8 query heads per KV head).
 //
 // "Where This Fits in the Inference Stack", TensorRT-LLM section: dequantise in registers
 // inside the attention kernel. Here the dequantised codes are written straight into the
@@ -8,9 +8,9 @@
 //   scores  S[16 tokens x 3 per head] = K^[16 x 2*128] . Q[2*128 x 3 per head]
 //     (mma.sync m16n8k32, int8 x int8 -> int32). Centroids are 16-bit fixed-point numbers
 //     c = 256 c_hi + c_lo, queries 24-bit ones q = 65536 q_hi + 256 q_mid + q_lo, each part an
-//     int8. K^ comes from a shared-memory LUT indexed by one code byte (two 4-bit codes) whose
-//     4-byte entry is {hi, hi, lo, lo} of the two centroids, i.e. four consecutive k slots of
-//     one A row. Per head three columns take {q_hi, 0}, {q_mid, q_hi} and {q_lo, q_mid} at the
+//     int8. K^ comes from a shared-memory LUT indexed by the codes of two adjacent coordinates
+//     (a code byte of 4-bit keys, 6 bits of 3-bit keys) whose 4-byte entry is
+//     {hi, hi, lo, lo} of the two centroids, i.e. four consecutive k slots of one A row. Per head three columns take {q_hi, 0}, {q_mid, q_hi} and {q_lo, q_mid} at the
 //     {hi, lo} slots, so c.q = 2^24 col0 + 2^16 col1 + 2^8 col2 up to c_lo q_lo (2^-24 of the
 //     scale); the rounding of the centroids to 16 bits, at a scale chosen to make it small, is
 //     the only other error.
@@ -20,9 +20,9 @@
 //     3/4-bit V^: one table word per token and pair of adjacent coordinates, two PRMTs per
 //     pair of operand registers. P' = p * ||v_t|| in fp16.
 //
-// The contraction order is free along k, so each thread owns a contiguous 16-byte slice of
-// every key record and one 32-bit word of every value record: all loads are 16- or 4-byte,
-// and the permutation is undone when the partial accumulators are written.
+// The contraction order is free along k, so each thread owns a contiguous slice of every key
+// record (16 bytes of 4-bit codes, 12 of 3-bit codes) and one or two 32-bit words of every
+// value record, and the permutation is undone when the partial accumulators are written.
 //
 // Work split: the (batch, KV head, 16-token tile) space is flattened and cut into equal
 // contiguous ranges, one per persistent CTA (12 warps with 2-bit values, else 4); within a
@@ -108,9 +108,10 @@ struct Tile {
 
 // Shared-memory tables of one configuration. Key rows: one code-pair index (4-bit keys: a
 // byte of two codes, 256 rows; 3-bit keys: 6 bits, 64 rows) x 32 lane copies of the 4-byte
-// int8 entry {hi, hi, lo, lo}, in a 256-byte row (the index lands above bit 8 of the address). Value rows, 2-bit values: one byte holding the
-// codes of two adjacent coordinates of two tokens (low nibble the first token) x 32 lane
-// copies of the two fp16x2 operand words = 256 bytes; 3/4-bit values: one index (the codes of
+// int8 entry {hi, hi, lo, lo}, in a 256-byte row of which the first 128 bytes are used (the
+// index lands at bit 8 of the address). Value rows, 2-bit values: one byte holding the codes
+// of two adjacent coordinates of two tokens (low nibble the first token) x 32 lane copies of
+// the two fp16x2 operand words = 256 bytes; 3/4-bit values: one index (the codes of
 // two adjacent coordinates of one token, the first in the low bits) x 32 lane copies of the
 // fp16x2 pair of their centroids = 128 bytes.
 // The 3-bit key table and the 3/4-bit value tables sit at addresses aligned to their size so
