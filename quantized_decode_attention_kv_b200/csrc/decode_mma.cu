@@ -25,7 +25,7 @@
 // value record, and the permutation is undone when the partial accumulators are written.
 //
 // Work split: the (batch, KV head, 16-token tile) space is flattened and cut into equal
-// contiguous ranges, one per persistent CTA (12 warps with 2-bit values, else 4); within a
+// contiguous ranges, one per persistent CTA (12 warps with 2-bit values or 4-bit keys, else 4); within a
 // range each maximal run of one (batch, KV head) is a segment, its tiles dealt round-robin to
 // the warps, each warp keeping its own online-softmax state (log2 domain); at the end of the
 // segment the warps store their rescaled accumulators in their own shared-memory slots, which
@@ -65,13 +65,15 @@ constexpr int kPrefetchSteps = TQ_DECODE_PREFETCH;
 constexpr uint32_t kFixedBase = 1024;
 
 // Warps per CTA and CTAs per SM. 2-bit values use a 64 KB value table beside the 64 KB key
-// table, so one CTA of 12 warps per SM shares both; other configurations run three CTAs of 4
-// warps (12 warps of up to 168 registers per SM either way; 16 warps of 128 registers were
-// measured slower).
+// table, and 4-bit keys keep the 3/4-bit value table in the unused halves of their 64 KB of
+// key rows, so these configurations run one CTA of 12 warps per SM sharing the tables; 3-bit
+// keys with 3/4-bit values run three CTAs of 4 warps (12 warps of up to 168 registers per SM
+// either way; 16 warps of 128 registers were measured slower).
 template <int KB, int VB>
 struct Cfg {
-  static constexpr int kWarps = VB == 2 ? 12 : 4;
-  static constexpr int kCtas = VB == 2 ? 1 : 3;
+  static constexpr bool kOneCta = VB == 2 || KB == 4;
+  static constexpr int kWarps = kOneCta ? 12 : 4;
+  static constexpr int kCtas = kOneCta ? 1 : 3;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kStep = kWarps * 16; // tokens a warp advances per step
 };
@@ -113,7 +115,7 @@ struct Tile {
 // of two adjacent coordinates of two tokens (low nibble the first token) x 32 lane copies of
 // the two fp16x2 operand words = 256 bytes; 3/4-bit values: one index (the codes of
 // two adjacent coordinates of one token, the first in the low bits) x 32 lane copies of the
-// fp16x2 pair of their centroids = 128 bytes.
+// fp16x2 pair of their centroids = 128 bytes (with 4-bit keys: the unused half of key row i).
 // The 3-bit key table and the 3/4-bit value tables sit at addresses aligned to their size so
 // that an index OR-ed above the lane offset is already the address.
 template <int KB, int VB>
@@ -121,9 +123,11 @@ struct Lut {
   static constexpr int kRows = KB == 4 ? 256 : 64;
   static constexpr int kBytes = kRows * 256;
   static constexpr int kAlign = KB == 4 ? 16 : kBytes;
+  // 4-bit keys with 3/4-bit values: value row i is the second 128 bytes of key row i
+  static constexpr bool kVInK = KB == 4 && VB >= 3;
   static constexpr int vRows = VB >= 3 ? 1 << (2 * VB) : 256;
-  static constexpr int vBytes = vRows * (VB >= 3 ? 128 : 256);
-  static constexpr int vAlign = VB >= 3 ? vBytes : 16;
+  static constexpr int vBytes = kVInK ? 0 : vRows * (VB >= 3 ? 128 : 256);
+  static constexpr int vAlign = VB >= 3 && !kVInK ? vBytes : 16;
   // merge area: per-warp maxima and sums [warps][8] each, merged [8] each, then the per-warp
   // value accumulators [warps][8 m-tiles][32 lanes] float4
   static constexpr int kMergeBytes = (2 * Cfg<KB, VB>::kWarps * 8 + 16) * 4 + Cfg<KB, VB>::kWarps * 256 * 16;
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
   const int r = lane >> 2, c = lane & 3;
 
   {
-    // key row e (256 bytes, the first 128 used): 32 lane copies of {hi(c0), hi(c1), lo(c0),
+    // key row e (first 128 of its 256 bytes): 32 lane copies of {hi(c0), hi(c1), lo(c0),
     // lo(c1)} for the two codes of index e, the first in the low bits
     uint32_t *kw = reinterpret_cast<uint32_t *>(kl_p);
     for (int idx = tid; idx < L::kRows * 32; idx += kThreads) {
@@ -296,7 +300,9 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
     uint32_t *vw = reinterpret_cast<uint32_t *>(vl_p);
     for (int idx = tid; idx < L::vRows * 32; idx += kThreads) {
       const int e = idx >> 5;
-      if constexpr (VB == 2) {
+      if constexpr (L::kVInK) {
+        kw[e * 64 + 32 + (idx & 31)] = pack_h2(a.vcent[e & ((1 << VB) - 1)], a.vcent[e >> VB]);
+      } else if constexpr (VB == 2) {
         // byte e: first token's codes at coordinates j, j+1 in bits 0-1, 2-3, the second
         // token's in bits 4-5, 6-7; words: coordinate j, coordinate j+1 (tokens in halves)
         const int l = idx & 31;
@@ -311,6 +317,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
   const uint32_t klane4 = static_cast<uint32_t>(lane) << 2; // lane's 4-byte key entry
   const uint32_t klb = klut | klane4;                          // 3-bit keys: base + lane offset
   const uint32_t vlb = vlut | lanebase;
+  [[maybe_unused]] const uint32_t vkb = klut + 128; // value rows inside the key rows
   const uint32_t one = a.one; // 1, opaque to the compiler so the add stays an IMAD
   __syncthreads();
   pdl_wait(); // the prepared queries and the cache are written by earlier kernels
@@ -698,12 +705,23 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
               run[t][1] = T.v[t][1];
             }
           }
-          constexpr uint32_t MI = ((1u << (2 * VB)) - 1u) << 7;
+          // row index above the lane offset: at bit 7 of a size-aligned table, or at bit 8 (rows
+          // 256 bytes apart) in the second halves of the 4-bit key rows
+          constexpr int kIxBit = L::kVInK ? 8 : 7;
+          constexpr uint32_t MI = ((1u << (2 * VB)) - 1u) << kIxBit;
 #pragma unroll
           for (int m = 0; m < 8; ++m) {
             uint32_t w[4];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) w[t] = lds32(lop_and_or(bits_at(run[t], 2 * VB * m, 7), MI, vlb));
+            for (int t = 0; t < 4; ++t) {
+              if constexpr (!L::kVInK) {
+                w[t] = lds32_off<0>(lop_and_or(bits_at(run[t], 2 * VB * m, kIxBit), MI, vlb));
+              } else if constexpr (kFixed) {
+                w[t] = lds32_off<kFixedBase + 128>(lop_and_or(bits_at(run[t], 2 * VB * m, kIxBit), MI, lanebase));
+              } else {
+                w[t] = lds32_off<0>(imad(lop_and_or(bits_at(run[t], 2 * VB * m, kIxBit), MI, lanebase), one, vkb));
+              }
+            }
             mma16816(o[m], prmt(w[0], w[1], 0x5410u), prmt(w[0], w[1], 0x7632u), prmt(w[2], w[3], 0x5410u),
                      prmt(w[2], w[3], 0x7632u), pb0, pb1);
           }
