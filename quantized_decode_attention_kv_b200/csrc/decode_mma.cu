@@ -25,11 +25,11 @@
 // value record, and the permutation is undone when the partial accumulators are written.
 //
 // Work split: the (batch, KV head, 16-token tile) space is flattened and cut into equal
-// contiguous ranges, one per persistent CTA (12 warps with 2-bit values or 4-bit keys, else 4); within a
-// range each maximal run of one (batch, KV head) is a segment, its tiles dealt round-robin to
-// the warps, each warp keeping its own online-softmax state (log2 domain); at the end of the
-// segment the warps store their rescaled accumulators in their own shared-memory slots, which
-// are summed into one partial record per query head.
+// contiguous ranges, one per persistent CTA (12 warps with 2-bit values or 4-bit keys, else
+// 4); within a range each maximal run of one (batch, KV head) is a segment, its tiles dealt
+// round-robin to the warps, each warp keeping its own online-softmax state (log2 domain); at
+// the end of the segment the warps store their rescaled accumulators in their own
+// shared-memory slots, which are summed into one partial record per query head.
 #include "mma_ops.cuh"
 
 #include <algorithm>
