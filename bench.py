@@ -336,6 +336,8 @@ def run_ours(args):
             line["ragged_decode"] = side["ragged"]
         if "paged" in side:
             line["paged_decode"] = side["paged"]
+        if "k4v3" in side:
+            line["decode_3p5bit"] = side["k4v3"]
     print(json.dumps(line), flush=True)
 
 
@@ -412,6 +414,18 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
                         "page_size": page, "layout": f"{npages} pages of {page} positions, scattered by a "
                                                      f"seeded permutation; every sequence at full length"}
         del pc, bt, wsp
+    # the pages' 3.5-bit operating point (4-bit keys, 3-bit values) on the same inputs
+    if w.d == 128 and w.k_mode == 0 and w.v_mode == 0 and (w.k_bits, w.v_bits) != (4, 3):
+        c35 = tq.TQCache(w.B, w.Hkv, w.T, w.d, 4, 3, seed=cache.seed)
+        tq.tq_quantize_kv(K, V, c35, stream=stream)
+        b35 = c35.packed_bytes(w.T)
+        ws35 = tq.workspace(tq.tq_decode_workspace_bytes(c35, w.Hq, w.T))
+        s35 = _time(lambda: tq.tq_decode_attention(q, c35, w.T, w.scale, out, ws35, stream=stream),
+                    stream, max(args.steps // 4, 20), torch)
+        res["k4v3"] = {"us": s35 * 1e6, "gbs": b35 / s35 / 1e9, "frac": b35 / s35 / 1e9 / hbm,
+                       "bytes": b35, "k": "4-bit MSE", "v": "3-bit MSE",
+                       "reading": "3.5 bits per cached coordinate as 4-bit keys + 3-bit values"}
+        del c35, ws35
     # end to end through the C ABI from pinned host buffers, as a serving loop runs it: every
     # step copies its inputs (query, the new token's K and V) in from pinned memory, runs the
     # two calls and reads its attention output back; the copies run on their own streams and
