@@ -188,8 +188,9 @@ __device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, 
     mx = fmaxf(mx, fabsf(x[e]));
   }
   mx = warp_max(mx);
-  // all-zero query: zero scores; a non-finite one makes the scores NaN
-  const bool ok = mx > 0.f && isfinite(mx);
+  // a query whose largest coordinate is below 1e-30 (zero included) gets zero scores (its
+  // exact scores are below 1e-30 times the key norms); a non-finite one makes them NaN
+  const bool ok = mx > 1e-30f && isfinite(mx);
   const float qsc = ok ? kQFixMax / mx : 0.f;
   uint32_t hw = 0, mw = 0, lw = 0;
 #pragma unroll
@@ -206,7 +207,7 @@ __device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, 
   reinterpret_cast<uint32_t *>(out->hi)[lane] = hw;
   reinterpret_cast<uint32_t *>(out->mid)[lane] = mw;
   reinterpret_cast<uint32_t *>(out->lo)[lane] = lw;
-  if (lane == 0) out->inv = ok ? 16777216.0f / (qsc * csc) : (mx == 0.f ? 0.f : __int_as_float(0x7fc00000));
+  if (lane == 0) out->inv = ok ? 16777216.0f / (qsc * csc) : (isfinite(mx) ? 0.f : __int_as_float(0x7fc00000));
 }
 
 struct FastArgs {

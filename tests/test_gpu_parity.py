@@ -226,13 +226,16 @@ def test_quantize_then_decode_end_to_end(case):
     P.assert_attention_close(P.to_np(out), want)
 
 
-def test_decode_zero_query_head_attends_uniformly():
+@pytest.mark.parametrize("q_dtype", [torch.bfloat16, torch.float32])
+def test_decode_zero_query_head_attends_uniformly(q_dtype):
     # an all-zero query has no fixed-point scale: its scores are all zero (uniform weights)
-    # while the other heads of the same KV head decode normally
+    # while the other heads of the same KV head decode normally; so has a query of subnormal
+    # size (exact scores below 1e-30)
     case = (128, 4, 2, (4, O.MSE), (2, O.MSE), 0, 333, 333)
-    B, Hq, K, V, q = _decode_case(case, torch.bfloat16, seed=12)
+    B, Hq, K, V, q = _decode_case(case, q_dtype, seed=12)
     q[0, 1] = 0.0
     q[1, 6] = 0.0
+    q[1, 5] = (q[1, 5].float() * 1e-39).to(q_dtype)
     cache = tq.TQCache(B, 2, 333, 128, 4, 2)
     k_recs = P.oracle_records(P.to_np(K), 4, O.MSE, 0, 1, None)
     v_recs = P.oracle_records(P.to_np(V), 2, O.MSE, 0, 1, None)
