@@ -433,3 +433,38 @@ def test_compressed_attention_converges_with_bits():
     ratios = np.array(errs[:-1]) / np.array(errs[1:])
     assert np.all((ratios > 1.4) & (ratios < 2.6)), errs
     assert errs[-1] < 0.06
+
+
+def test_prefill_reduces_to_decode_and_is_causal():
+    # prefill over the compressed cache (S16, Decode Throughput vs. TTFT): the last query of a
+    # chunk that ends the cache is a decode query; a query never sees later positions; the
+    # first position of a sequence attends to itself alone
+    rng = np.random.default_rng(21)
+    B, Hkv, G, T, d, lq = 2, 2, 3, 40, 32, 5
+    K, V = rng.standard_normal((2, B, Hkv, T, d))
+    k_recs = [O.quantize(K[b, h], 3) for b in range(B) for h in range(Hkv)]
+    v_recs = [O.quantize(V[b, h], 2) for b in range(B) for h in range(Hkv)]
+    q = rng.standard_normal((B, lq, Hkv * G, d))
+    t0 = T - lq
+    out = O.prefill_compressed(q, k_recs, v_recs, B, Hkv, t0, d ** -0.5)
+    assert out.shape == (B, lq, Hkv * G, d)
+    # (1) the chunk's last query over the whole cache is the decode of that query
+    dec = O.decode_compressed(q[:, -1], k_recs, v_recs, B, Hkv, d ** -0.5)
+    np.testing.assert_allclose(out[:, -1], dec, rtol=0, atol=1e-13)
+    # (2) causality: other keys and values after position t0 + i leave query i unchanged
+    K2, V2 = K.copy(), V.copy()
+    K2[:, :, t0 + 2:] = 5.0 * rng.standard_normal(K2[:, :, t0 + 2:].shape)
+    V2[:, :, t0 + 2:] = rng.standard_normal(V2[:, :, t0 + 2:].shape)
+    k2 = [O.quantize(K2[b, h], 3) for b in range(B) for h in range(Hkv)]
+    v2 = [O.quantize(V2[b, h], 2) for b in range(B) for h in range(Hkv)]
+    out2 = O.prefill_compressed(q, k2, v2, B, Hkv, t0, d ** -0.5)
+    np.testing.assert_array_equal(out2[:, :2], out[:, :2])
+    assert np.abs(out2[:, 2:] - out[:, 2:]).max() > 1e-3
+    # (3) a chunk at the start of a sequence: position 0 sees only itself, so its output is
+    # the dequantised value of token 0 whatever the query
+    first = O.prefill_compressed(q[:, :1] * 100.0, k_recs, v_recs, B, Hkv, 0, d ** -0.5)
+    for b in range(B):
+        for h in range(Hkv * G):
+            np.testing.assert_allclose(first[b, 0, h], O.dequantize(v_recs[b * Hkv + h // G])[0],
+                                       rtol=0, atol=1e-14)
+
