@@ -146,7 +146,11 @@ int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
                    const tq_cache *cache, void *stream);
 
 /* Workspace bytes tq_decode_attention needs for this shape (split-K partials: running
- * max, running sum and the rotated-domain accumulator per split and query head). 0 if
+ * max, running sum and the rotated-domain accumulator per split and query head). The pages
+ * place the attention over the compressed cache in the decode step ("Where This Fits in the
+ * Inference Stack", TensorRT-LLM section: flash-decoding splits the context); the partial
+ * records of those splits live in this caller-owned workspace, since the library never
+ * allocates. B is the batch, Hq the query heads, T_len the attended positions. 0 if
  * invalid. Depends on the current device's SM count. */
 size_t tq_decode_workspace_bytes(int B, int Hq, int T_len, const tq_cache *cache);
 
@@ -179,7 +183,10 @@ int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale
  * current; make that first call before any stream capture. Every call on a device shares the
  * same array and leaves its partials behind; a call writes every element it later reads, so
  * nothing needs clearing, but calls that overlap on the GPU (other streams, other host
- * threads) race on the array and must be serialised by the caller. */
+ * threads) race on the array and must be serialised by the caller. The looked-up address is
+ * kept for the life of the process: after a reset of the device (cudaDeviceReset, or another
+ * library destroying the primary context) the array may move, and this call must not be used
+ * on that device again. */
 int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, float scale,
                                 const tq_cache *cache, float *out, void *stream);
 
@@ -208,8 +215,13 @@ int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,
                      int *quantize_launches, int *decode_launches);
 
 /* Dequantise cache positions [0, T_len) of K (which = 0) or V (which = 1) into out
- * [B][Hkv][T_len][d] of `dtype` in the original domain: x_hat = n D H c / d (MSE), plus
- * the QJL residual estimate sqrt(d) gamma sqrt(pi/2)/m S^T s inside the bracket (PROD). */
+ * [B][Hkv][T_len][d] of `dtype` (TQ_F32 / TQ_BF16 / TQ_F16, device, caller-owned) in the
+ * original domain: x_hat = n D H c / d (MSE), plus the QJL residual estimate
+ * sqrt(d) gamma sqrt(pi/2)/m S^T s inside the bracket (PROD). This is the reconstruction
+ * the pages describe ("Closing - The Three-Step Summary", Steps 1-3: look up the centroids,
+ * undo the rotation, scale by the stored norm; Step 3 adds the QJL correction). Errors:
+ * TQ_ERR_INVALID_ARG (which not 0/1, dtype unknown, T_len outside 0..T_cap, null or
+ * misaligned out), TQ_ERR_CUDA. T_len = 0 is a no-op. */
 int tq_dequantize(const tq_cache *cache, int which, int T_len, void *out, int dtype,
                   void *stream);
 
@@ -242,7 +254,11 @@ int tq_decode_attention_paged(const void *q, int dtype, int Hq, const int *T_len
  * (tcgen05 write path of TurboQuant_prod records) gave up waiting for its MMAs after about a
  * second, recorded a fault, freed its tensor memory and returned without writing the rest of
  * its records. Reading synchronises the device and clears the bits. Writes *flags; returns
- * TQ_OK or TQ_ERR_CUDA. The pages have no counterpart to this call. */
+ * TQ_OK or TQ_ERR_CUDA. A set bit means a tensor-core
+ * operation may still have been in flight when its tensor memory was released: the
+ * library's device state (and the outputs of that call) are then undefined, and the caller
+ * should treat the CUDA context as lost and tear it down. The pages have no counterpart to
+ * this call. */
 int tq_device_faults(unsigned *flags);
 
 #ifdef __cplusplus

@@ -20,7 +20,8 @@ Every step the pages leave open takes a stated reading; each reading is marked "
 
 Parity pins: every public function here is pinned by tests/test_oracle.py against values
 the pages print, closed forms, invariants, library routines the oracle does not use, or
-brute force on tiny inputs. No function is "parity unpinned".
+brute force on tiny inputs; boundary_distance (the exemption band of the bit-exact code
+comparison) is pinned against the decision boundaries of Max's published Gaussian quantiser.
 """
 from __future__ import annotations
 

@@ -188,9 +188,14 @@ __device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, 
     mx = fmaxf(mx, fabsf(x[e]));
   }
   mx = warp_max(mx);
-  // a query whose largest coordinate is below 1e-30 (zero included) gets zero scores (its
-  // exact scores are below 1e-30 times the key norms); a non-finite one makes them NaN
-  const bool ok = mx > 1e-30f && isfinite(mx);
+  // fmaxf ignores NaN, so a NaN anywhere in the query (the rotation spreads it to every
+  // coordinate) is detected separately
+  const bool has_nan = __any_sync(0xffffffffu, isnan(x[0]) || isnan(x[1]) || isnan(x[2]) || isnan(x[3]));
+  // A query whose largest coordinate is below 1e-30 (zero included) gets zero scores (its
+  // exact scores are below 1e-30 times the key norms). A query holding a NaN or an infinity
+  // gets the score factor NaN: its scores, softmax weights and output are NaN, as exact
+  // attention would give.
+  const bool ok = !has_nan && mx > 1e-30f && isfinite(mx);
   const float qsc = ok ? kQFixMax / mx : 0.f;
   uint32_t hw = 0, mw = 0, lw = 0;
 #pragma unroll
@@ -207,7 +212,7 @@ __device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, 
   reinterpret_cast<uint32_t *>(out->hi)[lane] = hw;
   reinterpret_cast<uint32_t *>(out->mid)[lane] = mw;
   reinterpret_cast<uint32_t *>(out->lo)[lane] = lw;
-  if (lane == 0) out->inv = ok ? 16777216.0f / (qsc * csc) : (isfinite(mx) ? 0.f : __int_as_float(0x7fc00000));
+  if (lane == 0) out->inv = ok ? 16777216.0f / (qsc * csc) : (!has_nan && isfinite(mx) ? 0.f : __int_as_float(0x7fc00000));
 }
 
 struct FastArgs {

@@ -251,6 +251,67 @@ def test_decode_zero_query_head_attends_uniformly(q_dtype):
     np.testing.assert_allclose(want[0, 1], vh.mean(axis=0), rtol=1e-9, atol=1e-12)
 
 
+@pytest.mark.parametrize("case", [
+    (128, 4, 2, (4, O.MSE), (2, O.MSE), 0, 333, 333),    # tensor-core MSE kernel
+    (128, 8, 1, (3, O.MSE), (3, O.MSE), 0, 200, 200),    # tensor-core MSE kernel, two n-tiles
+    (256, 2, 2, (4, O.MSE), (2, O.MSE), 0, 150, 150),    # generic split-K kernel
+    (64, 1, 3, (2, O.PROD), (2, O.PROD), 64, 140, 140),  # TurboQuant_prod, one head per KV head
+    (64, 2, 2, (2, O.PROD), (2, O.PROD), 64, 140, 140),  # TurboQuant_prod, two heads per KV head
+], ids=lambda c: f"d{c[0]}-G{c[1]}-k{c[3]}-v{c[4]}")
+def test_decode_non_finite_query_heads_give_nan(case):
+    # a query head holding a NaN or an infinity has NaN scores in exact arithmetic, so its
+    # attention output is NaN; the other heads of the same KV head decode as usual
+    d, G, Hkv, (kb, km), (vb, vm), m, T, _ = case
+    B, Hq, K, V, q = _decode_case(case, torch.bfloat16, seed=14)
+    bad = [(0, 0), (1, Hq - 1)]
+    q[0, 0, 3] = float("nan")
+    q[1, Hq - 1, 7] = float("inf")
+    cache = tq.TQCache(B, Hkv, T, d, kb, vb, km, vm, m, m, seed=4, qjl_seed=2)
+    k_recs = P.oracle_records(P.to_np(K), kb, km, 4, 2, m or None)
+    v_recs = P.oracle_records(P.to_np(V), vb, vm, 4, 2, m or None)
+    P.upload(cache, "k", k_recs)
+    P.upload(cache, "v", v_recs)
+    out = torch.empty(B, Hq, d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, T))
+    tq.tq_decode_attention(q.cuda(), cache, T, d ** -0.5, out, ws)
+    torch.cuda.synchronize()
+    got = P.to_np(out)
+    qf = P.to_np(q)
+    for b, h in bad:
+        assert np.isnan(got[b, h]).all(), f"head ({b},{h}) should be NaN"
+        qf[b, h] = 0.0  # the oracle's answer for the finite heads does not depend on these
+    want = P.oracle_decode(qf, k_recs, v_recs, B, Hkv, d ** -0.5)
+    for b in range(B):
+        for h in range(Hq):
+            if (b, h) not in bad:
+                assert np.isfinite(got[b, h]).all()
+                assert P.rel_l2(got[b, h], want[b, h]) <= P.ATTN_RTOL, (b, h)
+
+
+def test_bf16_decode_non_finite_query_heads_give_nan():
+    for d, G, Hkv in ((128, 4, 2), (64, 1, 3)):
+        B, T = 2, 260
+        Hq = G * Hkv
+        K, V = random_kv(B, Hkv, T, d, dtype=torch.bfloat16, seed=d)
+        q = torch.randn(B, Hq, d, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+        q[0, 1, 0] = float("nan")
+        q[1, 0, 5] = float("-inf")
+        out = torch.empty(B, Hq, d, device="cuda")
+        ws = tq.workspace(tq.tq_decode_bf16_workspace_bytes(B, Hq, Hkv, T, d))
+        tq.tq_decode_attention_bf16(q.cuda(), K.cuda(), V.cuda(), T, d ** -0.5, out, ws)
+        torch.cuda.synchronize()
+        got = P.to_np(out)
+        qf = P.to_np(q)
+        for b, h in ((0, 1), (1, 0)):
+            assert np.isnan(got[b, h]).all()
+            qf[b, h] = 0.0
+        want = O.gqa_decode(qf, P.to_np(K), P.to_np(V), d ** -0.5)
+        for b in range(B):
+            for h in range(Hq):
+                if (b, h) not in ((0, 1), (1, 0)):
+                    assert P.rel_l2(got[b, h], want[b, h]) <= P.ATTN_RTOL
+
+
 def test_decode_rejects_small_workspace_and_empty_context():
     cache = tq.TQCache(1, 1, 64, 128, 4, 2)
     q = torch.zeros(1, 4, 128, device="cuda", dtype=torch.bfloat16)

@@ -125,6 +125,41 @@ def test_codebook_matches_max_table():
             assert abs(dist - vals[0]) / vals[0] < 2e-3, (bits, dist, vals)
 
 
+def test_boundary_distance_against_published_boundaries():
+    # The decision boundaries are the midpoints of adjacent optimum levels; Max's table (four
+    # decimals) fixes them to within 1e-4. Coordinates placed at a published boundary plus a
+    # small offset must report that offset; a record without Lloyd-Max codes reports +inf.
+    import dataclasses
+    pub = {}
+    for row in _read_rows("max1960_gaussian_quantizer.txt"):
+        parts = row.split()
+        if parts[1] == "centroid":
+            half = [float(v) for v in parts[2:]]
+            full = [-v for v in half[::-1]] + half
+            pub[int(parts[0])] = [(a + b) / 2 for a, b in zip(full[:-1], full[1:])]
+    base = O.quantize(np.ones((1, 8)), 4)
+    for bits, beta in pub.items():
+        offsets = np.array([0.003, -0.004, 0.01, -0.02])
+        z = (np.asarray(beta)[:, None] + offsets[None, :]).reshape(1, -1)
+        rec = dataclasses.replace(base, bits=bits, mode=O.MSE, z=z)
+        got = O.boundary_distance(rec)
+        want = np.broadcast_to(np.abs(offsets), (len(beta), len(offsets))).reshape(1, -1)
+        assert np.all(np.abs(got - want) <= 2e-4), (bits, got, want)
+        # half-way between two neighbouring boundaries: half the gap
+        if len(beta) > 1:
+            mid = np.array([[(beta[1] + beta[2]) / 2 if len(beta) > 2 else (beta[0] + beta[1]) / 2]])
+            gap = (beta[2] - beta[1]) / 2 if len(beta) > 2 else (beta[1] - beta[0]) / 2
+            got_mid = O.boundary_distance(dataclasses.replace(base, bits=bits, mode=O.MSE, z=mid))
+            assert abs(got_mid[0, 0] - gap) <= 2e-4
+    # TurboQuant_prod at 2 bits decides with the 1-bit codebook (boundary 0 only)
+    z = np.array([[0.9, -0.25, 1e-6]])
+    got = O.boundary_distance(dataclasses.replace(base, bits=2, mode=O.PROD, z=z))
+    assert np.allclose(got, [[0.9, 0.25, 1e-6]], atol=1e-12)
+    # 1-bit TurboQuant_prod stores no Lloyd-Max codes: nothing to exempt
+    got = O.boundary_distance(dataclasses.replace(base, bits=1, mode=O.PROD, z=z))
+    assert np.all(np.isinf(got)) and got.shape == z.shape
+
+
 def test_codebook_one_bit_closed_form():
     c, beta, dist = O.lloyd_max_gaussian(1)
     assert np.allclose(c, [-math.sqrt(2 / math.pi), math.sqrt(2 / math.pi)], atol=1e-12)

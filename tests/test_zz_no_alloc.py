@@ -26,6 +26,9 @@ from quantized_decode_attention_kv_b200.workloads import random_kv  # noqa: E402
 @pytest.mark.parametrize("d,G,Hkv,kcfg,vcfg,T", [
     (128, 4, 2, (4, tq.TQ_MSE), (2, tq.TQ_MSE), 3000),
     (64, 1, 3, (2, tq.TQ_PROD), (2, tq.TQ_PROD), 777),
+    (128, 4, 2, (4, tq.TQ_MSE), (3, tq.TQ_MSE), 1500),   # 3-bit values (the 3.5-bit reading)
+    (256, 2, 2, (4, tq.TQ_MSE), (2, tq.TQ_MSE), 390),    # generic split-K kernel + its combine
+    (32, 16, 1, (3, tq.TQ_MSE), (2, tq.TQ_MSE), 200),    # generic kernel, many heads per KV head
 ])
 def test_noalloc_decode_matches_workspace_decode_on_two_calls(d, G, Hkv, kcfg, vcfg, T):
     B, Hq = 3, G * Hkv
