@@ -338,13 +338,29 @@ def run_ours(args):
             line["paged_decode"] = side["paged"]
         if "k4v3" in side:
             line["decode_3p5bit"] = side["k4v3"]
+        if "boundary_flips" in side:
+            line["boundary_flips"] = side["boundary_flips"]
+        line["configs"] = side.get("configs", {})
     print(json.dumps(line), flush=True)
 
 
-def _time(fn, stream, reps, torch):
+MIN_CALLS, MIN_SECONDS = 200, 0.5
+
+
+def _time(fn, stream, torch, min_calls=MIN_CALLS, min_s=MIN_SECONDS):
+    """Mean device time of one call of fn (CUDA events on the launching stream) over at least
+    min_calls calls and at least min_s seconds, after three warm-up calls."""
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    fn()
+    for _ in range(3):
+        fn()
     torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(3):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    est = max(e0.elapsed_time(e1) / 3 * 1e-3, 1e-7)
+    reps = max(min_calls, int(min_s / est) + 1)
     e0.record(stream)
     for _ in range(reps):
         fn()
@@ -358,9 +374,9 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
     res = {}
     # decode call alone (split-K kernel + combine)
     res["decode_s"] = _time(lambda: tq.tq_decode_attention(q, cache, w.T, w.scale, out, ws, stream=stream),
-                            stream, max(args.steps, 20), torch)
+                            stream, torch)
     # bulk quantise of the whole layer: B*T token positions, all KV heads, K and V
-    qs = _time(lambda: tq.tq_quantize_kv(K, V, cache, stream=stream), stream, 5, torch)
+    qs = _time(lambda: tq.tq_quantize_kv(K, V, cache, stream=stream), stream, torch, min_calls=20)
     in_bytes = (K.numel() + V.numel()) * K.element_size()
     q_bytes = in_bytes + packed
     res["quantize"] = {"us": qs * 1e6, "mtok_s": w.B * w.T / qs / 1e6, "gbs": q_bytes / qs / 1e9,
@@ -371,7 +387,7 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
         wsb = tq.workspace(tq.tq_decode_bf16_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.d))
         qb = q.to(torch.bfloat16)
         bs = _time(lambda: tq.tq_decode_attention_bf16(qb, K, V, w.T, w.scale, out, wsb, stream=stream),
-                   stream, 10, torch)
+                   stream, torch)
         bbytes = (K.numel() + V.numel()) * 2
         res["bf16"] = {"us": bs * 1e6, "gbs": bbytes / bs / 1e9, "frac": bbytes / bs / 1e9 / hbm,
                        "bytes": bbytes}
@@ -388,10 +404,10 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
         rbytes = sum(lens) * per_tok
         wsr = tq.workspace(tq.tq_decode_varlen_workspace_bytes(cache, w.Hq, lens))
         rs = _time(lambda: tq.tq_decode_attention_varlen(q, cache, lens, w.scale, out, wsr, stream=stream),
-                   stream, max(args.steps // 4, 20), torch)
+                   stream, torch)
         wsp = tq.workspace(tq.tq_decode_workspace_bytes(cache, w.Hq, max(lens)))
         ps = _time(lambda: tq.tq_decode_attention(q, cache, max(lens), w.scale, out, wsp, stream=stream),
-                   stream, max(args.steps // 4, 20), torch)
+                   stream, torch)
         res["ragged"] = {"us": rs * 1e6, "gbs": rbytes / rs / 1e9, "frac": rbytes / rs / 1e9 / hbm,
                          "bytes": rbytes, "lengths": f"{w.B} sequences, seeded uniform in [T/4, T], "
                                                     f"min {min(lens)}, max {max(lens)}, sum {sum(lens)}",
@@ -409,7 +425,7 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
         lens = [w.T] * w.B
         wsp = tq.workspace(tq.tq_decode_paged_workspace_bytes(pc, w.Hq, lens))
         pgs = _time(lambda: tq.tq_decode_attention_paged(q, pc, lens, w.scale, out, wsp, stream=stream),
-                    stream, max(args.steps // 4, 20), torch)
+                    stream, torch)
         res["paged"] = {"us": pgs * 1e6, "gbs": packed / pgs / 1e9, "frac": packed / pgs / 1e9 / hbm,
                         "page_size": page, "layout": f"{npages} pages of {page} positions, scattered by a "
                                                      f"seeded permutation; every sequence at full length"}
@@ -421,7 +437,7 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
         b35 = c35.packed_bytes(w.T)
         ws35 = tq.workspace(tq.tq_decode_workspace_bytes(c35, w.Hq, w.T))
         s35 = _time(lambda: tq.tq_decode_attention(q, c35, w.T, w.scale, out, ws35, stream=stream),
-                    stream, max(args.steps // 4, 20), torch)
+                    stream, torch)
         res["k4v3"] = {"us": s35 * 1e6, "gbs": b35 / s35 / 1e9, "frac": b35 / s35 / 1e9 / hbm,
                        "bytes": b35, "k": "4-bit MSE", "v": "3-bit MSE",
                        "reading": "3.5 bits per cached coordinate as 4-bit keys + 3-bit values"}
@@ -478,10 +494,164 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
     res["e2e"] = {"value": packed / es / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                   "d2h_bytes_per_step": hout[0].numel() * hout[0].element_size(), "ms_per_step": es * 1e3,
                   "pipeline": "copy-in, compute and copy-out on three streams, double-buffered"}
-    # the oracle on the host cores, bounded sample
+    samples = {w.name: flip_sample(w, K, V, cache)}
+    res["configs"] = {}
+    for name in OTHER_WORKLOADS:
+        if name == w.name:
+            continue
+        entry, sample = measure_workload(WORKLOADS_BY_NAME()[name], tq, torch, stream, hbm)
+        res["configs"][name] = entry
+        samples[name] = sample
+        torch.cuda.empty_cache()
+    # the oracle on the host cores (bounded sample), and the oracle's codes for the sampled
+    # slice of every workload against the device's (the count of codes decided differently
+    # near a decision boundary)
     if args.gpus == 1:
         res["cpu_baseline"] = time_oracle_decode(w)
+        for name, sample in samples.items():
+            flips = oracle_boundary_flips(*sample)
+            if name == w.name:
+                res["boundary_flips"] = flips
+            else:
+                res["configs"][name]["boundary_flips"] = flips
     return res
+
+
+OTHER_WORKLOADS = ("tiny_single_head_fp32", "gpt2_prod_2bit", "llama3_8b_128k_3bit", "llama70b_asym_16k",
+                   "llama3_8b_decode_32k")
+FLIP_ROWS = 4096
+
+
+def WORKLOADS_BY_NAME():
+    from quantized_decode_attention_kv_b200.workloads import WORKLOADS
+    return WORKLOADS
+
+
+def flip_sample(w, K, V, cache, n=FLIP_ROWS):
+    """Inputs and device codes of the first n positions of (batch 0, KV head 0), K and V, as
+    host arrays, for the count of boundary flips."""
+    n = min(n, K.shape[2])
+    out = [w, n]
+    for side, X in (("k", K), ("v", V)):
+        out.append(X[0, 0, :n].float().cpu().numpy())
+        codes = cache[f"{side}_codes"]
+        out.append(None if codes is None else codes[0, 0, :n].cpu().numpy())
+        signs = cache[f"{side}_signs"]
+        out.append(None if signs is None else signs[0, 0, :n].cpu().numpy())
+    return tuple(out)
+
+
+def oracle_boundary_flips(w, n, kx, kcodes, ksigns, vx, vcodes, vsigns):
+    """CPU (oracle) leg: the oracle quantises the sampled rows in float64; device codes that
+    differ from its codes are counted, with the number of coordinates within 1e-5 of a decision
+    boundary (where the float32 device decision may legitimately differ) and, for
+    TurboQuant_prod, sign bits that differ with |(S r)_j| < 1e-5 ||r||."""
+    import numpy as np
+
+    import oracle as O
+    res = {}
+    for side, x, codes, signs, bits, mode in (("k", kx, kcodes, ksigns, w.k_bits, w.k_mode),
+                                              ("v", vx, vcodes, vsigns, w.v_bits, w.v_mode)):
+        rec = O.quantize(x.astype(np.float64), bits, mode, seed=w.seed, qjl_seed=w.qjl_seed, m=w.qjl_m or None)
+        wb = bits if mode == O.MSE else bits - 1
+        near = O.boundary_distance(rec) < 1e-5
+        if wb > 0:
+            got = O.unpack_bits(codes, wb, w.d)
+            diff = got != rec.codes
+        else:
+            diff = np.zeros_like(near)
+        e = {"rows": int(n), "coords": int(near.size), "near_boundary": int(near.sum()),
+             "flipped": int(diff.sum()), "flipped_away_from_boundary": int((diff & ~near).sum())}
+        if mode == O.PROD:
+            row_ok = ~np.any(diff, axis=1)
+            gb = O.unpack_bits(signs, 1, rec.m)
+            near_s = np.abs(rec.proj) < 1e-5 * rec.rnorm[:, None]
+            bad = (gb != rec.qjl_bits) & row_ok[:, None]
+            e["sign_bits"] = int(row_ok.sum() * rec.m)
+            e["signs_flipped"] = int(bad.sum())
+            e["signs_flipped_away_from_zero"] = int((bad & ~near_s).sum())
+        res[side] = e
+    return res
+
+
+def measure_workload(w, tq, torch, stream, hbm):
+    """One layer of workload w at full size: decode call (µs, GB/s, fraction of the HBM
+    peak) and bulk quantise of the layer (µs, Mtok/s, fraction); for the 128K-context workload
+    the 32-layer prefill write timed as one run; for the 70B-shaped one a bf16 boundary layer
+    and the 80-layer decode step timed as one run."""
+    from quantized_decode_attention_kv_b200.workloads import make_inputs
+    K, V, q = make_inputs(w, device="cuda")
+    cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, w.k_mode, w.v_mode, w.qjl_m,
+                       w.qjl_m, seed=w.seed, qjl_seed=w.qjl_seed)
+    tq.tq_quantize_kv(K, V, cache, stream=stream)
+    out = torch.empty(w.B, w.Hq, w.d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_workspace_bytes(cache, w.Hq, w.T))
+    packed = cache.packed_bytes(w.T)
+    dec = _time(lambda: tq.tq_decode_attention(q, cache, w.T, w.scale, out, ws, stream=stream), stream, torch)
+    qt = _time(lambda: tq.tq_quantize_kv(K, V, cache, stream=stream), stream, torch, min_calls=20)
+    qbytes = (K.numel() + V.numel()) * K.element_size() + packed
+    e = {"shape": f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d} T={w.T}",
+         "k": f"{w.k_bits}-bit {'MSE' if w.k_mode == 0 else 'PROD'}",
+         "v": f"{w.v_bits}-bit {'MSE' if w.v_mode == 0 else 'PROD'}",
+         "decode_us": dec * 1e6, "decode_gbs": packed / dec / 1e9, "decode_frac": packed / dec / 1e9 / hbm,
+         "packed_bytes": packed,
+         "quantize_us": qt * 1e6, "quantize_mtok_s": w.B * w.T / qt / 1e6, "quantize_gbs": qbytes / qt / 1e9,
+         "quantize_frac": qbytes / qt / 1e9 / hbm, "quantize_bytes": qbytes}
+    sample = flip_sample(w, K, V, cache)
+    if w.layers > 1 and not w.bf16_layers:
+        # prefill write of every layer, timed as one run: layer l's K, V (two input buffers in
+        # turn, each its own seeded draw) quantised into layer l's cache
+        K2, V2, _ = make_inputs(w, device="cuda", layer=1)
+        caches = [cache] + [tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, w.k_mode, w.v_mode,
+                                       seed=w.seed) for _ in range(w.layers - 1)]
+        ins = [(K, V), (K2, V2)]
+
+        def write_all():
+            for i, c in enumerate(caches):
+                tq.tq_quantize_kv(*ins[i % 2], c, stream=stream)
+        wt = _time(write_all, stream, torch, min_calls=3, min_s=0.5)
+        e["prefill_write_all_layers"] = {
+            "layers": w.layers, "us": wt * 1e6, "mtok_s": w.B * w.T / wt / 1e6,
+            "gbs": w.layers * qbytes / wt / 1e9, "frac": w.layers * qbytes / wt / 1e9 / hbm,
+            "bytes": w.layers * qbytes, "inputs": "two seeded input buffers used by alternate layers"}
+        del caches, ins, K2, V2
+    if w.bf16_layers:
+        # a layer kept in bf16 (the same split-K design over the unquantised cache)
+        wsb = tq.workspace(tq.tq_decode_bf16_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.d))
+        bt = _time(lambda: tq.tq_decode_attention_bf16(q, K, V, w.T, w.scale, out, wsb, stream=stream),
+                   stream, torch)
+        bbytes = (K.numel() + V.numel()) * 2
+        e["bf16_layer_decode"] = {"us": bt * 1e6, "gbs": bbytes / bt / 1e9, "frac": bbytes / bt / 1e9 / hbm,
+                                  "bytes": bbytes}
+        # the whole decode step over all layers: quantised layers write their new token and run
+        # the compressed decode, bf16 layers run the bf16 decode over their own K, V
+        layers = []
+        for l in range(w.layers):
+            Kl, Vl, ql = make_inputs(w, device="cuda", layer=l)
+            if l in w.bf16_layers:
+                layers.append(("bf16", Kl, Vl, ql, None))
+            else:
+                cl = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, seed=w.seed)
+                tq.tq_quantize_kv(Kl, Vl, cl, stream=stream)
+                layers.append(("tq", Kl[:, :, w.T - 1:].contiguous(), Vl[:, :, w.T - 1:].contiguous(), ql, cl))
+                del Kl, Vl
+        def step_all():
+            for kind, a0, a1, ql, cl in layers:
+                if kind == "bf16":
+                    tq.tq_decode_attention_bf16(ql, a0, a1, w.T, w.scale, out, wsb, stream=stream)
+                else:
+                    tq.tq_quantize_kv(a0, a1, cl, t_offset=w.T - 1, stream=stream)
+                    tq.tq_decode_attention(ql, cl, w.T, w.scale, out, ws, stream=stream)
+        st = _time(step_all, stream, torch, min_calls=3, min_s=0.5)
+        nq = w.layers - len(w.bf16_layers)
+        sbytes = nq * packed + len(w.bf16_layers) * bbytes
+        e["decode_step_all_layers"] = {
+            "layers": w.layers, "bf16_layers": list(w.bf16_layers), "us": st * 1e6, "gbs": sbytes / st / 1e9,
+            "frac": sbytes / st / 1e9 / hbm, "bytes": sbytes,
+            "step": "per quantised layer: write of the new token + compressed decode; per bf16 layer: bf16 decode"}
+        del layers
+    del K, V, q, cache, ws
+    return e, sample
 
 
 def main():
