@@ -180,10 +180,10 @@ __global__ void __launch_bounds__(kBThreads, 3) decode_bf16_mma_kernel(const Bf1
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float mn = fmaxf(m_run[e], mx);
-        alpha[e] = exp2f(m_run[e] - mn);
+        alpha[e] = softmax_exp2(m_run[e] - mn);
         moved |= mn != m_run[e];
         m_run[e] = mn;
-        const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
+        const float p0 = softmax_exp2(s0 - mn), p1 = softmax_exp2(s1 - mn);
         l_run[e] = fmaf(l_run[e], alpha[e], p0 + p1);
         split_bf16(p0, p1, phi[e], plo[e]); // (token r, token r + 8)
       }

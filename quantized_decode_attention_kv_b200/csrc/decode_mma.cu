@@ -496,10 +496,10 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           const float mn = fmaxf(m_run[nt], mx);
-          alpha[nt] = exp2f(m_run[nt] - mn);
+          alpha[nt] = softmax_exp2(m_run[nt] - mn);
           rescale |= mn != m_run[nt];
           m_run[nt] = mn;
-          const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
+          const float p0 = softmax_exp2(s0 - mn), p1 = softmax_exp2(s1 - mn);
           l_run[nt] = fmaf(l_run[nt], alpha[nt], p0 + p1);
           pk[nt] = pack_h2(p0 * vn0, p1 * vn1);
         }

@@ -333,10 +333,10 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const float mn = fmaxf(m_run, mx);
-      const float alpha = exp2f(m_run - mn);
+      const float alpha = softmax_exp2(m_run - mn);
       const bool moved = mn != m_run;
       m_run = mn;
-      const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
+      const float p0 = softmax_exp2(s0 - mn), p1 = softmax_exp2(s1 - mn);
       l_run = fmaf(l_run, alpha, p0 + p1);
       const uint32_t pkc = pack_h2(p0 * vn0, p1 * vn1);
       const uint32_t pks = pack_h2(p0 * vn0 * vg0, p1 * vn1 * vg1);
@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
       for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
       const float mn = fmaxf(m_run, mx);
       if (mn != m_run) {
-        const float alpha = exp2f(m_run - mn);
+        const float alpha = softmax_exp2(m_run - mn);
         l_run *= alpha;
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
         }
         m_run = mn;
       }
-      const float pr = exp2f(s - mn);
+      const float pr = softmax_exp2(s - mn);
       l_run += pr;
       const float vn = f16_bits_to_f32(T.vn), vg = f16_bits_to_f32(T.vg);
       const uint32_t pk = pack_h2(pr * vn, pr * vn * vg); // (code rows, sketch rows)

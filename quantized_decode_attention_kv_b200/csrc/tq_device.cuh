@@ -200,6 +200,15 @@ __device__ __forceinline__ float f16_bits_to_f32(uint16_t b) {
   return __half2float(__ushort_as_half(b));
 }
 
+// 2^x for online-softmax weights and rescale factors (x <= 0 or -inf): the hardware
+// approximation (MUFU.EX2, relative error ~2^-22) with results below 2^-126 flushed to zero,
+// which a softmax weight can afford; NaN stays NaN.
+__device__ __forceinline__ float softmax_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
