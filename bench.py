@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--no-side", action="store_true", help="skip side measurements")
     ap.add_argument("--T", type=int, default=0,
                     help="override the context length (profiling runs on smaller cases)")
+    ap.add_argument("--prefill-case", default="",
+                    help="T,Lq: run one prefill chunk of Lq queries at the end of a T-position cache "
+                         "(Llama-3.1-8B shape, batch 4, 4-bit keys, 2-bit values) and exit (profiling)")
     return ap.parse_args()
 
 
@@ -341,6 +344,7 @@ def run_ours(args):
         if "boundary_flips" in side:
             line["boundary_flips"] = side["boundary_flips"]
         line["configs"] = side.get("configs", {})
+        line["prefill"] = side.get("prefill", {})
     print(json.dumps(line), flush=True)
 
 
@@ -376,12 +380,15 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
     res["decode_s"] = _time(lambda: tq.tq_decode_attention(q, cache, w.T, w.scale, out, ws, stream=stream),
                             stream, torch)
     # bulk quantise of the whole layer: B*T token positions, all KV heads, K and V
-    qs = _time(lambda: tq.tq_quantize_kv(K, V, cache, stream=stream), stream, torch, min_calls=20)
+    qclk = Clocks(torch.cuda.current_device())
+    with qclk:
+        qs = _time(lambda: tq.tq_quantize_kv(K, V, cache, stream=stream), stream, torch, min_calls=20)
     in_bytes = (K.numel() + V.numel()) * K.element_size()
     q_bytes = in_bytes + packed
     res["quantize"] = {"us": qs * 1e6, "mtok_s": w.B * w.T / qs / 1e6, "gbs": q_bytes / qs / 1e9,
                        "frac": q_bytes / qs / 1e9 / hbm, "bytes": q_bytes,
-                       "token": "one (sequence, position) of one layer: all KV heads, K and V"}
+                       "token": "one (sequence, position) of one layer: all KV heads, K and V",
+                       "clocks": qclk.summary()}
     # the same split-K design over the unquantised bf16 cache
     if K.dtype == torch.bfloat16:
         wsb = tq.workspace(tq.tq_decode_bf16_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.d))
@@ -503,6 +510,7 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
         res["configs"][name] = entry
         samples[name] = sample
         torch.cuda.empty_cache()
+    res["prefill"] = measure_prefill(tq, torch, stream)
     # the oracle on the host cores (bounded sample), and the oracle's codes for the sampled
     # slice of every workload against the device's (the count of codes decided differently
     # near a decision boundary)
@@ -515,6 +523,49 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
             else:
                 res["configs"][name]["boundary_flips"] = flips
     return res
+
+
+def measure_prefill(tq, torch, stream):
+    """Chunked prefill attention over the compressed cache at long contexts (the
+    Llama-3.1-8B shape, batch 4): a chunk of 1024 queries at the end of a 64K-token cache
+    (4-bit keys, 2-bit values) and of a 128K-token cache (3-bit keys and values). The roofline is
+    the tensor cores': algorithmic FLOPs 4 d per (query row, visible key) against the measured
+    dense bf16 peak."""
+    import dataclasses
+
+    from quantized_decode_attention_kv_b200.workloads import WORKLOADS, make_inputs
+    pk = tensor_peak()
+    res = {}
+    for label, name, T in (("64k", "llama3_8b_decode_32k", 65536), ("128k", "llama3_8b_128k_3bit", 131072)):
+        w = dataclasses.replace(WORKLOADS[name], B=4, T=T)
+        Lq, t0 = 1024, T - 1024
+        K, V, _ = make_inputs(w, device="cuda")
+        cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, seed=w.seed)
+        tq.tq_quantize_kv(K, V, cache, stream=stream)
+        del K, V
+        g = torch.Generator(device="cuda").manual_seed(77)
+        q = torch.randn(w.B, Lq, w.Hq, w.d, generator=g, device="cuda").to(torch.bfloat16)
+        out = torch.empty(w.B, Lq, w.Hq, w.d, device="cuda")
+        ts = _time(lambda: tq.tq_prefill_attention(q, cache, t0, w.scale, out, stream=stream), stream, torch,
+                   min_calls=3, min_s=0.5)
+        flops = w.B * w.Hq * 4 * w.d * (Lq * t0 + Lq * (Lq + 1) // 2)
+        tf = flops / ts / 1e12
+        res[label] = {"shape": f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d}, cache {T} positions, chunk Lq={Lq} at t0={t0}",
+                      "k": f"{w.k_bits}-bit MSE", "v": f"{w.v_bits}-bit MSE", "us": ts * 1e6,
+                      "tflops": tf, "peak_tflops": pk[0], "frac": tf / pk[0], "peak_source": pk[1],
+                      "flops": flops, "flop_count": "4 d per (query row, visible cached key): q.k and p.v"}
+        del cache, q, out
+        torch.cuda.empty_cache()
+    return res
+
+
+def tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    return 1590.0, "fallback 1.59 PFLOP/s"
 
 
 OTHER_WORKLOADS = ("tiny_single_head_fp32", "gpt2_prod_2bit", "llama3_8b_128k_3bit", "llama70b_asym_16k",
@@ -654,8 +705,33 @@ def measure_workload(w, tq, torch, stream, hbm):
     return e, sample
 
 
+def run_prefill_case(spec: str):
+    """One prefill call on a stated case, for profilers (no timing, no JSON line)."""
+    import dataclasses
+
+    import torch
+
+    from quantized_decode_attention_kv_b200 import tq
+    from quantized_decode_attention_kv_b200.workloads import WORKLOADS, make_inputs
+    T, Lq = (int(x) for x in spec.split(","))
+    w = dataclasses.replace(WORKLOADS[DEFAULT_WORKLOAD], B=4, T=T)
+    K, V, _ = make_inputs(w, device="cuda")
+    cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, seed=w.seed)
+    tq.tq_quantize_kv(K, V, cache)
+    q = torch.randn(w.B, Lq, w.Hq, w.d, generator=torch.Generator(device="cuda").manual_seed(77),
+                    device="cuda").to(torch.bfloat16)
+    out = torch.empty(w.B, Lq, w.Hq, w.d, device="cuda")
+    for _ in range(2):
+        tq.tq_prefill_attention(q, cache, T - Lq, w.scale, out)
+    torch.cuda.synchronize()
+    print(json.dumps({"prefill_case": spec, "out_finite": bool(torch.isfinite(out).all())}))
+
+
 def main():
     args = parse_args()
+    if args.prefill_case:
+        run_prefill_case(args.prefill_case)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -195,9 +195,10 @@ int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, flo
  * positions. T_lens is a HOST array of B = cache->B ints, each in 1..T_cap; it is read during
  * the call only (the lengths travel to the kernels as launch parameters, so a captured graph
  * keeps the values of the capture). The work is split evenly over the ragged (sequence, KV
- * head, 16-token tile) space. Supported for the tensor-core MSE configuration (d = 128, MSE
- * keys of 3/4 bits, MSE values of 2..4 bits, at most 8 query heads per KV head) with
- * B <= 512; other configurations return TQ_ERR_UNSUPPORTED. Workspace size from
+ * head, 16-token tile) space. Supported for the tensor-core configurations: d = 128 with MSE
+ * keys of 3/4 bits, MSE values of 2..4 bits and at most 8 query heads per KV head, and d = 64
+ * with 2-bit TurboQuant_prod keys and values of 64 sketch rows and 1 or 2 query heads per KV
+ * head; B <= 512; other configurations return TQ_ERR_UNSUPPORTED. Workspace size from
  * tq_decode_varlen_workspace_bytes (0 on invalid arguments). Errors as tq_decode_attention.
  * This extends the pages' decode ("Where This Fits in the Inference Stack": real serving
  * batches sequences of different lengths). */
@@ -250,10 +251,27 @@ int tq_decode_attention_paged(const void *q, int dtype, int Hq, const int *T_len
                               const tq_paged_cache *cache, float *out, void *ws, size_t ws_bytes,
                               void *stream);
 
+/* Prefill (chunked) attention over the compressed cache ("Where This Fits in the Inference
+ * Stack", Decode Throughput vs. Time to First Token: at long contexts the attention of prefill
+ * reads the compressed cache as well; TensorRT-LLM section: chunked attention). A chunk of Lq
+ * queries q [B][Lq][Hq][d] of `dtype` at positions t0 .. t0 + Lq - 1 (their own keys and values
+ * already written to the cache, e.g. by tq_quantize_kv with t_offset = t0) attends causally:
+ * query i of sequence b and query head hq reads cache positions 0 .. t0 + i of KV head
+ * hq / (Hq / Hkv). out [B][Lq][Hq][d] float32 (device, caller-owned). The arithmetic is that
+ * of the decode call (scores from 16-bit fixed-point centroids and 24-bit fixed-point queries
+ * on int8 tensor cores, softmax in fp32, P.V with fp16 weights times ||v|| and fp32
+ * accumulation). No workspace. Supported: d = 128, TurboQuant_mse keys of 3 or 4 bits and
+ * values of 2..4 bits, Hq / Hkv dividing 128; other configurations return TQ_ERR_UNSUPPORTED.
+ * Errors: TQ_ERR_INVALID_ARG (pointers, shapes, t0 + Lq > T_cap), TQ_ERR_CUDA. */
+int tq_prefill_attention(const void *q, int dtype, int Hq, int Lq, int t0, float scale,
+                         const tq_cache *cache, float *out, void *stream);
+
 /* Device-side faults recorded since the last call, as bits: bit 0 = a tensor-core kernel
  * (tcgen05 write path of TurboQuant_prod records) gave up waiting for its MMAs after about a
  * second, recorded a fault, freed its tensor memory and returned without writing the rest of
- * its records. Reading synchronises the device and clears the bits. Writes *flags; returns
+ * its records; bit 1 = the prefill kernel gave up waiting on one of its pipeline stages the
+ * same way and ran to its end without further waits (its outputs undefined). Reading
+ * synchronises the device and clears the bits. Writes *flags; returns
  * TQ_OK or TQ_ERR_CUDA. A set bit means a tensor-core
  * operation may still have been in flight when its tensor memory was released: the
  * library's device state (and the outputs of that call) are then undefined, and the caller

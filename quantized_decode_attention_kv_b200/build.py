@@ -17,7 +17,7 @@ LIB = os.path.join(PKG, "libtq.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
           "-I", os.path.join(ROOT, "include")]
-SOURCES = ["host.cpp", "quantize.cu", "quantize_fast.cu", "quantize_prod.cu", "decode.cu", "decode_mma.cu", "decode_prod.cu", "decode_bf16.cu"]
+SOURCES = ["host.cpp", "quantize.cu", "quantize_fast.cu", "quantize_prod.cu", "decode.cu", "decode_mma.cu", "prefill.cu", "decode_prod.cu", "decode_bf16.cu"]
 
 
 def _nvcc() -> str:

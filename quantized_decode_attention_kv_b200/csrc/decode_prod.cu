@@ -23,6 +23,8 @@
 #include "mma_ops.cuh"
 
 #include <algorithm>
+#include <vector>
+#include <type_traits>
 
 namespace tq {
 namespace {
@@ -149,7 +151,34 @@ struct ProdArgs {
   int tiles_per_bh, tiles_per_cta, slots, stride;
   long long total_tiles;
   uint32_t one2; // fp16 (1, 1): 0x3C003C00
+  int B;
 };
+struct NoVarLenP {};
+
+// The segment of the flattened (b, KV head, 16-token tile) space that starts at tile `seg`:
+// its (b, KV head), first tile, end and context length. A ragged call gives sequence b
+// ceil(len[b] / 16) tiles per KV head, starting at tile boff[b] (vb: the sequence of the
+// previous segment, advanced in place).
+template <bool RAG>
+__device__ __forceinline__ void prod_segment(const ProdArgs &a, const std::conditional_t<RAG, VarLen, NoVarLenP> &vl,
+                                             long long seg, long long range1, int &vb, long long &bh,
+                                             long long &seg_end, int &tile0, int &T_len) {
+  if constexpr (RAG) {
+    while (vb + 1 < a.B && vl.boff[vb + 1] <= seg) ++vb;
+    T_len = vl.blen[vb];
+    const int tpb = (T_len + 15) >> 4;
+    const long long local = seg - vl.boff[vb];
+    const int hh = static_cast<int>(local / tpb);
+    tile0 = static_cast<int>(local - static_cast<long long>(hh) * tpb);
+    bh = static_cast<long long>(vb) * a.Hkv + hh;
+    seg_end = min(range1, vl.boff[vb] + static_cast<long long>(hh + 1) * tpb);
+  } else {
+    T_len = a.T_len;
+    bh = seg / a.tiles_per_bh;
+    seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
+    tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+  }
+}
 
 // +-1 fp16 pair from bits (j, j + 16) of w moved to the sign bits by a left shift of `sh`
 // (sh = 15 - j): bit set = -1. `one2` holds fp16 (1, 1) in a register so that the mask and
@@ -167,7 +196,9 @@ struct ProdTile {
   uint16_t kn[2], kg[2], vn[2], vg[2]; // norms and residual norms of tokens r, r + 8
 };
 
-__global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArgs a) {
+template <bool RAG>
+__global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArgs a,
+                                                                   const std::conditional_t<RAG, VarLen, NoVarLenP> vl) {
   __shared__ float mst[kPW * 8];
   __shared__ float gmx[8];
   __shared__ float lsum[8];
@@ -183,10 +214,11 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
   const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
   const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
   int slot = 0;
+  int vb = 0;
   for (long long seg = range0; seg < range1; ++slot) {
-    const long long bh = seg / a.tiles_per_bh;
-    const long long seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
-    const int tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+    long long bh, seg_end;
+    int tile0, T_len;
+    prod_segment<RAG>(a, vl, seg, range1, vb, bh, seg_end, tile0, T_len);
     const int ntiles = static_cast<int>(seg_end - seg);
     seg = seg_end;
     const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
@@ -220,7 +252,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
     for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
 
     const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
-    const int tlast = a.T_len - 1;
+    const int tlast = T_len - 1;
     const uint8_t *kbase = (c < 2 ? a.kc : a.ks) + 4 * (c & 1);
     const int vwo = 4 * (r >> 2);
     const uint32_t selx = static_cast<uint32_t>(r & 3) | (static_cast<uint32_t>(4 + (r & 3)) << 8);
@@ -253,12 +285,12 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
                              a.vg + rec0 + tw0 + r};
 
     auto load_next = [&](ProdTile &T) {
-      if (lane < 8 && tpf + 16 <= a.T_len && tpf < (tile0 + ntiles) * 16)
+      if (lane < 8 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
       pfp += pfstep;
       tpf += kPW * 16;
       const int t0 = (tile0 + jl) * 16;
-      if (t0 + 16 <= a.T_len) {
+      if (t0 + 16 <= T_len) {
         T.kw[0] = __ldcs(reinterpret_cast<const uint32_t *>(kp));
         T.kw[1] = __ldcs(reinterpret_cast<const uint32_t *>(kp + 64));
         const int toff[4] = {0, 8, 64, 72};
@@ -323,7 +355,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
       const float kg0 = f16_bits_to_f32(T.kg[0]), kg1 = f16_bits_to_f32(T.kg[1]);
       const float vn0 = f16_bits_to_f32(T.vn[0]), vn1 = f16_bits_to_f32(T.vn[1]);
       const float vg0 = f16_bits_to_f32(T.vg[0]), vg1 = f16_bits_to_f32(T.vg[1]);
-      const bool ok0 = t0 + r < a.T_len, ok1 = t0 + r + 8 < a.T_len;
+      const bool ok0 = t0 + r < T_len, ok1 = t0 + r + 8 < T_len;
       const float s0 = ok0 ? kn0 * fmaf(kg0, sk0, code0) * kPLog2e : -INFINITY;
       const float s1 = ok1 ? kn1 * fmaf(kg1, sk1, code1) * kPLog2e : -INFINITY;
 
@@ -443,7 +475,9 @@ struct LutTile {
   uint32_t vm[2][4], vq[2][4]; // value code / sketch word r/4 of tokens 16 h + {2c, 2c+1, 2c+8, 2c+9}
 };
 
-__global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const ProdArgs a) {
+template <bool RAG>
+__global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const ProdArgs a,
+                                                                       const std::conditional_t<RAG, VarLen, NoVarLenP> vl) {
   __shared__ float tab[16 * 256];
   __shared__ float mst[kPW];
   __shared__ float gmx, lsum;
@@ -458,10 +492,11 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
   const long long range0 = static_cast<long long>(blockIdx.x) * a.tiles_per_cta;
   const long long range1 = min(a.total_tiles, range0 + a.tiles_per_cta);
   int slot = 0;
+  int vb = 0;
   for (long long seg = range0; seg < range1; ++slot) {
-    const long long bh = seg / a.tiles_per_bh;
-    const long long seg_end = min(range1, (bh + 1) * a.tiles_per_bh);
-    const int tile0 = static_cast<int>(seg - bh * a.tiles_per_bh);
+    long long bh, seg_end;
+    int tile0, T_len;
+    prod_segment<RAG>(a, vl, seg, range1, vb, bh, seg_end, tile0, T_len);
     const int ntiles = static_cast<int>(seg_end - seg);
     seg = seg_end;
     const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
@@ -486,7 +521,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
     for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
 
     const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
-    const int ts = tile0 * 16, te = min((tile0 + ntiles) * 16, a.T_len); // segment tokens
+    const int ts = tile0 * 16, te = min((tile0 + ntiles) * 16, T_len); // segment tokens
     const int ngroups = (te - ts + 31) / 32;
     const int vwo = 4 * (r >> 2);
     const uint32_t selx = static_cast<uint32_t>(r & 3) | (static_cast<uint32_t>(4 + (r & 3)) << 8);
@@ -655,10 +690,12 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
 // Merge the partial records of one (b, q-head); u' = -c1 u, add sqrt(d) sqrt(pi/2)/m S^T w,
 // apply the inverse rotation D H / d and divide by the softmax sum. One warp per (b, q-head);
 // lane l owns coordinates 2 l, 2 l + 1 and sketch rows 2 l, 2 l + 1.
+template <bool RAG>
 __global__ void __launch_bounds__(128) combine_prod_kernel(const float *part, int B, int Hkv, int G,
                                                            int tiles_per_bh, int tiles_per_cta,
                                                            int slots, int stride, uint64_t seed,
-                                                           const float *Sv, float c1v, float *out) {
+                                                           const float *Sv, float c1v, float *out,
+                                                           const std::conditional_t<RAG, VarLen, NoVarLenP> vl) {
   const int lane = threadIdx.x & 31;
   const int Hq = Hkv * G;
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -667,10 +704,31 @@ __global__ void __launch_bounds__(128) combine_prod_kernel(const float *part, in
   const int b = gw / Hq, hq = gw - b * Hq;
   const int h = hq / G, g = hq - h * G;
   const long long bh = static_cast<long long>(b) * Hkv + h;
-  const long long first = bh * tiles_per_bh, last = first + tiles_per_bh - 1;
+  // the (b, KV head) of flattened tile f (ragged calls: sequence by binary search)
+  auto bh_of = [&](long long f) -> long long {
+    if constexpr (!RAG) {
+      return f / tiles_per_bh;
+    } else {
+      int lo = 0, hi = B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (vl.boff[mid] <= f) lo = mid;
+        else hi = mid - 1;
+      }
+      const int tpb = (vl.blen[lo] + 15) >> 4;
+      return static_cast<long long>(lo) * Hkv + (f - vl.boff[lo]) / tpb;
+    }
+  };
+  int tpb = tiles_per_bh;
+  long long first = bh * tiles_per_bh;
+  if constexpr (RAG) {
+    tpb = (vl.blen[b] + 15) >> 4;
+    first = vl.boff[b] + static_cast<long long>(h) * tpb;
+  }
+  const long long last = first + tpb - 1;
   const int cta0 = static_cast<int>(first / tiles_per_cta), cta1 = static_cast<int>(last / tiles_per_cta);
   auto rec = [&](int cta) {
-    const long long bh0 = static_cast<long long>(cta) * tiles_per_cta / tiles_per_bh;
+    const long long bh0 = bh_of(static_cast<long long>(cta) * tiles_per_cta);
     return part + ((static_cast<size_t>(cta) * slots + (bh - bh0)) * G + g) * stride;
   };
   float M = -INFINITY;
@@ -741,20 +799,37 @@ bool prod_decode_supported(int d, int k_mode, int k_bits, int k_m, int v_mode, i
          v_bits == 2 && v_m == kPM && G >= 1 && G <= 2;
 }
 
-void plan_prod(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p) {
+void plan_prod(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p, const int *T_lens) {
   const int G = Hq / Hkv;
   p->path = 2;
   p->tile = 16;
   p->gc = G;
   p->ws_stride = 2 + kPD + kPM + 2; // 132 floats
   p->tiles_per_bh = (T_len + 15) / 16;
-  const long long total = static_cast<long long>(B) * Hkv * p->tiles_per_bh;
+  long long total = static_cast<long long>(B) * Hkv * p->tiles_per_bh;
+  if (T_lens) {
+    total = 0;
+    for (int b = 0; b < B; ++b) total += static_cast<long long>(Hkv) * ((T_lens[b] + 15) / 16);
+  }
   long long ctas = static_cast<long long>(sm_count) * 3;
   ctas = std::min<long long>(ctas, (total + 7) / 8); // at least 8 tiles per CTA
   ctas = std::max<long long>(ctas, 1);
   p->tiles_per_cta = static_cast<int>((total + ctas - 1) / ctas);
   p->ctas = static_cast<int>((total + p->tiles_per_cta - 1) / p->tiles_per_cta);
   p->slots = (p->tiles_per_cta + p->tiles_per_bh - 1) / p->tiles_per_bh + 1;
+  if (T_lens) { // the most (b, KV head) segments any CTA's range touches
+    std::vector<int> nseg(p->ctas, 0);
+    long long off = 0;
+    for (int b = 0; b < B; ++b) {
+      const int tpb = (T_lens[b] + 15) / 16;
+      for (int h = 0; h < Hkv; ++h, off += tpb) {
+        const int c0 = static_cast<int>(off / p->tiles_per_cta);
+        const int c1 = static_cast<int>((off + tpb - 1) / p->tiles_per_cta);
+        for (int c = c0; c <= c1; ++c) ++nseg[c];
+      }
+    }
+    p->slots = *std::max_element(nseg.begin(), nseg.end());
+  }
   p->splits = 0;
   p->chunk = 0;
   p->part_bytes = static_cast<size_t>(p->ctas) * p->slots * G * p->ws_stride * sizeof(float);
@@ -790,12 +865,29 @@ cudaError_t launch_prod_decode(const DecodeArgs &a, cudaStream_t s) {
   f.stride = p.ws_stride;
   f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
   f.one2 = 0x3C003C00u;
-  e = launch_pdl(f.G == 1 ? decode_prod_lut_kernel : decode_prod_kernel, dim3(p.ctas),
-                 dim3(kPThreads), 0, s, f);
+  f.B = a.B;
+  if (a.T_lens) {
+    // ragged batch: the per-sequence lengths and tile offsets travel as launch parameters
+    VarLen vl;
+    vl.on = 1;
+    vl.boff[0] = 0;
+    for (int b = 0; b < a.B; ++b) {
+      vl.blen[b] = a.T_lens[b];
+      vl.boff[b + 1] = vl.boff[b] + a.Hkv * ((a.T_lens[b] + 15) / 16);
+    }
+    f.total_tiles = vl.boff[a.B];
+    e = launch_pdl(f.G == 1 ? decode_prod_lut_kernel<true> : decode_prod_kernel<true>, dim3(p.ctas),
+                   dim3(kPThreads), 0, s, f, vl);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(combine_prod_kernel<true>, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
+                      static_cast<const float *>(a.ws), a.B, a.Hkv, f.G, p.tiles_per_bh, p.tiles_per_cta,
+                      p.slots, p.ws_stride, a.seed, a.v.S, a.v.cb.c[1], a.out, vl);
+  }
+  e = launch_pdl(f.G == 1 ? decode_prod_lut_kernel<false> : decode_prod_kernel<false>, dim3(p.ctas),
+                 dim3(kPThreads), 0, s, f, NoVarLenP{});
   if (e != cudaSuccess) return e;
-  return launch_pdl(combine_prod_kernel, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
+  return launch_pdl(combine_prod_kernel<false>, dim3((a.B * a.Hq + 3) / 4), dim3(128), 0, s,
                     static_cast<const float *>(a.ws), a.B, a.Hkv, f.G, p.tiles_per_bh,
-                    p.tiles_per_cta, p.slots, p.ws_stride, a.seed, a.v.S, a.v.cb.c[1], a.out);
+                    p.tiles_per_cta, p.slots, p.ws_stride, a.seed, a.v.S, a.v.cb.c[1], a.out, NoVarLenP{});
 }
-
 } // namespace tq

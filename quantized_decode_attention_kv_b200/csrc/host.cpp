@@ -470,11 +470,22 @@ static int check_varlen(const tq_cache *cache, int Hq, const int *T_lens, int *T
     mx = std::max(mx, T_lens[b]);
   }
   const int fp = fast_path(*cache, Hq);
-  if (fp == 0 || fp == tq::kProdFast)
-    return fail(TQ_ERR_UNSUPPORTED, "ragged decode needs the tensor-core MSE configuration "
-                                    "(d = 128, MSE, 3/4-bit K, 2..4-bit V, <= 8 query heads per KV head)");
+  if (fp == 0)
+    return fail(TQ_ERR_UNSUPPORTED, "ragged decode needs a tensor-core configuration (d = 128, MSE, "
+                                    "3/4-bit K, 2..4-bit V, <= 8 query heads per KV head; or d = 64, "
+                                    "2-bit TurboQuant_prod K and V with 64 sketch rows, <= 2 query heads "
+                                    "per KV head)");
   *T_max = mx;
   return TQ_OK;
+}
+
+// Plan of a ragged call for the configuration's tensor-core kernel.
+static void plan_varlen(const tq_cache &c, int Hq, int mx, int sms, const int *T_lens, tq::DecodePlan *p) {
+  const int fp = fast_path(c, Hq);
+  if (fp == tq::kProdFast)
+    tq::plan_prod(c.B, Hq, c.Hkv, mx, sms, p, T_lens);
+  else
+    tq::plan_fast(c.B, Hq, c.Hkv, mx, sms, fp >> 4, fp & 15, p, T_lens);
 }
 
 size_t tq_decode_varlen_workspace_bytes(int Hq, const tq_cache *cache, const int *T_lens) {
@@ -486,8 +497,7 @@ size_t tq_decode_varlen_workspace_bytes(int Hq, const tq_cache *cache, const int
     return 0;
   }
   tq::DecodePlan p{};
-  const int fp = fast_path(*cache, Hq);
-  tq::plan_fast(cache->B, Hq, cache->Hkv, mx, sms, fp >> 4, fp & 15, &p, T_lens);
+  plan_varlen(*cache, Hq, mx, sms, T_lens, &p);
   return p.ws_bytes;
 }
 
@@ -509,8 +519,9 @@ static int decode_varlen_impl(const void *q, int dtype, int Hq, const int *T_len
   if (st) return st;
   int sms = sm_count();
   if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
-  const int fp = fast_path(*cache, Hq);
-  tq::plan_fast(cache->B, Hq, cache->Hkv, mx, sms, fp >> 4, fp & 15, &a.plan, T_lens);
+  if (pg.pshift >= 0 && fast_path(*cache, Hq) == tq::kProdFast)
+    return fail(TQ_ERR_UNSUPPORTED, "a paged cache holds TurboQuant_mse records only");
+  plan_varlen(*cache, Hq, mx, sms, T_lens, &a.plan);
   if (!ws || !aligned16(ws) || ws_bytes < a.plan.ws_bytes)
     return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
                 a.plan.ws_bytes, ws ? ws_bytes : 0);
@@ -528,7 +539,9 @@ static int decode_varlen_impl(const void *q, int dtype, int Hq, const int *T_len
   a.seed = cache->seed;
   a.out = out;
   a.ws = static_cast<float *>(ws);
-  return cuda_status(tq::launch_fast_decode(a, static_cast<cudaStream_t>(stream)), "decode launch");
+  return cuda_status(a.plan.path == 2 ? tq::launch_prod_decode(a, static_cast<cudaStream_t>(stream))
+                                      : tq::launch_fast_decode(a, static_cast<cudaStream_t>(stream)),
+                     "decode launch");
 }
 
 int tq_decode_attention_varlen(const void *q, int dtype, int Hq, const int *T_lens, float scale,
@@ -651,9 +664,56 @@ int tq_decode_attention_noalloc(const void *q, int dtype, int Hq, int T_len, flo
                      "decode (fixed scratch) launch");
 }
 
+int tq_prefill_attention(const void *q, int dtype, int Hq, int Lq, int t0, float scale,
+                         const tq_cache *cache, float *out, void *stream) {
+  int st = check_cache(cache);
+  if (st) return st;
+  if (!dtype_ok(dtype)) return fail(TQ_ERR_INVALID_ARG, "dtype=%d is not F32/BF16/F16", dtype);
+  if (!q || !out || !aligned16(q) || !aligned16(out))
+    return fail(TQ_ERR_INVALID_ARG, "q/out must be non-NULL and 16-byte aligned");
+  if (Hq < 1 || Hq % cache->Hkv || Hq > 65535)
+    return fail(TQ_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d (<= 65535)", Hq,
+                cache->Hkv);
+  if (Lq < 1 || t0 < 0 || static_cast<long long>(t0) + Lq > cache->T_cap)
+    return fail(TQ_ERR_INVALID_ARG, "Lq=%d, t0=%d: need Lq >= 1, t0 >= 0, t0 + Lq <= T_cap=%d", Lq, t0,
+                cache->T_cap);
+  if (!std::isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "scale is not finite");
+  tq::PrefillLaunch l;
+  std::memset(&l, 0, sizeof l);
+  st = resolve_tensor(*cache, 0, &l.k);
+  if (st) return st;
+  st = resolve_tensor(*cache, 1, &l.v);
+  if (st) return st;
+  if (!tq::prefill_supported(cache->d, l.k.mode, l.k.wbits, l.v.mode, l.v.wbits, Hq / cache->Hkv))
+    return fail(TQ_ERR_UNSUPPORTED,
+                "prefill supports head_dim 128, TurboQuant_mse keys of 3/4 bits and values of 2..4 bits, "
+                "and Hq/Hkv dividing 128");
+  const long long ctas = static_cast<long long>(cache->B) * cache->Hkv *
+                         ((Lq + 128 / (Hq / cache->Hkv) - 1) / (128 / (Hq / cache->Hkv)));
+  if (ctas > 0x7FFFFFFF) return fail(TQ_ERR_INVALID_ARG, "too many query blocks");
+  l.q = q;
+  l.q_dtype = dtype;
+  l.B = cache->B;
+  l.Hq = Hq;
+  l.Hkv = cache->Hkv;
+  l.Lq = Lq;
+  l.t0 = t0;
+  l.T_cap = cache->T_cap;
+  l.scale = scale;
+  l.seed = cache->seed;
+  l.out = out;
+  return cuda_status(tq::launch_prefill(l, static_cast<cudaStream_t>(stream)), "prefill launch");
+}
+
 int tq_device_faults(unsigned *flags) {
   if (!flags) return fail(TQ_ERR_INVALID_ARG, "flags is NULL");
-  return cuda_status(tq::read_and_clear_prod_faults(flags), "tq_device_faults");
+  unsigned prod = 0, pre = 0;
+  int st = cuda_status(tq::read_and_clear_prod_faults(&prod), "tq_device_faults");
+  if (st) return st;
+  st = cuda_status(tq::read_and_clear_prefill_faults(&pre), "tq_device_faults");
+  if (st) return st;
+  *flags = (prod ? 1u : 0u) | (pre ? 2u : 0u);
+  return TQ_OK;
 }
 
 int tq_launch_counts(const tq_cache *cache, int dtype, int T, int Hq, int T_len,

@@ -1,0 +1,519 @@
+// Prefill (chunked) attention over the compressed cache on the fifth-generation tensor cores:
+// head_dim 128, TurboQuant_mse keys of 3 or 4 bits and values of 2, 3 or 4 bits.
+//
+// "Where This Fits in the Inference Stack", Decode Throughput vs. Time to First Token: at long
+// contexts the attention of prefill reads the cache too; TensorRT-LLM section: chunked
+// attention is one of the kernels that needs the in-register dequantisation. A chunk of Lq
+// queries at positions t0 .. t0 + Lq - 1 (their own keys and values already in the cache)
+// attends causally: query i sees cache positions 0 .. t0 + i.
+//
+// With many queries per KV head the dequantisation of a key or value tile is shared by all of
+// them, so the tiles are dequantised once into shared-memory operands and the contractions are
+// ordinary tcgen05 MMAs with wide N:
+//   S_type = Q_type . K^T (kind::i8, M = 128 query rows, N = 64 tokens, K = 256): the key
+//     operand holds the 16-bit fixed-point centroids as {hi, hi, lo, lo} bytes per coordinate
+//     pair and the three query operands the 24-bit fixed-point query parts, exactly the score
+//     arithmetic of the decode kernels (c.q = 2^24 S_0 + 2^16 S_1 + 2^8 S_2 up to c_lo q_lo);
+//   O += P' . V (kind::f16, M = 128, N = 128 coordinates, K = 64 tokens): P' = p ||v|| in fp16
+//     written by the softmax threads into tensor memory (the A operand), V the fp16 centroids
+//     in shared memory (MN-major: each token's coordinates contiguous).
+// A CTA takes 128 query rows (128 / G positions x G query heads) of one (batch, KV head):
+//   softmax warps (4): thread = query row = TMEM lane; it prepares its queries (rotation,
+//     fixed point), and per KV tile reads its row's scores, keeps the row's running maximum and
+//     sum (no cross-thread reduction), rescales its output row in TMEM when the maximum moves,
+//     and at the end applies the inverse rotation to its row;
+//   producer warps (4): dequantise each 64-token tile of codes into the two operands (two
+//     buffers), with the tile's key and value norms;
+//   MMA warp (1 thread): S MMAs of tile j, then P.V of tile j - 1, with tcgen05.commit
+//     releasing the buffers.
+// TMEM: two score stages of 3 x 64 int32 columns (the tile's P' overwrites the first 32 columns
+// of its stage once read) and the 128 fp32 output columns. Every mbarrier wait is bounded.
+#include "decode_mse_common.cuh"
+#include "tc_ops.cuh"
+
+#include <algorithm>
+
+namespace tq {
+namespace {
+using namespace mma_ops;
+using namespace mse;
+
+constexpr int kRows = 128;                   // query rows per CTA (TMEM lanes)
+constexpr int kKT = 64;                      // KV tokens per tile
+constexpr int kSWp = 4, kPWp = 4;            // softmax warps, producer warps
+constexpr int kWarpMMAp = kSWp + kPWp;       // the MMA warp
+constexpr int kThreadsP = (kSWp + kPWp + 1) * 32;
+constexpr uint32_t kTmemColsP = 512;
+constexpr uint32_t kSCols = 3 * kKT;         // one score stage
+constexpr uint32_t kOCol = 2 * kSCols;       // output columns 384 .. 511
+constexpr long long kWaitCyclesP = 1ll << 31; // about a second
+
+__device__ unsigned g_prefill_fault;
+
+struct PrefillArgs {
+  const uint8_t *kc, *vc;
+  const uint16_t *kn, *vn;
+  const void *q; // [B][Lq][Hq][128] of q_dtype
+  int q_dtype;
+  float *out;    // [B][Lq][Hq][128] float32
+  float scale;
+  uint64_t seed;
+  int Hq, Hkv, G, Lq, t0, T_cap;
+  int P;      // query positions per CTA (128 / G)
+  int blocks; // CTAs per (batch, KV head)
+  float kcent[16];
+  float kcsc;
+  float vcent[16];
+};
+
+template <int KB, int VB>
+struct PfLayout {
+  static constexpr int oQ = 0;                       // 3 x [128 rows][256 bytes] int8, K-major
+  static constexpr int oK = oQ + 3 * kRows * 256;    // 2 x [64 tokens][256 bytes] int8, K-major
+  static constexpr int oV = oK + 2 * kKT * 256;      // 2 x [128 coords][64 tokens] fp16, MN-major
+  static constexpr int oKN = oV + 2 * kKT * 256;     // 2 x 64 key norms (float)
+  static constexpr int oVN = oKN + 2 * kKT * 4;      // 2 x 64 value norms (float)
+  static constexpr int oKT = oVN + 2 * kKT * 4;      // key entries {hi, hi, lo, lo} per code pair
+  static constexpr int kKRows = KB == 4 ? 256 : 64;
+  static constexpr int oVT = oKT + kKRows * 4;       // value table
+  static constexpr int kVRows = VB == 2 ? 256 : 1 << (2 * VB);
+  static constexpr int kVEntry = VB == 2 ? 8 : 4;    // 2-bit: 4 fp16 per code byte; else fp16x2 per pair
+  static constexpr int oQP = oVT + kVRows * kVEntry; // per softmax warp: one prepared query
+  static constexpr int oInv = oQP + kSWp * static_cast<int>(sizeof(QPrep));
+  static constexpr int oBar = (oInv + kRows * 4 + 7) & ~7;
+  static constexpr int nBar = 11;                    // KV_full[2] KV_free[2] S_full[2] S_free[2] P_full[2] PV_done Q_ready fin
+  static constexpr int oMisc = oBar + (nBar + 2) * 8;
+  static constexpr int kSmem = oMisc + 16 + 1024;    // + alignment of the base
+};
+
+__device__ __forceinline__ bool pf_try(uint32_t mbar, uint32_t parity) {
+  uint32_t done;
+  asm volatile("{\n\t.reg .pred P;\n\tmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+               "selp.u32 %0, 1, 0, P;\n\t}\n"
+               : "=r"(done)
+               : "r"(mbar), "r"(parity), "r"(500000u)
+               : "memory");
+  return done != 0;
+}
+
+__device__ __noinline__ void pf_wait_slow(uint32_t mbar, uint32_t parity, volatile int *dead) {
+  const long long t0 = clock64();
+  while (!pf_try(mbar, parity)) {
+    if (*dead) return;
+    if (clock64() - t0 > kWaitCyclesP) {
+      *dead = 1;
+      atomicOr(&g_prefill_fault, 1u);
+      return;
+    }
+  }
+}
+
+// Bounded wait on an mbarrier phase (about a second; after a timeout, or once another warp of
+// the CTA timed out, it returns without waiting and the CTA runs to its end).
+__device__ __forceinline__ void pf_wait(uint32_t mbar, uint32_t parity, volatile int *dead) {
+  if (!pf_try(mbar, parity)) pf_wait_slow(mbar, parity, dead);
+}
+
+template <int KB, int VB>
+__global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs a) {
+  using L = PfLayout<KB, VB>;
+  constexpr int KR = KB * 16, VR = VB * 16; // record bytes
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
+  const uint32_t sb = (raw + 1023) & ~1023u;
+  uint8_t *const sm = smem_raw + (sb - raw);
+  const uint32_t bar0 = sb + L::oBar;
+  auto KV_full = [&](int x) { return bar0 + 8u * x; };
+  auto KV_free = [&](int x) { return bar0 + 8u * (2 + x); };
+  auto S_full = [&](int x) { return bar0 + 8u * (4 + x); };
+  auto S_free = [&](int x) { return bar0 + 8u * (6 + x); };
+  auto P_full = [&](int x) { return bar0 + 8u * (8 + x); };
+  const uint32_t PV_done = bar0 + 8u * 10, Q_ready = bar0 + 8u * 11, fin_bar = bar0 + 8u * 12;
+  uint32_t *const misc = reinterpret_cast<uint32_t *>(sm + L::oMisc);
+  volatile int *const dead = reinterpret_cast<volatile int *>(misc + 1);
+  float *const knb = reinterpret_cast<float *>(sm + L::oKN);
+  float *const vnb = reinterpret_cast<float *>(sm + L::oVN);
+  float *const rinv = reinterpret_cast<float *>(sm + L::oInv);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int blk = blockIdx.x % a.blocks;
+  const long long bh = blockIdx.x / a.blocks;
+  const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
+  const int i0 = blk * a.P;
+  const int i_last = min(a.Lq, i0 + a.P) - 1;
+  const int pos_last = a.t0 + i_last;
+  const int ntiles = pos_last / kKT + 1;
+
+  // ---- tables: key entries {hi(c0), hi(c1), lo(c0), lo(c1)} of a code pair (the decode
+  //      kernels' 16-bit fixed point); values as fp16 centroids
+  {
+    uint32_t *kt = reinterpret_cast<uint32_t *>(sm + L::oKT);
+    for (int e = tid; e < L::kKRows; e += kThreadsP) {
+      const float c0 = a.kcent[e & (KB == 4 ? 15 : 7)], c1 = a.kcent[KB == 4 ? e >> 4 : e >> 3];
+      const int x0 = __float2int_rn(c0 * a.kcsc), x1 = __float2int_rn(c1 * a.kcsc);
+      const int l0 = ((x0 + 128) & 255) - 128, l1 = ((x1 + 128) & 255) - 128;
+      const int h0 = (x0 - l0) >> 8, h1 = (x1 - l1) >> 8;
+      kt[e] = static_cast<uint32_t>(h0 & 255) | (static_cast<uint32_t>(h1 & 255) << 8) |
+              (static_cast<uint32_t>(l0 & 255) << 16) | (static_cast<uint32_t>(l1 & 255) << 24);
+    }
+    uint32_t *vt = reinterpret_cast<uint32_t *>(sm + L::oVT);
+    for (int e = tid; e < L::kVRows; e += kThreadsP) {
+      if constexpr (VB == 2) {
+        vt[2 * e] = pack_h2(a.vcent[e & 3], a.vcent[(e >> 2) & 3]);
+        vt[2 * e + 1] = pack_h2(a.vcent[(e >> 4) & 3], a.vcent[(e >> 6) & 3]);
+      } else {
+        vt[e] = pack_h2(a.vcent[e & ((1 << VB) - 1)], a.vcent[e >> VB]);
+      }
+    }
+  }
+  if (tid == 0) {
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(KV_full(x), 32 * kPWp);
+      tc::mbar_init(KV_free(x), 1);
+      tc::mbar_init(S_full(x), 1);
+      tc::mbar_init(S_free(x), 1);
+      tc::mbar_init(P_full(x), 32 * kSWp);
+    }
+    tc::mbar_init(PV_done, 1);
+    tc::mbar_init(Q_ready, 32 * kSWp);
+    tc::mbar_init(fin_bar, 1);
+    *dead = 0;
+    tc::mbar_init_fence();
+  }
+  if (warp == kWarpMMAp) tc::tmem_alloc(sb + L::oMisc, kTmemColsP);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = misc[0];
+  pdl_wait(); // the queries and the cache are written by earlier kernels
+  pdl_trigger();
+
+  if (warp < kSWp) {
+    // =============================== softmax warps: thread = query row = TMEM lane
+    const int row = tid;
+    const int ri = row / a.G, rg = row - ri * a.G; // query position within the block, head
+    const bool row_ok = ri < a.P && i0 + ri < a.Lq;
+    const int my_pos = a.t0 + i0 + ri;
+    // ---- queries of the warp's 32 rows: rotation and 24-bit fixed point (one warp per query),
+    //      written as the three int8 operands {q_hi, q_hi, 0, 0}, {q_mid, q_mid, q_hi, q_hi},
+    //      {q_lo, q_lo, q_mid, q_mid} at the {hi, hi, lo, lo} slots of each coordinate pair
+    QPrep *qs = reinterpret_cast<QPrep *>(sm + L::oQP) + warp;
+#pragma unroll 1
+    for (int k = 0; k < 32; ++k) {
+      const int rr = 32 * warp + k;
+      const int qi = rr / a.G, qg = rr - qi * a.G;
+      const bool ok = qi < a.P && i0 + qi < a.Lq;
+      if (ok) {
+        const size_t bq = (static_cast<size_t>(b) * a.Lq + i0 + qi) * a.Hq + h * a.G + qg;
+        prep_query(a.q, a.q_dtype, bq, a.scale, a.seed, a.kcsc, qs, lane);
+      } else {
+        reinterpret_cast<uint32_t *>(qs->hi)[lane] = 0u;
+        reinterpret_cast<uint32_t *>(qs->mid)[lane] = 0u;
+        reinterpret_cast<uint32_t *>(qs->lo)[lane] = 0u;
+        if (lane == 0) qs->inv = 0.f;
+      }
+      __syncwarp();
+      // lane l: k bytes 8 l .. 8 l + 7 = code pairs 2 l, 2 l + 1 (coordinates 4 l .. 4 l + 3)
+      const uint32_t hi = reinterpret_cast<const uint32_t *>(qs->hi)[lane];
+      const uint32_t mid = reinterpret_cast<const uint32_t *>(qs->mid)[lane];
+      const uint32_t lo = reinterpret_cast<const uint32_t *>(qs->lo)[lane];
+      const uint32_t off = (rr & 7) * 16 + (rr >> 3) * 2048 + (lane >> 1) * 128 + 8 * (lane & 1);
+      *reinterpret_cast<uint2 *>(sm + L::oQ + off) = make_uint2(hi & 0xFFFFu, hi >> 16);
+      *reinterpret_cast<uint2 *>(sm + L::oQ + kRows * 256 + off) =
+          make_uint2((mid & 0xFFFFu) | (hi << 16), (mid >> 16) | (hi & 0xFFFF0000u));
+      *reinterpret_cast<uint2 *>(sm + L::oQ + 2 * kRows * 256 + off) =
+          make_uint2((lo & 0xFFFFu) | (mid << 16), (lo >> 16) | (mid & 0xFFFF0000u));
+      if (lane == 0) rinv[rr] = qs->inv * kLog2e;
+      __syncwarp();
+    }
+    tc::fence_async_smem();
+    tc::mbar_arrive(Q_ready);
+    __syncwarp();
+    const float qsc = rinv[row];
+    const uint32_t lrow = static_cast<uint32_t>(32 * warp) << 16;
+
+    float m_run = -INFINITY, l_run = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < ntiles; ++j) {
+      const int x = j & 1;
+      pf_wait(S_full(x), (j >> 1) & 1, dead);
+      tc::fence_after_sync();
+      const uint32_t st = tbase + lrow + x * kSCols;
+      float s[kKT];
+#pragma unroll
+      for (int cch = 0; cch < kKT / 16; ++cch) {
+        uint32_t r0[16], r1[16], r2[16];
+        tc::tmem_ld32x32_x16(st + 16 * cch, r0);
+        tc::tmem_ld32x32_x16(st + kKT + 16 * cch, r1);
+        tc::tmem_ld32x32_x16(st + 2 * kKT + 16 * cch, r2);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int tt = 16 * cch + t;
+          const float d = fmaf(__int_as_float(static_cast<int>(r2[t]) + kMagic), 1.0f / 65536.0f,
+                               fmaf(__int_as_float(static_cast<int>(r1[t]) + kMagic), 1.0f / 256.0f,
+                                    __int_as_float(static_cast<int>(r0[t]) + kMagic) - kMagicAdj));
+          s[tt] = kKT * j + tt <= my_pos ? knb[x * kKT + tt] * qsc * d : -INFINITY;
+        }
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int t = 1; t < kKT; ++t) mx = fmaxf(mx, s[t]);
+      const float mn = fmaxf(m_run, mx);
+      // a row whose maximum moved scales its sum and the output row accumulated so far (once the
+      // previous tile's P.V has landed; before the first P.V the output is undefined and is
+      // overwritten). The TMEM loads and stores are warp-collective (.sync.aligned), so the
+      // whole warp takes this path when any of its rows needs it, the others with factor 1.
+      const bool moved = mn != m_run;
+      const float alpha = moved ? softmax_exp2(m_run - mn) : 1.f;
+      l_run *= alpha;
+      m_run = mn;
+      if (j > 0 && __any_sync(0xffffffffu, moved)) {
+        // completion j - 1 of PV_done: S_full(j) implies P.V of tile j - 2 had completed, so
+        // the barrier is at completion j - 1 or j and the parity identifies it
+        pf_wait(PV_done, (j - 1) & 1, dead);
+        tc::fence_after_sync();
+#pragma unroll 1
+        for (int cch = 0; cch < 4; ++cch) {
+          uint32_t ov[32];
+          tc::tmem_ld32x32_x32u(tbase + lrow + kOCol + 32 * cch, ov);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tc::tmem_st32x32_x32(tbase + lrow + kOCol + 32 * cch, ov);
+        }
+      }
+      // weights p ||v|| as fp16 into the first 32 columns of the stage (already read)
+      uint32_t pw[kKT / 2];
+#pragma unroll
+      for (int t = 0; t < kKT; t += 2) {
+        const float p0 = s[t] == -INFINITY ? 0.f : softmax_exp2(s[t] - m_run);
+        const float p1 = s[t + 1] == -INFINITY ? 0.f : softmax_exp2(s[t + 1] - m_run);
+        l_run += p0 + p1;
+        pw[t >> 1] = pack_h2(p0 * vnb[x * kKT + t], p1 * vnb[x * kKT + t + 1]);
+      }
+      tc::tmem_st32x32_x32(st, pw);
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(P_full(x));
+    }
+    // ---- output row: O / l in the rotated domain, then the inverse rotation D H / d (after the
+    //      last P.V: the MMA thread commits every MMA of the CTA to fin_bar)
+    pf_wait(fin_bar, 0, dead);
+    tc::fence_after_sync();
+    float o[128];
+#pragma unroll
+    for (int cch = 0; cch < 4; ++cch) {
+      uint32_t ov[32];
+      tc::tmem_ld32x32_x32u(tbase + lrow + kOCol + 32 * cch, ov);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[32 * cch + e] = __uint_as_float(ov[e]);
+    }
+#pragma unroll
+    for (int span = 1; span < 128; span <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        if ((i & span) == 0) {
+          const float u = o[i], v = o[i + span];
+          o[i] = u + v;
+          o[i + span] = u - v;
+        }
+      }
+    }
+    if (row_ok) {
+      const float sc = 1.0f / (128.0f * l_run);
+      const uint64_t w0 = dev_splitmix64(a.seed, 0), w1 = dev_splitmix64(a.seed, 1);
+      float *dst = a.out + ((static_cast<size_t>(b) * a.Lq + i0 + ri) * a.Hq + h * a.G + rg) * 128;
+#pragma unroll
+      for (int i = 0; i < 128; i += 4) {
+        float4 v4;
+        float *vp = &v4.x;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int ii = i + e;
+          const bool neg = ((ii < 64 ? w0 >> ii : w1 >> (ii - 64)) & 1ull) != 0;
+          vp[e] = neg ? -o[ii] * sc : o[ii] * sc;
+        }
+        *reinterpret_cast<float4 *>(dst + i) = v4;
+      }
+    }
+  } else if (warp < kWarpMMAp) {
+    // =============================== producer warps: 64-token tiles of K and V operands
+    const int pt = tid - 32 * kSWp;   // 0..127
+    const int n = pt >> 1, half = pt & 1;
+    const uint32_t *kt = reinterpret_cast<const uint32_t *>(sm + L::oKT);
+    const uint8_t *vt = sm + L::oVT;
+#pragma unroll 1
+    for (int j = 0; j < ntiles; ++j) {
+      const int x = j & 1;
+      if (j >= 2) pf_wait(KV_free(x), ((j >> 1) - 1) & 1, dead);
+      const int tok = min(kKT * j + n, pos_last);
+      const size_t rec = static_cast<size_t>(bh) * a.T_cap + tok;
+      // keys: code pairs 32 half .. 32 half + 31 -> k bytes 128 half .. 128 half + 127 of row n
+      {
+        uint32_t w[KB * 2];
+        const uint32_t *kp = reinterpret_cast<const uint32_t *>(a.kc + rec * KR + KB * 8 * half);
+#pragma unroll
+        for (int k = 0; k < KB * 2; ++k) w[k] = __ldg(kp + k);
+        uint8_t *kdst = sm + L::oK + x * (kKT * 256) + (n & 7) * 16 + (n >> 3) * 2048 + half * 8 * 128;
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) { // 16 k bytes = 4 code pairs
+          uint32_t e4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int pp = 4 * c16 + u; // pair within this half
+            uint32_t idx;
+            if constexpr (KB == 4) {
+              idx = (w[pp >> 2] >> (8 * (pp & 3))) & 0xFFu;
+            } else {
+              idx = bits_at(w, 6 * pp, 0) & 0x3Fu;
+            }
+            e4[u] = kt[idx];
+          }
+          *reinterpret_cast<uint4 *>(kdst + c16 * 128) = make_uint4(e4[0], e4[1], e4[2], e4[3]);
+        }
+      }
+      // values: coordinates 64 half .. 64 half + 63 of token n as fp16, MN-major
+      {
+        uint32_t w[VB * 2];
+        const uint32_t *vp = reinterpret_cast<const uint32_t *>(a.vc + rec * VR + VB * 8 * half);
+#pragma unroll
+        for (int k = 0; k < VB * 2; ++k) w[k] = __ldg(vp + k);
+        uint8_t *vdst = sm + L::oV + x * (kKT * 256) + (n >> 3) * 128 + (n & 7) * 16 + half * 8 * 1024;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) { // 8 coordinates
+          uint32_t e4[4];
+          if constexpr (VB == 2) {
+            const uint32_t byte0 = (w[c8 >> 1] >> (16 * (c8 & 1))) & 0xFFu;
+            const uint32_t byte1 = (w[c8 >> 1] >> (16 * (c8 & 1) + 8)) & 0xFFu;
+            const uint2 q0 = *reinterpret_cast<const uint2 *>(vt + 8 * byte0);
+            const uint2 q1 = *reinterpret_cast<const uint2 *>(vt + 8 * byte1);
+            e4[0] = q0.x;
+            e4[1] = q0.y;
+            e4[2] = q1.x;
+            e4[3] = q1.y;
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int pp = 4 * c8 + u; // coordinate pair within this half
+              const uint32_t idx = bits_at(w, 2 * VB * pp, 0) & ((1u << (2 * VB)) - 1u);
+              e4[u] = reinterpret_cast<const uint32_t *>(vt)[idx];
+            }
+          }
+          *reinterpret_cast<uint4 *>(vdst + c8 * 1024) = make_uint4(e4[0], e4[1], e4[2], e4[3]);
+        }
+      }
+      if (half == 0) knb[x * kKT + n] = f16_bits_to_f32(__ldg(a.kn + rec));
+      else vnb[x * kKT + n] = f16_bits_to_f32(__ldg(a.vn + rec));
+      tc::fence_async_smem();
+      tc::mbar_arrive(KV_full(x));
+    }
+  } else {
+    // =============================== MMA warp: one thread issues every MMA
+    if (lane == 0) {
+      const uint32_t id_s = tc::idesc_i8(kRows, kKT);
+      const uint32_t id_o = tc::idesc_f16_bmn(kRows, 128);
+      pf_wait(Q_ready, 0, dead);
+      auto pv = [&](int jj) {
+        const int x = jj & 1;
+        pf_wait(P_full(x), (jj >> 1) & 1, dead);
+        tc::fence_after_sync();
+#pragma unroll
+        for (int s = 0; s < kKT / 16; ++s)
+          tc::mma_ts_f16(tbase + kOCol, tbase + x * kSCols + 8 * s,
+                         tc::desc_kmajor(sb + L::oV + x * (kKT * 256) + 256 * s, 128, 1024), id_o,
+                         (jj > 0 || s > 0) ? 1u : 0u);
+        tc::commit(S_free(x));
+        tc::commit(KV_free(x));
+        tc::commit(PV_done);
+      };
+#pragma unroll 1
+      for (int j = 0; j < ntiles; ++j) {
+        const int x = j & 1;
+        pf_wait(KV_full(x), (j >> 1) & 1, dead);
+        if (j >= 2) pf_wait(S_free(x), ((j >> 1) - 1) & 1, dead);
+        tc::fence_after_sync();
+#pragma unroll
+        for (int type = 0; type < 3; ++type)
+#pragma unroll
+          for (int s = 0; s < 8; ++s)
+            tc::mma_ss_i8(tbase + x * kSCols + kKT * type,
+                          tc::desc_kmajor8(sb + L::oQ + type * (kRows * 256) + 256 * s, 128, 2048),
+                          tc::desc_kmajor8(sb + L::oK + x * (kKT * 256) + 256 * s, 128, 2048), id_s,
+                          s > 0 ? 1u : 0u);
+        tc::commit(S_full(x));
+        if (j > 0) pv(j - 1);
+      }
+      pv(ntiles - 1);
+      tc::commit(fin_bar);
+      pf_wait(fin_bar, 0, dead);
+    }
+    __syncwarp();
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == kWarpMMAp) tc::tmem_dealloc(tbase, kTmemColsP);
+}
+
+template <int KB, int VB>
+cudaError_t run_prefill(const PrefillArgs &p, int ctas, cudaStream_t s) {
+  constexpr int smem = PfLayout<KB, VB>::kSmem;
+  auto kern = prefill_kernel<KB, VB>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(ctas), dim3(kThreadsP), smem, s, p);
+}
+
+} // namespace
+
+bool prefill_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G) {
+  return d == 128 && k_mode == TQ_MSE && (k_wbits == 3 || k_wbits == 4) && v_mode == TQ_MSE && v_wbits >= 2 &&
+         v_wbits <= 4 && G >= 1 && G <= kRows && kRows % G == 0;
+}
+
+cudaError_t launch_prefill(const PrefillLaunch &l, cudaStream_t s) {
+  PrefillArgs p;
+  p.kc = l.k.codes;
+  p.vc = l.v.codes;
+  p.kn = l.k.norm;
+  p.vn = l.v.norm;
+  p.q = l.q;
+  p.q_dtype = l.q_dtype;
+  p.out = l.out;
+  p.scale = l.scale;
+  p.seed = l.seed;
+  p.Hq = l.Hq;
+  p.Hkv = l.Hkv;
+  p.G = l.Hq / l.Hkv;
+  p.Lq = l.Lq;
+  p.t0 = l.t0;
+  p.T_cap = l.T_cap;
+  p.P = kRows / p.G;
+  p.blocks = (l.Lq + p.P - 1) / p.P;
+  for (int j = 0; j < 16; ++j) p.kcent[j] = l.k.cb.c[j];
+  p.kcsc = l.k.cb.fix_scale;
+  for (int j = 0; j < 16; ++j) p.vcent[j] = l.v.cb.c[j];
+  const int ctas = l.B * l.Hkv * p.blocks;
+  const int kb = l.k.wbits, vb = l.v.wbits;
+  if (kb == 4) return vb == 2 ? run_prefill<4, 2>(p, ctas, s) : vb == 3 ? run_prefill<4, 3>(p, ctas, s)
+                                                                      : run_prefill<4, 4>(p, ctas, s);
+  return vb == 2 ? run_prefill<3, 2>(p, ctas, s) : vb == 3 ? run_prefill<3, 3>(p, ctas, s)
+                                                           : run_prefill<3, 4>(p, ctas, s);
+}
+
+cudaError_t read_and_clear_prefill_faults(unsigned *flags) {
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_prefill_fault, sizeof v);
+  if (e != cudaSuccess) return e;
+  *flags = v;
+  if (v) {
+    const unsigned z = 0;
+    e = cudaMemcpyToSymbol(g_prefill_fault, &z, sizeof z);
+  }
+  return e;
+}
+
+} // namespace tq

@@ -126,6 +126,61 @@ __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint
                : "r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(z));
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T on int8 operands, both K-major. Issued by one thread.
+__device__ __forceinline__ void mma_ss_i8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n"
+               :
+               : "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(z));
+}
+
+// Instruction descriptor of kind::f16 with fp32 accumulation, fp16 A (K-major, from TMEM) and
+// fp16 B stored MN-major (N contiguous), M x N tile.
+__host__ __device__ constexpr uint32_t idesc_f16_bmn(int M, int N) {
+  return (1u << 4) | (1u << 16) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem] on fp16 operands (A M x 16 in TMEM: lane i = row i, two
+// consecutive k per 32-bit column, 8 columns). Issued by one thread.
+__device__ __forceinline__ void mma_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                           uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}\n"
+               :
+               : "r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(z));
+}
+
+// Warp-wide: thread i writes v[0..31] into 32 consecutive columns of TMEM lane (lane base + i).
+__device__ __forceinline__ void tmem_st32x32_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+               "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+               "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+               :
+               : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                 "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
+                 "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
+                 "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+                 "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+               : "memory");
+}
+
+// Warp-wide: thread i reads 32 consecutive 32-bit columns of TMEM lane (lane base + i).
+__device__ __forceinline__ void tmem_ld32x32_x32u(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+               "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+               "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+                 "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+                 "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+                 "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+                 "=r"(r[31])
+               : "r"(taddr));
+}
+
 // Warp-wide store of 16 TMEM lanes x 64 columns: thread (r = lane / 4, c = lane % 4) supplies,
 // for repetition i = 0..7, v[4i] = (lane r, column 8i + 2c), v[4i+1] = (lane r, column
 // 8i + 2c + 1), v[4i+2] = (lane r + 8, column 8i + 2c), v[4i+3] = (lane r + 8, 8i + 2c + 1).

@@ -146,12 +146,30 @@ void plan_fast(int B, int Hq, int Hkv, int T_len, int sm_count, int kb, int vb, 
                const int *T_lens = nullptr);
 cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s);
 
+// Prefill (chunked) attention over the compressed cache on tcgen05 tensor cores (prefill.cu):
+// head_dim 128, MSE keys of 3 or 4 bits, MSE values of 2..4 bits, G dividing 128. The Lq
+// queries q[B][Lq][Hq][128] at positions t0 .. t0 + Lq - 1 attend causally to the cache.
+struct PrefillLaunch {
+  const void *q;
+  int q_dtype;
+  int B, Hq, Hkv, Lq, t0, T_cap;
+  float scale;
+  uint64_t seed;
+  TensorArgs k, v;
+  float *out;
+};
+bool prefill_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G);
+cudaError_t launch_prefill(const PrefillLaunch &l, cudaStream_t s);
+cudaError_t read_and_clear_prefill_faults(unsigned *flags);
+
 // Tensor-core decode of TurboQuant_prod records (decode_prod.cu): head_dim 64, 2-bit keys and
 // values with 64 QJL rows each, 1..2 query heads per KV head. Plan code kProdFast.
 constexpr int kProdFast = 0x200;
 bool prod_decode_supported(int d, int k_mode, int k_bits, int k_m, int v_mode, int v_bits, int v_m,
                            int G);
-void plan_prod(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p);
+// T_lens: NULL (every sequence T_len long) or B per-sequence lengths (ragged call; T_len is then
+// the longest).
+void plan_prod(int B, int Hq, int Hkv, int T_len, int sm_count, DecodePlan *p, const int *T_lens = nullptr);
 cudaError_t launch_prod_decode(const DecodeArgs &a, cudaStream_t s);
 
 // Tensor-core bf16 decode (decode_bf16.cu): head_dim 128, 1..8 query heads per KV head.

@@ -92,6 +92,9 @@ EXPORTS = {
     "tq_decode_attention_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, ctypes.c_float, ctypes.POINTER(tq_cache),
                                                    ctypes.c_void_p, ctypes.c_void_p]),
+    "tq_prefill_attention": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_float, ctypes.POINTER(tq_cache),
+                                            ctypes.c_void_p, ctypes.c_void_p]),
     "tq_dequantize": (ctypes.c_int, [ctypes.POINTER(tq_cache), ctypes.c_int, ctypes.c_int,
                                      ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "tq_decode_bf16_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -385,6 +388,19 @@ def tq_decode_attention_noalloc(q: torch.Tensor, cache: TQCache, T_len: int, sca
         raise TQError(TQ_ERR_INVALID_ARG, f"unsupported dtype {q.dtype}")
     _check(lib.tq_decode_attention_noalloc(_dev(q, "q"), dt, q.shape[1], T_len, scale,
                                            ctypes.byref(cache.struct), _dev(out, "out"), _stream(stream)))
+
+
+def tq_prefill_attention(q: torch.Tensor, cache: TQCache, t0: int, scale: float, out: torch.Tensor,
+                         stream=None) -> None:
+    """Chunked prefill attention: q [B, Lq, Hq, d] at positions t0 .. t0 + Lq - 1 attends causally
+    to the compressed cache (the chunk's own K, V already written); out [B, Lq, Hq, d] float32."""
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise TQError(TQ_ERR_INVALID_ARG, f"unsupported dtype {q.dtype}")
+    if q.dim() != 4:
+        raise TQError(TQ_ERR_INVALID_ARG, "q must be [B, Lq, Hq, d]")
+    _check(lib.tq_prefill_attention(_dev(q, "q"), dt, q.shape[2], q.shape[1], t0, scale,
+                                    ctypes.byref(cache.struct), _dev(out, "out"), _stream(stream)))
 
 
 def tq_dequantize(cache: TQCache, which: int, T_len: int, out: torch.Tensor, stream=None) -> None:

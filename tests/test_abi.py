@@ -212,8 +212,8 @@ def test_varlen_decode_validates_before_any_device_work():
     assert tq.lib.tq_decode_attention_varlen(out, 1, 8, None, 0.1, ctypes.byref(c), out, out, 1 << 20,
                                              None) == tq.TQ_ERR_INVALID_ARG
     assert tq.lib.tq_decode_varlen_workspace_bytes(8, ctypes.byref(c), None) == 0
-    # TurboQuant_prod records and head_dim 64 have no ragged kernel
-    p = _fake_cache(3, 2, 64, 64, 2, O.PROD, 2, O.PROD, 64)
+    # TurboQuant_prod records with 32 sketch rows have no ragged (tensor-core) kernel
+    p = _fake_cache(3, 2, 64, 64, 2, O.PROD, 2, O.PROD, 32)
     lens[1] = 7
     assert tq.lib.tq_decode_attention_varlen(out, 1, 4, ctypes.cast(lens, ctypes.c_void_p), 0.1,
                                              ctypes.byref(p), out, out, 1 << 20, None) == tq.TQ_ERR_UNSUPPORTED

@@ -22,6 +22,10 @@ CASES = [
     (128, 4, 2, (4, O.MSE), (2, O.MSE), [1, 700, 16, 33, 1024, 257], 1024),  # 12-warp CTAs
     (128, 8, 1, (4, O.MSE), (2, O.MSE), [500, 3, 64, 1000], 1000),           # 8 query heads
     (128, 2, 3, (3, O.MSE), (3, O.MSE), [129, 2, 600], 640),                  # 4-warp CTAs
+    # TurboQuant_prod, d = 64, 64 sketch rows: one query head per KV head (byte-table scores)
+    # and two (tensor-core scores)
+    (64, 1, 3, (2, O.PROD), (2, O.PROD), [1, 520, 17, 64, 300], 520),
+    (64, 2, 2, (2, O.PROD), (2, O.PROD), [333, 5, 129, 2, 400, 48], 400),
 ]
 
 
@@ -86,7 +90,20 @@ def test_varlen_with_equal_lengths_equals_the_uniform_call():
 
 
 def test_varlen_rejects_unsupported_configurations():
-    cache = tq.TQCache(2, 2, 64, 64, 2, 2, O.PROD, O.PROD, 64, 64)
+    cache = tq.TQCache(2, 2, 64, 64, 2, 2, O.PROD, O.PROD, 32, 32)  # 32 sketch rows
     with pytest.raises(tq.TQError) as e:
         tq.tq_decode_varlen_workspace_bytes(cache, 2, [10, 20])
-    assert "tensor-core MSE" in str(e.value)
+    assert "tensor-core configuration" in str(e.value)
+
+
+def test_varlen_prod_with_equal_lengths_equals_the_uniform_call():
+    T_lens = [300] * 3
+    B, Hq, q, cache, _, _ = _setup(64, 2, 2, (2, O.PROD), (2, O.PROD), T_lens, 320, seed=7)
+    out_v = torch.empty(B, Hq, 64, device="cuda")
+    out_u = torch.empty(B, Hq, 64, device="cuda")
+    ws_v = tq.workspace(tq.tq_decode_varlen_workspace_bytes(cache, Hq, T_lens))
+    ws_u = tq.workspace(tq.tq_decode_workspace_bytes(cache, Hq, 300))
+    tq.tq_decode_attention_varlen(q.cuda(), cache, T_lens, 0.125, out_v, ws_v)
+    tq.tq_decode_attention(q.cuda(), cache, 300, 0.125, out_u, ws_u)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out_v, out_u, rtol=1e-5, atol=1e-6)
