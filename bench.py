@@ -98,11 +98,14 @@ def _code_only(src: str) -> str:
     return "".join(out)
 
 
+DECODE_SOURCES = ("decode_mma.cu", "decode_mse_common.cuh", "mma_ops.cuh", "tq_device.cuh")
+
+
 def decode_sources_digest() -> str:
     """sha256 over the code (comments and whitespace removed) of the bench's dominant kernel's
     sources (the tensor-core decode)."""
     h = hashlib.sha256()
-    for name in ("decode_mma.cu", "mma_ops.cuh"):
+    for name in DECODE_SOURCES:
         with open(os.path.join(ROOT, "quantized_decode_attention_kv_b200", "csrc", name)) as f:
             h.update(_code_only(f.read()).encode())
     return h.hexdigest()

@@ -15,19 +15,23 @@
 //     pair and the three query operands the 24-bit fixed-point query parts, exactly the score
 //     arithmetic of the decode kernels (c.q = 2^24 S_0 + 2^16 S_1 + 2^8 S_2 up to c_lo q_lo);
 //   O += P' . V (kind::f16, M = 128, N = 128 coordinates, K = 64 tokens): P' = p ||v|| in fp16
-//     written by the softmax threads into tensor memory (the A operand), V the fp16 centroids
-//     in shared memory (MN-major: each token's coordinates contiguous).
+//     written by the softmax threads into shared memory (the A operand, K-major), V the fp16
+//     centroids in shared memory (MN-major: each token's coordinates contiguous).
 // A CTA takes 128 query rows (128 / G positions x G query heads) of one (batch, KV head):
 //   softmax warps (4): thread = query row = TMEM lane; it prepares its queries (rotation,
 //     fixed point), and per KV tile reads its row's scores, keeps the row's running maximum and
 //     sum (no cross-thread reduction), rescales its output row in TMEM when the maximum moves,
 //     and at the end applies the inverse rotation to its row;
 //   producer warps (4): dequantise each 64-token tile of codes into the two operands (two
-//     buffers), with the tile's key and value norms;
+//     buffers each), with the tile's key and value norms, loading the next tile's codes while
+//     expanding the current one;
 //   MMA warp (1 thread): S MMAs of tile j, then P.V of tile j - 1, with tcgen05.commit
-//     releasing the buffers.
-// TMEM: two score stages of 3 x 64 int32 columns (the tile's P' overwrites the first 32 columns
-// of its stage once read) and the 128 fp32 output columns. Every mbarrier wait is bounded.
+//     signalling completion.
+// Every buffer is released by its last reader: a score stage and the tile's norms by the
+// softmax warps once read (so the score MMAs of tile j + 2 overlap the softmax of tile j + 1),
+// the key operand with them, the value operand and P' by the completion of P.V. TMEM: two
+// score stages of 3 x 64 int32 columns, refilled with the read-back constant by the softmax
+// threads, and the 128 fp32 output columns. Every mbarrier wait is bounded.
 #include "decode_mse_common.cuh"
 #include "tc_ops.cuh"
 
@@ -68,22 +72,24 @@ struct PrefillArgs {
 
 template <int KB, int VB>
 struct PfLayout {
-  static constexpr int oQ = 0;                       // 3 x [128 rows][256 bytes] int8, K-major
-  static constexpr int oK = oQ + 3 * kRows * 256;    // 2 x [64 tokens][256 bytes] int8, K-major
-  static constexpr int oV = oK + 2 * kKT * 256;      // 2 x [128 coords][64 tokens] fp16, MN-major
-  static constexpr int oKN = oV + 2 * kKT * 256;     // 2 x 64 key norms (float)
-  static constexpr int oVN = oKN + 2 * kKT * 4;      // 2 x 64 value norms (float)
-  static constexpr int oKT = oVN + 2 * kKT * 4;      // key entries {hi, hi, lo, lo} per code pair
+  static constexpr int oQ = 0;                           // 3 x [128 rows][256 bytes] int8, K-major
+  static constexpr int oK = oQ + 3 * kRows * 256;        // 2 x [64 tokens][256 bytes] int8, K-major
+  static constexpr int oV = oK + 2 * kKT * 256;          // 2 x [128 coords][64 tokens] fp16, MN-major
+  static constexpr int oP = oV + 2 * kKT * 256;          // 2 x [128 rows][64 tokens] fp16 P', K-major
+  static constexpr int oKN = oP + 2 * kRows * kKT * 2;   // 2 x 64 key norms (float)
+  static constexpr int oVN = oKN + 2 * kKT * 4;          // 2 x 64 value norms (float)
+  static constexpr int oKT = oVN + 2 * kKT * 4;          // key entries {hi, hi, lo, lo} per code pair
   static constexpr int kKRows = KB == 4 ? 256 : 64;
-  static constexpr int oVT = oKT + kKRows * 4;       // value table
+  static constexpr int oVT = oKT + kKRows * 4;           // value table
   static constexpr int kVRows = VB == 2 ? 256 : 1 << (2 * VB);
-  static constexpr int kVEntry = VB == 2 ? 8 : 4;    // 2-bit: 4 fp16 per code byte; else fp16x2 per pair
-  static constexpr int oQP = oVT + kVRows * kVEntry; // per softmax warp: one prepared query
+  static constexpr int kVEntry = VB == 2 ? 8 : 4;        // 2-bit: 4 fp16 per code byte; else fp16x2 per pair
+  static constexpr int oQP = oVT + kVRows * kVEntry;     // per softmax warp: one prepared query
   static constexpr int oInv = oQP + kSWp * static_cast<int>(sizeof(QPrep));
   static constexpr int oBar = (oInv + kRows * 4 + 7) & ~7;
-  static constexpr int nBar = 11;                    // KV_full[2] KV_free[2] S_full[2] S_free[2] P_full[2] PV_done Q_ready fin
-  static constexpr int oMisc = oBar + (nBar + 2) * 8;
-  static constexpr int kSmem = oMisc + 16 + 1024;    // + alignment of the base
+  // K_full[2] V_full[2] V_free[2] S_full[2] S_free[2] P_full[2] PV_done Q_ready fin
+  static constexpr int nBar = 15;
+  static constexpr int oMisc = oBar + nBar * 8;
+  static constexpr int kSmem = oMisc + 16 + 1024;        // + alignment of the base
 };
 
 __device__ __forceinline__ bool pf_try(uint32_t mbar, uint32_t parity) {
@@ -114,6 +120,19 @@ __device__ __forceinline__ void pf_wait(uint32_t mbar, uint32_t parity, volatile
   if (!pf_try(mbar, parity)) pf_wait_slow(mbar, parity, dead);
 }
 
+// The MMA thread's last wait: for the completion of every MMA it issued (which depends on no
+// other warp), whether or not the CTA has given up, so that TMEM is never released under a
+// running MMA; bounded all the same.
+__device__ __noinline__ void pf_wait_own_mmas(uint32_t mbar) {
+  const long long t0 = clock64();
+  while (!pf_try(mbar, 0)) {
+    if (clock64() - t0 > kWaitCyclesP) {
+      atomicOr(&g_prefill_fault, 1u);
+      return;
+    }
+  }
+}
+
 template <int KB, int VB>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs a) {
   using L = PfLayout<KB, VB>;
@@ -123,12 +142,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
   const uint32_t sb = (raw + 1023) & ~1023u;
   uint8_t *const sm = smem_raw + (sb - raw);
   const uint32_t bar0 = sb + L::oBar;
-  auto KV_full = [&](int x) { return bar0 + 8u * x; };
-  auto KV_free = [&](int x) { return bar0 + 8u * (2 + x); };
-  auto S_full = [&](int x) { return bar0 + 8u * (4 + x); };
-  auto S_free = [&](int x) { return bar0 + 8u * (6 + x); };
-  auto P_full = [&](int x) { return bar0 + 8u * (8 + x); };
-  const uint32_t PV_done = bar0 + 8u * 10, Q_ready = bar0 + 8u * 11, fin_bar = bar0 + 8u * 12;
+  auto K_full = [&](int x) { return bar0 + 8u * x; };
+  auto V_full = [&](int x) { return bar0 + 8u * (2 + x); };
+  auto V_free = [&](int x) { return bar0 + 8u * (4 + x); };
+  auto S_full = [&](int x) { return bar0 + 8u * (6 + x); };
+  auto S_free = [&](int x) { return bar0 + 8u * (8 + x); };
+  auto P_full = [&](int x) { return bar0 + 8u * (10 + x); };
+  const uint32_t PV_done = bar0 + 8u * 12, Q_ready = bar0 + 8u * 13, fin_bar = bar0 + 8u * 14;
   uint32_t *const misc = reinterpret_cast<uint32_t *>(sm + L::oMisc);
   volatile int *const dead = reinterpret_cast<volatile int *>(misc + 1);
   float *const knb = reinterpret_cast<float *>(sm + L::oKN);
@@ -168,10 +188,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
   }
   if (tid == 0) {
     for (int x = 0; x < 2; ++x) {
-      tc::mbar_init(KV_full(x), 32 * kPWp);
-      tc::mbar_init(KV_free(x), 1);
+      tc::mbar_init(K_full(x), 32 * kPWp);
+      tc::mbar_init(V_full(x), 32 * kPWp);
+      tc::mbar_init(V_free(x), 1);
       tc::mbar_init(S_full(x), 1);
-      tc::mbar_init(S_free(x), 1);
+      tc::mbar_init(S_free(x), kSWp);
       tc::mbar_init(P_full(x), 32 * kSWp);
     }
     tc::mbar_init(PV_done, 1);
@@ -194,6 +215,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
     const int ri = row / a.G, rg = row - ri * a.G; // query position within the block, head
     const bool row_ok = ri < a.P && i0 + ri < a.Lq;
     const int my_pos = a.t0 + i0 + ri;
+    const int pos_lo = a.t0 + i0 + (32 * warp) / a.G; // the smallest position among the warp's rows
+    const uint32_t lrow = static_cast<uint32_t>(32 * warp) << 16;
     // ---- queries of the warp's 32 rows: rotation and 24-bit fixed point (one warp per query),
     //      written as the three int8 operands {q_hi, q_hi, 0, 0}, {q_mid, q_mid, q_hi, q_hi},
     //      {q_lo, q_lo, q_mid, q_mid} at the {hi, hi, lo, lo} slots of each coordinate pair
@@ -226,19 +249,29 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       if (lane == 0) rinv[rr] = qs->inv * kLog2e;
       __syncwarp();
     }
+    // both score stages start at the magic constant: every score MMA accumulates onto it, so
+    // an int32 sum s reads back as the float 1.5 * 2^23 + s
+#pragma unroll 1
+    for (int c = 0; c < 2 * static_cast<int>(kSCols) / 32; ++c)
+      tc::tmem_fill32x32_x32(tbase + lrow + 32 * c, static_cast<uint32_t>(kMagic));
+    tc::tmem_wait_st();
+    tc::fence_before_sync();
     tc::fence_async_smem();
     tc::mbar_arrive(Q_ready);
     __syncwarp();
     const float qsc = rinv[row];
-    const uint32_t lrow = static_cast<uint32_t>(32 * warp) << 16;
 
+    // running maximum in units of ||k|| * (c . q~) (the exponent is qsc times it), running sum
     float m_run = -INFINITY, l_run = 0.f;
 #pragma unroll 1
     for (int j = 0; j < ntiles; ++j) {
       const int x = j & 1;
       pf_wait(S_full(x), (j >> 1) & 1, dead);
       tc::fence_after_sync();
+      // warp-uniform: some row of the warp sees only part of this tile (the causal diagonal)
+      const bool edge = kKT * j + kKT - 1 > pos_lo;
       const uint32_t st = tbase + lrow + x * kSCols;
+      const float4 *kn4 = reinterpret_cast<const float4 *>(knb + x * kKT);
       float s[kKT];
 #pragma unroll
       for (int cch = 0; cch < kKT / 16; ++cch) {
@@ -248,13 +281,26 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
         tc::tmem_ld32x32_x16(st + 2 * kKT + 16 * cch, r2);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int tt = 16 * cch + t;
-          const float d = fmaf(__int_as_float(static_cast<int>(r2[t]) + kMagic), 1.0f / 65536.0f,
-                               fmaf(__int_as_float(static_cast<int>(r1[t]) + kMagic), 1.0f / 256.0f,
-                                    __int_as_float(static_cast<int>(r0[t]) + kMagic) - kMagicAdj));
-          s[tt] = kKT * j + tt <= my_pos ? knb[x * kKT + tt] * qsc * d : -INFINITY;
+        for (int t4 = 0; t4 < 4; ++t4) {
+          const float4 k4 = kn4[4 * cch + t4];
+          const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = 4 * t4 + e;
+            const float d = fmaf(__uint_as_float(r2[t]), 1.0f / 65536.0f,
+                                 fmaf(__uint_as_float(r1[t]), 1.0f / 256.0f, __uint_as_float(r0[t]) - kMagicAdj));
+            s[16 * cch + t] = kk[e] * d;
+          }
         }
+      }
+      // the stage back to the magic constant for tile j + 2 (waited for before it is released)
+#pragma unroll
+      for (int c = 0; c < static_cast<int>(kSCols) / 32; ++c)
+        tc::tmem_fill32x32_x32(st + 32 * c, static_cast<uint32_t>(kMagic));
+      if (edge) {
+#pragma unroll
+        for (int t = 0; t < kKT; ++t)
+          if (kKT * j + t > my_pos) s[t] = -INFINITY;
       }
       float mx = s[0];
 #pragma unroll
@@ -262,15 +308,48 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       const float mn = fmaxf(m_run, mx);
       // a row whose maximum moved scales its sum and the output row accumulated so far (once the
       // previous tile's P.V has landed; before the first P.V the output is undefined and is
-      // overwritten). The TMEM loads and stores are warp-collective (.sync.aligned), so the
-      // whole warp takes this path when any of its rows needs it, the others with factor 1.
+      // overwritten)
       const bool moved = mn != m_run;
-      const float alpha = moved ? softmax_exp2(m_run - mn) : 1.f;
+      const float alpha = (moved && j > 0) ? softmax_exp2(qsc * (m_run - mn)) : 1.f;
       l_run *= alpha;
       m_run = mn;
+      const float mq = qsc * mn;
+      // weights p ||v|| as fp16 (P', the A operand of P.V)
+      const float4 *vn4 = reinterpret_cast<const float4 *>(vnb + x * kKT);
+      uint32_t pw[kKT / 2];
+#pragma unroll
+      for (int t4 = 0; t4 < kKT / 4; ++t4) {
+        const float4 v4 = vn4[t4];
+        float p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[e] = softmax_exp2(fmaf(s[4 * t4 + e], qsc, -mq));
+        if (edge) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (kKT * j + 4 * t4 + e > my_pos) p[e] = 0.f;
+        }
+        l_run += (p[0] + p[1]) + (p[2] + p[3]);
+        pw[2 * t4] = pack_h2(p[0] * v4.x, p[1] * v4.y);
+        pw[2 * t4 + 1] = pack_h2(p[2] * v4.z, p[3] * v4.w);
+      }
+      // the score stage and the tile's norms are no longer needed: release them to the next
+      // score MMAs and the producers
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(S_free(x));
+      // P' buffer x was last read by P.V of tile j - 2, complete once S_full(j) arrived (the MMA
+      // thread commits S_full(j) after issuing it)
+      uint8_t *pdst = sm + L::oP + x * (kRows * kKT * 2) + (row & 7) * 16 + (row >> 3) * 1024;
+#pragma unroll
+      for (int c = 0; c < kKT / 8; ++c)
+        *reinterpret_cast<uint4 *>(pdst + c * 128) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+      tc::fence_async_smem();
+      // the TMEM loads and stores are warp-collective (.sync.aligned), so the whole warp takes
+      // this path when any of its rows needs it, the others with factor 1
       if (j > 0 && __any_sync(0xffffffffu, moved)) {
-        // completion j - 1 of PV_done: S_full(j) implies P.V of tile j - 2 had completed, so
-        // the barrier is at completion j - 1 or j and the parity identifies it
+        // completion j - 1 of PV_done: S_full(j) implies P.V of tile j - 2 had completed, and
+        // P.V of tile j waits for this tile's P', so the parity identifies it
         pf_wait(PV_done, (j - 1) & 1, dead);
         tc::fence_after_sync();
 #pragma unroll 1
@@ -282,18 +361,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
           tc::tmem_st32x32_x32(tbase + lrow + kOCol + 32 * cch, ov);
         }
+        tc::tmem_wait_st();
       }
-      // weights p ||v|| as fp16 into the first 32 columns of the stage (already read)
-      uint32_t pw[kKT / 2];
-#pragma unroll
-      for (int t = 0; t < kKT; t += 2) {
-        const float p0 = s[t] == -INFINITY ? 0.f : softmax_exp2(s[t] - m_run);
-        const float p1 = s[t + 1] == -INFINITY ? 0.f : softmax_exp2(s[t + 1] - m_run);
-        l_run += p0 + p1;
-        pw[t >> 1] = pack_h2(p0 * vnb[x * kKT + t], p1 * vnb[x * kKT + t + 1]);
-      }
-      tc::tmem_st32x32_x32(st, pw);
-      tc::tmem_wait_st();
       tc::fence_before_sync();
       tc::mbar_arrive(P_full(x));
     }
@@ -339,23 +408,33 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       }
     }
   } else if (warp < kWarpMMAp) {
-    // =============================== producer warps: 64-token tiles of K and V operands
-    const int pt = tid - 32 * kSWp;   // 0..127
+    // =============================== producer warps: 64-token tiles of K and V operands; the
+    //      codes of the next tile are loaded while the current one is expanded
+    const int pt = tid - 32 * kSWp; // 0..127
     const int n = pt >> 1, half = pt & 1;
     const uint32_t *kt = reinterpret_cast<const uint32_t *>(sm + L::oKT);
     const uint8_t *vt = sm + L::oVT;
-#pragma unroll 1
-    for (int j = 0; j < ntiles; ++j) {
-      const int x = j & 1;
-      if (j >= 2) pf_wait(KV_free(x), ((j >> 1) - 1) & 1, dead);
+    struct Codes {
+      uint32_t k[KB * 2], v[VB * 2];
+      uint16_t nrm; // key norm (half 0) or value norm (half 1) of token n
+    };
+    auto load = [&](int j, Codes &c) {
       const int tok = min(kKT * j + n, pos_last);
       const size_t rec = static_cast<size_t>(bh) * a.T_cap + tok;
-      // keys: code pairs 32 half .. 32 half + 31 -> k bytes 128 half .. 128 half + 127 of row n
-      {
-        uint32_t w[KB * 2];
-        const uint32_t *kp = reinterpret_cast<const uint32_t *>(a.kc + rec * KR + KB * 8 * half);
+      const uint32_t *kp = reinterpret_cast<const uint32_t *>(a.kc + rec * KR + KB * 8 * half);
 #pragma unroll
-        for (int k = 0; k < KB * 2; ++k) w[k] = __ldg(kp + k);
+      for (int k = 0; k < KB * 2; ++k) c.k[k] = __ldg(kp + k);
+      const uint32_t *vp = reinterpret_cast<const uint32_t *>(a.vc + rec * VR + VB * 8 * half);
+#pragma unroll
+      for (int k = 0; k < VB * 2; ++k) c.v[k] = __ldg(vp + k);
+      c.nrm = __ldg((half == 0 ? a.kn : a.vn) + rec);
+    };
+    auto produce = [&](int j, const Codes &c) {
+      const int x = j & 1;
+      // keys: code pairs 32 half .. 32 half + 31 -> k bytes 128 half .. 128 half + 127 of row n.
+      // Buffer x and the norms of tile j - 2 are free once its softmax released the stage.
+      if (j >= 2) pf_wait(S_free(x), ((j >> 1) - 1) & 1, dead);
+      {
         uint8_t *kdst = sm + L::oK + x * (kKT * 256) + (n & 7) * 16 + (n >> 3) * 2048 + half * 8 * 128;
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) { // 16 k bytes = 4 code pairs
@@ -365,28 +444,30 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
             const int pp = 4 * c16 + u; // pair within this half
             uint32_t idx;
             if constexpr (KB == 4) {
-              idx = (w[pp >> 2] >> (8 * (pp & 3))) & 0xFFu;
+              idx = (c.k[pp >> 2] >> (8 * (pp & 3))) & 0xFFu;
             } else {
-              idx = bits_at(w, 6 * pp, 0) & 0x3Fu;
+              idx = bits_at(c.k, 6 * pp, 0) & 0x3Fu;
             }
             e4[u] = kt[idx];
           }
           *reinterpret_cast<uint4 *>(kdst + c16 * 128) = make_uint4(e4[0], e4[1], e4[2], e4[3]);
         }
       }
-      // values: coordinates 64 half .. 64 half + 63 of token n as fp16, MN-major
+      if (half == 0) knb[x * kKT + n] = f16_bits_to_f32(c.nrm);
+      else vnb[x * kKT + n] = f16_bits_to_f32(c.nrm);
+      tc::fence_async_smem();
+      tc::mbar_arrive(K_full(x));
+      // values: coordinates 64 half .. 64 half + 63 of token n as fp16, MN-major; buffer x is
+      // free once P.V of tile j - 2 completed
+      if (j >= 2) pf_wait(V_free(x), ((j >> 1) - 1) & 1, dead);
       {
-        uint32_t w[VB * 2];
-        const uint32_t *vp = reinterpret_cast<const uint32_t *>(a.vc + rec * VR + VB * 8 * half);
-#pragma unroll
-        for (int k = 0; k < VB * 2; ++k) w[k] = __ldg(vp + k);
         uint8_t *vdst = sm + L::oV + x * (kKT * 256) + (n >> 3) * 128 + (n & 7) * 16 + half * 8 * 1024;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) { // 8 coordinates
           uint32_t e4[4];
           if constexpr (VB == 2) {
-            const uint32_t byte0 = (w[c8 >> 1] >> (16 * (c8 & 1))) & 0xFFu;
-            const uint32_t byte1 = (w[c8 >> 1] >> (16 * (c8 & 1) + 8)) & 0xFFu;
+            const uint32_t byte0 = (c.v[c8 >> 1] >> (16 * (c8 & 1))) & 0xFFu;
+            const uint32_t byte1 = (c.v[c8 >> 1] >> (16 * (c8 & 1) + 8)) & 0xFFu;
             const uint2 q0 = *reinterpret_cast<const uint2 *>(vt + 8 * byte0);
             const uint2 q1 = *reinterpret_cast<const uint2 *>(vt + 8 * byte1);
             e4[0] = q0.x;
@@ -397,17 +478,25 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int pp = 4 * c8 + u; // coordinate pair within this half
-              const uint32_t idx = bits_at(w, 2 * VB * pp, 0) & ((1u << (2 * VB)) - 1u);
+              const uint32_t idx = bits_at(c.v, 2 * VB * pp, 0) & ((1u << (2 * VB)) - 1u);
               e4[u] = reinterpret_cast<const uint32_t *>(vt)[idx];
             }
           }
           *reinterpret_cast<uint4 *>(vdst + c8 * 1024) = make_uint4(e4[0], e4[1], e4[2], e4[3]);
         }
       }
-      if (half == 0) knb[x * kKT + n] = f16_bits_to_f32(__ldg(a.kn + rec));
-      else vnb[x * kKT + n] = f16_bits_to_f32(__ldg(a.vn + rec));
       tc::fence_async_smem();
-      tc::mbar_arrive(KV_full(x));
+      tc::mbar_arrive(V_full(x));
+    };
+    Codes c0, c1;
+    load(0, c0);
+#pragma unroll 1
+    for (int j = 0; j < ntiles; j += 2) {
+      if (j + 1 < ntiles) load(j + 1, c1);
+      produce(j, c0);
+      if (j + 1 >= ntiles) break;
+      if (j + 2 < ntiles) load(j + 2, c0);
+      produce(j + 1, c1);
     }
   } else {
     // =============================== MMA warp: one thread issues every MMA
@@ -415,24 +504,27 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       const uint32_t id_s = tc::idesc_i8(kRows, kKT);
       const uint32_t id_o = tc::idesc_f16_bmn(kRows, 128);
       pf_wait(Q_ready, 0, dead);
+      // after a timeout (dead) no further MMA is issued
       auto pv = [&](int jj) {
         const int x = jj & 1;
         pf_wait(P_full(x), (jj >> 1) & 1, dead);
+        pf_wait(V_full(x), (jj >> 1) & 1, dead);
+        if (*dead) return;
         tc::fence_after_sync();
 #pragma unroll
         for (int s = 0; s < kKT / 16; ++s)
-          tc::mma_ts_f16(tbase + kOCol, tbase + x * kSCols + 8 * s,
-                         tc::desc_kmajor(sb + L::oV + x * (kKT * 256) + 256 * s, 128, 1024), id_o,
-                         (jj > 0 || s > 0) ? 1u : 0u);
-        tc::commit(S_free(x));
-        tc::commit(KV_free(x));
+          tc::mma_ss(tbase + kOCol, tc::desc_kmajor(sb + L::oP + x * (kRows * kKT * 2) + 256 * s, 128, 1024),
+                     tc::desc_kmajor(sb + L::oV + x * (kKT * 256) + 256 * s, 128, 1024), id_o,
+                     (jj > 0 || s > 0) ? 1u : 0u);
+        tc::commit(V_free(x));
         tc::commit(PV_done);
       };
 #pragma unroll 1
       for (int j = 0; j < ntiles; ++j) {
         const int x = j & 1;
-        pf_wait(KV_full(x), (j >> 1) & 1, dead);
+        pf_wait(K_full(x), (j >> 1) & 1, dead);
         if (j >= 2) pf_wait(S_free(x), ((j >> 1) - 1) & 1, dead);
+        if (*dead) break;
         tc::fence_after_sync();
 #pragma unroll
         for (int type = 0; type < 3; ++type)
@@ -440,14 +532,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
           for (int s = 0; s < 8; ++s)
             tc::mma_ss_i8(tbase + x * kSCols + kKT * type,
                           tc::desc_kmajor8(sb + L::oQ + type * (kRows * 256) + 256 * s, 128, 2048),
-                          tc::desc_kmajor8(sb + L::oK + x * (kKT * 256) + 256 * s, 128, 2048), id_s,
-                          s > 0 ? 1u : 0u);
+                          tc::desc_kmajor8(sb + L::oK + x * (kKT * 256) + 256 * s, 128, 2048), id_s, 1u);
         tc::commit(S_full(x));
         if (j > 0) pv(j - 1);
       }
       pv(ntiles - 1);
       tc::commit(fin_bar);
-      pf_wait(fin_bar, 0, dead);
+      pf_wait_own_mmas(fin_bar);
     }
     __syncwarp();
   }

@@ -204,6 +204,14 @@ __device__ __forceinline__ void tmem_fill32x32_x16(uint32_t taddr, uint32_t x) {
                : "memory");
 }
 
+// Warp-wide: 32 consecutive 32-bit columns of TMEM lane (lane base + i) set to x.
+__device__ __forceinline__ void tmem_fill32x32_x32(uint32_t taddr, uint32_t x) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+               "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+               "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(x)
+               : "memory");
+}
+
 // Warp-wide: thread i reads 16 consecutive 32-bit columns of TMEM lane (lane base + i).
 __device__ __forceinline__ void tmem_ld32x32_x16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
