@@ -283,13 +283,18 @@ def run_ours(args):
         tq.tq_quantize_kv(k_new, v_new, cache, t_offset=w.T - 1, stream=stream)
         tq.tq_decode_attention(q, cache, w.T, w.scale, out, ws, stream=stream)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    barrier()
     clocks = Clocks(local)
     with clocks:
-        torch.cuda.synchronize()
+        # the W warm-up steps run inside the clock-sampling window, continued until the GPU has
+        # been busy for SETTLE_S (the sampler's start-up leaves it idle, and the first steps
+        # after an idle spell run at lower clocks)
+        warm = 0
+        t_warm = time.perf_counter()
+        while warm < args.warmup or time.perf_counter() - t_warm < SETTLE_S:
+            for _ in range(10):
+                step()
+            warm += 10
+            torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -313,7 +318,7 @@ def run_ours(args):
     hbm, hbm_src = peaks()
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "warmup_steps_run": warm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "i8+f16-mma/f32", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
                    "k": f"{w.k_bits}-bit {'MSE' if w.k_mode == 0 else 'PROD'}",
@@ -352,6 +357,7 @@ def run_ours(args):
 
 
 MIN_CALLS, MIN_SECONDS = 200, 0.5
+SETTLE_S = 0.05  # device-busy time of the warm-up before the timed steps
 
 
 def _time(fn, stream, torch, min_calls=MIN_CALLS, min_s=MIN_SECONDS):

@@ -44,7 +44,7 @@ using namespace mse;
 
 constexpr int kRows = 128;                   // query rows per CTA (TMEM lanes)
 constexpr int kKT = 64;                      // KV tokens per tile
-constexpr int kSWp = 4, kPWp = 4;            // softmax warps, producer warps
+constexpr int kSWp = 8, kPWp = 4;            // softmax warps (two per row: half a tile each), producer warps
 constexpr int kWarpMMAp = kSWp + kPWp;       // the MMA warp
 constexpr int kThreadsP = (kSWp + kPWp + 1) * 32;
 constexpr uint32_t kTmemColsP = 512;
@@ -85,7 +85,8 @@ struct PfLayout {
   static constexpr int kVEntry = VB == 2 ? 8 : 4;        // 2-bit: 4 fp16 per code byte; else fp16x2 per pair
   static constexpr int oQP = oVT + kVRows * kVEntry;     // per softmax warp: one prepared query
   static constexpr int oInv = oQP + kSWp * static_cast<int>(sizeof(QPrep));
-  static constexpr int oBar = (oInv + kRows * 4 + 7) & ~7;
+  static constexpr int oXch = oInv + kRows * 4;          // [2 tile parities][2 halves][128 rows] float
+  static constexpr int oBar = (oXch + 4 * kRows * 4 + 7) & ~7;
   // K_full[2] V_full[2] V_free[2] S_full[2] S_free[2] P_full[2] PV_done Q_ready fin
   static constexpr int nBar = 15;
   static constexpr int oMisc = oBar + nBar * 8;
@@ -210,20 +211,29 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
   pdl_trigger();
 
   if (warp < kSWp) {
-    // =============================== softmax warps: thread = query row = TMEM lane
-    const int row = tid;
+    // =============================== softmax warps: two per query row (= TMEM lane), warp
+    //      quarter qw holds lanes 32 qw .. 32 qw + 31 and half hf the tokens 32 hf .. 32 hf + 31
+    //      of every tile and output coordinates 64 hf .. 64 hf + 63 at the end
+    const int qw = warp & 3, hf = warp >> 2;
+    const int row = 32 * qw + lane;
     const int ri = row / a.G, rg = row - ri * a.G; // query position within the block, head
     const bool row_ok = ri < a.P && i0 + ri < a.Lq;
     const int my_pos = a.t0 + i0 + ri;
-    const int pos_lo = a.t0 + i0 + (32 * warp) / a.G; // the smallest position among the warp's rows
-    const uint32_t lrow = static_cast<uint32_t>(32 * warp) << 16;
-    // ---- queries of the warp's 32 rows: rotation and 24-bit fixed point (one warp per query),
+    const int pos_lo = a.t0 + i0 + (32 * qw) / a.G; // the smallest position among the warp's rows
+    const uint32_t lrow = static_cast<uint32_t>(32 * qw) << 16;
+    float *const xch = reinterpret_cast<float *>(sm + L::oXch);
+    // the two warps of a lane quarter meet at named barrier 1 + qw
+    auto pair_sync = [&]() {
+      __syncwarp();
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + qw) : "memory");
+    };
+    // ---- queries of the warp's 16 rows: rotation and 24-bit fixed point (one warp per query),
     //      written as the three int8 operands {q_hi, q_hi, 0, 0}, {q_mid, q_mid, q_hi, q_hi},
     //      {q_lo, q_lo, q_mid, q_mid} at the {hi, hi, lo, lo} slots of each coordinate pair
     QPrep *qs = reinterpret_cast<QPrep *>(sm + L::oQP) + warp;
 #pragma unroll 1
-    for (int k = 0; k < 32; ++k) {
-      const int rr = 32 * warp + k;
+    for (int k = 0; k < 16; ++k) {
+      const int rr = 32 * qw + 16 * hf + k;
       const int qi = rr / a.G, qg = rr - qi * a.G;
       const bool ok = qi < a.P && i0 + qi < a.Lq;
       if (ok) {
@@ -250,31 +260,36 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       __syncwarp();
     }
     // both score stages start at the magic constant: every score MMA accumulates onto it, so
-    // an int32 sum s reads back as the float 1.5 * 2^23 + s
-#pragma unroll 1
-    for (int c = 0; c < 2 * static_cast<int>(kSCols) / 32; ++c)
-      tc::tmem_fill32x32_x32(tbase + lrow + 32 * c, static_cast<uint32_t>(kMagic));
+    // an int32 sum s reads back as the float 1.5 * 2^23 + s (each warp its own tokens' columns)
+#pragma unroll
+    for (int x = 0; x < 2; ++x)
+#pragma unroll
+      for (int t = 0; t < 3; ++t)
+        tc::tmem_fill32x32_x32(tbase + lrow + x * kSCols + kKT * t + 32 * hf, static_cast<uint32_t>(kMagic));
     tc::tmem_wait_st();
     tc::fence_before_sync();
     tc::fence_async_smem();
     tc::mbar_arrive(Q_ready);
-    __syncwarp();
+    pair_sync(); // the row's scale factor is written by the other warp of the pair for half its rows
     const float qsc = rinv[row];
 
-    // running maximum in units of ||k|| * (c . q~) (the exponent is qsc times it), running sum
+    // running maximum in units of ||k|| * (c . q~) (the exponent is qsc times it), shared by the
+    // pair; running sums per half
+    constexpr int kH = kKT / 2; // tokens per warp and tile
     float m_run = -INFINITY, l_run = 0.f;
 #pragma unroll 1
     for (int j = 0; j < ntiles; ++j) {
       const int x = j & 1;
+      const int tb = kKT * j + kH * hf; // first token of this warp's half tile
       pf_wait(S_full(x), (j >> 1) & 1, dead);
       tc::fence_after_sync();
-      // warp-uniform: some row of the warp sees only part of this tile (the causal diagonal)
-      const bool edge = kKT * j + kKT - 1 > pos_lo;
-      const uint32_t st = tbase + lrow + x * kSCols;
-      const float4 *kn4 = reinterpret_cast<const float4 *>(knb + x * kKT);
-      float s[kKT];
+      // warp-uniform: some row of the warp sees only part of its half tile (the causal diagonal)
+      const bool edge = tb + kH - 1 > pos_lo;
+      const uint32_t st = tbase + lrow + x * kSCols + kH * hf;
+      const float4 *kn4 = reinterpret_cast<const float4 *>(knb + x * kKT + kH * hf);
+      float s[kH];
 #pragma unroll
-      for (int cch = 0; cch < kKT / 16; ++cch) {
+      for (int cch = 0; cch < kH / 16; ++cch) {
         uint32_t r0[16], r1[16], r2[16];
         tc::tmem_ld32x32_x16(st + 16 * cch, r0);
         tc::tmem_ld32x32_x16(st + kKT + 16 * cch, r1);
@@ -293,32 +308,37 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
           }
         }
       }
-      // the stage back to the magic constant for tile j + 2 (waited for before it is released)
+      // the columns back to the magic constant for tile j + 2 (waited for before release)
 #pragma unroll
-      for (int c = 0; c < static_cast<int>(kSCols) / 32; ++c)
-        tc::tmem_fill32x32_x32(st + 32 * c, static_cast<uint32_t>(kMagic));
+      for (int t = 0; t < 3; ++t) tc::tmem_fill32x32_x32(st + kKT * t, static_cast<uint32_t>(kMagic));
       if (edge) {
 #pragma unroll
-        for (int t = 0; t < kKT; ++t)
-          if (kKT * j + t > my_pos) s[t] = -INFINITY;
+        for (int t = 0; t < kH; ++t)
+          if (tb + t > my_pos) s[t] = -INFINITY;
       }
       float mx = s[0];
 #pragma unroll
-      for (int t = 1; t < kKT; ++t) mx = fmaxf(mx, s[t]);
+      for (int t = 1; t < kH; ++t) mx = fmaxf(mx, s[t]);
+      // the row's maximum over the whole tile: the halves' maxima meet in shared memory (one
+      // slot per tile parity, so that the next tile's write cannot meet this tile's read)
+      float *const xs = xch + (j & 1) * 2 * kRows;
+      xs[hf * kRows + row] = mx;
+      pair_sync();
+      mx = fmaxf(mx, xs[(1 - hf) * kRows + row]);
       const float mn = fmaxf(m_run, mx);
-      // a row whose maximum moved scales its sum and the output row accumulated so far (once the
-      // previous tile's P.V has landed; before the first P.V the output is undefined and is
-      // overwritten)
+      // a row whose maximum moved scales its sum and its half of the output row accumulated so
+      // far (once the previous tile's P.V has landed; before the first P.V the output is
+      // undefined and is overwritten)
       const bool moved = mn != m_run;
       const float alpha = (moved && j > 0) ? softmax_exp2(qsc * (m_run - mn)) : 1.f;
       l_run *= alpha;
       m_run = mn;
       const float mq = qsc * mn;
       // weights p ||v|| as fp16 (P', the A operand of P.V)
-      const float4 *vn4 = reinterpret_cast<const float4 *>(vnb + x * kKT);
-      uint32_t pw[kKT / 2];
+      const float4 *vn4 = reinterpret_cast<const float4 *>(vnb + x * kKT + kH * hf);
+      uint32_t pw[kH / 2];
 #pragma unroll
-      for (int t4 = 0; t4 < kKT / 4; ++t4) {
+      for (int t4 = 0; t4 < kH / 4; ++t4) {
         const float4 v4 = vn4[t4];
         float p[4];
 #pragma unroll
@@ -326,23 +346,23 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
         if (edge) {
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (kKT * j + 4 * t4 + e > my_pos) p[e] = 0.f;
+            if (tb + 4 * t4 + e > my_pos) p[e] = 0.f;
         }
         l_run += (p[0] + p[1]) + (p[2] + p[3]);
         pw[2 * t4] = pack_h2(p[0] * v4.x, p[1] * v4.y);
         pw[2 * t4 + 1] = pack_h2(p[2] * v4.z, p[3] * v4.w);
       }
-      // the score stage and the tile's norms are no longer needed: release them to the next
+      // the score columns and the tile's norms are no longer needed: release them to the next
       // score MMAs and the producers
       tc::tmem_wait_st();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(S_free(x));
       // P' buffer x was last read by P.V of tile j - 2, complete once S_full(j) arrived (the MMA
-      // thread commits S_full(j) after issuing it)
-      uint8_t *pdst = sm + L::oP + x * (kRows * kKT * 2) + (row & 7) * 16 + (row >> 3) * 1024;
+      // thread commits S_full(j) after issuing it); this warp's tokens are k chunks 4 hf .. 4 hf + 3
+      uint8_t *pdst = sm + L::oP + x * (kRows * kKT * 2) + (row & 7) * 16 + (row >> 3) * 1024 + hf * 512;
 #pragma unroll
-      for (int c = 0; c < kKT / 8; ++c)
+      for (int c = 0; c < kH / 8; ++c)
         *reinterpret_cast<uint4 *>(pdst + c * 128) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
       tc::fence_async_smem();
       // the TMEM loads and stores are warp-collective (.sync.aligned), so the whole warp takes
@@ -353,13 +373,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
         pf_wait(PV_done, (j - 1) & 1, dead);
         tc::fence_after_sync();
 #pragma unroll 1
-        for (int cch = 0; cch < 4; ++cch) {
+        for (int cch = 0; cch < 2; ++cch) {
           uint32_t ov[32];
-          tc::tmem_ld32x32_x32u(tbase + lrow + kOCol + 32 * cch, ov);
+          const uint32_t oc = tbase + lrow + kOCol + 64 * hf + 32 * cch;
+          tc::tmem_ld32x32_x32u(oc, ov);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tc::tmem_st32x32_x32(tbase + lrow + kOCol + 32 * cch, ov);
+          tc::tmem_st32x32_x32(oc, ov);
         }
         tc::tmem_wait_st();
       }
@@ -367,22 +388,27 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       tc::mbar_arrive(P_full(x));
     }
     // ---- output row: O / l in the rotated domain, then the inverse rotation D H / d (after the
-    //      last P.V: the MMA thread commits every MMA of the CTA to fin_bar)
+    //      last P.V: the MMA thread commits every MMA of the CTA to fin_bar). Each warp of the
+    //      pair transforms its 64 coordinates over the butterfly spans 1 .. 32, the span-64 stage
+    //      pairs coordinate i of one half with i of the other through TMEM.
+    // the half's sum goes to the slot of parity ntiles (its last reads, at tile ntiles - 2, were
+    // done before the partner passed the last tile's pair_sync)
+    xch[(ntiles & 1) * 2 * kRows + hf * kRows + row] = l_run;
     pf_wait(fin_bar, 0, dead);
     tc::fence_after_sync();
-    float o[128];
+    float o[64];
 #pragma unroll
-    for (int cch = 0; cch < 4; ++cch) {
+    for (int cch = 0; cch < 2; ++cch) {
       uint32_t ov[32];
-      tc::tmem_ld32x32_x32u(tbase + lrow + kOCol + 32 * cch, ov);
+      tc::tmem_ld32x32_x32u(tbase + lrow + kOCol + 64 * hf + 32 * cch, ov);
       tc::tmem_wait_ld();
 #pragma unroll
       for (int e = 0; e < 32; ++e) o[32 * cch + e] = __uint_as_float(ov[e]);
     }
 #pragma unroll
-    for (int span = 1; span < 128; span <<= 1) {
+    for (int span = 1; span < 64; span <<= 1) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < 64; ++i) {
         if ((i & span) == 0) {
           const float u = o[i], v = o[i + span];
           o[i] = u + v;
@@ -390,18 +416,44 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
         }
       }
     }
-    if (row_ok) {
-      const float sc = 1.0f / (128.0f * l_run);
-      const uint64_t w0 = dev_splitmix64(a.seed, 0), w1 = dev_splitmix64(a.seed, 1);
-      float *dst = a.out + ((static_cast<size_t>(b) * a.Lq + i0 + ri) * a.Hq + h * a.G + rg) * 128;
+    {
+      uint32_t ov[32];
 #pragma unroll
-      for (int i = 0; i < 128; i += 4) {
+      for (int cch = 0; cch < 2; ++cch) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(o[32 * cch + e]);
+        tc::tmem_st32x32_x32(tbase + lrow + kOCol + 64 * hf + 32 * cch, ov);
+      }
+      tc::tmem_wait_st();
+    }
+    tc::fence_before_sync();
+    pair_sync();
+    tc::fence_after_sync();
+    const float l_tot = l_run + xch[(ntiles & 1) * 2 * kRows + (1 - hf) * kRows + row];
+#pragma unroll
+    for (int cch = 0; cch < 2; ++cch) {
+      uint32_t ov[32];
+      tc::tmem_ld32x32_x32u(tbase + lrow + kOCol + 64 * (1 - hf) + 32 * cch, ov);
+      tc::tmem_wait_ld();
+      // half 0 keeps u + v (coordinates 0 .. 63), half 1 u - v (64 .. 127), u being half 0's value
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float other = __uint_as_float(ov[e]);
+        o[32 * cch + e] = hf == 0 ? o[32 * cch + e] + other : other - o[32 * cch + e];
+      }
+    }
+    if (row_ok) {
+      const float sc = 1.0f / (128.0f * l_tot);
+      const uint64_t w = dev_splitmix64(a.seed, hf); // sign bits of coordinates 64 hf .. 64 hf + 63
+      float *dst = a.out + ((static_cast<size_t>(b) * a.Lq + i0 + ri) * a.Hq + h * a.G + rg) * 128 + 64 * hf;
+#pragma unroll
+      for (int i = 0; i < 64; i += 4) {
         float4 v4;
         float *vp = &v4.x;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int ii = i + e;
-          const bool neg = ((ii < 64 ? w0 >> ii : w1 >> (ii - 64)) & 1ull) != 0;
+          const bool neg = ((w >> ii) & 1ull) != 0;
           vp[e] = neg ? -o[ii] * sc : o[ii] * sc;
         }
         *reinterpret_cast<float4 *>(dst + i) = v4;
