@@ -92,10 +92,14 @@ typedef struct {
  * page. All pointers are device pointers owned by the caller. Per tensor:
  *   codes  [num_pages][Hkv][page_size][tq_code_bytes]  uint8   Lloyd-Max codes
  *   norm   [num_pages][Hkv][page_size]                 uint16  fp16 bits of ||x||
+ *   signs  [num_pages][Hkv][page_size][tq_sign_bytes]  uint8   PROD only: QJL sign bits, else NULL
+ *   rnorm  [num_pages][Hkv][page_size]                 uint16  PROD only: fp16 ||r||, else NULL
+ *   qjl    [m][d]                                      float   PROD only: the projection S, else NULL
  *   block_table [B][max_pages]                         int32   physical page of each logical
  *                                                              page (entries in 0..num_pages-1)
- * Supported: head_dim 128, TurboQuant_mse keys and values (3/4-bit keys, 2..4-bit values for
- * decode). A sequence may hold at most max_pages * page_size positions. */
+ * Supported: head_dim 128 TurboQuant_mse keys and values (3/4-bit keys, 2..4-bit values for
+ * decode), or head_dim 64 TurboQuant_prod keys and values with m = 64 (2-bit for decode);
+ * writes take 16-bit input. A sequence may hold at most max_pages * page_size positions. */
 typedef struct {
   int B, Hkv, d, page_size, num_pages, max_pages;
   uint64_t seed;
@@ -103,6 +107,9 @@ typedef struct {
   uint8_t *k_codes, *v_codes;
   uint16_t *k_norm, *v_norm;
   const int32_t *block_table;
+  uint8_t *k_signs, *v_signs;
+  uint16_t *k_rnorm, *v_rnorm;
+  const float *k_qjl, *v_qjl;
 } tq_paged_cache;
 
 /* Message for the last failure on the calling thread ("" if none). */

@@ -152,7 +152,16 @@ struct ProdArgs {
   long long total_tiles;
   uint32_t one2; // fp16 (1, 1): 0x3C003C00
   int B;
+  const int *bt; // paged cache (ragged calls only): block table [B][maxp]; record (b, h, t) at
+  int pshift, maxp; // ((bt[b][t >> pshift] * Hkv + h) << pshift) + (t mod page); else nullptr
 };
+
+// Record index of token t of (b, KV head) bh in a paged cache.
+__device__ __forceinline__ long long prod_page_rec(const ProdArgs &a, long long bh, int t) {
+  const long long b = bh / a.Hkv, h = bh - b * a.Hkv;
+  const long long page = __ldg(a.bt + b * a.maxp + (t >> a.pshift));
+  return ((page * a.Hkv + h) << a.pshift) + (t & ((1 << a.pshift) - 1));
+}
 struct NoVarLenP {};
 
 // The segment of the flattened (b, KV head, 16-token tile) space that starts at tile `seg`:
@@ -252,6 +261,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
     for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
 
     const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
+    const bool paged = RAG && a.bt != nullptr; // paged: every tile through the block table
     const int tlast = T_len - 1;
     const uint8_t *kbase = (c < 2 ? a.kc : a.ks) + 4 * (c & 1);
     const int vwo = 4 * (r >> 2);
@@ -285,12 +295,12 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
                              a.vg + rec0 + tw0 + r};
 
     auto load_next = [&](ProdTile &T) {
-      if (lane < 8 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16)
+      if (!paged && lane < 8 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
       pfp += pfstep;
       tpf += kPW * 16;
       const int t0 = (tile0 + jl) * 16;
-      if (t0 + 16 <= T_len) {
+      if (!paged && t0 + 16 <= T_len) {
         T.kw[0] = __ldcs(reinterpret_cast<const uint32_t *>(kp));
         T.kw[1] = __ldcs(reinterpret_cast<const uint32_t *>(kp + 64));
         const int toff[4] = {0, 8, 64, 72};
@@ -308,24 +318,26 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
         T.vg[0] = __ldcs(np[3]);
         T.vg[1] = __ldcs(np[3] + 8);
       } else {
+        // record of token t (within this 16-token tile, so within one page) = base + t
+        const long long base = paged ? prod_page_rec(a, bh, t0) - t0 : static_cast<long long>(rec0);
         const int tr = min(t0 + r, tlast), tr8 = min(t0 + r + 8, tlast);
         const int tv = t0 + 2 * c;
         const int tvs[4] = {min(tv, tlast), min(tv + 1, tlast), min(tv + 8, tlast), min(tv + 9, tlast)};
-        T.kw[0] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (rec0 + tr) * 8));
-        T.kw[1] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (rec0 + tr8) * 8));
+        T.kw[0] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (base + tr) * 8));
+        T.kw[1] = __ldcs(reinterpret_cast<const uint32_t *>(kbase + (base + tr8) * 8));
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          T.vm[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (rec0 + tvs[e]) * 8 + vwo));
-          T.vq[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (rec0 + tvs[e]) * 8 + vwo));
+          T.vm[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (base + tvs[e]) * 8 + vwo));
+          T.vq[e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (base + tvs[e]) * 8 + vwo));
         }
-        T.kn[0] = __ldcs(a.kn + rec0 + tr);
-        T.kn[1] = __ldcs(a.kn + rec0 + tr8);
-        T.kg[0] = __ldcs(a.kg + rec0 + tr);
-        T.kg[1] = __ldcs(a.kg + rec0 + tr8);
-        T.vn[0] = __ldcs(a.vn + rec0 + tr);
-        T.vn[1] = __ldcs(a.vn + rec0 + tr8);
-        T.vg[0] = __ldcs(a.vg + rec0 + tr);
-        T.vg[1] = __ldcs(a.vg + rec0 + tr8);
+        T.kn[0] = __ldcs(a.kn + base + tr);
+        T.kn[1] = __ldcs(a.kn + base + tr8);
+        T.kg[0] = __ldcs(a.kg + base + tr);
+        T.kg[1] = __ldcs(a.kg + base + tr8);
+        T.vn[0] = __ldcs(a.vn + base + tr);
+        T.vn[1] = __ldcs(a.vn + base + tr8);
+        T.vg[0] = __ldcs(a.vg + base + tr);
+        T.vg[1] = __ldcs(a.vg + base + tr8);
       }
       kp += kPW * 16 * 8;
       vcp += kPW * 16 * 8;
@@ -521,6 +533,10 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
     for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
 
     const size_t rec0 = static_cast<size_t>(bh) * a.T_cap;
+    const bool paged = RAG && a.bt != nullptr; // paged: every record through the block table
+    auto recof = [&](int t) -> long long {
+      return paged ? prod_page_rec(a, bh, t) : static_cast<long long>(rec0) + t;
+    };
     const int ts = tile0 * 16, te = min((tile0 + ntiles) * 16, T_len); // segment tokens
     const int ngroups = (te - ts + 31) / 32;
     const int vwo = 4 * (r >> 2);
@@ -537,7 +553,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
 
     auto load_next = [&](LutTile &T) {
       const int t0 = ts + 32 * jl;
-      if (t0 + 32 <= te) {
+      if (!paged && t0 + 32 <= te) {
         T.kc = __ldcs(kcp);
         T.ks = __ldcs(ksp);
         T.kn = __ldcs(np[0]);
@@ -553,7 +569,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
             T.vq[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(vsp + 128 * hh + toff[e]));
           }
       } else {
-        const size_t tk = rec0 + min(t0 + lane, te - 1);
+        const long long tk = recof(min(t0 + lane, te - 1));
         T.kc = __ldcs(reinterpret_cast<const uint2 *>(a.kc) + tk);
         T.ks = __ldcs(reinterpret_cast<const uint2 *>(a.ks) + tk);
         T.kn = __ldcs(a.kn + tk);
@@ -566,8 +582,9 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
           const int tvs[4] = {min(tv, te - 1), min(tv + 1, te - 1), min(tv + 8, te - 1), min(tv + 9, te - 1)};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            T.vm[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + (rec0 + tvs[e]) * 8 + vwo));
-            T.vq[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + (rec0 + tvs[e]) * 8 + vwo));
+            const long long tr = recof(tvs[e]);
+            T.vm[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vc + tr * 8 + vwo));
+            T.vq[hh][e] = __ldcs(reinterpret_cast<const uint32_t *>(a.vs + tr * 8 + vwo));
           }
         }
       }
@@ -866,6 +883,9 @@ cudaError_t launch_prod_decode(const DecodeArgs &a, cudaStream_t s) {
   f.total_tiles = static_cast<long long>(a.B) * a.Hkv * p.tiles_per_bh;
   f.one2 = 0x3C003C00u;
   f.B = a.B;
+  f.bt = a.pg.bt;
+  f.pshift = a.pg.pshift;
+  f.maxp = a.pg.maxp;
   if (a.T_lens) {
     // ragged batch: the per-sequence lengths and tile offsets travel as launch parameters
     VarLen vl;

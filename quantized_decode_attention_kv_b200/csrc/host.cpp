@@ -363,8 +363,10 @@ static int quantize_impl(const void *K, const void *V, int dtype, int T, int t_o
     if (!x) continue;
     if (tq::quantize_fast_supported(a[which])) fast[which] = &a[which];
     else if (tq::quantize_prod_supported(a[which])) prod[which] = &a[which];
-    if (pg.bt && !fast[which]) // the paged layout is written by the 16-bit MSE kernels only
-      return fail(TQ_ERR_UNSUPPORTED, "paged writes need 16-bit input and TurboQuant_mse records");
+    // the paged layout is written by the 16-bit MSE and TurboQuant_prod (d = 64, m = 64) kernels
+    if (pg.bt && !fast[which] && !prod[which])
+      return fail(TQ_ERR_UNSUPPORTED, "paged writes need 16-bit input and a head_dim-128 TurboQuant_mse "
+                                      "or head_dim-64 TurboQuant_prod (m = 64) tensor");
   }
   if (fast[0] || fast[1] || prod[0] || prod[1]) {
     const int sms = sm_count();
@@ -519,8 +521,6 @@ static int decode_varlen_impl(const void *q, int dtype, int Hq, const int *T_len
   if (st) return st;
   int sms = sm_count();
   if (sms <= 0) return fail(TQ_ERR_CUDA, "cannot query the device's SM count");
-  if (pg.pshift >= 0 && fast_path(*cache, Hq) == tq::kProdFast)
-    return fail(TQ_ERR_UNSUPPORTED, "a paged cache holds TurboQuant_mse records only");
   plan_varlen(*cache, Hq, mx, sms, T_lens, &a.plan);
   if (!ws || !aligned16(ws) || ws_bytes < a.plan.ws_bytes)
     return fail(TQ_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
@@ -561,9 +561,11 @@ static int paged_view(const tq_paged_cache *pc, tq_cache *view, tq::Paging *pg) 
   if (pc->page_size < 16 || (pc->page_size & (pc->page_size - 1)))
     return fail(TQ_ERR_INVALID_ARG, "page_size=%d must be a power of two >= 16", pc->page_size);
   if (!pc->block_table) return fail(TQ_ERR_INVALID_ARG, "block_table is NULL");
-  if (pc->d != 128) return fail(TQ_ERR_UNSUPPORTED, "paged caches support d = 128, got %d", pc->d);
-  if (pc->kc.mode != TQ_MSE || pc->vc.mode != TQ_MSE)
-    return fail(TQ_ERR_UNSUPPORTED, "paged caches support TurboQuant_mse records only");
+  const bool mse = pc->kc.mode == TQ_MSE && pc->vc.mode == TQ_MSE;
+  const bool prod = pc->kc.mode == TQ_PROD && pc->vc.mode == TQ_PROD;
+  if (!(mse && pc->d == 128) && !(prod && pc->d == 64))
+    return fail(TQ_ERR_UNSUPPORTED, "paged caches hold head_dim-128 TurboQuant_mse or head_dim-64 "
+                                    "TurboQuant_prod records (d=%d, modes %d/%d)", pc->d, pc->kc.mode, pc->vc.mode);
   const long long cap = static_cast<long long>(pc->max_pages) * pc->page_size;
   const long long recs = static_cast<long long>(pc->num_pages) * pc->Hkv * pc->page_size;
   if (cap > (1ll << 30) || recs > (1ll << 40))
@@ -580,6 +582,12 @@ static int paged_view(const tq_paged_cache *pc, tq_cache *view, tq::Paging *pg) 
   view->v_codes = pc->v_codes;
   view->k_norm = pc->k_norm;
   view->v_norm = pc->v_norm;
+  view->k_signs = pc->k_signs;
+  view->v_signs = pc->v_signs;
+  view->k_rnorm = pc->k_rnorm;
+  view->v_rnorm = pc->v_rnorm;
+  view->k_qjl = pc->k_qjl;
+  view->v_qjl = pc->v_qjl;
   int st = check_cache(view);
   if (st) return st;
   int shift = 0;

@@ -35,8 +35,19 @@ struct ProdQuantTensor {
   const float *S; // [64][64]
   unsigned nvec;
   int T, T_cap, t_offset, wbits;
-  float c1; // the positive 1-bit centroid (wbits = 1)
+  float c1;      // the positive 1-bit centroid (wbits = 1)
+  const int *bt; // paged cache: block table [B][maxp] (nullptr: dense [B][Hkv][T_cap] layout)
+  int pshift, maxp, Hkv;
 };
+
+// Record index of new position tt of (b, KV head) bh: dense, or through the block table.
+__device__ __forceinline__ size_t prod_rec(const ProdQuantTensor &t, unsigned bh, unsigned tt) {
+  const unsigned pos = static_cast<unsigned>(t.t_offset) + tt;
+  if (!t.bt) return static_cast<size_t>(bh) * t.T_cap + pos;
+  const unsigned b = bh / static_cast<unsigned>(t.Hkv), h = bh - b * static_cast<unsigned>(t.Hkv);
+  const unsigned page = static_cast<unsigned>(__ldg(t.bt + static_cast<size_t>(b) * t.maxp + (pos >> t.pshift)));
+  return ((static_cast<size_t>(page) * t.Hkv + h) << t.pshift) + (pos & ((1u << t.pshift) - 1u));
+}
 
 struct ProdQuantArgs {
   ProdQuantTensor t[2];
@@ -250,7 +261,7 @@ __global__ void __launch_bounds__(kRWarps * 32, 3) quantize_prod_kernel(const Pr
             tt -= T;
             ++bh;
           }
-          const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
+          const size_t rec = prod_rec(t, bh, tt);
           const uint32_t s0 = u ? sg[1][0] : sg[0][0], s1 = u ? sg[1][1] : sg[0][1];
           reinterpret_cast<uint2 *>(t.signs)[rec] = make_uint2(s0, s1);
           if constexpr (WB == 1)
@@ -484,7 +495,7 @@ __global__ void __launch_bounds__(kTcRows, 3) quantize_prod_tc_kernel(const Prod
       const unsigned v = v0 + tid;
       if (v < t.nvec) {
         const unsigned bh = v / T, tt = v - bh * T;
-        const size_t rec = static_cast<size_t>(bh) * t.T_cap + t.t_offset + tt;
+        const size_t rec = prod_rec(t, bh, tt);
         reinterpret_cast<uint2 *>(t.signs)[rec] = make_uint2(sg[0], sg[1]);
         if constexpr (WB == 1) reinterpret_cast<uint2 *>(t.codes)[rec] = make_uint2(~cw[0], ~cw[1]);
         t.norm[rec] = f32_to_f16_bits(nrm);
@@ -546,6 +557,10 @@ cudaError_t launch_quantize_prod(const QuantArgs *k, const QuantArgs *v, int sms
     t.T = q.T;
     t.T_cap = q.T_cap;
     t.t_offset = q.t_offset;
+    t.bt = q.pg.bt;
+    t.pshift = q.pg.pshift;
+    t.maxp = q.pg.maxp;
+    t.Hkv = q.Hkv;
     t.wbits = q.t.wbits;
     t.c1 = q.t.wbits == 1 ? q.t.cb.c[1] : 0.f;
     f.groups[nt] = (t.nvec + 15) / 16;

@@ -53,6 +53,9 @@ class tq_paged_cache(ctypes.Structure):
         ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
         ("k_norm", ctypes.c_void_p), ("v_norm", ctypes.c_void_p),
         ("block_table", ctypes.c_void_p),
+        ("k_signs", ctypes.c_void_p), ("v_signs", ctypes.c_void_p),
+        ("k_rnorm", ctypes.c_void_p), ("v_rnorm", ctypes.c_void_p),
+        ("k_qjl", ctypes.c_void_p), ("v_qjl", ctypes.c_void_p),
     ]
 
 
@@ -236,30 +239,44 @@ class TQCache:
 
 
 class TQPagedCache:
-    """One layer's paged compressed KV cache (TurboQuant_mse, head_dim 128): torch owns the
-    page pools; ``block_table`` is an int32 [B][max_pages] device tensor the caller fills with
-    physical page indices (it may be rewritten between calls). Shapes follow include/tq.h."""
+    """One layer's paged compressed KV cache (head_dim-128 TurboQuant_mse or head_dim-64
+    TurboQuant_prod records): torch owns the page pools; ``block_table`` is an int32
+    [B][max_pages] device tensor the caller fills with physical page indices (it may be
+    rewritten between calls). Shapes follow include/tq.h."""
 
     def __init__(self, B: int, Hkv: int, d: int, page_size: int, num_pages: int, max_pages: int,
-                 k_bits: int, v_bits: int, block_table: torch.Tensor, seed: int = 0, device: str = "cuda"):
+                 k_bits: int, v_bits: int, block_table: torch.Tensor, seed: int = 0, device: str = "cuda",
+                 k_mode: int = TQ_MSE, v_mode: int = TQ_MSE, k_qjl_m: int = 0, v_qjl_m: int = 0,
+                 qjl_seed: int = 1):
         dev = torch.device(device)
         self.B, self.Hkv, self.d, self.page_size = B, Hkv, d, page_size
         self.num_pages, self.max_pages, self.k_bits, self.v_bits, self.seed = num_pages, max_pages, k_bits, v_bits, seed
+        self.k_mode, self.v_mode, self.k_qjl_m, self.v_qjl_m, self.qjl_seed = k_mode, v_mode, k_qjl_m, v_qjl_m, qjl_seed
         if block_table.dtype != torch.int32 or tuple(block_table.shape) != (B, max_pages) or not block_table.is_cuda:
             raise TQError(TQ_ERR_INVALID_ARG, "block_table must be an int32 CUDA tensor [B][max_pages]")
         self.block_table = block_table.contiguous()
         self.tensors = {}
-        for side, bits in (("k", k_bits), ("v", v_bits)):
-            cb = tq_code_bytes(d, bits, TQ_MSE, 0)
+        for side, bits, mode, m in (("k", k_bits, k_mode, k_qjl_m), ("v", v_bits, v_mode, v_qjl_m)):
+            cb = tq_code_bytes(d, bits, mode, m)
             shape = (num_pages, Hkv, page_size)
-            self.tensors[f"{side}_codes"] = torch.zeros(shape + (cb,), dtype=torch.uint8, device=dev)
+            self.tensors[f"{side}_codes"] = torch.zeros(shape + (max(cb, 1),), dtype=torch.uint8, device=dev) if cb else None
             self.tensors[f"{side}_norm"] = torch.zeros(shape, dtype=torch.int16, device=dev)
+            if mode == TQ_PROD:
+                self.tensors[f"{side}_signs"] = torch.zeros(shape + (tq_sign_bytes(d, bits, mode, m),),
+                                                            dtype=torch.uint8, device=dev)
+                self.tensors[f"{side}_rnorm"] = torch.zeros(shape, dtype=torch.int16, device=dev)
+                self.tensors[f"{side}_qjl"] = torch.from_numpy(tq_make_qjl_matrix(qjl_seed, m or d, d)).to(dev)
+            else:
+                for key in ("signs", "rnorm", "qjl"):
+                    self.tensors[f"{side}_{key}"] = None
         t = self.tensors
+        ptr = lambda x: x.data_ptr() if x is not None else None  # noqa: E731
         self.struct = tq_paged_cache(B, Hkv, d, page_size, num_pages, max_pages, seed,
-                                     tq_qcfg(k_bits, TQ_MSE, 0), tq_qcfg(v_bits, TQ_MSE, 0),
-                                     t["k_codes"].data_ptr(), t["v_codes"].data_ptr(),
-                                     t["k_norm"].data_ptr(), t["v_norm"].data_ptr(),
-                                     self.block_table.data_ptr())
+                                     tq_qcfg(k_bits, k_mode, k_qjl_m), tq_qcfg(v_bits, v_mode, v_qjl_m),
+                                     ptr(t["k_codes"]), ptr(t["v_codes"]), ptr(t["k_norm"]), ptr(t["v_norm"]),
+                                     self.block_table.data_ptr(),
+                                     ptr(t["k_signs"]), ptr(t["v_signs"]), ptr(t["k_rnorm"]), ptr(t["v_rnorm"]),
+                                     ptr(t["k_qjl"]), ptr(t["v_qjl"]))
 
     def __getitem__(self, key):
         return self.tensors[key]
