@@ -186,8 +186,8 @@ int tq_decode_attention(const void *q, int dtype, int Hq, int T_len, float scale
  * caller-owned. The split-K partials live in one fixed 8 MiB device array inside libtq
  * (present on every GPU that loads the library, until the process exits); a shape whose
  * tq_decode_workspace_bytes exceeds 8 MiB is rejected with TQ_ERR_WORKSPACE and nothing is
- * launched. The first call on a device looks up the array's device address with that device
- * current; make that first call before any stream capture. Every call on a device shares the
+ * launched. The first call on a device looks up the array's device address (a host-side
+ * symbol lookup) with that device current. Every call on a device shares the
  * same array and leaves its partials behind; a call writes every element it later reads, so
  * nothing needs clearing, but calls that overlap on the GPU (other streams, other host
  * threads) race on the array and must be serialised by the caller. The looked-up address is
