@@ -55,6 +55,16 @@ extern "C" {
 
 #define TQ_MSE 0  /* TurboQuant_mse: b-bit Lloyd-Max codes                                  */
 #define TQ_PROD 1 /* TurboQuant_prod: (b-1)-bit codes + 1-bit QJL residual sketch + ||r||   */
+/* TurboQuant_mse records whose 4-bit codes live on Blackwell's FP4 (E2M1) grid instead of the
+ * Lloyd-Max levels ("Where This Fits in the Inference Stack", Blackwell FP4: whether the
+ * centroids map onto E2M1 is an open question there). Levels, ascending: s * (-6, -4, -3, -2,
+ * -1.5, -1, -0.5, -0, +0, 0.5, 1, 1.5, 2, 3, 4, 6) on the N(0,1) scale of the rotated
+ * coordinates (divided by sqrt(d) for a unit vector), s = 0.48708 the Gaussian-MSE-optimal
+ * stretch; boundaries at the midpoints, 0 between the two zeros (a coordinate takes the zero
+ * of its own sign). Code i is the level's index, as for TQ_MSE; its E2M1 bit pattern is
+ * i - 8 for i >= 8 and 15 - i for i < 8. Gaussian MSE 0.01268, 1.335x the 4-bit Lloyd-Max
+ * codebook's. bits must be 4; records are laid out as 4-bit TQ_MSE records. */
+#define TQ_E2M1 2
 
 #define TQ_F32 0
 #define TQ_BF16 1
@@ -63,7 +73,7 @@ extern "C" {
 /* Quantiser of one tensor (keys or values). */
 typedef struct {
   int bits;  /* total bits per coordinate, 1..4                                          */
-  int mode;  /* TQ_MSE or TQ_PROD ("Closing", Step 3: PROD is meant for bits <= 2)        */
+  int mode;  /* TQ_MSE, TQ_PROD ("Closing", Step 3: PROD is meant for bits <= 2) or TQ_E2M1 */
   int qjl_m; /* PROD only: QJL rows m (0 = d); ignored for TQ_MSE                          */
 } tq_qcfg;
 

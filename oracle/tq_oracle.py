@@ -33,7 +33,7 @@ from statistics import NormalDist
 import numpy as np
 
 __all__ = [
-    "MSE", "PROD", "splitmix64", "rotation_signs", "hadamard", "rotate", "inverse_rotate",
+    "MSE", "PROD", "E2M1", "e2m1_value", "e2m1_codebook", "code_to_e2m1", "splitmix64", "rotation_signs", "hadamard", "rotate", "inverse_rotate",
     "qjl_matrix", "lloyd_max_gaussian", "codebook", "Records", "quantize", "dequantize",
     "pack_bits", "unpack_bits", "code_bytes", "sign_bytes", "record_bytes",
     "boundary_distance", "attention", "gqa_decode", "decode_compressed", "records_from_packed",
@@ -42,6 +42,7 @@ __all__ = [
 
 MSE = 0   # TurboQuant_mse: b-bit Lloyd-Max codes only
 PROD = 1  # TurboQuant_prod: (b-1)-bit Lloyd-Max codes + 1-bit QJL residual sketch
+E2M1 = 2  # TurboQuant_mse with 4-bit codes on Blackwell's FP4 (E2M1) grid [S16 Blackwell FP4]
 
 _MASK64 = (1 << 64) - 1
 _ROWS = 1024  # vectors per chunk in quantize/boundary_distance (memory only)
@@ -195,6 +196,88 @@ def _lloyd_max(bits: int, tol: float, max_iter: int):
     return np.array(c), np.array(beta), dist
 
 
+# ----------------------------------------------------------------------------------------
+# The E2M1 grid [S16 "Blackwell FP4: The Natural Convergence Point": whether the Lloyd-Max
+# centroids map onto NVFP4's E2M1 values is left open there]. E2M1 is the 4-bit float of
+# the OCP microscaling formats: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit; it
+# holds 0, 0.5, 1, 1.5, 2, 3, 4, 6 with either sign (+0 and -0 both exist).
+# Reading: the rotated coordinates are i.i.d. N(0,1) for every block, so one stretch s of the
+# grid (no per-block scale) is the quantiser: 16 levels s * (-6, -4, -3, -2, -1.5, -1, -0.5,
+# -0, +0, 0.5, 1, 1.5, 2, 3, 4, 6) in ascending order, the two zeros kept as two codes (a
+# coordinate takes the zero of its own sign), boundaries at the midpoints (0 between the two
+# zeros), s minimising the Gaussian MSE. Code i is stored like a Lloyd-Max code (its index in
+# that order); its E2M1 bit pattern is code_to_e2m1(i).
+# ----------------------------------------------------------------------------------------
+_E2M1_SORTED = (-6.0, -4.0, -3.0, -2.0, -1.5, -1.0, -0.5, -0.0, 0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def e2m1_value(bits: int) -> float:
+    """The value of a 4-bit E2M1 pattern: (-1)^s * (m / 2 if e == 0 else 2^(e-1) * (1 + m/2))."""
+    sign = -1.0 if (bits >> 3) & 1 else 1.0
+    e, m = (bits >> 1) & 3, bits & 1
+    return sign * (m / 2.0 if e == 0 else 2.0 ** (e - 1) * (1.0 + m / 2.0))
+
+
+def code_to_e2m1(code):
+    """E2M1 bit pattern of code i of the ascending E2M1 codebook: the positive half (i >= 8)
+    is i - 8, the negative half the magnitude order reversed under the sign bit."""
+    code = np.asarray(code, dtype=np.int64)
+    return np.where(code >= 8, code - 8, 8 + (7 - code))
+
+
+def _grid_mse(levels: np.ndarray) -> float:
+    """E[(z - Q(z))^2] for z ~ N(0,1) and the nearest-level quantiser on ascending ``levels``
+    (cells between the midpoints), from the exact Gaussian moments of each cell."""
+    edges = [-math.inf] + [(levels[j] + levels[j + 1]) / 2.0 for j in range(len(levels) - 1)] + [math.inf]
+    total = 0.0
+    for j, c in enumerate(levels):
+        a, b = edges[j], edges[j + 1]
+        p = _cdf(b) - _cdf(a)
+        m1 = _pdf(a) - _pdf(b)
+        m2 = p + (0.0 if math.isinf(a) else a * _pdf(a)) - (0.0 if math.isinf(b) else b * _pdf(b))
+        total += m2 - 2.0 * c * m1 + c * c * p
+    return total
+
+
+@functools.lru_cache(maxsize=None)
+def _e2m1_cached():
+    grid = np.array(_E2M1_SORTED)
+    lo, hi = 0.3, 0.8  # the Gaussian MSE of the stretched grid is unimodal here
+    g = (math.sqrt(5.0) - 1.0) / 2.0
+    a, b = hi - g * (hi - lo), lo + g * (hi - lo)
+    fa, fb = _grid_mse(grid * a), _grid_mse(grid * b)
+    while hi - lo > 1e-12:  # golden-section search
+        if fa < fb:
+            hi, b, fb = b, a, fa
+            a = hi - g * (hi - lo)
+            fa = _grid_mse(grid * a)
+        else:
+            lo, a, fa = a, b, fb
+            b = lo + g * (hi - lo)
+            fb = _grid_mse(grid * b)
+    s = (lo + hi) / 2.0
+    c = grid * s
+    beta = np.array([(c[j] + c[j + 1]) / 2.0 for j in range(15)])
+    beta[7] = 0.0
+    return c, beta, _grid_mse(c), s
+
+
+def e2m1_codebook():
+    """(levels ascending [16], boundaries ascending [15], Gaussian MSE, stretch s) of the E2M1
+    codebook on the N(0,1) scale (see the reading above)."""
+    c, beta, dist, s = _e2m1_cached()
+    return c.copy(), beta.copy(), dist, s
+
+
+def _levels(wbits: int, mode: int):
+    """Centroids and boundaries (N(0,1) scale) of a tensor's codes."""
+    if mode == E2M1:
+        c, beta, _, _ = e2m1_codebook()
+        return c, beta
+    c, beta, _ = lloyd_max_gaussian(wbits)
+    return c, beta
+
+
 def codebook(bits: int, d: int):
     """Centroids and boundaries for a unit-norm vector's rotated coordinates: the N(0,1)
     Lloyd-Max codebook scaled by 1/sqrt(d) [S17 Step 2; One-Slide Version]."""
@@ -231,7 +314,7 @@ def unpack_bits(packed: np.ndarray, width: int, k: int) -> np.ndarray:
 
 
 def _mse_bits(bits: int, mode: int) -> int:
-    return bits if mode == MSE else bits - 1
+    return bits - 1 if mode == PROD else bits
 
 
 def code_bytes(d: int, bits: int, mode: int) -> int:
@@ -241,7 +324,7 @@ def code_bytes(d: int, bits: int, mode: int) -> int:
 
 def sign_bytes(d: int, bits: int, mode: int, m: int | None = None) -> int:
     """Bytes of QJL sign bits per vector (0 in MSE mode)."""
-    return 0 if mode == MSE else (m or d) // 8
+    return (m or d) // 8 if mode == PROD else 0
 
 
 def record_bytes(d: int, bits: int, mode: int, m: int | None = None) -> int:
@@ -250,7 +333,7 @@ def record_bytes(d: int, bits: int, mode: int, m: int | None = None) -> int:
     At d=128 a 3-bit MSE record is 48 + 2 = 50 bytes, 5.12x smaller than 256 bytes of fp16
     [S15 Finding 3, "block_size=128: 5.12x"]; a 4-bit record is 66 bytes (~4x).
     """
-    extra = 2 if mode == MSE else 4
+    extra = 4 if mode == PROD else 2
     return code_bytes(d, bits, mode) + sign_bytes(d, bits, mode, m) + extra
 
 
@@ -294,6 +377,8 @@ def quantize(x: np.ndarray, bits: int, mode: int = MSE, seed: int = 0, qjl_seed:
     3. MSE: code_i = the nearest centroid of the ``bits``-bit N(0,1) Lloyd-Max codebook,
        found by brute force over all centroids; an exact tie goes to the lower index
        [S17 Step 2]. This equals the count of boundaries strictly below z_i (checked).
+    3''. E2M1 (bits = 4): as 3 on the E2M1 codebook; a coordinate between the two zero levels
+       takes the zero of its own sign (the count of boundaries strictly below z; 0 -> -0).
     3'. PROD (b <= 2, [S17 Step 3; S15 Finding 2]): (bits-1)-bit codes as in 3 (none when
        bits = 1); residual r = (z - c[code]) / sqrt(d) in the unit-norm rotated domain;
        gamma = ||r|| stored as float16; QJL bit j = 1 iff (S r)_j < 0 (sign(0) = +1).
@@ -304,7 +389,7 @@ def quantize(x: np.ndarray, bits: int, mode: int = MSE, seed: int = 0, qjl_seed:
     n_vec, d = x.shape
     m = d if (m is None or m == 0) else m
     wbits = _mse_bits(bits, mode)
-    if mode not in (MSE, PROD) or bits < 1 or wbits < 0:
+    if mode not in (MSE, PROD, E2M1) or bits < 1 or wbits < 0 or (mode == E2M1 and bits != 4):
         raise ValueError("bad bits/mode")
 
     norm = np.sqrt(np.sum(x * x, axis=1))
@@ -315,15 +400,22 @@ def quantize(x: np.ndarray, bits: int, mode: int = MSE, seed: int = 0, qjl_seed:
     z[nz] = y[nz] / norm[nz, None]
 
     if wbits > 0:
-        cent, beta, _ = lloyd_max_gaussian(wbits)
+        cent, beta = _levels(wbits, mode)
         codes = np.empty(z.shape, dtype=np.int64)
         for lo in range(0, n_vec, _ROWS):  # rows are independent; chunks bound the temporaries
             zc = z[lo:lo + _ROWS]
-            codes[lo:lo + _ROWS] = np.argmin(np.abs(zc[:, :, None] - cent[None, None, :]), axis=2)
+            dist_all = np.abs(zc[:, :, None] - cent[None, None, :])
+            nearest = np.argmin(dist_all, axis=2)
             counted = np.searchsorted(beta, zc, side="left")
             exact_tie = np.min(np.abs(zc[:, :, None] - beta[None, None, :]), axis=2) < 1e-12
-            assert np.all((codes[lo:lo + _ROWS] == counted) | exact_tie), \
-                "nearest centroid != boundary count"
+            if mode == E2M1:
+                # the two zero levels are equally near; the count picks the zero of z's sign
+                codes[lo:lo + _ROWS] = counted
+                got = np.take_along_axis(dist_all, counted[:, :, None], axis=2)[:, :, 0]
+                assert np.all((got == dist_all.min(axis=2)) | exact_tie), "count is not a nearest level"
+            else:
+                codes[lo:lo + _ROWS] = nearest
+                assert np.all((nearest == counted) | exact_tie), "nearest centroid != boundary count"
         chat = cent[codes]
     else:
         codes = np.zeros((n_vec, d), dtype=np.int64)
@@ -380,7 +472,7 @@ def dequantize(rec: Records) -> np.ndarray:
     """
     d = rec.d
     wbits = _mse_bits(rec.bits, rec.mode)
-    inner = lloyd_max_gaussian(wbits)[0][rec.codes] if wbits > 0 else np.zeros(rec.codes.shape)
+    inner = _levels(wbits, rec.mode)[0][rec.codes] if wbits > 0 else np.zeros(rec.codes.shape)
     if rec.mode == PROD:
         s_mat = qjl_matrix(rec.qjl_seed, rec.m, d)
         signs = 1.0 - 2.0 * rec.qjl_bits
@@ -398,7 +490,7 @@ def boundary_distance(rec: Records) -> np.ndarray:
     wbits = _mse_bits(rec.bits, rec.mode)
     if wbits == 0:
         return np.full(rec.z.shape, np.inf)
-    beta = lloyd_max_gaussian(wbits)[1]
+    beta = _levels(wbits, rec.mode)[1]
     out = np.empty(rec.z.shape)
     for lo in range(0, rec.z.shape[0], _ROWS):
         zc = rec.z[lo:lo + _ROWS]

@@ -53,14 +53,11 @@ struct QPrep {
 };
 
 
-// Query prep of one query by one warp: rotate (q'' = H D q), scale (q~ = scale q'' / d),
-// round to 24-bit fixed point at the full range and split into int8 hi, mid and lo; csc is
-// the centroids' fixed-point scale. Lane l holds coordinates 4 l .. 4 l + 3; the butterflies of span 1, 2 run in the
-// lane, those of span 4 .. 64 across lanes (the lane with the span bit set keeps
-// partner - own).
-__device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, float scale,
-                                           uint64_t seed, float csc, QPrep *out, int lane) {
-  float x[4];
+// Rotation and scaling of one query by one warp: q~ = scale (H D q) / d. Lane l holds
+// coordinates 4 l .. 4 l + 3; the butterflies of span 1, 2 run in the lane, those of span
+// 4 .. 64 across lanes (the lane with the span bit set keeps partner - own).
+__device__ __forceinline__ void rotate_query(const void *q, int dtype, size_t bq, float scale,
+                                             uint64_t seed, int lane, float (&x)[4]) {
   const uint64_t sw = dev_splitmix64(seed, static_cast<uint64_t>(lane >> 4)); // coordinates 64 k ..
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
@@ -84,12 +81,20 @@ __device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, 
       x[e] = upper ? o - x[e] : x[e] + o;
     }
   }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] *= scale / static_cast<float>(kD);
+}
+
+// Query prep of one query by one warp: rotate and scale (rotate_query), round to 24-bit fixed
+// point at the full range and split into int8 hi, mid and lo; csc is the centroids'
+// fixed-point scale.
+__device__ __forceinline__ void prep_query(const void *q, int dtype, size_t bq, float scale,
+                                           uint64_t seed, float csc, QPrep *out, int lane) {
+  float x[4];
+  rotate_query(q, dtype, bq, scale, seed, lane, x);
   float mx = 0.f;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    x[e] *= scale / static_cast<float>(kD);
-    mx = fmaxf(mx, fabsf(x[e]));
-  }
+  for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(x[e]));
   mx = warp_max(mx);
   // fmaxf ignores NaN, so a NaN anywhere in the query (the rotation spreads it to every
   // coordinate) is detected separately

@@ -98,6 +98,67 @@ double fixed_point_scale(const double *c, int L) {
   return best;
 }
 
+// The E2M1 codebook on the N(0,1) scale: the 16 ascending levels s * (-6, -4, -3, -2, -1.5, -1,
+// -0.5, -0, +0, 0.5, 1, 1.5, 2, 3, 4, 6) of Blackwell's FP4 format (+0 and -0 kept as two
+// codes: a coordinate takes the zero of its sign), boundaries at the midpoints (0 between the
+// zeros), s minimising the Gaussian MSE by golden-section search over [0.3, 0.8] ("Where This
+// Fits in the Inference Stack", Blackwell FP4: can the codes live on the E2M1 grid).
+double grid_mse(const double *c, int L) {
+  double total = 0.0;
+  for (int j = 0; j < L; ++j) {
+    const double a = j == 0 ? -INFINITY : 0.5 * (c[j - 1] + c[j]);
+    const double b = j == L - 1 ? INFINITY : 0.5 * (c[j] + c[j + 1]);
+    const double p = ncdf(b) - ncdf(a);
+    const double m1 = npdf(a) - npdf(b);
+    const double m2 = p + (std::isinf(a) ? 0.0 : a * npdf(a)) - (std::isinf(b) ? 0.0 : b * npdf(b));
+    total += m2 - 2.0 * c[j] * m1 + c[j] * c[j] * p;
+  }
+  return total;
+}
+
+DoubleCodebook compute_e2m1() {
+  static const double grid[16] = {-6, -4, -3, -2, -1.5, -1, -0.5, -0.0, 0.0, 0.5, 1, 1.5, 2, 3, 4, 6};
+  auto mse_at = [](double s) {
+    double c[16];
+    for (int j = 0; j < 16; ++j) c[j] = grid[j] * s;
+    return grid_mse(c, 16);
+  };
+  const double g = 0.5 * (std::sqrt(5.0) - 1.0);
+  double lo = 0.3, hi = 0.8, a = hi - g * (hi - lo), b = lo + g * (hi - lo);
+  double fa = mse_at(a), fb = mse_at(b);
+  while (hi - lo > 1e-12) {
+    if (fa < fb) {
+      hi = b;
+      b = a;
+      fb = fa;
+      a = hi - g * (hi - lo);
+      fa = mse_at(a);
+    } else {
+      lo = a;
+      a = b;
+      fa = fb;
+      b = lo + g * (hi - lo);
+      fb = mse_at(b);
+    }
+  }
+  const double s = 0.5 * (lo + hi);
+  DoubleCodebook cb{};
+  cb.levels = 16;
+  cb.ok = true;
+  for (int j = 0; j < 16; ++j) cb.c[j] = grid[j] * s;
+  for (int j = 0; j < 15; ++j) cb.beta[j] = 0.5 * (cb.c[j] + cb.c[j + 1]);
+  cb.beta[7] = 0.0;
+  cb.fix_scale = fixed_point_scale(cb.c, 16);
+  return cb;
+}
+
+const DoubleCodebook &e2m1_codebook() {
+  static DoubleCodebook table;
+  static std::once_flag once;
+  std::call_once(once, [] { table = compute_e2m1(); });
+  return table;
+}
+
 DoubleCodebook compute_lloyd_max(int wbits) {
   DoubleCodebook cb{};
   const int L = 1 << wbits;
@@ -148,8 +209,10 @@ int check_qcfg(int d, const tq_qcfg &c, const char *name) {
     return fail(TQ_ERR_UNSUPPORTED, "d=%d: head_dim must be a power of two in 16..256", d);
   if (c.bits < 1 || c.bits > 4)
     return fail(TQ_ERR_UNSUPPORTED, "%s.bits=%d: bits must be 1..4", name, c.bits);
-  if (c.mode != TQ_MSE && c.mode != TQ_PROD)
-    return fail(TQ_ERR_UNSUPPORTED, "%s.mode=%d: mode must be TQ_MSE or TQ_PROD", name, c.mode);
+  if (c.mode != TQ_MSE && c.mode != TQ_PROD && c.mode != TQ_E2M1)
+    return fail(TQ_ERR_UNSUPPORTED, "%s.mode=%d: mode must be TQ_MSE, TQ_PROD or TQ_E2M1", name, c.mode);
+  if (c.mode == TQ_E2M1 && c.bits != 4)
+    return fail(TQ_ERR_UNSUPPORTED, "%s.bits=%d: TQ_E2M1 codes are 4 bits", name, c.bits);
   if (c.mode == TQ_PROD) {
     int m = c.qjl_m == 0 ? d : c.qjl_m;
     if (m < 8 || m > tq::kMaxM || m % 8)
@@ -166,8 +229,8 @@ int resolve_tensor(const tq_cache &c, int which, tq::TensorArgs *t) {
   if (st) return st;
   std::memset(t, 0, sizeof *t);
   t->bits = q.bits;
-  t->mode = q.mode;
-  t->wbits = q.mode == TQ_MSE ? q.bits : q.bits - 1;
+  t->mode = q.mode == TQ_PROD ? TQ_PROD : TQ_MSE; // E2M1 codes are MSE codes on another codebook
+  t->wbits = q.mode == TQ_PROD ? q.bits - 1 : q.bits;
   t->m = q.mode == TQ_PROD ? (q.qjl_m == 0 ? c.d : q.qjl_m) : 0;
   t->code_bytes = c.d * t->wbits / 8;
   t->sign_bytes = t->m / 8;
@@ -193,7 +256,7 @@ int resolve_tensor(const tq_cache &c, int which, tq::TensorArgs *t) {
   if (t->wbits == 0) {
     cb.levels = 1;
   } else {
-    const DoubleCodebook &d = lloyd_max(t->wbits);
+    const DoubleCodebook &d = q.mode == TQ_E2M1 ? e2m1_codebook() : lloyd_max(t->wbits);
     if (!d.ok) return fail(TQ_ERR_UNSUPPORTED, "Lloyd-Max iteration did not converge");
     cb.levels = d.levels;
     for (int j = 0; j < d.levels; ++j) cb.c[j] = static_cast<float>(d.c[j]);
@@ -234,13 +297,14 @@ bool dtype_ok(int dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
 // Whether the cache's bit-widths and shape take a tensor-core decode kernel: 0 if not,
 // kProdFast for the TurboQuant_prod kernel, else (key bits << 4) | value bits.
 int fast_path(const tq_cache &c, int Hq) {
-  const int kw = c.kc.mode == TQ_MSE ? c.kc.bits : c.kc.bits - 1;
-  const int vw = c.vc.mode == TQ_MSE ? c.vc.bits : c.vc.bits - 1;
+  const int kw = c.kc.mode == TQ_PROD ? c.kc.bits - 1 : c.kc.bits;
+  const int vw = c.vc.mode == TQ_PROD ? c.vc.bits - 1 : c.vc.bits;
   const int km = c.kc.qjl_m ? c.kc.qjl_m : c.d, vm = c.vc.qjl_m ? c.vc.qjl_m : c.d;
+  // the kernels see E2M1 tensors as MSE tensors with their own codebook
+  const int kmode = c.kc.mode == TQ_PROD ? TQ_PROD : TQ_MSE, vmode = c.vc.mode == TQ_PROD ? TQ_PROD : TQ_MSE;
   if (tq::prod_decode_supported(c.d, c.kc.mode, c.kc.bits, km, c.vc.mode, c.vc.bits, vm, Hq / c.Hkv))
     return tq::kProdFast;
-  return tq::fast_decode_supported(c.d, c.kc.mode, kw, c.vc.mode, vw, Hq / c.Hkv) ? (kw << 4) | vw
-                                                                                    : 0;
+  return tq::fast_decode_supported(c.d, kmode, kw, vmode, vw, Hq / c.Hkv) ? (kw << 4) | vw : 0;
 }
 
 } // namespace
@@ -294,7 +358,7 @@ int tq_make_qjl_matrix(uint64_t seed, int m, int d, float *S) {
 
 size_t tq_code_bytes(int d, tq_qcfg c) {
   if (check_qcfg(d, c, "cfg")) return 0;
-  int w = c.mode == TQ_MSE ? c.bits : c.bits - 1;
+  int w = c.mode == TQ_PROD ? c.bits - 1 : c.bits;
   return static_cast<size_t>(d) * w / 8;
 }
 
@@ -561,7 +625,7 @@ static int paged_view(const tq_paged_cache *pc, tq_cache *view, tq::Paging *pg) 
   if (pc->page_size < 16 || (pc->page_size & (pc->page_size - 1)))
     return fail(TQ_ERR_INVALID_ARG, "page_size=%d must be a power of two >= 16", pc->page_size);
   if (!pc->block_table) return fail(TQ_ERR_INVALID_ARG, "block_table is NULL");
-  const bool mse = pc->kc.mode == TQ_MSE && pc->vc.mode == TQ_MSE;
+  const bool mse = pc->kc.mode != TQ_PROD && pc->vc.mode != TQ_PROD; // MSE or E2M1 codes
   const bool prod = pc->kc.mode == TQ_PROD && pc->vc.mode == TQ_PROD;
   if (!(mse && pc->d == 128) && !(prod && pc->d == 64))
     return fail(TQ_ERR_UNSUPPORTED, "paged caches hold head_dim-128 TurboQuant_mse or head_dim-64 "
@@ -710,6 +774,7 @@ int tq_prefill_attention(const void *q, int dtype, int Hq, int Lq, int t0, float
   l.scale = scale;
   l.seed = cache->seed;
   l.out = out;
+  l.k_e2m1 = cache->kc.mode == TQ_E2M1;
   return cuda_status(tq::launch_prefill(l, static_cast<cudaStream_t>(stream)), "prefill launch");
 }
 

@@ -35,6 +35,8 @@
 #include "decode_mse_common.cuh"
 #include "tc_ops.cuh"
 
+#include <cuda_fp8.h>
+
 #include <algorithm>
 
 namespace tq {
@@ -47,10 +49,16 @@ constexpr int kKT = 64;                      // KV tokens per tile
 constexpr int kSWp = 8, kPWp = 4;            // softmax warps (two per row: half a tile each), producer warps
 constexpr int kWarpMMAp = kSWp + kPWp;       // the MMA warp
 constexpr int kThreadsP = (kSWp + kPWp + 1) * 32;
-constexpr uint32_t kTmemColsP = 512;
-constexpr uint32_t kSCols = 3 * kKT;         // one score stage
-constexpr uint32_t kOCol = 2 * kSCols;       // output columns 384 .. 511
 constexpr long long kWaitCyclesP = 1ll << 31; // about a second
+// Score stages: three int32 columns per token (the int8 parts), or one fp32 column per token
+// when the keys are E2M1 (F4); two stages, then the 128 fp32 output columns.
+template <bool F4>
+struct PfTmem {
+  static constexpr uint32_t S = F4 ? kKT : 3 * kKT;  // one score stage
+  static constexpr uint32_t O = 2 * S;               // first output column
+  static constexpr uint32_t alloc = F4 ? 256 : 512;
+};
+constexpr int kQParts4 = 4; // E4M3 parts of the query (F4): about 16 significant bits
 
 __device__ unsigned g_prefill_fault;
 
@@ -68,18 +76,24 @@ struct PrefillArgs {
   float kcent[16];
   float kcsc;
   float vcent[16];
+  float kstretch; // F4: the E2M1 grid's stretch (levels = kstretch * E2M1 values)
 };
 
-template <int KB, int VB>
+template <int KB, int VB, bool F4>
 struct PfLayout {
-  static constexpr int oQ = 0;                           // 3 x [128 rows][256 bytes] int8, K-major
-  static constexpr int oK = oQ + 3 * kRows * 256;        // 2 x [64 tokens][256 bytes] int8, K-major
-  static constexpr int oV = oK + 2 * kKT * 256;          // 2 x [128 coords][64 tokens] fp16, MN-major
+  // query operands, K-major: 3 x [128 rows][256 bytes] int8, or (F4) 4 x [128 rows][128] E4M3
+  static constexpr int kQBytes = F4 ? kQParts4 * kRows * 128 : 3 * kRows * 256;
+  // key operand stages, K-major: [64 tokens][256 bytes] int8, or (F4) [64 tokens][8 groups of
+  // 16 E2M1 codes: 8 bytes of packed codes + 8 bytes of padding]
+  static constexpr int kKStage = F4 ? kKT * 128 : kKT * 256;
+  static constexpr int oQ = 0;
+  static constexpr int oK = oQ + kQBytes;
+  static constexpr int oV = oK + 2 * kKStage;            // 2 x [128 coords][64 tokens] fp16, MN-major
   static constexpr int oP = oV + 2 * kKT * 256;          // 2 x [128 rows][64 tokens] fp16 P', K-major
   static constexpr int oKN = oP + 2 * kRows * kKT * 2;   // 2 x 64 key norms (float)
   static constexpr int oVN = oKN + 2 * kKT * 4;          // 2 x 64 value norms (float)
   static constexpr int oKT = oVN + 2 * kKT * 4;          // key entries {hi, hi, lo, lo} per code pair
-  static constexpr int kKRows = KB == 4 ? 256 : 64;
+  static constexpr int kKRows = F4 ? 0 : KB == 4 ? 256 : 64;
   static constexpr int oVT = oKT + kKRows * 4;           // value table
   static constexpr int kVRows = VB == 2 ? 256 : 1 << (2 * VB);
   static constexpr int kVEntry = VB == 2 ? 8 : 4;        // 2-bit: 4 fp16 per code byte; else fp16x2 per pair
@@ -134,9 +148,10 @@ __device__ __noinline__ void pf_wait_own_mmas(uint32_t mbar) {
   }
 }
 
-template <int KB, int VB>
+template <int KB, int VB, bool F4>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs a) {
-  using L = PfLayout<KB, VB>;
+  using L = PfLayout<KB, VB, F4>;
+  constexpr uint32_t kSCols = PfTmem<F4>::S, kOCol = PfTmem<F4>::O, kTmemColsP = PfTmem<F4>::alloc;
   constexpr int KR = KB * 16, VR = VB * 16; // record bytes
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
@@ -169,7 +184,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
   //      kernels' 16-bit fixed point); values as fp16 centroids
   {
     uint32_t *kt = reinterpret_cast<uint32_t *>(sm + L::oKT);
-    for (int e = tid; e < L::kKRows; e += kThreadsP) {
+    for (int e = tid; e < L::kKRows; e += kThreadsP) { // none for E2M1 keys
       const float c0 = a.kcent[e & (KB == 4 ? 15 : 7)], c1 = a.kcent[KB == 4 ? e >> 4 : e >> 3];
       const int x0 = __float2int_rn(c0 * a.kcsc), x1 = __float2int_rn(c1 * a.kcsc);
       const int l0 = ((x0 + 128) & 255) - 128, l1 = ((x1 + 128) & 255) - 128;
@@ -236,6 +251,43 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       const int rr = 32 * qw + 16 * hf + k;
       const int qi = rr / a.G, qg = rr - qi * a.G;
       const bool ok = qi < a.P && i0 + qi < a.Lq;
+      if constexpr (F4) {
+        // E2M1 keys: the query as the sum of four E4M3 parts (each the rounding of what the
+        // earlier ones left), scaled so that its largest coordinate is 224; the score MMAs
+        // accumulate all four in fp32. Part p of row rr, coordinate i: byte (rr & 7) * 16 +
+        // (rr >> 3) * 1024 + (i >> 4) * 128 + (i & 15) of part p's operand.
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ok) {
+          const size_t bq = (static_cast<size_t>(b) * a.Lq + i0 + qi) * a.Hq + h * a.G + qg;
+          rotate_query(a.q, a.q_dtype, bq, a.scale, a.seed, lane, x);
+        }
+        float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+        mx = warp_max(mx);
+        const bool has_nan = __any_sync(0xffffffffu, isnan(x[0]) || isnan(x[1]) || isnan(x[2]) || isnan(x[3]));
+        const bool good = !has_nan && mx > 1e-30f && isfinite(mx);
+        const float qsc = good ? 224.0f / mx : 0.f;
+        float r[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) r[e] = x[e] * qsc;
+        const uint32_t off = (rr & 7) * 16 + (rr >> 3) * 1024 + (lane >> 2) * 128 + 4 * (lane & 3);
+#pragma unroll
+        for (int part = 0; part < kQParts4; ++part) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_fp8_storage_t f = __nv_cvt_float_to_fp8(r[e], __NV_SATFINITE, __NV_E4M3);
+            w |= static_cast<uint32_t>(f) << (8 * e);
+            r[e] -= __half2float(__half(__nv_cvt_fp8_to_halfraw(f, __NV_E4M3)));
+          }
+          *reinterpret_cast<uint32_t *>(sm + L::oQ + part * (kRows * 128) + off) = w;
+        }
+        // score = ||k|| * (c . q~) = ||k|| * S * kstretch / qsc, S the MMAs' sum over E2M1
+        // values; a query with a NaN or an infinity gets NaN, a (near) zero one zero scores
+        if (lane == 0)
+          rinv[rr] = (good ? a.kstretch / qsc : (!has_nan && isfinite(mx) ? 0.f : __int_as_float(0x7fc00000))) * kLog2e;
+        __syncwarp();
+        continue;
+      }
       if (ok) {
         const size_t bq = (static_cast<size_t>(b) * a.Lq + i0 + qi) * a.Hq + h * a.G + qg;
         prep_query(a.q, a.q_dtype, bq, a.scale, a.seed, a.kcsc, qs, lane);
@@ -261,12 +313,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
     }
     // both score stages start at the magic constant: every score MMA accumulates onto it, so
     // an int32 sum s reads back as the float 1.5 * 2^23 + s (each warp its own tokens' columns)
+    if constexpr (!F4) {
 #pragma unroll
-    for (int x = 0; x < 2; ++x)
+      for (int x = 0; x < 2; ++x)
 #pragma unroll
-      for (int t = 0; t < 3; ++t)
-        tc::tmem_fill32x32_x32(tbase + lrow + x * kSCols + kKT * t + 32 * hf, static_cast<uint32_t>(kMagic));
-    tc::tmem_wait_st();
+        for (int t = 0; t < 3; ++t)
+          tc::tmem_fill32x32_x32(tbase + lrow + x * kSCols + kKT * t + 32 * hf, static_cast<uint32_t>(kMagic));
+      tc::tmem_wait_st();
+    }
     tc::fence_before_sync();
     tc::fence_async_smem();
     tc::mbar_arrive(Q_ready);
@@ -288,29 +342,47 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       const uint32_t st = tbase + lrow + x * kSCols + kH * hf;
       const float4 *kn4 = reinterpret_cast<const float4 *>(knb + x * kKT + kH * hf);
       float s[kH];
+      if constexpr (F4) {
+        // one fp32 column per token
 #pragma unroll
-      for (int cch = 0; cch < kH / 16; ++cch) {
-        uint32_t r0[16], r1[16], r2[16];
-        tc::tmem_ld32x32_x16(st + 16 * cch, r0);
-        tc::tmem_ld32x32_x16(st + kKT + 16 * cch, r1);
-        tc::tmem_ld32x32_x16(st + 2 * kKT + 16 * cch, r2);
-        tc::tmem_wait_ld();
+        for (int cch = 0; cch < kH / 16; ++cch) {
+          uint32_t r0[16];
+          tc::tmem_ld32x32_x16(st + 16 * cch, r0);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int t4 = 0; t4 < 4; ++t4) {
-          const float4 k4 = kn4[4 * cch + t4];
-          const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int t = 4 * t4 + e;
-            const float d = fmaf(__uint_as_float(r2[t]), 1.0f / 65536.0f,
-                                 fmaf(__uint_as_float(r1[t]), 1.0f / 256.0f, __uint_as_float(r0[t]) - kMagicAdj));
-            s[16 * cch + t] = kk[e] * d;
+          for (int t4 = 0; t4 < 4; ++t4) {
+            const float4 k4 = kn4[4 * cch + t4];
+            s[16 * cch + 4 * t4] = k4.x * __uint_as_float(r0[4 * t4]);
+            s[16 * cch + 4 * t4 + 1] = k4.y * __uint_as_float(r0[4 * t4 + 1]);
+            s[16 * cch + 4 * t4 + 2] = k4.z * __uint_as_float(r0[4 * t4 + 2]);
+            s[16 * cch + 4 * t4 + 3] = k4.w * __uint_as_float(r0[4 * t4 + 3]);
           }
         }
-      }
-      // the columns back to the magic constant for tile j + 2 (waited for before release)
+      } else {
 #pragma unroll
-      for (int t = 0; t < 3; ++t) tc::tmem_fill32x32_x32(st + kKT * t, static_cast<uint32_t>(kMagic));
+        for (int cch = 0; cch < kH / 16; ++cch) {
+          uint32_t r0[16], r1[16], r2[16];
+          tc::tmem_ld32x32_x16(st + 16 * cch, r0);
+          tc::tmem_ld32x32_x16(st + kKT + 16 * cch, r1);
+          tc::tmem_ld32x32_x16(st + 2 * kKT + 16 * cch, r2);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int t4 = 0; t4 < 4; ++t4) {
+            const float4 k4 = kn4[4 * cch + t4];
+            const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int t = 4 * t4 + e;
+              const float d = fmaf(__uint_as_float(r2[t]), 1.0f / 65536.0f,
+                                   fmaf(__uint_as_float(r1[t]), 1.0f / 256.0f, __uint_as_float(r0[t]) - kMagicAdj));
+              s[16 * cch + t] = kk[e] * d;
+            }
+          }
+      }
+        // the columns back to the magic constant for tile j + 2 (waited for before release)
+#pragma unroll
+        for (int t = 0; t < 3; ++t) tc::tmem_fill32x32_x32(st + kKT * t, static_cast<uint32_t>(kMagic));
+      }
       if (edge) {
 #pragma unroll
         for (int t = 0; t < kH; ++t)
@@ -486,7 +558,19 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       // keys: code pairs 32 half .. 32 half + 31 -> k bytes 128 half .. 128 half + 127 of row n.
       // Buffer x and the norms of tile j - 2 are free once its softmax released the stage.
       if (j >= 2) pf_wait(S_free(x), ((j >> 1) - 1) & 1, dead);
-      {
+      if constexpr (F4) {
+        // E2M1 keys: the stored codes are indices of the ascending E2M1 levels; index i has
+        // the bit pattern i ^ 8 (i >= 8) or i ^ 15 (i < 8): per nibble, XOR with 15 - 7 t, t its
+        // top bit. Group g of 16 coordinates: 8 bytes of patterns, then 8 bytes of padding.
+        uint8_t *kdst = sm + L::oK + x * L::kKStage + (n & 7) * 16 + (n >> 3) * 1024 + half * 4 * 128;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t w0 = c.k[2 * g], w1 = c.k[2 * g + 1];
+          const uint32_t e0 = w0 ^ (0xFFFFFFFFu - 7u * ((w0 >> 3) & 0x11111111u));
+          const uint32_t e1 = w1 ^ (0xFFFFFFFFu - 7u * ((w1 >> 3) & 0x11111111u));
+          *reinterpret_cast<uint4 *>(kdst + g * 128) = make_uint4(e0, e1, 0u, 0u);
+        }
+      } else {
         uint8_t *kdst = sm + L::oK + x * (kKT * 256) + (n & 7) * 16 + (n >> 3) * 2048 + half * 8 * 128;
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) { // 16 k bytes = 4 code pairs
@@ -553,7 +637,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
   } else {
     // =============================== MMA warp: one thread issues every MMA
     if (lane == 0) {
-      const uint32_t id_s = tc::idesc_i8(kRows, kKT);
+      const uint32_t id_s = F4 ? tc::idesc_e4m3_e2m1(kRows, kKT) : tc::idesc_i8(kRows, kKT);
       const uint32_t id_o = tc::idesc_f16_bmn(kRows, 128);
       pf_wait(Q_ready, 0, dead);
       // after a timeout (dead) no further MMA is issued
@@ -578,13 +662,26 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
         if (j >= 2) pf_wait(S_free(x), ((j >> 1) - 1) & 1, dead);
         if (*dead) break;
         tc::fence_after_sync();
+        if constexpr (F4) {
+          // S = sum over the four E4M3 query parts and 4 k-steps of 32 coordinates: E4M3 x E2M1,
+          // fp32 accumulation into one column per token
 #pragma unroll
-        for (int type = 0; type < 3; ++type)
+          for (int part = 0; part < kQParts4; ++part)
 #pragma unroll
-          for (int s = 0; s < 8; ++s)
-            tc::mma_ss_i8(tbase + x * kSCols + kKT * type,
-                          tc::desc_kmajor8(sb + L::oQ + type * (kRows * 256) + 256 * s, 128, 2048),
-                          tc::desc_kmajor8(sb + L::oK + x * (kKT * 256) + 256 * s, 128, 2048), id_s, 1u);
+            for (int s = 0; s < 4; ++s)
+              tc::mma_ss_f8f6f4(tbase + x * kSCols,
+                                tc::desc_kmajor(sb + L::oQ + part * (kRows * 128) + 256 * s, 128, 1024),
+                                tc::desc_kmajor(sb + L::oK + x * L::kKStage + 256 * s, 128, 1024), id_s,
+                                (part > 0 || s > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int type = 0; type < 3; ++type)
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+              tc::mma_ss_i8(tbase + x * kSCols + kKT * type,
+                            tc::desc_kmajor8(sb + L::oQ + type * (kRows * 256) + 256 * s, 128, 2048),
+                            tc::desc_kmajor8(sb + L::oK + x * (kKT * 256) + 256 * s, 128, 2048), id_s, 1u);
+        }
         tc::commit(S_full(x));
         if (j > 0) pv(j - 1);
       }
@@ -601,10 +698,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
   if (warp == kWarpMMAp) tc::tmem_dealloc(tbase, kTmemColsP);
 }
 
-template <int KB, int VB>
+template <int KB, int VB, bool F4 = false>
 cudaError_t run_prefill(const PrefillArgs &p, int ctas, cudaStream_t s) {
-  constexpr int smem = PfLayout<KB, VB>::kSmem;
-  auto kern = prefill_kernel<KB, VB>;
+  constexpr int smem = PfLayout<KB, VB, F4>::kSmem;
+  auto kern = prefill_kernel<KB, VB, F4>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(ctas), dim3(kThreadsP), smem, s, p);
@@ -639,8 +736,12 @@ cudaError_t launch_prefill(const PrefillLaunch &l, cudaStream_t s) {
   for (int j = 0; j < 16; ++j) p.kcent[j] = l.k.cb.c[j];
   p.kcsc = l.k.cb.fix_scale;
   for (int j = 0; j < 16; ++j) p.vcent[j] = l.v.cb.c[j];
+  p.kstretch = l.k.cb.c[15] / 6.0f; // the largest E2M1 level is 6 x the stretch
   const int ctas = l.B * l.Hkv * p.blocks;
   const int kb = l.k.wbits, vb = l.v.wbits;
+  if (l.k_e2m1)
+    return vb == 2 ? run_prefill<4, 2, true>(p, ctas, s) : vb == 3 ? run_prefill<4, 3, true>(p, ctas, s)
+                                                                  : run_prefill<4, 4, true>(p, ctas, s);
   if (kb == 4) return vb == 2 ? run_prefill<4, 2>(p, ctas, s) : vb == 3 ? run_prefill<4, 3>(p, ctas, s)
                                                                       : run_prefill<4, 4>(p, ctas, s);
   return vb == 2 ? run_prefill<3, 2>(p, ctas, s) : vb == 3 ? run_prefill<3, 3>(p, ctas, s)

@@ -647,6 +647,10 @@ cudaError_t run_fast(const FastQuantArgs &f, int sms, cudaStream_t s) {
 
 bool quantize_fast_supported(const QuantArgs &a) {
   if (a.t.mode != TQ_MSE || a.t.wbits < 1 || a.t.wbits > 4) return false;
+  // the cell-table code search needs adjacent boundaries more than one cell (1/4) apart: true
+  // of every Lloyd-Max codebook of <= 4 bits, not of the E2M1 grid near zero
+  for (int j = 0; j + 2 < a.t.cb.levels; ++j)
+    if (a.t.cb.beta[j + 1] - a.t.cb.beta[j] <= 0.25f) return false;
   if (a.dtype != TQ_BF16 && a.dtype != TQ_F16) return false;
   if (a.d != 64 && a.d != 128) return false;
   if (static_cast<long long>(a.B) * a.Hkv * a.T >= (1ll << 32) - kQThreads) return false;

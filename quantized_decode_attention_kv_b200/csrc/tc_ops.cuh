@@ -136,6 +136,24 @@ __device__ __forceinline__ void mma_ss_i8(uint32_t d_tmem, uint64_t a, uint64_t 
                : "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(z));
 }
 
+// Instruction descriptor of kind::f8f6f4: fp32 accumulation, A E4M3 (format 0), B E2M1
+// (format 5), both K-major (the only major order E2M1 takes), M x N tile.
+__host__ __device__ constexpr uint32_t idesc_e4m3_e2m1(int M, int N) {
+  return (1u << 4) | (0u << 7) | (5u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (K = 32 per instruction; a 4-bit operand sits
+// in shared memory as groups of 16 packed codes in 8 bytes, each group padded to 16 bytes).
+__device__ __forceinline__ void mma_ss_f8f6f4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n"
+               :
+               : "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(z));
+}
+
 // Instruction descriptor of kind::f16 with fp32 accumulation, fp16 A (K-major, from TMEM) and
 // fp16 B stored MN-major (N contiguous), M x N tile.
 __host__ __device__ constexpr uint32_t idesc_f16_bmn(int M, int N) {

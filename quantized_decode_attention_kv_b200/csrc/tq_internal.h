@@ -157,6 +157,7 @@ struct PrefillLaunch {
   uint64_t seed;
   TensorArgs k, v;
   float *out;
+  bool k_e2m1; // keys on the E2M1 grid (TQ_E2M1): the kernel feeds them to E2M1 tensor-core MMAs
 };
 bool prefill_supported(int d, int k_mode, int k_wbits, int v_mode, int v_wbits, int G);
 cudaError_t launch_prefill(const PrefillLaunch &l, cudaStream_t s);

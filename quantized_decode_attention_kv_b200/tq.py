@@ -17,7 +17,7 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtq.so")
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA = 0, 1, 2, 3, 4
-TQ_MSE, TQ_PROD = 0, 1
+TQ_MSE, TQ_PROD, TQ_E2M1 = 0, 1, 2
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 _DTYPES = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.float16: TQ_F16}

@@ -71,7 +71,7 @@ def compare_records(cache: tq.TQCache, side: str, recs, t_offset: int = 0, heads
     ``heads`` lists the (b, h) of each record; by default records cover every (b, h) in
     row-major order."""
     H = cache.Hkv
-    wbits = recs[0].bits if recs[0].mode == O.MSE else recs[0].bits - 1
+    wbits = recs[0].bits - 1 if recs[0].mode == O.PROD else recs[0].bits
     d = recs[0].d
     codes_dev = _Lazy(cache[f"{side}_codes"]) if cache[f"{side}_codes"] is not None else None
     norm_dev = _Lazy(cache[f"{side}_norm"], np.float16)

@@ -128,6 +128,10 @@ def test_device_entry_points_validate_before_launch():
     assert lib.tq_quantize_kv(P, P, 1, 4, 0, ref(bad_d), None) == tq.TQ_ERR_UNSUPPORTED
     bad_bits = _cache(kc=tq.tq_qcfg(5, 0, 0))
     assert lib.tq_quantize_kv(P, P, 1, 4, 0, ref(bad_bits), None) == tq.TQ_ERR_UNSUPPORTED
+    e2m1_3bit = _cache(kc=tq.tq_qcfg(3, tq.TQ_E2M1, 0))  # E2M1 codes are 4 bits
+    assert lib.tq_quantize_kv(P, P, 1, 4, 0, ref(e2m1_3bit), None) == tq.TQ_ERR_UNSUPPORTED
+    assert "TQ_E2M1" in tq.last_error()
+    assert tq.tq_record_bytes(128, 4, tq.TQ_E2M1) == tq.tq_record_bytes(128, 4, tq.TQ_MSE) == 66
     prod_missing = _cache(kc=tq.tq_qcfg(2, 1, 0))
     assert lib.tq_quantize_kv(P, P, 1, 4, 0, ref(prod_missing), None) == tq.TQ_ERR_INVALID_ARG
     assert "TQ_PROD" in tq.last_error()
