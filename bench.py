@@ -537,7 +537,8 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
 def measure_prefill(tq, torch, stream):
     """Chunked prefill attention over the compressed cache at long contexts (the
     Llama-3.1-8B shape, batch 4): a chunk of 1024 queries at the end of a 64K-token cache
-    (4-bit keys, 2-bit values) and of a 128K-token cache (3-bit keys and values). The roofline is
+    (4-bit keys, 2-bit values; also with the keys on the E2M1 grid) and of a 128K-token cache
+    (3-bit keys and values). The roofline is
     the tensor cores': algorithmic FLOPs 4 d per (query row, visible key) against the measured
     dense bf16 peak."""
     import dataclasses
@@ -545,11 +546,13 @@ def measure_prefill(tq, torch, stream):
     from quantized_decode_attention_kv_b200.workloads import WORKLOADS, make_inputs
     pk = tensor_peak()
     res = {}
-    for label, name, T in (("64k", "llama3_8b_decode_32k", 65536), ("128k", "llama3_8b_128k_3bit", 131072)):
+    for label, name, T, kmode in (("64k", "llama3_8b_decode_32k", 65536, tq.TQ_MSE),
+                                  ("128k", "llama3_8b_128k_3bit", 131072, tq.TQ_MSE),
+                                  ("64k_e2m1_keys", "llama3_8b_decode_32k", 65536, tq.TQ_E2M1)):
         w = dataclasses.replace(WORKLOADS[name], B=4, T=T)
         Lq, t0 = 1024, T - 1024
         K, V, _ = make_inputs(w, device="cuda")
-        cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, seed=w.seed)
+        cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, kmode, tq.TQ_MSE, seed=w.seed)
         tq.tq_quantize_kv(K, V, cache, stream=stream)
         del K, V
         g = torch.Generator(device="cuda").manual_seed(77)
@@ -560,7 +563,8 @@ def measure_prefill(tq, torch, stream):
         flops = w.B * w.Hq * 4 * w.d * (Lq * t0 + Lq * (Lq + 1) // 2)
         tf = flops / ts / 1e12
         res[label] = {"shape": f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d}, cache {T} positions, chunk Lq={Lq} at t0={t0}",
-                      "k": f"{w.k_bits}-bit MSE", "v": f"{w.v_bits}-bit MSE", "us": ts * 1e6,
+                      "k": f"{w.k_bits}-bit " + ("E2M1 (score MMAs on E2M1 operands)" if kmode == tq.TQ_E2M1 else "MSE"),
+                      "v": f"{w.v_bits}-bit MSE", "us": ts * 1e6,
                       "tflops": tf, "peak_tflops": pk[0], "frac": tf / pk[0], "peak_source": pk[1],
                       "flops": flops, "flop_count": "4 d per (query row, visible cached key): q.k and p.v"}
         del cache, q, out

@@ -277,8 +277,11 @@ int tq_decode_attention_paged(const void *q, int dtype, int Hq, const int *T_len
  * hq / (Hq / Hkv). out [B][Lq][Hq][d] float32 (device, caller-owned). The arithmetic is that
  * of the decode call (scores from 16-bit fixed-point centroids and 24-bit fixed-point queries
  * on int8 tensor cores, softmax in fp32, P.V with fp16 weights times ||v|| and fp32
- * accumulation). No workspace. Supported: d = 128, TurboQuant_mse keys of 3 or 4 bits and
- * values of 2..4 bits, Hq / Hkv dividing 128; other configurations return TQ_ERR_UNSUPPORTED.
+ * accumulation). Keys on the E2M1 grid (TQ_E2M1) enter the score MMAs as E2M1 operands
+ * (tcgen05 kind::f8f6f4) against the query as the sum of four E4M3 parts ("Where This Fits in
+ * the Inference Stack", Blackwell FP4), within the same 2e-3 bar. No workspace. Supported:
+ * d = 128, TurboQuant_mse keys of 3 or 4 bits or TQ_E2M1 keys, values of 2..4 bits, Hq / Hkv
+ * dividing 128; other configurations return TQ_ERR_UNSUPPORTED.
  * Errors: TQ_ERR_INVALID_ARG (pointers, shapes, t0 + Lq > T_cap), TQ_ERR_CUDA. */
 int tq_prefill_attention(const void *q, int dtype, int Hq, int Lq, int t0, float scale,
                          const tq_cache *cache, float *out, void *stream);
