@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--no-side", action="store_true", help="skip side measurements")
     ap.add_argument("--T", type=int, default=0,
                     help="override the context length (profiling runs on smaller cases)")
+    ap.add_argument("--paged-case", type=int, default=0,
+                    help="T: run the Llama-3.1-8B-shaped decode (batch 16, K4/V2) over a T-position paged "
+                         "cache (64-position pages, seeded scatter) twice and exit (profiling)")
     ap.add_argument("--prefill-case", default="",
                     help="T,Lq: run one prefill chunk of Lq queries at the end of a T-position cache "
                          "(Llama-3.1-8B shape, batch 4, 4-bit keys, 2-bit values) and exit (profiling)")
@@ -442,9 +445,15 @@ def side_measurements(args, w, tq, torch, K, V, q, cache, out, ws, k_new, v_new,
         wsp = tq.workspace(tq.tq_decode_paged_workspace_bytes(pc, w.Hq, lens))
         pgs = _time(lambda: tq.tq_decode_attention_paged(q, pc, lens, w.scale, out, wsp, stream=stream),
                     stream, torch)
+        # the dense layout through the same per-sequence-length call, for comparison
+        wsd = tq.workspace(tq.tq_decode_varlen_workspace_bytes(cache, w.Hq, lens))
+        dvs = _time(lambda: tq.tq_decode_attention_varlen(q, cache, lens, w.scale, out, wsd, stream=stream),
+                    stream, torch)
         res["paged"] = {"us": pgs * 1e6, "gbs": packed / pgs / 1e9, "frac": packed / pgs / 1e9 / hbm,
                         "page_size": page, "layout": f"{npages} pages of {page} positions, scattered by a "
-                                                     f"seeded permutation; every sequence at full length"}
+                                                     f"seeded permutation; every sequence at full length",
+                        "dense_varlen_us": dvs * 1e6}
+        del wsd
         del pc, bt, wsp
     # the pages' 3.5-bit operating point (4-bit keys, 3-bit values) on the same inputs
     if w.d == 128 and w.k_mode == 0 and w.v_mode == 0 and (w.k_bits, w.v_bits) != (4, 3):
@@ -740,8 +749,36 @@ def run_prefill_case(spec: str):
     print(json.dumps({"prefill_case": spec, "out_finite": bool(torch.isfinite(out).all())}))
 
 
+def run_paged_case(T: int):
+    """Two paged decode calls on a stated case, for profilers (no timing, no JSON line)."""
+    import dataclasses
+
+    import torch
+
+    from quantized_decode_attention_kv_b200 import tq
+    from quantized_decode_attention_kv_b200.workloads import WORKLOADS, make_inputs
+    w = dataclasses.replace(WORKLOADS[DEFAULT_WORKLOAD], T=T)
+    K, V, q = make_inputs(w, device="cuda")
+    page = 64
+    maxp = (T + page - 1) // page
+    bt = torch.randperm(w.B * maxp, generator=torch.Generator().manual_seed(4321)).to(torch.int32)
+    pc = tq.TQPagedCache(w.B, w.Hkv, w.d, page, w.B * maxp, maxp, w.k_bits, w.v_bits,
+                         bt.reshape(w.B, maxp).cuda(), seed=w.seed)
+    tq.tq_quantize_kv_paged(K, V, pc, 0)
+    lens = [T] * w.B
+    out = torch.empty(w.B, w.Hq, w.d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_paged_workspace_bytes(pc, w.Hq, lens))
+    for _ in range(2):
+        tq.tq_decode_attention_paged(q, pc, lens, w.scale, out, ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"paged_case": T, "out_finite": bool(torch.isfinite(out).all())}))
+
+
 def main():
     args = parse_args()
+    if args.paged_case:
+        run_paged_case(args.paged_case)
+        return
     if args.prefill_case:
         run_prefill_case(args.prefill_case)
         return

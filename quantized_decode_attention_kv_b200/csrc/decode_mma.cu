@@ -910,6 +910,9 @@ cudaError_t launch_fast_decode(const DecodeArgs &a, cudaStream_t s) {
       vl.blen[b] = a.T_lens[b];
       vl.boff[b + 1] = vl.boff[b] + a.Hkv * ((a.T_lens[b] + 15) / 16);
     }
+    // the ragged tile space ends at boff[B]: the last CTA's range stops there (past it lies no
+    // (sequence, KV head), and its records, queries and block-table entries are out of bounds)
+    f.total_tiles = vl.boff[a.B];
     vlp = &vl;
   }
   const int kb = a.k.wbits, vb = a.v.wbits;
