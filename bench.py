@@ -51,8 +51,9 @@ def parse_args():
                     help="T: run the Llama-3.1-8B-shaped decode (batch 16, K4/V2) over a T-position paged "
                          "cache (64-position pages, seeded scatter) twice and exit (profiling)")
     ap.add_argument("--prefill-case", default="",
-                    help="T,Lq: run one prefill chunk of Lq queries at the end of a T-position cache "
-                         "(Llama-3.1-8B shape, batch 4, 4-bit keys, 2-bit values) and exit (profiling)")
+                    help="T,Lq[,e2m1]: run one prefill chunk of Lq queries at the end of a T-position cache "
+                         "(Llama-3.1-8B shape, batch 4, 4-bit keys (Lloyd-Max, or E2M1 with ',e2m1'), "
+                         "2-bit values) and exit (profiling)")
     return ap.parse_args()
 
 
@@ -735,10 +736,12 @@ def run_prefill_case(spec: str):
 
     from quantized_decode_attention_kv_b200 import tq
     from quantized_decode_attention_kv_b200.workloads import WORKLOADS, make_inputs
-    T, Lq = (int(x) for x in spec.split(","))
+    parts = spec.split(",")
+    T, Lq = int(parts[0]), int(parts[1])
+    kmode = tq.TQ_E2M1 if len(parts) > 2 and parts[2] == "e2m1" else tq.TQ_MSE
     w = dataclasses.replace(WORKLOADS[DEFAULT_WORKLOAD], B=4, T=T)
     K, V, _ = make_inputs(w, device="cuda")
-    cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, seed=w.seed)
+    cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, kmode, tq.TQ_MSE, seed=w.seed)
     tq.tq_quantize_kv(K, V, cache)
     q = torch.randn(w.B, Lq, w.Hq, w.d, generator=torch.Generator(device="cuda").manual_seed(77),
                     device="cuda").to(torch.bfloat16)
