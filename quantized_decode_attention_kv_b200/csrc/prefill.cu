@@ -50,13 +50,19 @@ constexpr int kSWp = 8, kPWp = 4;            // softmax warps (two per row: half
 constexpr int kWarpMMAp = kSWp + kPWp;       // the MMA warp
 constexpr int kThreadsP = (kSWp + kPWp + 1) * 32;
 constexpr long long kWaitCyclesP = 1ll << 31; // about a second
-// Score stages: three int32 columns per token (the int8 parts), or one fp32 column per token
-// when the keys are E2M1 (F4); two stages, then the 128 fp32 output columns.
+// TMEM columns. Int8 scores: two score stages of three int32 columns per token, then the 128
+// fp32 output columns (512 in all). E2M1 keys (F4): one fp32 score column per token leaves
+// room for the MMAs' A operands: the four E4M3 query parts (32 columns each: 4 bytes of a row
+// per column), two score stages, two P' buffers (fp16 pairs: 32 columns per 64 tokens), then
+// the output columns.
 template <bool F4>
 struct PfTmem {
-  static constexpr uint32_t S = F4 ? kKT : 3 * kKT;  // one score stage
-  static constexpr uint32_t O = 2 * S;               // first output column
-  static constexpr uint32_t alloc = F4 ? 256 : 512;
+  static constexpr uint32_t Q = 0;                          // F4: query parts
+  static constexpr uint32_t S0 = F4 ? 128 : 0;              // first score stage
+  static constexpr uint32_t S = F4 ? kKT : 3 * kKT;         // one score stage
+  static constexpr uint32_t P = S0 + 2 * S;                 // F4: P' buffers
+  static constexpr uint32_t O = F4 ? P + 2 * (kKT / 2) : 2 * S; // first output column
+  static constexpr uint32_t alloc = 512;
 };
 constexpr int kQParts4 = 4; // E4M3 parts of the query (F4): about 16 significant bits
 
@@ -152,6 +158,7 @@ template <int KB, int VB, bool F4>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs a) {
   using L = PfLayout<KB, VB, F4>;
   constexpr uint32_t kSCols = PfTmem<F4>::S, kOCol = PfTmem<F4>::O, kTmemColsP = PfTmem<F4>::alloc;
+  constexpr uint32_t kS0 = PfTmem<F4>::S0, kPCol = PfTmem<F4>::P, kQCol = PfTmem<F4>::Q;
   constexpr int KR = KB * 16, VR = VB * 16; // record bytes
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
@@ -318,7 +325,27 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       for (int x = 0; x < 2; ++x)
 #pragma unroll
         for (int t = 0; t < 3; ++t)
-          tc::tmem_fill32x32_x32(tbase + lrow + x * kSCols + kKT * t + 32 * hf, static_cast<uint32_t>(kMagic));
+          tc::tmem_fill32x32_x32(tbase + lrow + (kS0 + x * kSCols) + kKT * t + 32 * hf, static_cast<uint32_t>(kMagic));
+      tc::tmem_wait_st();
+    } else {
+      // the query parts move from their shared-memory staging (written above by the warp pair,
+      // one warp per row) into tensor memory, each thread its own row: parts 2 hf, 2 hf + 1
+      pair_sync();
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {
+        const int part = 2 * hf + pp;
+        const uint8_t *src = sm + L::oQ + part * (kRows * 128) + (row & 7) * 16 + (row >> 3) * 1024;
+        uint32_t qw32[32];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(src + g * 128);
+          qw32[4 * g] = v.x;
+          qw32[4 * g + 1] = v.y;
+          qw32[4 * g + 2] = v.z;
+          qw32[4 * g + 3] = v.w;
+        }
+        tc::tmem_st32x32_x32(tbase + lrow + kQCol + 32 * part, qw32);
+      }
       tc::tmem_wait_st();
     }
     tc::fence_before_sync();
@@ -339,7 +366,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       tc::fence_after_sync();
       // warp-uniform: some row of the warp sees only part of its half tile (the causal diagonal)
       const bool edge = tb + kH - 1 > pos_lo;
-      const uint32_t st = tbase + lrow + x * kSCols + kH * hf;
+      const uint32_t st = tbase + lrow + (kS0 + x * kSCols) + kH * hf;
       const float4 *kn4 = reinterpret_cast<const float4 *>(knb + x * kKT + kH * hf);
       float s[kH];
       if constexpr (F4) {
@@ -432,11 +459,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
       if (lane == 0) tc::mbar_arrive(S_free(x));
       // P' buffer x was last read by P.V of tile j - 2, complete once S_full(j) arrived (the MMA
       // thread commits S_full(j) after issuing it); this warp's tokens are k chunks 4 hf .. 4 hf + 3
-      uint8_t *pdst = sm + L::oP + x * (kRows * kKT * 2) + (row & 7) * 16 + (row >> 3) * 1024 + hf * 512;
+      if constexpr (F4) {
+        // P' into its TMEM buffer (the A operand of P.V): 16 columns of fp16 pairs per half tile
+        tc::tmem_st32x32_x16(tbase + lrow + kPCol + x * (kKT / 2) + (kH / 2) * hf, pw);
+      } else {
+        uint8_t *pdst = sm + L::oP + x * (kRows * kKT * 2) + (row & 7) * 16 + (row >> 3) * 1024 + hf * 512;
 #pragma unroll
-      for (int c = 0; c < kH / 8; ++c)
-        *reinterpret_cast<uint4 *>(pdst + c * 128) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-      tc::fence_async_smem();
+        for (int c = 0; c < kH / 8; ++c)
+          *reinterpret_cast<uint4 *>(pdst + c * 128) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+        tc::fence_async_smem();
+      }
       // the TMEM loads and stores are warp-collective (.sync.aligned), so the whole warp takes
       // this path when any of its rows needs it, the others with factor 1
       if (j > 0 && __any_sync(0xffffffffu, moved)) {
@@ -456,6 +488,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
         }
         tc::tmem_wait_st();
       }
+      if constexpr (F4) tc::tmem_wait_st(); // P' has landed in tensor memory
       tc::fence_before_sync();
       tc::mbar_arrive(P_full(x));
     }
@@ -648,10 +681,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
         if (*dead) return;
         tc::fence_after_sync();
 #pragma unroll
-        for (int s = 0; s < kKT / 16; ++s)
-          tc::mma_ss(tbase + kOCol, tc::desc_kmajor(sb + L::oP + x * (kRows * kKT * 2) + 256 * s, 128, 1024),
-                     tc::desc_kmajor(sb + L::oV + x * (kKT * 256) + 256 * s, 128, 1024), id_o,
-                     (jj > 0 || s > 0) ? 1u : 0u);
+        for (int s = 0; s < kKT / 16; ++s) {
+          if constexpr (F4)
+            tc::mma_ts_f16(tbase + kOCol, tbase + kPCol + x * (kKT / 2) + 8 * s,
+                           tc::desc_kmajor(sb + L::oV + x * (kKT * 256) + 256 * s, 128, 1024), id_o,
+                           (jj > 0 || s > 0) ? 1u : 0u);
+          else
+            tc::mma_ss(tbase + kOCol, tc::desc_kmajor(sb + L::oP + x * (kRows * kKT * 2) + 256 * s, 128, 1024),
+                       tc::desc_kmajor(sb + L::oV + x * (kKT * 256) + 256 * s, 128, 1024), id_o,
+                       (jj > 0 || s > 0) ? 1u : 0u);
+        }
         tc::commit(V_free(x));
         tc::commit(PV_done);
       };
@@ -669,8 +708,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
           for (int part = 0; part < kQParts4; ++part)
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-              tc::mma_ss_f8f6f4(tbase + x * kSCols,
-                                tc::desc_kmajor(sb + L::oQ + part * (kRows * 128) + 256 * s, 128, 1024),
+              tc::mma_ts_f8f6f4(tbase + (kS0 + x * kSCols), tbase + kQCol + 32 * part + 8 * s,
                                 tc::desc_kmajor(sb + L::oK + x * L::kKStage + 256 * s, 128, 1024), id_s,
                                 (part > 0 || s > 0) ? 1u : 0u);
         } else {
@@ -678,7 +716,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillArgs
           for (int type = 0; type < 3; ++type)
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-              tc::mma_ss_i8(tbase + x * kSCols + kKT * type,
+              tc::mma_ss_i8(tbase + (kS0 + x * kSCols) + kKT * type,
                             tc::desc_kmajor8(sb + L::oQ + type * (kRows * 256) + 256 * s, 128, 2048),
                             tc::desc_kmajor8(sb + L::oK + x * (kKT * 256) + 256 * s, 128, 2048), id_s, 1u);
         }

@@ -154,6 +154,17 @@ __device__ __forceinline__ void mma_ss_f8f6f4(uint32_t d_tmem, uint64_t a, uint6
                : "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(z));
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f8f6f4: A in tensor memory (lane = row, four 8-bit
+// elements of a row per 32-bit column, K = 32 per instruction).
+__device__ __forceinline__ void mma_ts_f8f6f4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                              uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}\n"
+               :
+               : "r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(z));
+}
+
 // Instruction descriptor of kind::f16 with fp32 accumulation, fp16 A (K-major, from TMEM) and
 // fp16 B stored MN-major (N contiguous), M x N tile.
 __host__ __device__ constexpr uint32_t idesc_f16_bmn(int M, int N) {
@@ -219,6 +230,15 @@ __device__ __forceinline__ void tmem_st16x256_x8(uint32_t taddr, const uint32_t 
 __device__ __forceinline__ void tmem_fill32x32_x16(uint32_t taddr, uint32_t x) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
                "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(x)
+               : "memory");
+}
+
+// Warp-wide: thread i writes v[0..15] into 16 consecutive columns of TMEM lane (lane base + i).
+__device__ __forceinline__ void tmem_st32x32_x16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+               "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+               "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
                : "memory");
 }
 
