@@ -76,3 +76,43 @@ def test_full_size_bf16_boundary_layer():
         want = O.gqa_decode(P.to_np(q[b:b + 1, h * G:(h + 1) * G]), P.to_np(K[b:b + 1, h:h + 1]),
                             P.to_np(V[b:b + 1, h:h + 1]), w.scale)
         P.assert_attention_close(P.to_np(out[b:b + 1, h * G:(h + 1) * G]), want)
+
+
+@pytest.mark.parametrize("name,T,kmode", [
+    ("llama3_8b_decode_32k", 65536, tq.TQ_MSE),    # the bench's 64K prefill chunk (K4/V2)
+    ("llama3_8b_128k_3bit", 131072, tq.TQ_MSE),    # the bench's 128K prefill chunk (K3/V3)
+    ("llama3_8b_decode_32k", 65536, tq.TQ_E2M1),   # 64K with keys on the E2M1 grid
+])
+def test_full_size_prefill_sampled_parity(name, T, kmode):
+    # the chunk bench.py times: batch 4, 1024 queries at the end of the cache; sampled
+    # (batch, KV head) slices: records against the oracle, and the first and last query rows of
+    # the slice's query heads against the oracle's causal attention over its dequantised records
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS[name], B=4, T=T)
+    Lq, t0 = 1024, T - 1024
+    K, V, _ = make_inputs(w, device="cuda")
+    cache = tq.TQCache(w.B, w.Hkv, w.T, w.d, w.k_bits, w.v_bits, kmode, tq.TQ_MSE, seed=w.seed)
+    tq.tq_quantize_kv(K, V, cache)
+    q = torch.randn(w.B, Lq, w.Hq, w.d, generator=torch.Generator(device="cuda").manual_seed(77),
+                    device="cuda").to(torch.bfloat16)
+    out = torch.empty(w.B, Lq, w.Hq, w.d, device="cuda")
+    tq.tq_prefill_attention(q, cache, t0, w.scale, out)
+    torch.cuda.synchronize()
+    assert tq.tq_device_faults() == 0
+    G = w.G
+    for b, h in ((0, 0), (w.B - 1, w.Hkv - 1)):
+        recs = {}
+        for side, X, bits, mode in (("k", K, w.k_bits, O.E2M1 if kmode == tq.TQ_E2M1 else O.MSE),
+                                    ("v", V, w.v_bits, O.MSE)):
+            r = O.quantize(P.to_np(X[b, h]), bits, mode, seed=w.seed)
+            P.compare_records(cache, side, [r], heads=[(b, h)])
+            recs[side] = r
+        # the first and the last 8 query rows of the chunk (each block the oracle's own causal
+        # chunk starting at its position)
+        for i0 in (0, Lq - 8):
+            qs = P.to_np(q[b:b + 1, i0:i0 + 8, h * G:(h + 1) * G])
+            want = O.prefill_compressed(qs, [recs["k"]], [recs["v"]], 1, 1, t0 + i0, w.scale)
+            got = P.to_np(out[b:b + 1, i0:i0 + 8, h * G:(h + 1) * G])
+            P.assert_attention_close(got.reshape(8, G, w.d), want.reshape(8, G, w.d))
+    del K, V, cache
+    torch.cuda.empty_cache()
