@@ -27,9 +27,10 @@
 // Work split: the (batch, KV head, 16-token tile) space is flattened and cut into equal
 // contiguous ranges, one per persistent CTA (12 warps with 2-bit values or 4-bit keys, else
 // 4); within a range each maximal run of one (batch, KV head) is a segment, its tiles dealt
-// round-robin to the warps, each warp keeping its own online-softmax state (log2 domain); at
-// the end of the segment the warps store their rescaled accumulators in their own
-// shared-memory slots, which are summed into one partial record per query head.
+// round-robin to the warps (a paged cache: page-aligned chunks of up to 4 tiles), each warp
+// keeping its own online-softmax state (log2 domain); at the end of the segment the warps
+// store their rescaled accumulators in their own shared-memory slots, which are summed into
+// one partial record per query head.
 #include "decode_mse_common.cuh"
 
 #include <algorithm>
@@ -294,12 +295,9 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
 
       const size_t rec0 = PG ? 0 : static_cast<size_t>(bh) * a.T_cap;
       // paged cache: record index of token t0 (a multiple of 16: a tile never straddles a
-      // page) on a given page, and the page of the warp's tile jj (0 past the segment)
+      // page) on a given page
       [[maybe_unused]] auto page_rec = [&](int page, int t0) -> long long {
         return ((static_cast<long long>(page) * a.Hkv + h) << a.pshift) + (t0 & ((1 << a.pshift) - 1));
-      };
-      [[maybe_unused]] auto page_of = [&](int jj) -> int {
-        return jj < ntiles ? __ldg(a.bt + static_cast<size_t>(b) * a.maxp + (((tile0 + jj) * 16) >> a.pshift)) : 0;
       };
       const int tlast = T_len - 1;
       // word offset of this lane's value run within a record (3-bit runs start mid-word for odd r)
@@ -331,13 +329,6 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
         pfstep = kStep * 2;
       }
       int tpf = tp0;
-      // page pipeline: pages of the warp's next two tiles, looked up two steps ahead of use
-      [[maybe_unused]] int pg_a = 0, pg_b = 0;
-      if constexpr (PG) {
-        static_assert(kPrefetchSteps <= 1, "the page pipeline serves a prefetch one step ahead");
-        pg_a = page_of(warp);
-        pg_b = page_of(warp + kWarps);
-      }
 
       auto load_k = [&](uint32_t (&dst)[KB], const uint8_t *p) {
         if constexpr (KB == 4) {
@@ -356,35 +347,12 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
         for (int k = 0; k < TileT::VW; ++k) dst[k] = __ldcs(reinterpret_cast<const uint32_t *>(p) + k);
       };
 
-      // Full tiles load at fixed offsets from the lane pointers; the ragged last tile of a
-      // (batch, KV head) clamps each token to T_len - 1 (those tokens are masked later).
-      auto load_next = [&](TileT &T) {
-        if (kPrefetchSteps > 0) {
-          if (lane < KL + VL + 2 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16) {
-            if constexpr (PG) {
-              const long long rp = page_rec(pg_b, tpf);
-              pfp = lane < KL ? reinterpret_cast<const char *>(a.kc + rp * KR + 128 * lane)
-                    : lane < KL + VL ? reinterpret_cast<const char *>(a.vc + rp * VR + 128 * (lane - KL))
-                                     : reinterpret_cast<const char *>((lane == KL + VL ? a.kn : a.vn) + rp);
-            }
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
-          }
-          pfp += pfstep;
-          tpf += kWarps * 16;
-        }
-        const int t0 = (tile0 + jl) * 16;
-        [[maybe_unused]] long long rb = 0;
-        if constexpr (PG) {
-          rb = page_rec(pg_a, t0);
-          const int pg_c = page_of(jl + 2 * kWarps);
-          pg_a = pg_b;
-          pg_b = pg_c;
-          kp = a.kc + (rb + r) * KR + 4 * KB * c;
-          vp = a.vc + (rb + c) * VR + 4 * vwo;
-          knp = a.kn + rb + r;
-          vnp = a.vn + rb + r;
-        }
+      // One tile from the lane pointers: full tiles load at fixed offsets from them; the ragged
+      // last tile of a (batch, KV head) clamps each token to T_len - 1 (those tokens are masked
+      // later).
+      auto load_tile = [&](TileT &T, int t0) {
         if (t0 + 16 <= T_len) {
+
           load_k(T.k[0], kp);
           load_k(T.k[1], kp + 8 * KR);
           load_v(T.v[0], vp);
@@ -397,7 +365,7 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           T.vn[1] = __ldcs(vnp + 8);
         } else {
           // record of token t (within this tile, so within one page) = base + t
-          const long long base = PG ? rb - t0 : static_cast<long long>(rec0);
+          const long long base = PG ? (knp - a.kn) - r - t0 : static_cast<long long>(rec0);
           const long long tr = base + min(t0 + r, tlast), tr8 = base + min(t0 + r + 8, tlast);
           const uint8_t *kb = a.kc + 4 * KB * c;
           load_k(T.k[0], kb + tr * KR);
@@ -413,6 +381,18 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
           T.vn[0] = __ldcs(a.vn + tr);
           T.vn[1] = __ldcs(a.vn + tr8);
         }
+      };
+
+      // the warp's next tile (dense and per-sequence-length walks: every kWarps-th tile)
+      auto load_next = [&](TileT &T) {
+        if (kPrefetchSteps > 0) {
+          if (lane < KL + VL + 2 && tpf + 16 <= T_len && tpf < (tile0 + ntiles) * 16)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(pfp));
+          pfp += pfstep;
+          tpf += kWarps * 16;
+        }
+        const int t0 = (tile0 + jl) * 16;
+        load_tile(T, t0);
         kp += kStep * KR;
         vp += kStep * VR;
         knp += kStep;
@@ -423,12 +403,17 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
       auto compute = [&](const TileT &T, int t0) {
         // ---- scores. A rows r and r + 8 are tokens r and r + 8; k-step s takes the lane's
         //      coordinate pairs 2s (a0: token r, a1: token r + 8) and 2s + 1 (a2, a3), one
-        //      32-bit table load each.
-        int acc[NT + 1][4];
+        //      32-bit table load each. With one score n-tile pair the even and odd k-steps
+        //      accumulate into separate registers (two dependent MMA chains of four instead of
+        //      one of eight), added as integers at the end; with two there is no register room.
+        int acc[NT + 1][4], acc2[NT + 1][4];
 #pragma unroll
         for (int nt = 0; nt <= NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] = kMagic;
+          for (int e = 0; e < 4; ++e) {
+            acc[nt][e] = kMagic;
+            acc2[nt][e] = 0;
+          }
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           uint32_t ad0, ad1, ad2, ad3;
@@ -468,7 +453,14 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
             e3 = lds32_off<0>(ad3);
           }
 #pragma unroll
-          for (int nt = 0; nt <= NT; ++nt) imma16832(acc[nt], e0, e1, e2, e3, qb[nt][2 * s], qb[nt][2 * s + 1]);
+          for (int nt = 0; nt <= NT; ++nt)
+            imma16832((NT == 1 && (s & 1)) ? acc2[nt] : acc[nt], e0, e1, e2, e3, qb[nt][2 * s], qb[nt][2 * s + 1]);
+        }
+        if constexpr (NT == 1) {
+#pragma unroll
+          for (int nt = 0; nt <= NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] += acc2[nt][e];
         }
 
         // ---- online softmax (log2 domain); lane (r, c) owns head 4 nt + c, tokens r, r+8
@@ -606,16 +598,84 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
 
       // Two tile buffers in turn: the next tile loads while the current one computes.
       TileT ta, tb;
-      int jt = warp;
-      if (jl < ntiles) load_next(ta);
-      while (jt < ntiles) {
-        if (jl < ntiles) load_next(tb);
-        compute(ta, (tile0 + jt) * 16);
-        jt += kWarps;
-        if (jt >= ntiles) break;
+      if constexpr (!PG) {
+        int jt = warp;
         if (jl < ntiles) load_next(ta);
-        compute(tb, (tile0 + jt) * 16);
-        jt += kWarps;
+        while (jt < ntiles) {
+          if (jl < ntiles) load_next(tb);
+          compute(ta, (tile0 + jt) * 16);
+          jt += kWarps;
+          if (jt >= ntiles) break;
+          if (jl < ntiles) load_next(ta);
+          compute(tb, (tile0 + jt) * 16);
+          jt += kWarps;
+        }
+      } else {
+        // Paged cache: the segment's tiles are grouped into aligned chunks of ct = min(tiles
+        // per page, 4) tiles, which never straddle a page, and the warps take the chunks in
+        // turn, so the block table and the page arithmetic are visited once per chunk; inside
+        // a chunk the records are consecutive. Pages are looked up two chunks ahead, and each
+        // chunk is prefetched into L2 one chunk ahead.
+        const int lc = min(a.pshift - 4, 2), ct = 1 << lc;
+        const int tend = tile0 + ntiles; // absolute tile end of the segment
+        const int cw = (tile0 >> lc) + warp;
+        const int *btrow = a.bt + static_cast<size_t>(b) * a.maxp;
+        auto chunk_page = [&](int ch) -> int {
+          const int u = ch << lc;
+          return u < tend ? __ldg(btrow + (u >> (a.pshift - 4))) : 0;
+        };
+        auto set_ptrs = [&](int page, int u) {
+          const long long rb = page_rec(page, u * 16);
+          kp = a.kc + (rb + r) * KR + 4 * KB * c;
+          vp = a.vc + (rb + c) * VR + 4 * vwo;
+          knp = a.kn + rb + r;
+          vnp = a.vn + rb + r;
+        };
+        auto prefetch_chunk = [&](int ch, int page) {
+          const int u = ch << lc;
+          if (u >= tend) return;
+          const long long rc = page_rec(page, u * 16);
+          const int kls = ct * KR / 8, vls = ct * VR / 8; // 128-byte lines of the chunk
+          for (int i = lane; i < kls + vls + 2; i += 32) {
+            const char *pp = i < kls ? reinterpret_cast<const char *>(a.kc + rc * KR) + 128 * i
+                             : i < kls + vls ? reinterpret_cast<const char *>(a.vc + rc * VR) + 128 * (i - kls)
+                                             : reinterpret_cast<const char *>((i == kls + vls ? a.kn : a.vn) + rc);
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(pp));
+          }
+        };
+        // the tile after u in the warp's walk
+        auto nxt = [&](int u) { return ((u + 1) & (ct - 1)) ? u + 1 : u + 1 + (kWarps - 1) * ct; };
+        int ul = max(tile0, cw << lc), ut = ul; // next tile to load, next tile to compute
+        int pg_b = chunk_page(cw + kWarps), pg_c = chunk_page(cw + 2 * kWarps);
+        if (ul < tend) set_ptrs(chunk_page(cw), ul);
+        prefetch_chunk(cw + kWarps, pg_b);
+        auto load_pg = [&](TileT &T) {
+          load_tile(T, ul * 16);
+          ul = nxt(ul);
+          if ((ul & (ct - 1)) == 0) {
+            // the next tile starts the warp's next chunk, on page pg_b
+            const int ch = ul >> lc;
+            if (ul < tend) set_ptrs(pg_b, ul);
+            prefetch_chunk(ch + kWarps, pg_c);
+            pg_b = pg_c;
+            pg_c = chunk_page(ch + 2 * kWarps);
+          } else {
+            kp += 16 * KR;
+            vp += 16 * VR;
+            knp += 16;
+            vnp += 16;
+          }
+        };
+        if (ul < tend) load_pg(ta);
+        while (ut < tend) {
+          if (ul < tend) load_pg(tb);
+          compute(ta, ut * 16);
+          ut = nxt(ut);
+          if (ut >= tend) break;
+          if (ul < tend) load_pg(ta);
+          compute(tb, ut * 16);
+          ut = nxt(ut);
+        }
       }
 
       // ---- merge the warps: common max and sum per head, then each warp stores its rescaled

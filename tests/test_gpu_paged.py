@@ -127,7 +127,9 @@ def test_paged_decode_matches_oracle(page_size, G, Hkv, kb, vb):
         want = P.oracle_decode(qn[b:b + 1], k_recs[b * Hkv:(b + 1) * Hkv], v_recs[b * Hkv:(b + 1) * Hkv],
                                1, Hkv, scale, T)
         P.assert_attention_close(on[b:b + 1], want)
-    # the same records in the dense layout give the same outputs
+    # the same records in the dense layout give the same outputs up to rounding: the paged walk
+    # deals page chunks to the warps, so each warp's softmax reference (and with it the fp16
+    # rounding of its weights) can differ from the dense walk's
     dense = tq.TQCache(B, Hkv, T_cap, 128, kb, vb, seed=31)
     P.upload(dense, "k", k_recs)
     P.upload(dense, "v", v_recs)
@@ -135,7 +137,7 @@ def test_paged_decode_matches_oracle(page_size, G, Hkv, kb, vb):
     ws_d = tq.workspace(tq.tq_decode_varlen_workspace_bytes(dense, Hq, T_lens))
     tq.tq_decode_attention_varlen(q.cuda(), dense, T_lens, scale, out_d, ws_d)
     torch.cuda.synchronize()
-    torch.testing.assert_close(out, out_d, rtol=1e-5, atol=1e-6)
+    P.assert_attention_close(P.to_np(out), P.to_np(out_d))
 
 
 @pytest.mark.parametrize("page_size,B,Hkv,T", [

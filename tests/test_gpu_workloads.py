@@ -116,3 +116,49 @@ def test_full_size_prefill_sampled_parity(name, T, kmode):
             P.assert_attention_close(got.reshape(8, G, w.d), want.reshape(8, G, w.d))
     del K, V, cache
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("page,ragged", [(64, False), (16, True), (32, True), (256, True)],
+                         ids=["page64-full", "page16-ragged", "page32-ragged", "page256-ragged"])
+def test_full_size_paged_decode_sampled_parity(page, ragged):
+    # the bench's paged case (Llama-3.1-8B-shaped layer, batch 16, 32K context, pages scattered
+    # over the pool by a seeded permutation) and ragged lengths in [T/4, T] at other page sizes:
+    # every CTA walks many page chunks. The paged call must agree with the dense
+    # per-sequence-length call on the same inputs (the two writers store the same records), and sampled
+    # (batch, KV head) slices must match the oracle over their own lengths.
+    w = WORKLOADS["llama3_8b_decode_32k"]
+    K, V, q = make_inputs(w, device="cuda")
+    if ragged:
+        g = torch.Generator().manual_seed(99 + page)
+        lens = torch.randint(w.T // 4, w.T + 1, (w.B,), generator=g).tolist()
+    else:
+        lens = [w.T] * w.B
+    maxp = (w.T + page - 1) // page
+    npages = w.B * maxp
+    bt = torch.randperm(npages, generator=torch.Generator().manual_seed(4321)).to(torch.int32)
+    pc = tq.TQPagedCache(w.B, w.Hkv, w.d, page, npages, maxp, w.k_bits, w.v_bits,
+                         bt.reshape(w.B, maxp).cuda(), seed=w.seed)
+    tq.tq_quantize_kv_paged(K, V, pc, 0)
+    out = torch.empty(w.B, w.Hq, w.d, device="cuda")
+    ws = tq.workspace(tq.tq_decode_paged_workspace_bytes(pc, w.Hq, lens))
+    tq.tq_decode_attention_paged(q, pc, lens, w.scale, out, ws)
+    dense = _cache_for(w)
+    tq.tq_quantize_kv(K, V, dense)
+    out_d = torch.empty_like(out)
+    ws_d = tq.workspace(tq.tq_decode_varlen_workspace_bytes(dense, w.Hq, lens))
+    tq.tq_decode_attention_varlen(q, dense, lens, w.scale, out_d, ws_d)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    # same records, another assignment of tiles to warps: only rounding differs (each warp's
+    # softmax reference sets the fp16 rounding of its weights)
+    P.assert_attention_close(P.to_np(out), P.to_np(out_d))
+    G = w.G
+    for b, h in ((0, 0), (w.B - 1, w.Hkv - 1)):
+        T = lens[b]
+        recs = {side: O.quantize(P.to_np(X[b, h, :T]), bits, O.MSE, seed=w.seed)
+                for side, X, bits in (("k", K, w.k_bits), ("v", V, w.v_bits))}
+        qs = P.to_np(q[b:b + 1, h * G:(h + 1) * G])
+        want = O.decode_compressed(qs, [recs["k"]], [recs["v"]], 1, 1, w.scale)
+        P.assert_attention_close(P.to_np(out[b:b + 1, h * G:(h + 1) * G]), want)
+    del K, V, pc, dense, ws, ws_d
+    torch.cuda.empty_cache()
