@@ -469,9 +469,12 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
         const float vn0 = f16_bits_to_f32(T.vn[0]);
         const float vn1 = f16_bits_to_f32(T.vn[1]);
         const bool ok0 = t0 + r < T_len, ok1 = t0 + r + 8 < T_len;
-        uint32_t pk[NT];
-        float alpha[NT];
-        bool rescale = false;
+        // The softmax reference of a head moves only when a score of the tile exceeds it: one
+        // vote decides, and only then are the tile's maxima reduced across the row group
+        // (three shuffles) and the accumulators rescaled. Otherwise the weights are taken
+        // against the current reference directly (they are at most 1 either way).
+        float s0[NT], s1[NT];
+        bool over = false;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           // token r: columns 2c (2^24 terms) and 2c + 1 (2^16) in acc 0, 1 of n-tile nt and the
@@ -481,22 +484,24 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
                                 fmaf(__int_as_float(acc[nt][1]), 1.0f / 256.0f, __int_as_float(acc[nt][0]) - kMagicAdj));
           const float d1 = fmaf(__int_as_float(acc[NT][2 + nt]), 1.0f / 65536.0f,
                                 fmaf(__int_as_float(acc[nt][3]), 1.0f / 256.0f, __int_as_float(acc[nt][2]) - kMagicAdj));
-          const float s0 = ok0 ? kn0 * qscale[nt] * d0 : -INFINITY;
-          const float s1 = ok1 ? kn1 * qscale[nt] * d1 : -INFINITY;
-          float mx = fmaxf(s0, s1);
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          const float mn = fmaxf(m_run[nt], mx);
-          alpha[nt] = softmax_exp2(m_run[nt] - mn);
-          rescale |= mn != m_run[nt];
-          m_run[nt] = mn;
-          const float p0 = softmax_exp2(s0 - mn), p1 = softmax_exp2(s1 - mn);
-          l_run[nt] = fmaf(l_run[nt], alpha[nt], p0 + p1);
-          pk[nt] = pack_h2(p0 * vn0, p1 * vn1);
+          s0[nt] = ok0 ? kn0 * qscale[nt] * d0 : -INFINITY;
+          s1[nt] = ok1 ? kn1 * qscale[nt] * d1 : -INFINITY;
+          over |= s0[nt] > m_run[nt] || s1[nt] > m_run[nt];
         }
-        // rescale the value accumulators (lane owns heads 2c, 2c+1) when any max moved
-        if (__any_sync(0xffffffffu, rescale)) {
+        if (__any_sync(0xffffffffu, over)) {
+          float alpha[NT];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            float mx = fmaxf(s0[nt], s1[nt]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mn = fmaxf(m_run[nt], mx);
+            alpha[nt] = softmax_exp2(m_run[nt] - mn);
+            l_run[nt] *= alpha[nt];
+            m_run[nt] = mn;
+          }
+          // rescale the value accumulators (lane owns heads 2c, 2c+1)
           float a0[NT], a1[NT];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
@@ -512,6 +517,13 @@ __global__ void __launch_bounds__(Cfg<KB, VB>::kThreads, Cfg<KB, VB>::kCtas)
             o[m][2] *= al0;
             o[m][3] *= al1;
           }
+        }
+        uint32_t pk[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const float p0 = softmax_exp2(s0[nt] - m_run[nt]), p1 = softmax_exp2(s1[nt] - m_run[nt]);
+          l_run[nt] += p0 + p1;
+          pk[nt] = pack_h2(p0 * vn0, p1 * vn1);
         }
 
         // ---- P'^T as the B operand: lane (r, c) needs head g = r at k rows 2c, 2c+1, 2c+8, 2c+9,
