@@ -371,20 +371,18 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
       const float s0 = ok0 ? kn0 * fmaf(kg0, sk0, code0) * kPLog2e : -INFINITY;
       const float s1 = ok1 ? kn1 * fmaf(kg1, sk1, code1) * kPLog2e : -INFINITY;
 
-      // ---- online softmax (log2 domain) over the lane's head
-      float mx = fmaxf(s0, s1);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const float mn = fmaxf(m_run, mx);
-      const float alpha = softmax_exp2(m_run - mn);
-      const bool moved = mn != m_run;
-      m_run = mn;
-      const float p0 = softmax_exp2(s0 - mn), p1 = softmax_exp2(s1 - mn);
-      l_run = fmaf(l_run, alpha, p0 + p1);
-      const uint32_t pkc = pack_h2(p0 * vn0, p1 * vn1);
-      const uint32_t pks = pack_h2(p0 * vn0 * vg0, p1 * vn1 * vg1);
-      if (__any_sync(0xffffffffu, moved)) {
+      // ---- online softmax (log2 domain) over the lane's head. The reference moves only when a
+      //      score of the tile exceeds it: one vote decides, and only then are the maxima
+      //      reduced across the row group and the accumulators rescaled.
+      if (__any_sync(0xffffffffu, s0 > m_run || s1 > m_run)) {
+        float mx = fmaxf(s0, s1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float mn = fmaxf(m_run, mx);
+        const float alpha = softmax_exp2(m_run - mn);
+        l_run *= alpha;
+        m_run = mn;
         // lane (r, c) accumulates heads 2c, 2c + 1: head 0 lives on lanes c = 0, head 1 on c = 2
         const float al0 = __shfl_sync(0xffffffffu, alpha, lane & ~3);
         const float al1 = __shfl_sync(0xffffffffu, alpha, (lane & ~3) | 2);
@@ -396,6 +394,10 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
           o[m][3] *= al1;
         }
       }
+      const float p0 = softmax_exp2(s0 - m_run), p1 = softmax_exp2(s1 - m_run);
+      l_run += p0 + p1;
+      const uint32_t pkc = pack_h2(p0 * vn0, p1 * vn1);
+      const uint32_t pks = pack_h2(p0 * vn0 * vg0, p1 * vn1 * vg1);
 
       // ---- P' operands (column r = head r): tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1)
       const int srca = 8 * c + 2 * (r & 1), srcb = srca + 4;
@@ -528,6 +530,7 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
     __syncthreads();
 
     float m_run = -INFINITY, l_run = 0.f;
+    float s_code = 0.f, s_sketch = 0.f; // the lane's running sums of P' (code rows, sketch rows)
     float o[8][4];
 #pragma unroll
     for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
@@ -613,14 +616,18 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
       }
       const float kn = f16_bits_to_f32(T.kn), kg = f16_bits_to_f32(T.kg);
       const float s = t0 + lane < te ? kn * (csum + sc + kg * (ssum + sk)) * kPLog2e : -INFINITY;
-      // ---- online softmax over the 32 tokens of the group (one head: the max is warp-uniform)
-      float mx = s;
+      // ---- online softmax over the 32 tokens of the group (one head: the reference is
+      //      warp-uniform); the group's maximum is reduced only when a vote finds a score above
+      //      the reference
+      if (__any_sync(0xffffffffu, s > m_run)) {
+        float mx = s;
 #pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
-      const float mn = fmaxf(m_run, mx);
-      if (mn != m_run) {
+        for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+        const float mn = fmaxf(m_run, mx);
         const float alpha = softmax_exp2(m_run - mn);
         l_run *= alpha;
+        s_code *= alpha;
+        s_sketch *= alpha;
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
           o[m][0] *= alpha;
@@ -630,30 +637,54 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
         }
         m_run = mn;
       }
-      const float pr = softmax_exp2(s - mn);
+      const float pr = softmax_exp2(s - m_run);
       l_run += pr;
       const float vn = f16_bits_to_f32(T.vn), vg = f16_bits_to_f32(T.vg);
       const uint32_t pk = pack_h2(pr * vn, pr * vn * vg); // (code rows, sketch rows)
 
-      // ---- values: two 16-token MMA groups; P' column 0 = the head (other columns zero)
+      // ---- values: two 16-token MMA groups; P' column 0 = the head (other columns zero).
+      //      The operand is the record bit itself, not a +-1 factor: an A register masks bit p of
+      //      both halves of the byte-pair word, which is the fp16 value 2^(p-24) where the bit is
+      //      set (an exact subnormal) and 0 where it is clear. The group's two MMAs start from
+      //      zero, so M = 2^(p-24) sum_t b_t P'_t is small and exact up to the fp32 sum, and the
+      //      accumulator takes -2^(25-p) M = -2 sum_t b_t P'_t; the running sums of P' (code and
+      //      sketch rows) supply the sum_t P'_t of sum_t P'_t (1 - 2 b_t) at the merge.
+      s_code += __low2float(*reinterpret_cast<const __half2 *>(&pk));
+      s_sketch += __high2float(*reinterpret_cast<const __half2 *>(&pk));
+      uint32_t pbc[2][2], pbs[2][2], xm[2][2], xq[2][2];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int base = 16 * hh + 2 * c;
         const uint32_t x0 = __shfl_sync(0xffffffffu, pk, base), x1 = __shfl_sync(0xffffffffu, pk, base + 1);
         const uint32_t x8 = __shfl_sync(0xffffffffu, pk, base + 8), x9 = __shfl_sync(0xffffffffu, pk, base + 9);
-        uint32_t pbc0 = prmt(x0, x1, 0x5410u), pbc1 = prmt(x8, x9, 0x5410u);
-        uint32_t pbs0 = prmt(x0, x1, 0x7632u), pbs1 = prmt(x8, x9, 0x7632u);
-        if (r != 0) pbc0 = pbc1 = pbs0 = pbs1 = 0u;
-        const uint32_t xm0 = prmt(T.vm[hh][0], T.vm[hh][1], selx), xm1 = prmt(T.vm[hh][2], T.vm[hh][3], selx);
-        const uint32_t xq0 = prmt(T.vq[hh][0], T.vq[hh][1], selx), xq1 = prmt(T.vq[hh][2], T.vq[hh][3], selx);
+        pbc[hh][0] = r == 0 ? prmt(x0, x1, 0x5410u) : 0u;
+        pbc[hh][1] = r == 0 ? prmt(x8, x9, 0x5410u) : 0u;
+        pbs[hh][0] = r == 0 ? prmt(x0, x1, 0x7632u) : 0u;
+        pbs[hh][1] = r == 0 ? prmt(x8, x9, 0x7632u) : 0u;
+        xm[hh][0] = prmt(T.vm[hh][0], T.vm[hh][1], selx);
+        xm[hh][1] = prmt(T.vm[hh][2], T.vm[hh][3], selx);
+        xq[hh][0] = prmt(T.vq[hh][0], T.vq[hh][1], selx);
+        xq[hh][1] = prmt(T.vq[hh][2], T.vq[hh][3], selx);
+      }
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int sh0 = 15 - 2 * m, sh1 = 14 - 2 * m;
-          mma16816(o[m], pm1(xm0, sh0, one2), pm1(xm0, sh1, one2), pm1(xm1, sh0, one2),
-                   pm1(xm1, sh1, one2), pbc0, pbc1);
-          mma16816(o[4 + m], pm1(xq0, sh0, one2), pm1(xq0, sh1, one2), pm1(xq1, sh0, one2),
-                   pm1(xq1, sh1, one2), pbs0, pbs1);
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t mk0 = 0x10001u << (2 * m), mk1 = 0x10001u << (2 * m + 1);
+        float mc[4] = {0.f, 0.f, 0.f, 0.f}, ms[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          mma16816(mc, xm[hh][0] & mk0, xm[hh][0] & mk1, xm[hh][1] & mk0, xm[hh][1] & mk1, pbc[hh][0], pbc[hh][1]);
+          mma16816(ms, xq[hh][0] & mk0, xq[hh][0] & mk1, xq[hh][1] & mk0, xq[hh][1] & mk1, pbs[hh][0], pbs[hh][1]);
         }
+        // rows r (bit 2m) and r + 8 (bit 2m + 1)
+        const float c0 = -static_cast<float>(1 << (25 - 2 * m)), c1 = -static_cast<float>(1 << (24 - 2 * m));
+        o[m][0] = fmaf(mc[0], c0, o[m][0]);
+        o[m][1] = fmaf(mc[1], c0, o[m][1]);
+        o[m][2] = fmaf(mc[2], c1, o[m][2]);
+        o[m][3] = fmaf(mc[3], c1, o[m][3]);
+        o[4 + m][0] = fmaf(ms[0], c0, o[4 + m][0]);
+        o[4 + m][1] = fmaf(ms[1], c0, o[4 + m][1]);
+        o[4 + m][2] = fmaf(ms[2], c1, o[4 + m][2]);
+        o[4 + m][3] = fmaf(ms[3], c1, o[4 + m][3]);
       }
     };
 
@@ -670,10 +701,15 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
       jt += kPW;
     }
 
-    // ---- merge the warps (one head)
+    // ---- merge the warps (one head); a row's value is sum_t P'_t (1 - 2 b_t) = (the sum of
+    //      P' over the warp's tokens) + the accumulator
     float l = l_run;
 #pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o2);
+    for (int o2 = 16; o2 > 0; o2 >>= 1) {
+      l += __shfl_xor_sync(0xffffffffu, l, o2);
+      s_code += __shfl_xor_sync(0xffffffffu, s_code, o2);
+      s_sketch += __shfl_xor_sync(0xffffffffu, s_sketch, o2);
+    }
     if (lane == 0) mst[warp] = m_run;
     for (int idx = tid; idx < kPD + kPM; idx += kPThreads) obuf[idx] = 0.f;
     if (tid == 0) lsum = 0.f;
@@ -690,8 +726,9 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_lut_kernel(const Pro
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         const int i0 = (m < 4 ? 0 : kPD) + 8 * r + 2 * (m & 3);
-        atomicAdd(&obuf[i0], o[m][0] * f);
-        atomicAdd(&obuf[i0 + 1], o[m][2] * f);
+        const float sp = m < 4 ? s_code : s_sketch;
+        atomicAdd(&obuf[i0], (sp + o[m][0]) * f);
+        atomicAdd(&obuf[i0 + 1], (sp + o[m][2]) * f);
       }
     }
     __syncthreads();
