@@ -19,7 +19,9 @@
 //           u' = -c1 u (the codes' centroids), adds sqrt(d) sqrt(pi/2)/m S^T w, applies the
 //           inverse rotation D H / d once and divides by the softmax sum.
 //
-// The work split, online softmax and partial records follow the MSE tensor-core kernel.
+// The work split, online softmax and partial records follow the MSE tensor-core kernel. The
+// one-query-head kernel below scores on the CUDA cores instead and feeds the value MMAs the
+// masked record bits (0 or an exact fp16 subnormal) with the sum of P' added back at the merge.
 #include "mma_ops.cuh"
 
 #include <algorithm>
@@ -482,7 +484,8 @@ __global__ void __launch_bounds__(kPThreads, 3) decode_prod_kernel(const ProdArg
 // one query with 128 +-1 factors, so it is computed on the CUDA cores, one token per lane, from
 // per-query tables T_p[byte] = -2 * (sum of the values of the set bits of byte p of a record):
 // sum_k v_k (1 - 2 bit_k) = sum_k v_k + sum_p T_p[byte_p], 16 table reads per token instead of
-// an MMA whose score columns would be 3/4 empty. The values keep the tensor-core path above.
+// an MMA whose score columns would be 3/4 empty. The values stay on the tensor cores, with the
+// record bits themselves (not +-1 factors) as the A operand, one mask per register (below).
 struct LutTile {
   uint2 kc, ks;                // key codes and sketch of token `lane` of the group
   uint16_t kn, kg, vn, vg;     // its norms
