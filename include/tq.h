@@ -168,7 +168,9 @@ int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
  * Inference Stack", TensorRT-LLM section: flash-decoding splits the context); the partial
  * records of those splits live in this caller-owned workspace, since the library never
  * allocates. B is the batch, Hq the query heads, T_len the attended positions. 0 if
- * invalid. Depends on the current device's SM count. */
+ * invalid. Depends on the current device's SM count. The plain sizes come first and the
+ * cache last (rather than the cache before T_len): B must equal cache->B, and the call reads
+ * only the cache's shape and bit widths. */
 size_t tq_decode_workspace_bytes(int B, int Hq, int T_len, const tq_cache *cache);
 
 /* Decode attention over cache positions [0, T_len) of every (b, KV head) ("Where This
