@@ -775,6 +775,7 @@ __global__ void __launch_bounds__(128) combine_fast_kernel(const float *part, in
   const int Hq = Hkv * G;
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5); // (b, q-head) of this warp
   pdl_wait(); // the partials come from the decode kernel
+  pdl_trigger(); // the next kernel's prologue may overlap this one (it waits for its end)
   if (gw >= B * Hq) return;
   const int b = gw / Hq, hq = gw - b * Hq;
   const int h = hq / G, g = hq - h * G;
