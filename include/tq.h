@@ -156,9 +156,10 @@ size_t tq_record_bytes(int d, tq_qcfg c);
 /* Quantise-on-write ("Closing", Steps 1-3). K and V are device arrays [B][Hkv][T][d] of
  * `dtype` (TQ_F32 / TQ_BF16 / TQ_F16); either may be NULL to write only the other. Token t
  * is stored at cache position t_offset + t (0 <= t_offset, t_offset + T <= T_cap). T = 0
- * is a no-op. Per vector: n = ||x|| (fp32, stored fp16); z = H D x / n; codes by the
- * boundary count (fp32 decisions); PROD: r = (z - c[code]) / sqrt(d), rnorm = ||r||,
- * QJL bits of S r. A zero vector stores norm 0 (its reconstruction is 0). */
+ * is a no-op. Per vector: n = ||x|| (fp32, stored fp16, rounded to nearest: a norm of 65520
+ * or more is stored as +inf, and attention over such a record is not finite); z = H D x / n;
+ * codes by the boundary count (fp32 decisions); PROD: r = (z - c[code]) / sqrt(d),
+ * rnorm = ||r||, QJL bits of S r. A zero vector stores norm 0 (its reconstruction is 0). */
 int tq_quantize_kv(const void *K, const void *V, int dtype, int T, int t_offset,
                    const tq_cache *cache, void *stream);
 

@@ -338,8 +338,10 @@ def record_bytes(d: int, bits: int, mode: int, m: int | None = None) -> int:
 
 
 def _fp16_of(v: np.ndarray) -> np.ndarray:
-    """Round a float64 value to float32 then float16 (both round-to-nearest-even)."""
-    return np.asarray(v, dtype=np.float64).astype(np.float32).astype(np.float16)
+    """Round a float64 value to float32 then float16 (both round-to-nearest-even); values at or
+    above 65520 in magnitude become infinite, as IEEE rounding prescribes."""
+    with np.errstate(over="ignore"):
+        return np.asarray(v, dtype=np.float64).astype(np.float32).astype(np.float16)
 
 
 # ----------------------------------------------------------------------------------------

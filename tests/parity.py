@@ -53,16 +53,18 @@ def upload(cache: tq.TQCache, side: str, recs, t_offset: int = 0) -> None:
 
 
 def _fp16_ambiguous(exact: np.ndarray) -> np.ndarray:
-    lo = (exact * (1 - 1e-5)).astype(np.float32).astype(np.float16)
-    hi = (exact * (1 + 1e-5)).astype(np.float32).astype(np.float16)
+    with np.errstate(over="ignore"):  # norms past the fp16 range round to inf on both sides
+        lo = (exact * (1 - 1e-5)).astype(np.float32).astype(np.float16)
+        hi = (exact * (1 + 1e-5)).astype(np.float32).astype(np.float16)
     return lo != hi
 
 
 def _fp16_close(got16: np.ndarray, want16: np.ndarray, exact: np.ndarray) -> np.ndarray:
     same = got16.view(np.int16) == want16.view(np.int16)
     amb = _fp16_ambiguous(exact)
-    nbr = np.abs(got16.astype(np.float64) - exact) <= np.abs(
-        np.spacing(np.abs(exact).astype(np.float16)).astype(np.float64))
+    with np.errstate(over="ignore", invalid="ignore"):
+        nbr = np.abs(got16.astype(np.float64) - exact) <= np.abs(
+            np.spacing(np.abs(exact).astype(np.float16)).astype(np.float64))
     return same | (amb & nbr)
 
 

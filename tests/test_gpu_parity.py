@@ -66,6 +66,29 @@ def test_quantize_matches_oracle(case, dtype):
     assert int(cache["v_norm"][:, :, t_off + T:].abs().sum()) == 0
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", [(128, (4, O.MSE), (2, O.MSE), 0), (64, (2, O.PROD), (2, O.PROD), 64)],
+                         ids=["d128-mse", "d64-prod"])
+def test_quantize_norms_beyond_fp16_range(case, dtype):
+    # per-token scales from 1e2 to 3e6: norms from ~1e3 to ~3e7, so about half of them exceed
+    # the largest fp16 value and round to +inf in the stored norm (round to nearest, as the
+    # oracle's float32 -> float16 conversion does); the codes are those of the unit vector
+    d, (kb, km), (vb, vm), m = case
+    B, Hkv, T = 2, 2, 40
+    K, V = random_kv(B, Hkv, T, d, dtype=torch.float32, seed=77)
+    sc = torch.logspace(2, 6.5, T, dtype=torch.float32).view(1, 1, T, 1)
+    K, V = (K * sc).to(DT[dtype]), (V * sc.flip(2)).to(DT[dtype])
+    cache = tq.TQCache(B, Hkv, T, d, kb, vb, km, vm, m, m, seed=3, qjl_seed=9)
+    tq.tq_quantize_kv(K.cuda(), V.cuda(), cache)
+    torch.cuda.synchronize()
+    saturated = 0
+    for side, X, bits, mode in (("k", K, kb, km), ("v", V, vb, vm)):
+        recs = P.oracle_records(P.to_np(X), bits, mode, 3, 9, m or None)
+        P.compare_records(cache, side, recs)
+        saturated += sum(int(np.sum(np.isinf(r.norm16.astype(np.float64)))) for r in recs)
+    assert 0.3 * 2 * B * Hkv * T <= saturated <= 0.7 * 2 * B * Hkv * T
+
+
 def test_quantize_only_keys_or_values():
     d = 64
     K, V = _inputs(1, 2, 20, d, torch.bfloat16, seed=3)

@@ -377,6 +377,21 @@ def test_codeword_input_round_trips_exactly():
                        atol=1e-9)
 
 
+def test_norm_rounds_to_fp16_and_saturates_to_inf():
+    # the stored norm is the IEEE round-to-nearest fp16 of the float32 norm: 65504 is the
+    # largest finite fp16 value, the halfway point 65520 and anything above round to +inf
+    d = 16
+    e0 = np.zeros((4, d))
+    e0[:, 3] = [65504.0, 65519.0, 65520.0, 1.0e6]
+    r = O.quantize(e0, 3, O.MSE, seed=0)
+    got = r.norm16.astype(np.float64)
+    assert got[0] == 65504.0 and got[1] == 65504.0
+    assert np.isinf(got[2]) and np.isinf(got[3]) and np.all(got[2:] > 0)
+    # the codes are those of the unit vector, whatever the norm
+    r1 = O.quantize(e0[:1] / 65504.0, 3, O.MSE, seed=0)
+    assert np.array_equal(r.codes, np.repeat(r1.codes, 4, axis=0))
+
+
 def test_zero_vector():
     x = np.zeros((2, 64))
     x[1, 3] = 1.0
